@@ -1,0 +1,242 @@
+"""Pins of the oracle's attention, decode, smoothing and identification functions.
+
+Anchors: closed forms, invariants that hold by construction, special cases
+that reduce to plain softmax attention, and a scalar brute-force restatement of
+the tiled loop on tiny inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import attention as A
+from oracle import decode as D
+from oracle import formats as F
+from oracle import hyquant as H
+from oracle import smooth as SM
+
+
+def _rand(shape, seed, scale=1.0):
+    return (np.random.default_rng(seed).normal(size=shape) * scale).astype(np.float32)
+
+
+# ----------------------------------------------------------------------------- tiled loop
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("S", [64, 200, 256])
+def test_tiled_loop_identity_quantizer_is_softmax(causal, S):
+    q, k, v = _rand((S, 32), 1), _rand((S, 32), 2, 2.0), _rand((S, 32), 3)
+    out = A.attention_pnq(q, k, v, causal=causal, fmt="nvfp4", p_quantizer=lambda p: p)
+    ref = A.attention_plain(q, k, v, causal=causal)
+    assert np.max(np.abs(out - ref)) <= 1e-12
+
+
+def _scalar_pnq(q, k, v, causal, fmt, qmax_p=0.0):
+    """Brute-force restatement with scalar Python loops (tiny inputs only)."""
+    Sq, d = q.shape
+    Sk = k.shape[0]
+    sm = 1.0 / math.sqrt(d)
+    blk = F.block_size(fmt)
+    g = A.p_tensor_scale(fmt)
+    out = np.zeros((Sq, v.shape[1]))
+    for i in range(Sq):
+        m, l, o = -math.inf, 0.0, np.zeros(v.shape[1])
+        for t0 in range(0, Sk, 128):
+            keys = [j for j in range(t0, min(Sk, t0 + 128)) if not (causal and j > i)]
+            if not keys:
+                continue
+            s = {j: float(np.dot(q[i].astype(np.float64), k[j].astype(np.float64))) * sm for j in keys}
+            m_new = max(m, max(s.values()))
+            ptil = np.zeros(128, dtype=np.float32)
+            for j in keys:
+                ptil[j - t0] = np.float32(math.exp(s[j] - m_new))
+            c, sb = F.quantize_blocks(ptil.reshape(128 // blk, blk), fmt, qmax_p if fmt == "mxfp4" else 0.0, g)
+            phat = F.dequantize_blocks(c, sb, fmt, g).reshape(128)
+            alpha = math.exp(m - m_new) if m != -math.inf else 0.0
+            l = alpha * l + sum(phat[j - t0] for j in keys)
+            o = alpha * o + sum(phat[j - t0] * v[j].astype(np.float64) for j in keys)
+            m = m_new
+        out[i] = o / l
+    return out
+
+
+@pytest.mark.parametrize("fmt,causal,qmax_p", [("nvfp4", True, 0.0), ("mxfp4", False, 0.0),
+                                               ("mxfp4", True, 7.25)])
+def test_tiled_pnq_matches_scalar_bruteforce(fmt, causal, qmax_p):
+    S = 150                                       # two key tiles, the second ragged
+    q, k, v = _rand((S, 16), 4, 2.0), _rand((S, 16), 5, 2.0), _rand((S, 16), 6)
+    rows = np.array([0, 1, 63, 127, 128, 129, 149])
+    out = A.attention_pnq(q, k, v, causal=causal, fmt=fmt, qmax_p=qmax_p, rows=rows)
+    ref = _scalar_pnq(q[rows] if not causal else q, k, v, causal, fmt, qmax_p)
+    ref = ref if not causal else ref[rows]
+    assert np.max(np.abs(out - ref)) <= 1e-12
+
+
+# ----------------------------------------------------------------------------- PNQ invariants
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_pnq_weights_are_convex(fmt, causal):
+    S = 300
+    q, k, v = _rand((S, 64), 7, 1.5), _rand((S, 64), 8, 1.5), _rand((S, 64), 9)
+    out, w = A.attention_pnq(q, k, v, causal=causal, fmt=fmt, return_weights=True)
+    assert np.all(w >= 0)
+    assert np.max(np.abs(w.sum(axis=1) - 1.0)) <= 1e-12
+    assert np.max(np.abs(w @ v.astype(np.float64) - out)) <= 1e-12
+    if causal:
+        assert np.all(w[np.triu_indices(S, 1)] == 0)
+    lo = np.min(v, axis=0) if not causal else None
+    if lo is not None:
+        assert np.all(out >= lo - 1e-12) and np.all(out <= np.max(v, axis=0) + 1e-12)
+
+
+def test_constant_v_is_preserved_only_with_consistent_normaliser():
+    S = 384
+    q, k = _rand((S, 64), 10, 2.0), _rand((S, 64), 11, 2.0)
+    v = np.ones((S, 64), dtype=np.float32)
+    _, _, vh = A.quantize_qkv(q, k, v, "nvfp4")
+    assert np.all(vh == 1.03125)                  # 1.0 under NVFP4: scale 0.171875, code 6
+    out = A.attention_pnq(q, k, vh, causal=True, fmt="nvfp4")
+    assert np.max(np.abs(out - 1.03125)) <= 1e-12
+    bad = A.attention_pnq(q, k, vh, causal=True, fmt="nvfp4", consistent=False)
+    assert np.max(np.abs(bad - 1.03125)) > 1e-3
+
+
+def test_inconsistent_normaliser_loses_mass():
+    """HiFA4: the normaliser from unquantised exponentials overstates the mass of P_hat."""
+    S = 1024
+    q, k, v = _rand((S, 64), 12, 1.5), _rand((S, 64), 13, 1.5), _rand((S, 64), 14)
+    _, eps = A.attention_pnq(q, k, v, causal=False, fmt="nvfp4", consistent=False,
+                             rows=np.arange(0, S, 8), return_eps=True)
+    assert np.median(eps) < 0
+
+
+# ----------------------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_zero_query_gives_mean_of_values(fmt):
+    S = 260
+    q = np.zeros((S, 32), dtype=np.float32)
+    k, v = _rand((S, 32), 15), _rand((S, 32), 16)
+    out = A.attention_pnq(q, k, v, causal=False, fmt=fmt)
+    assert np.max(np.abs(out - v.astype(np.float64).mean(axis=0))) <= 1e-12
+    outc = A.attention_pnq(q, k, v, causal=True, fmt=fmt)
+    pref = np.cumsum(v.astype(np.float64), axis=0) / np.arange(1, S + 1)[:, None]
+    assert np.max(np.abs(outc - pref)) <= 1e-12
+
+
+def test_first_causal_row_and_single_key():
+    q, k, v = _rand((130, 32), 17), _rand((130, 32), 18), _rand((130, 32), 19)
+    out = A.attention_pnq(q, k, v, causal=True, fmt="nvfp4", rows=[0])
+    assert np.max(np.abs(out[0] - v[0])) <= 1e-12
+    out1 = A.attention_pnq(q[:5], k[:1], v[:1], causal=False, fmt="mxfp4")
+    assert np.max(np.abs(out1 - v[0])) <= 1e-12
+
+
+def test_quantized_attention_is_close_to_unquantized():
+    S = 256
+    q, k, v = _rand((S, 64), 20), _rand((S, 64), 21), _rand((S, 64), 22)
+    qh, kh, vh = A.quantize_qkv(q, k, v, "nvfp4")
+    out = A.attention_pnq(qh, kh, vh, causal=True, fmt="nvfp4")
+    ref = A.attention_plain(q, k, v, causal=True)
+    rel = np.abs(out - ref).sum() / np.abs(ref).sum()
+    assert 1e-3 < rel < 0.2
+
+
+def test_lse_of_a_single_tile():
+    S = 100
+    q, k, v = _rand((S, 32), 23), _rand((S, 32), 24), _rand((S, 32), 25)
+    _, lse = A.attention_pnq(q, k, v, causal=False, fmt="nvfp4", return_lse=True)
+    s = (q.astype(np.float64) @ k.astype(np.float64).T) / math.sqrt(32)
+    m = s.max(axis=1)
+    p = np.exp(s - m[:, None])
+    ph = A.quantize_p(np.pad(p, ((0, 0), (0, 28))).astype(np.float32), "nvfp4")[:, :S]
+    assert np.max(np.abs(lse - (m + np.log(ph.sum(axis=1))))) <= 1e-12
+
+
+# ----------------------------------------------------------------------------- decode
+def test_decode_without_hybrid_parts_is_quantized_attention():
+    L, d = 320, 32
+    q, k, v = _rand((4, d), 26), _rand((L, d), 27), _rand((L, d), 28)
+    out = D.decode_group(q, k, v, np.zeros(0, dtype=np.int64), 0, "nvfp4")
+    kh, vh = D.quantize_fp4_region(k, v, np.zeros(0, dtype=np.int64), "nvfp4")
+    ref = np.stack([A.attention_pnq(q[i:i + 1], kh, vh, causal=False, fmt="nvfp4",
+                                    p_quantizer=lambda p: p)[0] for i in range(4)])
+    assert np.max(np.abs(out - ref)) <= 1e-12
+    # the FP4 region quantises exactly like the tensor quantiser (K along d, V along tokens)
+    kh2 = F.dequantize_rows(*F.quantize_rows(k, "nvfp4"), "nvfp4")
+    assert np.array_equal(kh, kh2)
+
+
+def test_decode_all_full_precision_is_plain_attention():
+    L, d, W = 256, 32, 64
+    q, k, v = _rand((4, d), 29), _rand((L, d), 30), _rand((L, d), 31)
+    hp = np.arange(L - W)
+    out = D.decode_group(q, k, v, hp, W, "nvfp4")
+    ref = A.attention_plain(q, k, v, causal=False)
+    assert np.max(np.abs(out - ref)) <= 1e-12
+
+
+def test_decode_key_classes_each_count_once():
+    L, d, W = 256, 32, 32
+    q, k, v = _rand((2, d), 32), _rand((L, d), 33), _rand((L, d), 34)
+    hp = np.array([3, 70, 150])
+    out = D.decode_group(q, k, v, hp, W, "mxfp4")
+    kh, vh = D.quantize_fp4_region(k[:L - W], v[:L - W], hp, "mxfp4")
+    keep = np.setdiff1d(np.arange(L - W), hp)
+    keys = np.concatenate([kh[keep], k[hp], k[L - W:]])
+    vals = np.concatenate([vh[keep], v[hp], v[L - W:]])
+    assert len(keys) == L
+    assert np.max(np.abs(out - A.attention_plain(q, keys, vals, causal=False))) <= 1e-12
+    # zero-filling excluded slots keeps them out of the V block maxima
+    v2 = v.copy()
+    v2[hp] = 1e4
+    _, vh2 = D.quantize_fp4_region(k[:L - W], v2[:L - W], hp, "mxfp4")
+    assert np.array_equal(vh2[keep], vh[keep])
+
+
+# ----------------------------------------------------------------------------- smoothing
+def test_smoothing_is_exact_and_nearest_power_of_two():
+    rng = np.random.default_rng(35)
+    qc = rng.normal(size=(8, 64, 32)).astype(np.float32)
+    kc = rng.normal(size=(2, 64, 32)).astype(np.float32)
+    kc[:, :, 5] *= 20
+    lam = SM.calibrate(qc, kc)
+    assert lam.shape == (2, 32)
+    assert np.all(np.log2(lam) == np.round(np.log2(lam)))
+    # independent evaluation through log2/sqrt, away from ties
+    qmax = np.abs(qc).reshape(2, 4 * 64, 32).max(axis=1)
+    kmax = np.abs(kc).max(axis=1)
+    r = (kmax / qmax).astype(np.float32)
+    e = np.log2(np.sqrt(r.astype(np.float64)))
+    safe = np.abs(e - np.floor(e) - 0.5) > 1e-6
+    assert np.array_equal(np.log2(lam)[safe], np.clip(np.round(e), -8, 8)[safe])
+    assert np.all(lam[:, 5] >= 4)                           # the outlier channel moves to Q
+    # exact invariance of Q K^T
+    for h in range(2):
+        qq = qc[4 * h].astype(np.float64)
+        kk = kc[h].astype(np.float64)
+        lhs = (qq * lam[h]) @ (kk / lam[h]).T
+        assert np.array_equal(lhs, qq @ kk.T)
+
+
+def test_smoothing_ties_and_edges():
+    assert SM.nearest_pow2_exponent_of_sqrt(np.array([2.0, 0.5, 8.0, 1.0, 1.99, 0.26])).tolist() == [1, 0, 2, 0, 0, -1]
+    qc = np.zeros((1, 4, 3), dtype=np.float32)
+    kc = np.zeros((1, 4, 3), dtype=np.float32)
+    qc[0, 0, 0] = 1.0
+    kc[0, 0, 1] = 1.0
+    lam = SM.calibrate(qc, kc)
+    assert lam.tolist() == [[2.0 ** -8, 2.0 ** 8, 1.0]]
+
+
+# ----------------------------------------------------------------------------- identification
+def test_vertical_lines_recover_planted_positions():
+    rng = np.random.default_rng(36)
+    N, d = 2000, 64
+    u = rng.normal(size=d)
+    u /= np.linalg.norm(u)
+    k = rng.normal(size=(N, d))
+    planted = np.sort(rng.choice(N, 100, replace=False))
+    k[planted] += 6.0 * u
+    q = rng.normal(size=(64, d)) + 3.0 * u
+    sel = H.select_vertical_lines(q, k, 0.05)
+    assert len(sel) == 100
+    assert len(np.intersect1d(sel, planted)) >= 95
