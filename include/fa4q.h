@@ -1,0 +1,232 @@
+/*
+ * fa4q.h - C ABI of the fused 4-bit microscaled FlashAttention library (B200, sm_100a).
+ *
+ * Plain pointers and sizes only.  Unless stated otherwise every pointer is a CUDA device
+ * pointer owned by the caller, 16-byte aligned, and every call is asynchronous on `stream`
+ * (a cudaStream_t passed as void*; NULL = the legacy default stream).  The library keeps
+ * no per-call state; its only global state is one device status word written by kernels
+ * whose bounded waits expire (read it with fa4q_device_status).
+ *
+ * Errors: argument errors are caught on the host before any launch and return
+ * FA4Q_ERR_INVALID_ARG; shapes outside the supported set return FA4Q_ERR_UNSUPPORTED;
+ * a failed launch returns FA4Q_ERR_CUDA.  No call ever falls back to a CPU path.
+ *
+ * Formats (BitDecoding-FP4: Algorithm-System Co-Design for Native FP4 KV Cache Decoding,
+ * section "The KV Cache Bottleneck in Long-Context LLM Serving"; MXAttention, Abstract):
+ *   elements are E2M1 (+-{0, .5, 1, 1.5, 2, 3, 4, 6}), two per byte, element 2i in the low
+ *   nibble of byte i;
+ *   NVFP4: 16-element blocks, one unsigned E4M3 scale byte each, optional FP32 tensor scale g;
+ *   MXFP4: 32-element blocks, one E8M0 scale byte each (2^(b-127)).
+ *
+ * Scale-factor layouts:
+ *   FA4Q_SF_ROWMAJOR: matrix [R][C] -> bytes [R][C/blk].
+ *   FA4Q_SF_TILED   : the layout the block-scaled tensor-core MMA consumes.  Rows are
+ *     grouped in tiles of 128 and scale columns in groups of 4; each (row tile, group)
+ *     is a 512-byte atom.  nRT = ceil(R/128), nG = ceil(C/128) * (32/blk) (the columns
+ *     are padded to whole 128-element tiles).  Atom (rt, g) starts at (rt*nG + g)*512;
+ *     row r, scale column k sits at byte (r%32)*16 + ((r%128)/32)*4 + (k%4) of atom
+ *     (r/128, k/4).  Padding bytes hold the scale of an all-zero block (0).
+ *     Size: fa4q_sf_tiled_bytes(R, C, fmt).
+ */
+#ifndef FA4Q_H_
+#define FA4Q_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FA4Q_NVFP4 = 0, FA4Q_MXFP4 = 1 } fa4q_format;
+
+typedef enum {
+  FA4Q_OK = 0,
+  FA4Q_ERR_INVALID_ARG = 1,
+  FA4Q_ERR_UNSUPPORTED = 2,
+  FA4Q_ERR_CUDA = 3,
+  FA4Q_ERR_TIMEOUT = 4
+} fa4q_status;
+
+typedef enum {
+  FA4Q_AXIS_INNER = 0, /* blocks along the contiguous axis (Q, K: along the head dim)      */
+  FA4Q_AXIS_OUTER = 1  /* blocks along rows (tokens); the output is transposed (V -> V^T)  */
+} fa4q_axis;
+
+typedef enum { FA4Q_SF_ROWMAJOR = 0, FA4Q_SF_TILED = 1 } fa4q_sf_layout;
+
+/* Human-readable name of a status code (static string). */
+const char* fa4q_status_string(fa4q_status s);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int fa4q_version(void);
+
+/* Bytes of a FA4Q_SF_TILED scale array for an [rows][cols] matrix. */
+size_t fa4q_sf_tiled_bytes(int64_t rows, int64_t cols, fa4q_format fmt);
+
+/*
+ * fa4q_quantize - blockwise E2M1 quantisation with per-block scales.
+ *
+ * Source: BitDecoding-FP4, "The KV Cache Bottleneck ..." (block microscaling, E2M1
+ * elements, E8M0 / E4M3 scales); MXAttention, Abstract (power-of-two scaling, scale
+ * bound Qmax = 7.25); HiFA4, Abstract (Smooth-QK: a static per-channel multiplier applied
+ * after RoPE, before quantisation).
+ *
+ * x           bf16, logically [groups][rows][cols]; element (g, r, c) at
+ *             x[(g*rows + r)*row_stride + c].  row_stride >= cols, multiple of 8.
+ * fmt         FA4Q_NVFP4 or FA4Q_MXFP4.
+ * axis        INNER: blocks of blk consecutive columns; cols % blk == 0.
+ *               packed_out [groups][rows][cols/2]; scales per `sf_layout` over the
+ *               [rows][cols] matrix of each group (groups stacked, each group's tiled
+ *               array is fa4q_sf_tiled_bytes(rows, cols) bytes).
+ *             OUTER: blocks of blk consecutive rows of each column; output transposed.
+ *               rows_pad = rows rounded up to 32 (zero tokens in the padding);
+ *               packed_out [groups][cols][rows_pad/2]; scales over the [cols][rows_pad]
+ *               transposed matrix of each group.
+ * qmax        scale bound.  NVFP4: 0 -> 6; scale = UE4M3(amax / (qmax * g)).
+ *             MXFP4: 0 -> OCP rule (e = floor(log2 amax) - 2); > 0 -> UOS rule (the
+ *             smallest e with amax <= qmax * 2^e), e.g. 7.25.
+ * tensor_scale  NVFP4 second-level FP32 scale g (must be > 0; 1 = none); ignored for MXFP4.
+ * smooth_mul  nullable FP32 [n][cols]; row r of group g is multiplied elementwise by
+ *             smooth_mul[((g % smooth_heads) / smooth_ratio)*cols + c] before the block
+ *             maximum (INNER only).  Pass the Q multipliers with smooth_ratio = Hq/Hkv and
+ *             the K multipliers (1/lambda) with smooth_ratio = 1; smooth_heads = heads.
+ * The FP32 order of operations is fixed (product qmax*g first, IEEE division), so the
+ * output is bit-identical to the reference rules.
+ */
+fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows, int64_t cols,
+                          int64_t row_stride, fa4q_format fmt, fa4q_axis axis, float qmax,
+                          float tensor_scale, const float* smooth_mul, int64_t smooth_heads,
+                          int64_t smooth_ratio, fa4q_sf_layout sf_layout, uint8_t* packed_out,
+                          uint8_t* scales_out, void* stream);
+
+/*
+ * fa4q_smooth_calibrate - static per-channel Smooth-QK multipliers from a calibration draw.
+ *
+ * Source: HiFA4, Abstract (calibration-static per-channel equivalent rescaling of Q and K
+ * after RoPE, moving quantisation difficulty from K to Q); BitDecoding-FP4, "Outlier-Aware
+ * Key Quantization" (static smoothing coefficients estimated during calibration).
+ * Rule: r_c = max_t|K_tc| / max_{t, q-heads of the kv-head}|Q_tc| (FP32 division);
+ * lambda_c = sqrt(r_c) rounded to the nearest power of two (log domain, ties up), clamped
+ * to [2^-8, 2^8]; r = 0 -> 2^-8, r = inf -> 2^8, NaN -> 1.
+ *
+ * q_cal bf16 [Hq][T][d], k_cal bf16 [Hkv][T][d]; outputs FP32 [Hkv][d]:
+ * mul_q = lambda, mul_k = 1/lambda (both exact powers of two).
+ */
+fa4q_status fa4q_smooth_calibrate(const void* q_cal, const void* k_cal, int Hq, int Hkv, int T,
+                                  int d, float* mul_q, float* mul_k, void* stream);
+
+/*
+ * fa4q_attn_fwd - fused 4-bit prefill attention (one launch).
+ *
+ * Source: HiFA4, Abstract (QK^T and PV as 4-bit GEMMs under an online softmax;
+ * P-Reordering: the normaliser accumulates the same quantised P_hat that feeds the PV
+ * GEMM, fused into that GEMM); MXAttention, Abstract (Pre-Normalization Quantization:
+ * the unnormalised exponentials are quantised before the row sum); BitDecoding-FP4,
+ * "Underflow-Aware Probability Scaling" (NVFP4 P uses the static tensor scale
+ * g_P = 1/(6*448)).  Key tiles are 128 wide; P blocks run along keys.
+ *
+ * q, q_sf     packed [B][Hq][S_q][d/2]; tiled scales, one [S_q][d] matrix per (b, h).
+ * k, k_sf     packed [B][Hkv][S_k][d/2]; tiled scales per (b, kv-head).
+ * vt, vt_sf   V^T packed [B][Hkv][d][S_kpad/2], S_kpad = S_k rounded up to 32 (the OUTER
+ *             output of fa4q_quantize); tiled scales per (b, kv-head) over [d][S_kpad].
+ * g_q,g_k,g_v NVFP4 tensor scales used when quantising (1 for MXFP4).
+ * d           64 or 128.  Hq % Hkv == 0; q-head h reads kv-head h*Hkv/Hq.
+ * qmax_p      MXFP4 P scale rule (0 = OCP, > 0 = UOS bound); ignored for NVFP4.
+ * causal      top-left aligned (query i sees keys <= i); requires S_q == S_k.
+ * sm_scale    0 -> 1/sqrt(d).
+ * out         [B][Hq][S_q][d], bf16 (out_is_fp32 = 0) or fp32.
+ * lse         nullable FP32 [B][Hq][S_q]: natural log-sum-exp m + ln(sum P_hat).
+ */
+fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                          const uint8_t* k_sf, const uint8_t* vt, const uint8_t* vt_sf,
+                          float g_q, float g_k, float g_v, int B, int Hq, int Hkv, int S_q,
+                          int S_k, int d, fa4q_format fmt, float qmax_p, int causal,
+                          float sm_scale, void* out, int out_is_fp32, float* lse, void* stream);
+
+/*
+ * Paged FP4 KV cache (BitDecoding-FP4, "System-Level Optimization": fixed-size token
+ * blocks mapped to physical memory through a block table).  Page size 64 tokens.
+ * For physical page p and kv-head h:
+ *   k_pages  [P][Hkv][64][d/2]      K rows, blocks along d
+ *   k_sf     [P][Hkv][64][d/blk]    row-major scales
+ *   vt_pages [P][Hkv][d][32]        V^T rows (64 tokens), blocks along tokens
+ *   vt_sf    [P][Hkv][d][64/blk]
+ * block_table [B][max_pages] int32 maps logical page j of sequence b to a physical page.
+ * fp4_len [B] int32: positions [0, fp4_len[b]) of sequence b live in the FP4 pages.
+ * excl_mask nullable uint64 [B][Hkv][max_pages]: bit t of word j marks position 64*j + t
+ *   as held in the full-precision set instead (its FP4 slot is zero and is skipped).
+ */
+
+/*
+ * fa4q_quantize_kv_pages - quantise K and V of positions [0, fp4_len[b]) into the paged
+ * FP4 cache, zero-filling excluded slots before quantisation.
+ * Source: HyQuant (Hybrid-Precision Quantization for LLM Attention): the KV cache is
+ * stored in the hybrid way, vertical-line tokens in full precision, the rest in 4 bits.
+ *
+ * k, v bf16 [B][Hkv][L][d] (contiguous; L >= max fp4_len).  Writes only the pages that
+ * block_table maps for j < ceil(fp4_len[b]/64); slots >= fp4_len in the last page are zero.
+ */
+fa4q_status fa4q_quantize_kv_pages(const void* k, const void* v, int B, int Hkv, int L, int d,
+                                   const int32_t* fp4_len, const uint64_t* excl_mask,
+                                   const int32_t* block_table, int max_pages, fa4q_format fmt,
+                                   float g_k, float g_v, uint8_t* k_pages, uint8_t* k_sf,
+                                   uint8_t* vt_pages, uint8_t* vt_sf, void* stream);
+
+/* Workspace bytes fa4q_decode needs for `num_splits` (0 = the automatic choice). */
+size_t fa4q_decode_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int num_splits);
+
+/*
+ * fa4q_decode - one query token per sequence over the hybrid cache: FP4 paged remainder
+ * (dequantised inside the scan), a BF16 vertical-line set and a BF16 window, under one
+ * softmax; split-K over pages with a combine of the (m, l, o) partials.
+ * Source: HyQuant (vertical-line + window tokens in full precision, fused-dequant decode
+ * scan, no full-precision cache materialised); BitDecoding-FP4, "System-Level
+ * Optimization" (paged cache, block table).
+ *
+ * q        bf16 [B][Hq][d]; out bf16 [B][Hq][d].  d == 128, Hq % Hkv == 0, Hq/Hkv <= 8.
+ * hp_k, hp_v  nullable bf16 [B][Hkv][max_hp][d]; hp_count int32 [B][Hkv] (<= max_hp).
+ * win_k, win_v nullable bf16 [B][Hkv][W][d]; win_len int32 [B] (<= W).
+ * g_k, g_v NVFP4 tensor scales of the pages (1 for MXFP4).  sm_scale 0 -> 1/sqrt(d).
+ * workspace  device scratch of fa4q_decode_workspace_size bytes (caller-owned).
+ */
+fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
+                        const uint8_t* vt_pages, const uint8_t* vt_sf,
+                        const int32_t* block_table, const int32_t* fp4_len,
+                        const uint64_t* excl_mask, const void* hp_k, const void* hp_v,
+                        const int32_t* hp_count, const void* win_k, const void* win_v,
+                        const int32_t* win_len, int B, int Hq, int Hkv, int d, int max_pages,
+                        int max_hp, int W, fa4q_format fmt, float g_k, float g_v,
+                        float sm_scale, void* out, void* workspace, size_t workspace_bytes,
+                        int num_splits, void* stream);
+
+/*
+ * fa4q_selftest_block_mma - diagnostic: one 128 x N x K block-scaled FP4 tensor-core
+ * product D = A * B^T (FP32), the same MMA path the prefill kernel uses.
+ * a packed [128][K/2], b packed [N][K/2] (K-major), a_sf / b_sf FA4Q_SF_TILED over
+ * [128][K] and [N][K]; d_out FP32 [128][N].  K in {64, 128}; N in {16, 32, ..., 256}.
+ */
+fa4q_status fa4q_selftest_block_mma(const uint8_t* a, const uint8_t* a_sf, const uint8_t* b,
+                                    const uint8_t* b_sf, int N, int K, fa4q_format fmt,
+                                    float* d_out, void* stream);
+
+/*
+ * fa4q_device_status - synchronise `stream`, then read and clear the device status word.
+ * Returns FA4Q_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call
+ * (*detail, if non-null, receives the kernel-specific code), FA4Q_OK otherwise.
+ */
+fa4q_status fa4q_device_status(void* stream, uint32_t* detail);
+
+/*
+ * fa4q_selftest_wait_timeout - diagnostic: launch one kernel that waits, with the same
+ * bounded-wait helper every pipelined kernel uses, on a barrier nothing will complete, for
+ * `polls` polls.  The wait expires, the kernel records FA4Q_ERR_TIMEOUT in the device status
+ * word and returns; no GPU hang or fault is involved.  Read it with fa4q_device_status.
+ */
+fa4q_status fa4q_selftest_wait_timeout(uint32_t polls, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA4Q_H_ */

@@ -1,0 +1,719 @@
+// attn_fwd.cu - fused 4-bit microscaled FlashAttention prefill for B200 (sm_100a).
+//
+// What it computes (per (batch, q-head), 128-row query tile, key tiles of 128):
+//   S_j = Q_hat K_hat_j^T                 block-scaled FP4 tensor-core MMA, FP32 in TMEM
+//   m   = max(m, rowmax S_j)              exact running maximum every tile
+//   P~  = exp(S_j - m)                    unnormalised exponentials (FP32)
+//   P^  = E2M1 blocks of P~ along keys    pre-normalisation quantisation (PNQ)
+//   [O | l] = alpha [O | l] + P^ [V_hat | 1]   both FP4 MMAs; l accumulates the same P^
+//   out = O / l * g_v
+// Sources: HiFA4 (Training-Free 4-bit FlashAttention on Ascend HIF4 NPUs), Abstract -
+// QK^T and PV as 4-bit GEMMs under an online softmax, P-Reordering (normaliser from the
+// quantised P^, fused into the PV GEMM); MXAttention, Abstract - Pre-Normalization
+// Quantization of the unnormalised exponentials before the row sum; BitDecoding-FP4,
+// "Underflow-Aware Probability Scaling" - NVFP4 P with the static tensor scale 1/(6*448);
+// "System-Level Optimization" - transposed softmax: P blocks run along the MMA reduction
+// (key) axis so P is quantised in registers and never leaves the SM.
+//
+// Kernel structure (one CTA per query tile, 256 threads, one CTA per SM):
+//   warp 0      TMA producer: Q tile once, then K, V^T tiles and their scale atoms through
+//               an NST-deep shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
+//   warp 1      TMEM owner and MMA issuer (one elected thread): tcgen05.cp of the scale
+//               atoms into TMEM, tcgen05.mma kind::mxf4nvf4 (NVFP4) or kind::mxf4 (MXFP4).
+//   warps 4-7   softmax: one query row per thread; tcgen05.ld of S, mask, running max,
+//               exp2, block scales, cvt to E2M1, P^ to shared memory (the A operand of the
+//               PV MMA), rescale of O and l in TMEM when the maximum moves, epilogue.
+// TMEM (512 columns): S double buffer [0,256), O [256,256+D), l [384,400), scale factors
+// [400,464).  Every mbarrier wait is bounded; on expiry the CTA records a status bit,
+// skips the remaining waits, drains its own copies and MMAs and exits.
+#include <math.h>
+
+#include "fa4q_common.cuh"
+#include "fa4q_internal.h"
+
+namespace fa4q {
+
+static __device__ uint32_t g_attn_status;
+
+constexpr int kBM = 128;
+constexpr int kBN = 128;
+constexpr int kThreads = 256;
+constexpr int kStages = 3;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kGpNvfp4 = 1.0f / 2688.0f;  // g_P = 1/(6*448), rounded to FP32
+
+// TMEM column map
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColL = 384;
+constexpr uint32_t kColSfQ = 400, kColSfK = 408, kColSfP = 424, kColSfV = 440, kColSfOne = 456;
+
+template <int D, bool MX>
+struct Cfg {
+  static constexpr int kBlk = MX ? 32 : 16;
+  static constexpr int kQBytes = kBM * D / 2;
+  static constexpr int kKBytes = kBN * D / 2;
+  static constexpr int kVBytes = D * kBN / 2;
+  static constexpr int kPBytes = kBM * kBN / 2;
+  static constexpr int kSfQAtoms = (D / kBlk + 3) / 4;  // atoms per row tile actually read
+  static constexpr int kSfGroups = 32 / kBlk;           // padded groups per 128 columns
+  static constexpr int kSfTileAtoms = 32 / kBlk;        // atoms per 128-key tile (P, V)
+  static constexpr int kKStepsQK = D / 64;
+  static constexpr int kQKSwizzle = D == 128 ? kSwiz64 : kSwiz32;
+  static constexpr int kQKSbo = D == 128 ? 512 : 256;
+};
+
+template <int D, bool MX>
+struct __align__(1024) Smem {
+  using C = Cfg<D, MX>;
+  uint8_t q[C::kQBytes];
+  uint8_t k[kStages][C::kKBytes];
+  uint8_t v[kStages][C::kVBytes];
+  uint8_t p[2][C::kPBytes];
+  uint8_t ones[1024];
+  uint8_t sfq[2 * 512];
+  uint8_t sfk[kStages][2 * 512];
+  uint8_t sfv[kStages][2 * 512];
+  uint8_t sfp[2][2 * 512];
+  uint8_t sfone[2 * 512];
+  uint64_t bar_q;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full[2];
+  uint64_t s_free[2];
+  uint64_t p_full[2];
+  uint64_t o_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
+
+struct AttnParams {
+  const uint8_t* q_sf;
+  const uint8_t* k_sf;
+  const uint8_t* vt_sf;
+  void* out;
+  float* lse;
+  int B, Hq, Hkv, S_q, S_k, S_kpad;
+  int n_qtiles;
+  float score_scale_log2;  // sm_scale * g_q * g_k * log2(e)
+  float g_v;
+  float qmax_p;
+  int causal;
+  int out_fp32;
+};
+
+// Bounded wait that gives up at once when another role of the CTA already gave up.
+FA4Q_DEVINL bool cta_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
+                          uint32_t code) {
+  if (*abort_flag) return false;
+  for (uint32_t i = 0; i < kWaitPolls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023) == 1023 && *abort_flag) return false;
+  }
+  atomicOr(&g_attn_status, code);
+  *abort_flag = 1;
+  return false;
+}
+
+FA4Q_DEVINL float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+FA4Q_DEVINL float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+FA4Q_DEVINL void tmem_ld1(uint32_t taddr, uint32_t& r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+}
+FA4Q_DEVINL void tmem_st1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
+
+// byte offset of (row r, 16-byte chunk c) in a K-major tile with 64-byte rows, 64B swizzle
+FA4Q_DEVINL uint32_t swz64_offset(uint32_t r, uint32_t c) {
+  return (r >> 3) * 512 + (r & 7) * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+}
+// ... 32-byte rows, 32B swizzle
+FA4Q_DEVINL uint32_t swz32_offset(uint32_t r, uint32_t c) {
+  return (r >> 3) * 256 + (r & 7) * 32 + ((c ^ ((r >> 2) & 1)) << 4);
+}
+
+// Issue one block-scaled FP4 MMA step.  For MXFP4 the two scales of a 64-element step sit
+// at byte 2*(step%2) of the 4-byte TMEM scale word (selected by the descriptor's sf id).
+template <bool MX>
+FA4Q_DEVINL void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, int N, int step,
+                          uint32_t sfa_col, uint32_t sfb_col, uint32_t acc) {
+  if constexpr (MX) {
+    const uint32_t id = 2u * (step & 1);
+    const uint32_t idesc = make_idesc_fp4(N, true, id, id);
+    mma_mxf4(d_tmem, adesc, bdesc, idesc, sfa_col + 4u * (step >> 1), sfb_col + 4u * (step >> 1),
+             acc);
+  } else {
+    const uint32_t idesc = make_idesc_fp4(N, false, 0, 0);
+    mma_nvf4(d_tmem, adesc, bdesc, idesc, sfa_col + 4u * step, sfb_col + 4u * step, acc);
+  }
+}
+
+template <int D, bool MX, bool CAUSAL>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = Cfg<D, MX>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D, MX>& sm = *reinterpret_cast<Smem<D, MX>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  volatile uint32_t* abort_flag = &sm.abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // causal: heaviest query tiles first
+  const int qt = CAUSAL ? (p.n_qtiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (p.Hq / p.Hkv);
+  const int bh_q = b * p.Hq + h, bh_k = b * p.Hkv + hk;
+  const int n_ktiles_all = (p.S_k + kBN - 1) / kBN;
+  const int n_tiles = CAUSAL ? min(qt + 1, n_ktiles_all) : n_ktiles_all;
+
+  // ---------------------------------------------------------------- setup
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar_q, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_free[s], 4);
+      mbar_init(&sm.p_full[s], 4);
+    }
+    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 2) {
+    // constant B operand of the normaliser MMA: 16 rows of E2M1 ones (code 2) and unit scales
+    uint32_t* o32 = reinterpret_cast<uint32_t*>(sm.ones);
+    for (int i = lane; i < 256; i += 32) o32[i] = 0x22222222u;
+    uint32_t* s32 = reinterpret_cast<uint32_t*>(sm.sfone);
+    const uint32_t one = MX ? 0x7F7F7F7Fu : 0x38383838u;
+    for (int i = lane; i < 256; i += 32) s32[i] = one;
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const int nrt_q = (p.S_q + 127) / 128, nrt_k = (p.S_k + 127) / 128;
+      const int ng_v = ((p.S_kpad + 127) / 128) * C::kSfGroups;
+      mbar_arrive_expect_tx(&sm.bar_q, C::kQBytes + C::kSfQAtoms * 512);
+      tma_load_3d(sm.q, &tm_q, 0, qt * kBM, bh_q, &sm.bar_q);
+      bulk_load(sm.sfq, p.q_sf + ((int64_t)bh_q * nrt_q + qt) * C::kSfGroups * 512,
+                C::kSfQAtoms * 512, &sm.bar_q);
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int s = j % kStages;
+        if (j >= kStages && !cta_wait(&sm.kv_empty[s], ((j / kStages) - 1) & 1, abort_flag,
+                                      kStatusTimeoutTmaFull))
+          break;
+        mbar_arrive_expect_tx(&sm.kv_full[s], C::kKBytes + C::kVBytes + C::kSfQAtoms * 512 +
+                                                  C::kSfTileAtoms * 512);
+        tma_load_3d(sm.k[s], &tm_k, 0, j * kBN, bh_k, &sm.kv_full[s]);
+        bulk_load(sm.sfk[s], p.k_sf + ((int64_t)bh_k * nrt_k + j) * C::kSfGroups * 512,
+                  C::kSfQAtoms * 512, &sm.kv_full[s]);
+        tma_load_3d(sm.v[s], &tm_v, j * (kBN / 2), 0, bh_k, &sm.kv_full[s]);
+        bulk_load(sm.sfv[s], p.vt_sf + (int64_t)bh_k * ng_v * 512 + (int64_t)j * C::kSfTileAtoms * 512,
+                  C::kSfTileAtoms * 512, &sm.kv_full[s]);
+        issued = j + 1;
+      }
+      // drain: every issued stage must have landed before the CTA may exit
+      for (int j = max(0, issued - kStages); j < issued; ++j)
+        mbar_wait(&sm.kv_full[j % kStages], (j / kStages) & 1, &g_attn_status, kStatusTimeoutDrain);
+      if (!(*abort_flag)) mbar_wait(&sm.bar_q, 0, &g_attn_status, kStatusTimeoutDrain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      const uint32_t q_addr = smem_u32(sm.q);
+      const uint32_t ones_addr = smem_u32(sm.ones);
+      bool ok = cta_wait(&sm.bar_q, 0, abort_flag, kStatusTimeoutMma);
+      tc_fence_after();
+      for (int a = 0; a < C::kSfQAtoms; ++a) tmem_cp_sf_atom(tmem + kColSfQ + 4 * a, smem_u32(sm.sfq + 512 * a));
+      for (int a = 0; a < C::kSfTileAtoms; ++a)
+        tmem_cp_sf_atom(tmem + kColSfOne + 4 * a, smem_u32(sm.sfone + 512 * a));
+      for (int j = 0; ok && j <= n_tiles; ++j) {
+        if (j < n_tiles) {
+          const int s = j % kStages, sb = j & 1;
+          if (!cta_wait(&sm.kv_full[s], (j / kStages) & 1, abort_flag, kStatusTimeoutMma)) break;
+          if (j >= 2 && !cta_wait(&sm.s_free[sb], ((j - 2) >> 1) & 1, abort_flag, kStatusTimeoutMma))
+            break;
+          tc_fence_after();
+          for (int a = 0; a < C::kSfQAtoms; ++a)
+            tmem_cp_sf_atom(tmem + kColSfK + 8 * sb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
+          const uint32_t k_addr = smem_u32(sm.k[s]);
+#pragma unroll
+          for (int ks = 0; ks < C::kKStepsQK; ++ks) {
+            const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+            const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+            mma_step<MX>(tmem + (sb ? kColS1 : kColS0), ad, bd, kBN, ks, tmem + kColSfQ,
+                         tmem + kColSfK + 8 * sb, ks > 0);
+          }
+          tc_commit(&sm.s_full[sb]);
+        }
+        if (j >= 1) {
+          const int jp = j - 1, s = jp % kStages, pb = jp & 1;
+          if (!cta_wait(&sm.p_full[pb], (jp >> 1) & 1, abort_flag, kStatusTimeoutMma)) break;
+          tc_fence_after();
+          for (int a = 0; a < C::kSfTileAtoms; ++a) {
+            tmem_cp_sf_atom(tmem + kColSfP + 8 * pb + 4 * a, smem_u32(sm.sfp[pb] + 512 * a));
+            tmem_cp_sf_atom(tmem + kColSfV + 8 * pb + 4 * a, smem_u32(sm.sfv[s] + 512 * a));
+          }
+          const uint32_t p_addr = smem_u32(sm.p[pb]);
+          const uint32_t v_addr = smem_u32(sm.v[s]);
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
+            const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
+            const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
+            const uint32_t acc = (jp > 0 || ks > 0) ? 1u : 0u;
+            mma_step<MX>(tmem + kColO, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
+            mma_step<MX>(tmem + kColL, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
+          }
+          tc_commit(&sm.o_done);
+          tc_commit(&sm.kv_empty[s]);
+        }
+      }
+      // drain: all MMAs this thread issued complete before TMEM is released
+      tc_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, &g_attn_status, kStatusTimeoutDrain);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / PNQ / epilogue
+    const int wq = warp - 4;                       // TMEM lane quadrant
+    const int r = wq * 32 + lane;                  // row within the query tile
+    const int row = qt * kBM + r;                  // query index
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const float sc = p.score_scale_log2;
+    float m = -INFINITY;                            // running max (log2 domain)
+    bool ok = true;
+    for (int j = 0; j < n_tiles && ok; ++j) {
+      const int sb = j & 1;
+      // warp-uniform outcome: every lane waits, all lanes take the same branch
+      if (!__all_sync(0xffffffffu, cta_wait(&sm.s_full[sb], (j >> 1) & 1, abort_flag, kStatusTimeoutSoftmax))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[kBN];
+#pragma unroll
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + 32 * c, raw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free[sb]);
+      // masking: keys beyond S_k, and (causal) keys after this query
+      const int key0 = j * kBN;
+      const bool edge = (key0 + kBN > p.S_k) || (CAUSAL && key0 + kBN - 1 > qt * kBM);
+      if (edge) {
+        const int lim = CAUSAL ? min(p.S_k - key0, row - key0 + 1) : (p.S_k - key0);
+#pragma unroll
+        for (int i = 0; i < kBN; ++i)
+          if (i >= lim) s[i] = -INFINITY;
+      }
+      // block maxima of the raw scores (the scale is positive), then the tile maximum
+      constexpr int kNB = kBN / C::kBlk;
+      float bmax[kNB];
+#pragma unroll
+      for (int bi = 0; bi < kNB; ++bi) {
+        float mx = s[bi * C::kBlk];
+#pragma unroll
+        for (int i = 1; i < C::kBlk; ++i) mx = fmaxf(mx, s[bi * C::kBlk + i]);
+        bmax[bi] = mx;
+      }
+      float tmax = bmax[0];
+#pragma unroll
+      for (int bi = 1; bi < kNB; ++bi) tmax = fmaxf(tmax, bmax[bi]);
+      const float m_new = fmaxf(m, tmax * sc);
+      const float alpha = ex2_approx(m - m_new);    // 0 on the first tile
+      // per block: amax = exp2(bmax*sc - m_new); scale; y_i = exp2(s_i*sc - m_new - log2(scale))
+      uint32_t packed[kBN / 8];
+      uint32_t sfw[kNB / 4 > 0 ? kNB / 4 : 1];
+#pragma unroll
+      for (int w = 0; w < (kNB / 4 > 0 ? kNB / 4 : 1); ++w) sfw[w] = 0;
+#pragma unroll
+      for (int bi = 0; bi < kNB; ++bi) {
+        const float amax = ex2_approx(fmaf(bmax[bi], sc, -m_new));
+        float off;
+        uint32_t code;
+        if constexpr (MX) {
+          const int e = mx_exponent(amax, p.qmax_p);
+          code = static_cast<uint32_t>(e + 127);
+          off = m_new + static_cast<float>(e);
+          if (!(amax > 0.0f)) off = INFINITY;
+        } else {
+          const float t = __fdiv_rn(amax, 6.0f * kGpNvfp4);       // amax / (6 * g_P)
+          code = ue4m3_encode(t);
+          const float sf = ue4m3_decode(code);
+          off = sf > 0.0f ? m_new + lg2_approx(sf * kGpNvfp4) : INFINITY;
+        }
+        sfw[bi >> 2] |= code << (8 * (bi & 3));
+#pragma unroll
+        for (int g8 = 0; g8 < C::kBlk / 8; ++g8) {
+          const int base = bi * C::kBlk + g8 * 8;
+          float y[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[i] = ex2_approx(fmaf(s[base + i], sc, -off));
+          packed[base / 8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+        }
+      }
+      // P^ (64 bytes of this row) and its scales into the shared-memory A operand
+      uint8_t* pbuf = sm.p[sb];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(pbuf + swz64_offset(r, c)) =
+            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+#pragma unroll
+      for (int a = 0; a < C::kSfTileAtoms; ++a)
+        *reinterpret_cast<uint32_t*>(sm.sfp[sb] + 512 * a + (r & 31) * 16 + (r >> 5) * 4) = sfw[a];
+      fence_proxy_async_smem();
+      // rescale O and l once the previous PV product has landed
+      if (j >= 1) {
+        if (!__all_sync(0xffffffffu, cta_wait(&sm.o_done, (j - 1) & 1, abort_flag, kStatusTimeoutSoftmax))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t raw[32];
+            tmem_ld32(lane_base + kColO + 32 * c, raw);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+            tmem_st32(lane_base + kColO + 32 * c, raw);
+          }
+          uint32_t lr;
+          tmem_ld1(lane_base + kColL, lr);
+          tmem_wait_ld();
+          tmem_st1(lane_base + kColL, __float_as_uint(__uint_as_float(lr) * alpha));
+          tmem_wait_st();
+        }
+      }
+      m = m_new;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.p_full[sb]);
+    }
+    // ---------------------------------------------------------------- epilogue
+    if (ok && __all_sync(0xffffffffu, cta_wait(&sm.o_done, (n_tiles - 1) & 1, abort_flag, kStatusTimeoutSoftmax))) {
+      tc_fence_after();
+      uint32_t lr;
+      tmem_ld1(lane_base + kColL, lr);
+      tmem_wait_ld();
+      const float l = __uint_as_float(lr);
+      const float inv = p.g_v / l;
+      const bool store = row < p.S_q;
+      const int64_t orow = (int64_t)bh_q * p.S_q + row;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t raw[32];
+        tmem_ld32(lane_base + kColO + 32 * c, raw);
+        tmem_wait_ld();
+        if (store) {
+          if (p.out_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * D + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(raw[4 * i]) * inv, __uint_as_float(raw[4 * i + 1]) * inv,
+                                   __uint_as_float(raw[4 * i + 2]) * inv, __uint_as_float(raw[4 * i + 3]) * inv);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * D + 32 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint32_t w[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(raw[8 * i + 2 * q]) * inv,
+                                                          __uint_as_float(raw[8 * i + 2 * q + 1]) * inv);
+                w[q] = *reinterpret_cast<uint32_t*>(&pr);
+              }
+              dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
+        }
+      }
+      if (store && p.lse != nullptr) {
+        const float lscale = MX ? 1.0f : kGpNvfp4;
+        p.lse[orow] = m * 0.69314718055994531f + logf(l * lscale);
+      }
+    }
+  }
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// =======================================================================================
+// self-test: one block-scaled MMA through the same descriptors and scale path
+// =======================================================================================
+template <bool MX>
+__global__ void __launch_bounds__(128, 1)
+    selftest_mma_kernel(const uint8_t* __restrict__ a, const uint8_t* __restrict__ a_sf,
+                        const uint8_t* __restrict__ bmat, const uint8_t* __restrict__ b_sf, int N,
+                        int K, float* __restrict__ d_out) {
+  constexpr int kBlk = MX ? 32 : 16;
+  __shared__ __align__(1024) uint8_t sa[128 * 64];
+  __shared__ __align__(1024) uint8_t sb[256 * 64];
+  __shared__ __align__(1024) uint8_t ssfa[2 * 512];
+  __shared__ __align__(1024) uint8_t ssfb[4 * 512];
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rb = K / 2;                                        // bytes per row (32 or 64)
+  // operands -> swizzled K-major shared-memory tiles (same pattern TMA produces)
+  for (int i = threadIdx.x; i < 128 * rb / 16; i += 128) {
+    const int r = i / (rb / 16), c = i % (rb / 16);
+    const uint4 v = *reinterpret_cast<const uint4*>(a + r * rb + c * 16);
+    *reinterpret_cast<uint4*>(sa + (rb == 64 ? swz64_offset(r, c) : swz32_offset(r, c))) = v;
+  }
+  for (int i = threadIdx.x; i < N * rb / 16; i += 128) {
+    const int r = i / (rb / 16), c = i % (rb / 16);
+    const uint4 v = *reinterpret_cast<const uint4*>(bmat + r * rb + c * 16);
+    *reinterpret_cast<uint4*>(sb + (rb == 64 ? swz64_offset(r, c) : swz32_offset(r, c))) = v;
+  }
+  // scale atoms: A has one row tile; B has ceil(N/128); groups per row tile = 32/kBlk
+  const int ng = 32 / kBlk, nrt_b = (N + 127) / 128;
+  for (int i = threadIdx.x; i < ng * 512 / 16; i += 128)
+    reinterpret_cast<uint4*>(ssfa)[i] = reinterpret_cast<const uint4*>(a_sf)[i];
+  for (int i = threadIdx.x; i < nrt_b * ng * 512 / 16; i += 128)
+    reinterpret_cast<uint4*>(ssfb)[i] = reinterpret_cast<const uint4*>(b_sf)[i];
+  fence_proxy_async_smem();
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tbase, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tbase;
+  // TMEM: D [0, N), SFA at 256 (4 columns per group), SFB at 272 (8 columns per group:
+  // row tile rt of group g at 272 + 8g + 4rt)
+  if (warp == 0 && elect_one()) {
+    for (int g = 0; g < ng; ++g) {
+      tmem_cp_sf_atom(tmem + 256 + 4 * g, smem_u32(ssfa + 512 * g));
+      for (int rt = 0; rt < nrt_b; ++rt)
+        tmem_cp_sf_atom(tmem + 272 + 8 * g + 4 * rt, smem_u32(ssfb + 512 * (rt * ng + g)));
+    }
+    const int steps = K / 64;
+    const uint32_t swz = rb == 64 ? kSwiz64 : kSwiz32;
+    const uint32_t sbo = rb == 64 ? 512 : 256;
+    for (int ks = 0; ks < steps; ++ks) {
+      const uint64_t ad = make_smem_desc(smem_u32(sa) + 32 * ks, 16, sbo, swz);
+      const uint64_t bd = make_smem_desc(smem_u32(sb) + 32 * ks, 16, sbo, swz);
+      if constexpr (MX) {
+        const uint32_t id = 2u * (ks & 1);
+        mma_mxf4(tmem, ad, bd, make_idesc_fp4(N, true, id, id), tmem + 256 + 4 * (ks >> 1),
+                 tmem + 272 + 8 * (ks >> 1), ks > 0);
+      } else {
+        mma_nvf4(tmem, ad, bd, make_idesc_fp4(N, false, 0, 0), tmem + 256 + 4 * ks,
+                 tmem + 272 + 8 * ks, ks > 0);
+      }
+    }
+    tc_commit(&bar);
+  }
+  __syncwarp();
+  mbar_wait(&bar, 0, &g_attn_status, kStatusTimeoutProbe);
+  tc_fence_after();
+  const int r = warp * 32 + lane;
+  const uint32_t lb = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  for (int c = 0; c < N; c += 16) {
+    uint32_t raw[16];
+    tmem_ld16(lb + c, raw);
+    tmem_wait_ld();
+    for (int i = 0; i < 16; ++i) d_out[r * N + c + i] = __uint_as_float(raw[i]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// bounded-wait probe: waits on a barrier nothing will complete, for `polls` polls
+__global__ void wait_probe_kernel(uint32_t polls) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &g_attn_status, kStatusTimeoutProbe, polls);
+}
+
+cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(host_word, g_attn_status, sizeof(uint32_t), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_attn_status, &zero, sizeof(uint32_t), 0, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(st);
+}
+
+// ---------------------------------------------------------------------------------------
+// host: tensor maps
+// ---------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D byte tensor [d2][d1][d0 bytes] with box (box0 bytes, box1 rows, 1)
+static bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0, d0 * d1};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, bool MX, bool CAUSAL>
+static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t* vt,
+                               const AttnParams& prm, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  const CUtensorMapSwizzle qk_swz = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  if (!make_map_3d(&tq, q, D / 2, prm.S_q, (uint64_t)prm.B * prm.Hq, D / 2, kBM, qk_swz) ||
+      !make_map_3d(&tk, k, D / 2, prm.S_k, (uint64_t)prm.B * prm.Hkv, D / 2, kBN, qk_swz) ||
+      !make_map_3d(&tv, vt, prm.S_kpad / 2, D, (uint64_t)prm.B * prm.Hkv, kBN / 2, D,
+                   CU_TENSOR_MAP_SWIZZLE_64B))
+    return FA4Q_ERR_CUDA;
+  const size_t smem = sizeof(Smem<D, MX>) + 1024;
+  auto kern = attn_fwd_kernel<D, MX, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return FA4Q_ERR_CUDA;
+  dim3 grid(prm.n_qtiles, prm.Hq, prm.B);
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
+  return launch_status();
+}
+
+}  // namespace fa4q
+
+using namespace fa4q;
+
+extern "C" fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                     const uint8_t* k_sf, const uint8_t* vt, const uint8_t* vt_sf,
+                                     float g_q, float g_k, float g_v, int B, int Hq, int Hkv,
+                                     int S_q, int S_k, int d, fa4q_format fmt, float qmax_p,
+                                     int causal, float sm_scale, void* out, int out_is_fp32,
+                                     float* lse, void* stream) {
+  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (!q || !q_sf || !k || !k_sf || !vt || !vt_sf || !out) return FA4Q_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || S_q < 0 || S_k < 0) return FA4Q_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA4Q_ERR_INVALID_ARG;
+  if (causal && S_q != S_k) return FA4Q_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA4Q_ERR_UNSUPPORTED;
+  if (!(qmax_p >= 0.0f) || !isfinite(qmax_p)) return FA4Q_ERR_INVALID_ARG;
+  if (fmt == FA4Q_MXFP4) { g_q = g_k = g_v = 1.0f; }
+  if (!(g_q > 0.0f) || !(g_k > 0.0f) || !(g_v > 0.0f)) return FA4Q_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(q_sf) || !aligned16(k_sf) ||
+      !aligned16(vt_sf) || !aligned16(out))
+    return FA4Q_ERR_INVALID_ARG;
+  if (B == 0 || S_q == 0) return FA4Q_OK;
+  if (S_k == 0) return FA4Q_ERR_INVALID_ARG;
+  const int n_qtiles = (S_q + kBM - 1) / kBM;
+  if (B > 65535 || Hq > 65535) return FA4Q_ERR_UNSUPPORTED;
+  AttnParams prm;
+  prm.q_sf = q_sf;
+  prm.k_sf = k_sf;
+  prm.vt_sf = vt_sf;
+  prm.out = out;
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.S_q = S_q;
+  prm.S_k = S_k;
+  prm.S_kpad = (S_k + 31) / 32 * 32;
+  prm.n_qtiles = n_qtiles;
+  const float sms = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)d);
+  prm.score_scale_log2 = sms * g_q * g_k * kLog2e;
+  prm.g_v = g_v;
+  prm.qmax_p = qmax_p;
+  prm.causal = causal;
+  prm.out_fp32 = out_is_fp32;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool mx = fmt == FA4Q_MXFP4;
+  if (d == 128) {
+    if (mx) return causal ? launch_attn<128, true, true>(q, k, vt, prm, st) : launch_attn<128, true, false>(q, k, vt, prm, st);
+    return causal ? launch_attn<128, false, true>(q, k, vt, prm, st) : launch_attn<128, false, false>(q, k, vt, prm, st);
+  }
+  if (mx) return causal ? launch_attn<64, true, true>(q, k, vt, prm, st) : launch_attn<64, true, false>(q, k, vt, prm, st);
+  return causal ? launch_attn<64, false, true>(q, k, vt, prm, st) : launch_attn<64, false, false>(q, k, vt, prm, st);
+}
+
+extern "C" fa4q_status fa4q_selftest_block_mma(const uint8_t* a, const uint8_t* a_sf, const uint8_t* b,
+                                               const uint8_t* b_sf, int N, int K, fa4q_format fmt,
+                                               float* d_out, void* stream) {
+  if (!a || !a_sf || !b || !b_sf || !d_out) return FA4Q_ERR_INVALID_ARG;
+  if (K != 64 && K != 128) return FA4Q_ERR_UNSUPPORTED;
+  if (N < 16 || N > 256 || N % 16 != 0) return FA4Q_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fmt == FA4Q_MXFP4)
+    selftest_mma_kernel<true><<<1, 128, 0, st>>>(a, a_sf, b, b_sf, N, K, d_out);
+  else if (fmt == FA4Q_NVFP4)
+    selftest_mma_kernel<false><<<1, 128, 0, st>>>(a, a_sf, b, b_sf, N, K, d_out);
+  else
+    return FA4Q_ERR_INVALID_ARG;
+  return launch_status();
+}
+
+extern "C" fa4q_status fa4q_selftest_wait_timeout(uint32_t polls, void* stream) {
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(polls);
+  return launch_status();
+}

@@ -1,0 +1,26 @@
+// fa4q_internal.h - host-side helpers shared by the fa4q translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "fa4q.h"
+
+namespace fa4q {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Map the launch result of the kernels just enqueued to a status code.
+inline fa4q_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA4Q_OK : FA4Q_ERR_CUDA;
+}
+
+// Each translation unit with bounded device waits owns one status word; these host
+// functions read-and-clear them (stream-ordered, then synchronised by the caller).
+cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word);
+cudaError_t decode_status_fetch(cudaStream_t st, uint32_t* host_word);
+
+}  // namespace fa4q

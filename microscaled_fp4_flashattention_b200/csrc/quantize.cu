@@ -1,0 +1,430 @@
+// quantize.cu - blockwise E2M1 quantisation kernels and their C-ABI entry points.
+//
+// Block microscaling: BitDecoding-FP4 (Algorithm-System Co-Design for Native FP4 KV Cache
+// Decoding), "The KV Cache Bottleneck in Long-Context LLM Serving" - blocks share one scale,
+// elements are E2M1, MX blocks have 32 elements with E8M0 scales, NVFP4 blocks 16 elements
+// with E4M3 scales.  Scale bound: MXAttention, Abstract (OCP MXFP4 and the universal optimal
+// scaling bound Qmax = 7.25).  Smoothing: HiFA4, Abstract (Smooth-QK multiplier before
+// quantisation).  Hybrid cache: HyQuant (vertical-line tokens kept in full precision; their
+// 4-bit slots are zero here).
+//
+// All three kernels are HBM-bound streaming passes: 16-byte coalesced loads of bf16,
+// FP32 scale arithmetic in the fixed IEEE order, packed E2M1 stores.
+#include <math.h>
+#include <stdio.h>
+
+#include "fa4q_common.cuh"
+#include "fa4q_internal.h"
+
+namespace fa4q {
+
+// ---------------------------------------------------------------------------------------
+// per-block quantisation (FP32 values in registers)
+// ---------------------------------------------------------------------------------------
+// NVFP4: s = UE4M3(amax / (qmax*g)); y = x / (float(s)*g); 16 elements -> 8 bytes.
+FA4Q_DEVINL uint32_t quant_block16_nvfp4(const float* v, float denom, float g, uint2& packed) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float t = __fdiv_rn(amax, denom);
+  const uint32_t s = ue4m3_encode(t);
+  const float div = __fmul_rn(ue4m3_decode(s), g);
+  float y[16];
+  if (div > 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(v[i], div);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = v[i] * 0.0f;
+  }
+  packed.x = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+  packed.y = e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+  return s;
+}
+
+// MXFP4: e from the OCP or UOS rule, y = x * 2^-e (exact); 32 elements -> 16 bytes.
+FA4Q_DEVINL uint32_t quant_block32_mxfp4(const float* v, float qmax, uint4& packed) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const int e = mx_exponent(amax, qmax);
+  const float inv = exp2i(-e);
+  float y[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) y[i] = v[i] * inv;
+  packed.x = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+  packed.y = e2m1x8(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+  packed.z = e2m1x8(y[16], y[17], y[18], y[19], y[20], y[21], y[22], y[23]);
+  packed.w = e2m1x8(y[24], y[25], y[26], y[27], y[28], y[29], y[30], y[31]);
+  return static_cast<uint32_t>(e + 127);
+}
+
+FA4Q_DEVINL void load_bf16x8(const uint16_t* p, float* out) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    out[2 * i] = __uint_as_float(w[i] << 16);
+    out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// Byte offset of (row r, scale column k) in one matrix's tiled scale array with nG groups.
+FA4Q_DEVINL int64_t sf_tiled_offset(int64_t r, int64_t k, int64_t nG) {
+  return ((r >> 7) * nG + (k >> 2)) * 512 + (r & 31) * 16 + ((r & 127) >> 5) * 4 + (k & 3);
+}
+
+// ---------------------------------------------------------------------------------------
+// AXIS_INNER: one thread per (row, group of 4 blocks)
+// ---------------------------------------------------------------------------------------
+template <int BLK>
+__global__ void __launch_bounds__(128) quant_inner_kernel(
+    const uint16_t* __restrict__ x, int64_t groups, int64_t rows, int64_t cols,
+    int64_t row_stride, float qmax, float g, const float* __restrict__ mul, int64_t mheads,
+    int64_t mratio, int tiled, uint8_t* __restrict__ packed, uint8_t* __restrict__ sf) {
+  const int64_t nblk = cols / BLK;
+  const int64_t rows_sp = tiled ? ((rows + 127) / 128) * 128 : rows;   // rows in SF space
+  const int64_t nG = tiled ? ((cols + 127) / 128) * (32 / BLK) : (nblk + 3) / 4;
+  const int64_t per_group = rows_sp * nG;
+  const int64_t total = groups * per_group;
+  const int64_t sf_group_bytes = tiled ? ((rows + 127) / 128) * nG * 512 : rows * nblk;
+  const float denom = __fmul_rn(qmax, g);
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t gi = idx / per_group;
+    const int64_t rem = idx - gi * per_group;
+    const int64_t r = rem / nG;
+    const int64_t j = rem - r * nG;
+    uint32_t sword = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t kb = 4 * j + i;
+      uint32_t s = 0;
+      if (r < rows && kb < nblk) {
+        const uint16_t* src = x + (gi * rows + r) * row_stride + kb * BLK;
+        float v[BLK];
+#pragma unroll
+        for (int c = 0; c < BLK; c += 8) load_bf16x8(src + c, v + c);
+        if (mul != nullptr) {
+          const float* m = mul + ((gi % mheads) / mratio) * cols + kb * BLK;
+#pragma unroll
+          for (int c = 0; c < BLK; c += 4) {
+            const float4 mm = *reinterpret_cast<const float4*>(m + c);
+            v[c] = __fmul_rn(v[c], mm.x);
+            v[c + 1] = __fmul_rn(v[c + 1], mm.y);
+            v[c + 2] = __fmul_rn(v[c + 2], mm.z);
+            v[c + 3] = __fmul_rn(v[c + 3], mm.w);
+          }
+        }
+        uint8_t* dst = packed + (gi * rows + r) * (cols / 2) + kb * (BLK / 2);
+        if constexpr (BLK == 16) {
+          uint2 p;
+          s = quant_block16_nvfp4(v, denom, g, p);
+          *reinterpret_cast<uint2*>(dst) = p;
+        } else {
+          uint4 p;
+          s = quant_block32_mxfp4(v, qmax, p);
+          *reinterpret_cast<uint4*>(dst) = p;
+        }
+      }
+      sword |= s << (8 * i);
+      if (!tiled && r < rows && kb < nblk) sf[gi * sf_group_bytes + r * nblk + kb] = (uint8_t)s;
+    }
+    if (tiled) {
+      *reinterpret_cast<uint32_t*>(sf + gi * sf_group_bytes + sf_tiled_offset(r, 4 * j, nG)) =
+          sword;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// AXIS_OUTER: blocks along tokens, transposed output.  CTA = (group, 128 tokens, 64 ch).
+// ---------------------------------------------------------------------------------------
+template <int BLK>
+__global__ void __launch_bounds__(128) quant_outer_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t row_stride, float qmax,
+    float g, int tiled, uint8_t* __restrict__ packed, uint8_t* __restrict__ sf) {
+  __shared__ float tile[64][129];
+  const int64_t gi = blockIdx.z;
+  const int64_t tok0 = (int64_t)blockIdx.x * 128;
+  const int64_t ch0 = (int64_t)blockIdx.y * 64;
+  const int64_t rows_pad = (rows + 31) / 32 * 32;
+  const int t = threadIdx.x;
+  // load [128 tokens][64 channels] -> tile[ch][tok]
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int u = t + 128 * i;
+    const int tr = u >> 3, c8 = (u & 7) * 8;
+    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (tok0 + tr < rows && ch0 + c8 < cols)
+      load_bf16x8(x + (gi * rows + tok0 + tr) * row_stride + ch0 + c8, v);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) tile[c8 + k][tr] = v[k];
+  }
+  __syncthreads();
+  const float denom = __fmul_rn(qmax, g);
+  // thread -> (channel, 4 consecutive blocks of tokens)
+  constexpr int kGroupTok = 4 * BLK;                  // 64 (NVFP4) or 128 (MXFP4)
+  constexpr int kGroupsPerTile = 128 / kGroupTok;     // 2 or 1
+  if (t >= 64 * kGroupsPerTile) return;
+  const int c = t / kGroupsPerTile;
+  const int tg = t % kGroupsPerTile;
+  const int64_t ch = ch0 + c;
+  if (ch >= cols) return;
+  const int64_t nblk_t = rows_pad / BLK;               // blocks per channel row
+  const int64_t nG = ((rows_pad + 127) / 128) * (32 / BLK);
+  const int64_t sf_group_bytes = tiled ? ((cols + 127) / 128) * nG * 512 : cols * nblk_t;
+  uint32_t sword = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int lt = tg * kGroupTok + i * BLK;           // local token of the block
+    const int64_t kb = (tok0 + lt) / BLK;              // block index along the channel row
+    float v[BLK];
+#pragma unroll
+    for (int k = 0; k < BLK; ++k) v[k] = tile[c][lt + k];
+    uint32_t s;
+    uint8_t* dst = packed + (gi * cols + ch) * (rows_pad / 2) + (tok0 + lt) / 2;
+    const bool inside = tok0 + lt < rows_pad;
+    if constexpr (BLK == 16) {
+      uint2 p;
+      s = quant_block16_nvfp4(v, denom, g, p);
+      if (inside) *reinterpret_cast<uint2*>(dst) = p;
+    } else {
+      uint4 p;
+      s = quant_block32_mxfp4(v, qmax, p);
+      if (inside) *reinterpret_cast<uint4*>(dst) = p;
+    }
+    sword |= s << (8 * i);
+    if (!tiled && inside) sf[gi * sf_group_bytes + ch * nblk_t + kb] = (uint8_t)s;
+  }
+  if (tiled) {
+    const int64_t k0 = (tok0 + tg * kGroupTok) / BLK;
+    *reinterpret_cast<uint32_t*>(sf + gi * sf_group_bytes + sf_tiled_offset(ch, k0, nG)) = sword;
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Paged KV quantisation: CTA = (page j, kv-head h, sequence b)
+// ---------------------------------------------------------------------------------------
+template <int BLK>
+__global__ void __launch_bounds__(128) quant_kv_pages_kernel(
+    const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int Hkv, int L, int d,
+    const int32_t* __restrict__ fp4_len, const uint64_t* __restrict__ excl, const int32_t* __restrict__ table,
+    int max_pages, float g_k, float g_v, uint8_t* __restrict__ k_pages, uint8_t* __restrict__ k_sf,
+    uint8_t* __restrict__ vt_pages, uint8_t* __restrict__ vt_sf) {
+  __shared__ float tile[128][65];                      // V^T: [channel][token]
+  const int j = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int n = min(fp4_len[b], L);
+  if (j * 64 >= n) return;
+  const int64_t phys = table[(int64_t)b * max_pages + j];
+  const uint64_t ex = excl ? excl[((int64_t)b * Hkv + h) * max_pages + j] : 0ull;
+  const int t = threadIdx.x;
+  const int64_t base = (((int64_t)b * Hkv + h) * L + (int64_t)j * 64) * d;
+  // ---- K rows: thread -> (token, group of 4 blocks along d)
+  const int ngrp = d / (4 * BLK);                      // 2 (NVFP4, d=128) / 1
+  const float denom_k = __fmul_rn(6.0f, g_k);
+  for (int u = t; u < 64 * ngrp; u += 128) {
+    const int tok = u / ngrp, gq = u % ngrp;
+    const bool valid = (j * 64 + tok < n) && !((ex >> tok) & 1ull);
+    uint32_t sword = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c0 = (gq * 4 + i) * BLK;
+      float vals[BLK];
+      if (valid) {
+#pragma unroll
+        for (int c = 0; c < BLK; c += 8) load_bf16x8(k + base + (int64_t)tok * d + c0 + c, vals + c);
+      } else {
+#pragma unroll
+        for (int c = 0; c < BLK; ++c) vals[c] = 0.0f;
+      }
+      uint8_t* dst = k_pages + ((phys * Hkv + h) * 64 + tok) * (d / 2) + c0 / 2;
+      uint32_t s;
+      if constexpr (BLK == 16) {
+        uint2 p;
+        s = quant_block16_nvfp4(vals, denom_k, g_k, p);
+        *reinterpret_cast<uint2*>(dst) = p;
+      } else {
+        uint4 p;
+        s = quant_block32_mxfp4(vals, 0.0f, p);
+        *reinterpret_cast<uint4*>(dst) = p;
+      }
+      sword |= s << (8 * i);
+    }
+    uint8_t* sdst = k_sf + ((phys * Hkv + h) * 64 + tok) * (d / BLK) + gq * 4;
+    *reinterpret_cast<uint32_t*>(sdst) = sword;
+  }
+  // ---- V: stage [64 tokens][d] as tile[ch][tok], invalid tokens zero
+  for (int u = t; u < 64 * (d / 8); u += 128) {
+    const int tok = u / (d / 8), c8 = (u % (d / 8)) * 8;
+    float vals[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const bool valid = (j * 64 + tok < n) && !((ex >> tok) & 1ull);
+    if (valid) load_bf16x8(v + base + (int64_t)tok * d + c8, vals);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) tile[c8 + q][tok] = vals[q];
+  }
+  __syncthreads();
+  const float denom_v = __fmul_rn(6.0f, g_v);
+  for (int c = t; c < d; c += 128) {
+    uint8_t* dst = vt_pages + ((phys * Hkv + h) * d + c) * 32;
+    uint8_t* sdst = vt_sf + ((phys * Hkv + h) * d + c) * (64 / BLK);
+#pragma unroll
+    for (int i = 0; i < 64 / BLK; ++i) {
+      float vals[BLK];
+#pragma unroll
+      for (int q = 0; q < BLK; ++q) vals[q] = tile[c][i * BLK + q];
+      uint32_t s;
+      if constexpr (BLK == 16) {
+        uint2 p;
+        s = quant_block16_nvfp4(vals, denom_v, g_v, p);
+        *reinterpret_cast<uint2*>(dst + i * 8) = p;
+      } else {
+        uint4 p;
+        s = quant_block32_mxfp4(vals, 0.0f, p);
+        *reinterpret_cast<uint4*>(dst + i * 16) = p;
+      }
+      sdst[i] = (uint8_t)s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// Smooth-QK calibration: CTA = kv-head, thread = channel
+// ---------------------------------------------------------------------------------------
+__global__ void smooth_calibrate_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                                        int Hq, int Hkv, int T, int d, float* __restrict__ mul_q,
+                                        float* __restrict__ mul_k) {
+  const int h = blockIdx.x;
+  const int grp = Hq / Hkv;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    float qm = 0.0f, km = 0.0f;
+    for (int hq = h * grp; hq < (h + 1) * grp; ++hq)
+      for (int t = 0; t < T; ++t) qm = fmaxf(qm, fabsf(bf16_to_f32(q[((int64_t)hq * T + t) * d + c])));
+    for (int t = 0; t < T; ++t) km = fmaxf(km, fabsf(bf16_to_f32(k[((int64_t)h * T + t) * d + c])));
+    const float r = __fdiv_rn(km, qm);
+    int e;
+    if (r != r) {
+      e = 0;
+    } else if (r == 0.0f) {
+      e = -8;
+    } else if (isinf(r)) {
+      e = 8;
+    } else {
+      const int E1 = floor_log2(r) + 1;               // e = floor((floor(log2 r) + 1) / 2)
+      e = E1 >= 0 ? E1 / 2 : -((1 - E1) / 2);
+      e = e < -8 ? -8 : (e > 8 ? 8 : e);
+    }
+    mul_q[h * d + c] = exp2i(e);
+    mul_k[h * d + c] = exp2i(-e);
+  }
+}
+
+}  // namespace fa4q
+
+using namespace fa4q;
+
+// =======================================================================================
+// C ABI
+// =======================================================================================
+extern "C" size_t fa4q_sf_tiled_bytes(int64_t rows, int64_t cols, fa4q_format fmt) {
+  if (rows <= 0 || cols <= 0) return 0;
+  const int64_t blk = fmt == FA4Q_MXFP4 ? 32 : 16;
+  return (size_t)(((rows + 127) / 128) * ((cols + 127) / 128) * (32 / blk) * 512);
+}
+
+extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows, int64_t cols,
+                                     int64_t row_stride, fa4q_format fmt, fa4q_axis axis,
+                                     float qmax, float tensor_scale, const float* smooth_mul,
+                                     int64_t smooth_heads, int64_t smooth_ratio,
+                                     fa4q_sf_layout sf_layout, uint8_t* packed_out,
+                                     uint8_t* scales_out, void* stream) {
+  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (axis != FA4Q_AXIS_INNER && axis != FA4Q_AXIS_OUTER) return FA4Q_ERR_INVALID_ARG;
+  if (sf_layout != FA4Q_SF_ROWMAJOR && sf_layout != FA4Q_SF_TILED) return FA4Q_ERR_INVALID_ARG;
+  if (groups < 0 || rows < 0 || cols < 0) return FA4Q_ERR_INVALID_ARG;
+  if (groups == 0 || rows == 0 || cols == 0) return FA4Q_OK;
+  if (!x || !packed_out || !scales_out) return FA4Q_ERR_INVALID_ARG;
+  if (row_stride < cols || row_stride % 8 != 0 || cols % 8 != 0) return FA4Q_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed_out)) return FA4Q_ERR_INVALID_ARG;
+  if (sf_layout == FA4Q_SF_TILED && !aligned16(scales_out)) return FA4Q_ERR_INVALID_ARG;
+  if (!(qmax >= 0.0f) || !isfinite(qmax)) return FA4Q_ERR_INVALID_ARG;
+  const float g = fmt == FA4Q_NVFP4 ? tensor_scale : 1.0f;
+  if (!(g > 0.0f) || !isfinite(g)) return FA4Q_ERR_INVALID_ARG;
+  const int blk = fmt == FA4Q_MXFP4 ? 32 : 16;
+  const float qm = (fmt == FA4Q_NVFP4 && qmax == 0.0f) ? 6.0f : qmax;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int tiled = sf_layout == FA4Q_SF_TILED;
+  if (axis == FA4Q_AXIS_INNER) {
+    if (cols % blk != 0) return FA4Q_ERR_UNSUPPORTED;
+    if (smooth_mul && (smooth_heads <= 0 || smooth_ratio <= 0 || !aligned16(smooth_mul)))
+      return FA4Q_ERR_INVALID_ARG;
+    const int64_t nblk = cols / blk;
+    const int64_t rows_sp = tiled ? (rows + 127) / 128 * 128 : rows;
+    const int64_t nG = tiled ? (cols + 127) / 128 * (32 / blk) : (nblk + 3) / 4;
+    const int64_t total = groups * rows_sp * nG;
+    const int64_t nblocks = std::min<int64_t>((total + 127) / 128, 148LL * 64);
+    if (blk == 16)
+      quant_inner_kernel<16><<<(unsigned)nblocks, 128, 0, st>>>(
+          (const uint16_t*)x, groups, rows, cols, row_stride, qm, g, smooth_mul,
+          smooth_heads > 0 ? smooth_heads : 1, smooth_ratio > 0 ? smooth_ratio : 1, tiled,
+          packed_out, scales_out);
+    else
+      quant_inner_kernel<32><<<(unsigned)nblocks, 128, 0, st>>>(
+          (const uint16_t*)x, groups, rows, cols, row_stride, qm, g, smooth_mul,
+          smooth_heads > 0 ? smooth_heads : 1, smooth_ratio > 0 ? smooth_ratio : 1, tiled,
+          packed_out, scales_out);
+  } else {
+    if (smooth_mul) return FA4Q_ERR_UNSUPPORTED;
+    if (groups > 65535) return FA4Q_ERR_UNSUPPORTED;
+    const int64_t rows_pad = (rows + 31) / 32 * 32;
+    dim3 grid((unsigned)((rows_pad + 127) / 128), (unsigned)((cols + 63) / 64), (unsigned)groups);
+    if (grid.y > 65535) return FA4Q_ERR_UNSUPPORTED;
+    if (blk == 16)
+      quant_outer_kernel<16><<<grid, 128, 0, st>>>((const uint16_t*)x, rows, cols, row_stride,
+                                                   qm, g, tiled, packed_out, scales_out);
+    else
+      quant_outer_kernel<32><<<grid, 128, 0, st>>>((const uint16_t*)x, rows, cols, row_stride,
+                                                   qm, g, tiled, packed_out, scales_out);
+  }
+  return launch_status();
+}
+
+extern "C" fa4q_status fa4q_smooth_calibrate(const void* q_cal, const void* k_cal, int Hq, int Hkv,
+                                             int T, int d, float* mul_q, float* mul_k,
+                                             void* stream) {
+  if (!q_cal || !k_cal || !mul_q || !mul_k) return FA4Q_ERR_INVALID_ARG;
+  if (Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0 || Hq % Hkv != 0) return FA4Q_ERR_INVALID_ARG;
+  smooth_calibrate_kernel<<<Hkv, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      (const uint16_t*)q_cal, (const uint16_t*)k_cal, Hq, Hkv, T, d, mul_q, mul_k);
+  return launch_status();
+}
+
+extern "C" fa4q_status fa4q_quantize_kv_pages(const void* k, const void* v, int B, int Hkv, int L,
+                                              int d, const int32_t* fp4_len,
+                                              const uint64_t* excl_mask,
+                                              const int32_t* block_table, int max_pages,
+                                              fa4q_format fmt, float g_k, float g_v,
+                                              uint8_t* k_pages, uint8_t* k_sf, uint8_t* vt_pages,
+                                              uint8_t* vt_sf, void* stream) {
+  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (!k || !v || !fp4_len || !block_table || !k_pages || !k_sf || !vt_pages || !vt_sf)
+    return FA4Q_ERR_INVALID_ARG;
+  if (B <= 0 || Hkv <= 0 || L <= 0 || max_pages <= 0) return FA4Q_ERR_INVALID_ARG;
+  if (d != 128) return FA4Q_ERR_UNSUPPORTED;
+  if ((int64_t)max_pages * 64 < 1 || B > 65535 || Hkv > 65535) return FA4Q_ERR_UNSUPPORTED;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_pages) || !aligned16(vt_pages))
+    return FA4Q_ERR_INVALID_ARG;
+  const float gk = fmt == FA4Q_NVFP4 ? g_k : 1.0f, gv = fmt == FA4Q_NVFP4 ? g_v : 1.0f;
+  if (!(gk > 0.0f) || !(gv > 0.0f)) return FA4Q_ERR_INVALID_ARG;
+  dim3 grid(max_pages, Hkv, B);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fmt == FA4Q_NVFP4)
+    quant_kv_pages_kernel<16><<<grid, 128, 0, st>>>((const uint16_t*)k, (const uint16_t*)v, Hkv, L,
+                                                    d, fp4_len, excl_mask, block_table, max_pages,
+                                                    gk, gv, k_pages, k_sf, vt_pages, vt_sf);
+  else
+    quant_kv_pages_kernel<32><<<grid, 128, 0, st>>>((const uint16_t*)k, (const uint16_t*)v, Hkv, L,
+                                                    d, fp4_len, excl_mask, block_table, max_pages,
+                                                    gk, gv, k_pages, k_sf, vt_pages, vt_sf);
+  return launch_status();
+}
