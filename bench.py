@@ -1,0 +1,420 @@
+"""Benchmark of the fused 4-bit microscaled FlashAttention path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 2|3|5] [--no-decode] [--no-cpu-baseline]
+
+One step = one pass of the prefill hot path over one synthetic batch of the causal GQA
+MXFP4 workload (B=1, 32/8 heads, S=4096, d=128, Smooth-QK on): block quantisation of Q and K
+(with the calibrated per-channel multipliers) and of V (transposed), then the fused FP4
+attention kernel.  Inputs are resident in HBM; L2 (126 MB) is flushed by a 256 MB write
+before every timed step.  The metric is prefill TFLOP/s (4*B*Hq*S^2*d, halved for causal).
+The decode path (batch 32, 32/8 heads, 32768 keys, NVFP4 pages + 5% BF16 vertical lines +
+128-token BF16 window) is timed in the same run and reported under "decode" (us/step, GB/s).
+
+N > 1 (torchrun): every rank runs its own independent batch (weak scaling, no collective on
+the data path); the step time is the max over ranks.  `--impl reference` times the CPU oracle
+on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "FP4 attention prefill TFLOPS & 32K decode µs/step; % of FP4 tensor / HBM roofline"
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
+FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
+
+
+# ------------------------------------------------------------------------------ helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained", d["bf16_tflops"]), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+# ------------------------------------------------------------------------------ prefill workload
+class PrefillRun:
+    """Device-resident inputs and outputs of one prefill batch, and the step itself."""
+
+    def __init__(self, w, dev, fa4q, seed_offset: int = 0):
+        import torch
+        self.w, self.dev, self.fa4q = w, dev, fa4q
+        q, k, v = synth.prefill_inputs(w) if seed_offset == 0 else self._shifted(w, seed_offset)
+        self.host = (q, k, v)
+        self.flops = w.flops
+        self.q = torch.from_numpy(q).to(dev).to(torch.bfloat16)
+        self.k = torch.from_numpy(k).to(dev).to(torch.bfloat16)
+        self.v = torch.from_numpy(v).to(dev).to(torch.bfloat16)
+        self.mq = self.mk = None
+        if w.smooth:
+            qc, kc = synth.calibration_inputs(w)
+            self.mq, self.mk = fa4q.smooth_calibrate(torch.from_numpy(qc).to(dev).to(torch.bfloat16),
+                                                     torch.from_numpy(kc).to(dev).to(torch.bfloat16))
+        self.out = torch.empty((w.B, w.Hq, w.S, w.d), dtype=torch.bfloat16, device=dev)
+        self.launches_per_step = 4
+
+    @staticmethod
+    def _shifted(w, off):
+        import dataclasses
+        ww = dataclasses.replace(w, wid=w.wid + 100 * off)
+        return synth.prefill_inputs(ww)
+
+    def step(self, attn_events=None, q=None, k=None, v=None):
+        fa4q, w = self.fa4q, self.w
+        q = self.q if q is None else q
+        k = self.k if k is None else k
+        v = self.v if v is None else v
+        pq, sq = fa4q.quantize(q, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax, 1.0, self.mq, w.Hq, w.Hq // w.Hkv)
+        pk, sk = fa4q.quantize(k, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax, 1.0, self.mk, w.Hkv, 1)
+        pv, sv = fa4q.quantize(v, w.fmt, fa4q.FA4Q_AXIS_OUTER, w.qmax)
+        if attn_events is not None:
+            attn_events[0].record()
+        fa4q.attn_fwd(pq, sq, pk, sk, pv, sv, B=w.B, Hq=w.Hq, Hkv=w.Hkv, S_q=w.S, S_k=w.S, d=w.d,
+                      fmt=w.fmt, causal=w.causal, qmax_p=w.qmax_p, out=self.out)
+        if attn_events is not None:
+            attn_events[1].record()
+        return self.out
+
+
+# ------------------------------------------------------------------------------ decode workload
+class DecodeRun:
+    def __init__(self, dw, dev, fa4q):
+        import torch
+        self.dw, self.dev, self.fa4q = dw, dev, fa4q
+        B, Hq, Hkv, d, L, W = dw.B, dw.Hq, dw.Hkv, dw.d, dw.L, dw.window
+        n_fp4, P, n_hp = dw.fp4_len, dw.n_pages, dw.n_hp
+        tK = torch.empty((B, Hkv, L, d), dtype=torch.bfloat16, device=dev)
+        tV = torch.empty((B, Hkv, L, d), dtype=torch.bfloat16, device=dev)
+        for b in range(B):
+            for h in range(Hkv):
+                tK[b, h] = torch.from_numpy(synth.decode_kv_slice(dw, "k", b, h)).to(dev).to(torch.bfloat16)
+                tV[b, h] = torch.from_numpy(synth.decode_kv_slice(dw, "v", b, h)).to(dev).to(torch.bfloat16)
+        Q = np.stack([synth.decode_query(dw, b) for b in range(B)])
+        hp = np.stack([np.stack([synth.decode_hp_positions(dw, b, h) for h in range(Hkv)]) for b in range(B)])
+        excl = np.zeros((B, Hkv, P), dtype=np.uint64)
+        bb, hh, jj = np.meshgrid(np.arange(B), np.arange(Hkv), np.arange(n_hp), indexing="ij")
+        np.bitwise_or.at(excl, (bb.ravel(), hh.ravel(), hp.ravel() // 64),
+                         np.left_shift(np.uint64(1), (hp.ravel() % 64).astype(np.uint64)))
+        i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a).astype(np.int32)).to(dev)
+        self.table = i32(synth.decode_block_table(dw))
+        self.fp4_len = i32(np.full(B, n_fp4))
+        self.excl = torch.from_numpy(excl.view(np.int64)).to(dev)
+        self.kp, self.ks, self.vp, self.vs = fa4q.quantize_kv_pages(tK, tV, self.fp4_len, self.excl,
+                                                                    self.table, B * P)
+        idx = torch.from_numpy(hp).to(dev)
+        self.hpk = torch.gather(tK[:, :, :n_fp4], 2, idx[..., None].expand(-1, -1, -1, d)).contiguous()
+        self.hpv = torch.gather(tV[:, :, :n_fp4], 2, idx[..., None].expand(-1, -1, -1, d)).contiguous()
+        self.hpc = i32(np.full((B, Hkv), n_hp))
+        self.wk, self.wv = tK[:, :, n_fp4:].contiguous(), tV[:, :, n_fp4:].contiguous()
+        self.wl = i32(np.full(B, W))
+        del tK, tV
+        torch.cuda.empty_cache()
+        self.q = torch.from_numpy(Q).to(dev).to(torch.bfloat16)
+        self.out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(fa4q.decode_workspace_size(B, Hq, Hkv, d, P), dtype=torch.uint8, device=dev)
+        blk = 16
+        self.bytes = (2 * B * Hkv * P * 64 * (d // 2 + d // blk)          # FP4 K and V^T pages + scales
+                      + 2 * B * Hkv * n_hp * d * 2 + 2 * B * Hkv * W * d * 2  # BF16 set and window
+                      + B * Hkv * P * 8 + B * P * 4                      # exclusion masks, block table
+                      + 2 * B * Hq * d * 2 + B * 4 * 2 + B * Hkv * 4)     # q, out, lengths, counts
+
+    def step(self):
+        fa4q = self.fa4q
+        return fa4q.decode(self.q, self.kp, self.ks, self.vp, self.vs, self.table, self.fp4_len, self.excl,
+                           self.hpk, self.hpv, self.hpc, self.wk, self.wv, self.wl, out=self.out,
+                           workspace=self.ws)
+
+
+# ------------------------------------------------------------------------------ CPU oracle timing
+def oracle_prefill_sample(w, budget_s: float, host=None):
+    """Time the oracle on sampled (head, row) work of workload w for about budget_s seconds;
+    returns (TFLOP/s, description, seconds)."""
+    from oracle import attention as OA
+    from oracle import smooth as OS
+    q, k, v = host if host is not None else synth.prefill_inputs(w)
+    lam = OS.calibrate(*synth.calibration_inputs(w)) if w.smooth else None
+    rng = np.random.default_rng(0)
+    done_flops, t_used, n_rows, heads_used = 0.0, 0.0, 0, 0
+    R = 64
+    while t_used < budget_s and heads_used < w.Hq:
+        h = int(rng.integers(w.Hq))
+        rows = np.sort(rng.choice(w.S, R, replace=False))
+        t0 = time.perf_counter()
+        OA.prefill(q, k, v, causal=w.causal, fmt=w.fmt, qmax=w.qmax, qmax_p=w.qmax_p, lam=lam, rows=rows,
+                   heads=[(0, h)])
+        dt = time.perf_counter() - t0
+        keys = (rows + 1) if w.causal else np.full(R, w.S)
+        done_flops += float(4.0 * w.d * keys.sum())
+        t_used += dt
+        n_rows += R
+        heads_used += 1
+        if dt < budget_s / 8:
+            R = min(w.S, R * 2)
+    desc = f"{n_rows} query rows over {heads_used} heads of {w.name} (all keys per row, oracle as is)"
+    return done_flops / t_used / 1e12, desc, t_used
+
+
+# ------------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--soak-s", type=float, default=2.0)
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        steps, warm = max(1, args.steps), max(0, args.warmup)
+        per_step = 2.5
+        for _ in range(warm):
+            oracle_prefill_sample(w, per_step / 4)
+        tf, desc, secs = [], None, 0.0
+        for _ in range(steps):
+            v, desc, s = oracle_prefill_sample(w, per_step)
+            tf.append(v)
+            secs += s
+        value = statistics.mean(tf)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+                "steps": steps, "warmup": warm, "ms_per_step": 1e3 * secs / steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": w.fmt, "data": "synthetic",
+                "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d,
+                           "causal": w.causal, "fmt": w.fmt},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import torch
+    import microscaled_fp4_flashattention_b200 as fa4q
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = load_peaks()
+
+    run = PrefillRun(w, dev, fa4q, seed_offset=rank)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(max(3, args.warmup)):
+        run.step()
+    barrier()
+    # soak: run steps back to back so the clock sampler sees the part under load
+    sampler = ClockSampler(dev.index if world == 1 else local_rank)
+    with sampler:
+        t_end = time.time() + args.soak_s
+        while time.time() < t_end:
+            for _ in range(20):
+                run.step()
+            torch.cuda.synchronize()
+        barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        aev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.fill_(float(i))                      # evict L2 (untimed)
+            ev[i][0].record()
+            run.step(attn_events=aev[i])
+            ev[i][1].record()
+        barrier()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    attn_ms = [a.elapsed_time(b) for a, b in aev]
+    t_ms = float(np.mean(step_ms))
+    a_ms = float(np.mean(attn_ms))
+    if world > 1:
+        t = torch.tensor([t_ms, a_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_ms, a_ms = float(t[0]), float(t[1])
+    value = world * run.flops / (t_ms * 1e-3) / 1e12
+
+    # end to end through the public API: pinned host inputs -> device, quantise, attend, output -> host
+    q_h = torch.from_numpy(run.host[0]).to(torch.bfloat16).pin_memory()
+    k_h = torch.from_numpy(run.host[1]).to(torch.bfloat16).pin_memory()
+    v_h = torch.from_numpy(run.host[2]).to(torch.bfloat16).pin_memory()
+    o_h = torch.empty(run.out.shape, dtype=torch.bfloat16).pin_memory()
+    qd, kd, vd = torch.empty_like(run.q), torch.empty_like(run.k), torch.empty_like(run.v)
+
+    def e2e_step():
+        qd.copy_(q_h, non_blocking=True)
+        kd.copy_(k_h, non_blocking=True)
+        vd.copy_(v_h, non_blocking=True)
+        out = run.step(q=qd, k=kd, v=vd)
+        o_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(5, args.steps // 2)
+    e0.record()
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record()
+    barrier()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    if world > 1:
+        t = torch.tensor([e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e_ms = float(t[0])
+    h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
+    d2h = o_h.numel() * 2
+
+    fp4_peak = bf16_tf * FP4_PER_BF16
+    achieved = run.flops / (a_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.fmt, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d, "causal": w.causal,
+                   "fmt": w.fmt, "smooth": w.smooth, "qmax": w.qmax, "parallelism": f"replicas x{world}",
+                   "step": "quantize Q,K,V + fused FP4 attention",
+                   "l2": "flushed before each timed step (256 MB write, untimed)"},
+        "gpu_launches": run.launches_per_step * args.steps,
+        "e2e": {"value": world * run.flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
+        "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+                     "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": None,
+                     "peak_source": f"{peak_kind} bf16 burst {bf16_tf:.1f} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4/BF16)",
+                     "ms_per_launch": a_ms},
+        "clocks": sampler.summary(),
+    }
+
+    if not args.no_decode:
+        del run, flush
+        torch.cuda.empty_cache()
+        dw = synth.WORKLOADS[4]
+        drun = DecodeRun(dw, dev, fa4q)
+        for _ in range(max(3, args.warmup)):
+            drun.step()
+        barrier()
+        dsteps = max(20, args.steps)
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dsampler = ClockSampler(dev.index)
+        with dsampler:
+            t_end = time.time() + 1.0
+            while time.time() < t_end:
+                for _ in range(20):
+                    drun.step()
+                torch.cuda.synchronize()
+            d0.record()
+            for _ in range(dsteps):
+                drun.step()
+            d1.record()
+            barrier()
+        d_ms = d0.elapsed_time(d1) / dsteps
+        gbs = drun.bytes / (d_ms * 1e-3) / 1e9
+        line["decode"] = {"workload": dw.name, "us_per_step": d_ms * 1e3, "higher_is_better": False,
+                          "GBps": gbs, "bytes_per_step": drun.bytes, "gpu_launches": 2 * dsteps,
+                          "roofline": {"kernel": "decode_split_kernel+decode_combine_kernel", "bound": "hbm",
+                                       "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                                       "traffic": None, "peak_source": f"{peak_kind} hbm copy"},
+                          "l2": "working set 1.4 GB > L2", "clocks": dsampler.summary()}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, _ = oracle_prefill_sample(w, 12.0)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -308,7 +308,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = qt * kBM + r;                  // query index
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float sc = p.score_scale_log2;
-    float m = -INFINITY;                            // running max (log2 domain)
+    // Running maximum kept in the raw MMA-score domain.  Block maxima are taken from the
+    // exact difference (bmax - m) * sc, so the block holding the row maximum gets amax = 1
+    // exactly: the MX OCP exponent floor(log2 amax) - 2 jumps at every power of two, and a
+    // fused s*sc - round(m*sc) that lands 1 ulp below 0 would move that block's scale.
+    float m = -INFINITY;
     bool ok = true;
     for (int j = 0; j < n_tiles && ok; ++j) {
       const int sb = j & 1;
@@ -319,13 +323,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       float s[kBN];
+      {
+        uint32_t raw[kBN / 32][32];
 #pragma unroll
-      for (int c = 0; c < kBN / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + 32 * c, raw);
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + 32 * c, raw[c]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[i]);
+        for (int c = 0; c < kBN / 32; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[c][i]);
       }
       tc_fence_before();
       __syncwarp();
@@ -352,28 +358,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       float tmax = bmax[0];
 #pragma unroll
       for (int bi = 1; bi < kNB; ++bi) tmax = fmaxf(tmax, bmax[bi]);
-      const float m_new = fmaxf(m, tmax * sc);
-      const float alpha = ex2_approx(m - m_new);    // 0 on the first tile
-      // per block: amax = exp2(bmax*sc - m_new); scale; y_i = exp2(s_i*sc - m_new - log2(scale))
+      const float m_new = fmaxf(m, tmax);
+      const float alpha = ex2_approx((m - m_new) * sc);   // 0 on the first tile
+      const float mref = m_new * sc;
+      // per block: amax = exp2((bmax - m)*sc); scale; y_i = exp2(s_i*sc - m*sc - log2(scale))
       uint32_t packed[kBN / 8];
       uint32_t sfw[kNB / 4 > 0 ? kNB / 4 : 1];
 #pragma unroll
       for (int w = 0; w < (kNB / 4 > 0 ? kNB / 4 : 1); ++w) sfw[w] = 0;
 #pragma unroll
       for (int bi = 0; bi < kNB; ++bi) {
-        const float amax = ex2_approx(fmaf(bmax[bi], sc, -m_new));
+        const float amax = ex2_approx((bmax[bi] - m_new) * sc);
         float off;
         uint32_t code;
         if constexpr (MX) {
           const int e = mx_exponent(amax, p.qmax_p);
           code = static_cast<uint32_t>(e + 127);
-          off = m_new + static_cast<float>(e);
+          off = mref + static_cast<float>(e);
           if (!(amax > 0.0f)) off = INFINITY;
         } else {
           const float t = __fdiv_rn(amax, 6.0f * kGpNvfp4);       // amax / (6 * g_P)
           code = ue4m3_encode(t);
           const float sf = ue4m3_decode(code);
-          off = sf > 0.0f ? m_new + lg2_approx(sf * kGpNvfp4) : INFINITY;
+          off = sf > 0.0f ? mref + lg2_approx(sf * kGpNvfp4) : INFINITY;
         }
         sfw[bi >> 2] |= code << (8 * (bi & 3));
 #pragma unroll
@@ -464,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (store && p.lse != nullptr) {
         const float lscale = MX ? 1.0f : kGpNvfp4;
-        p.lse[orow] = m * 0.69314718055994531f + logf(l * lscale);
+        p.lse[orow] = m * sc * 0.69314718055994531f + logf(l * lscale);
       }
     }
   }

@@ -170,7 +170,10 @@ __global__ void __launch_bounds__(128) quant_outer_kernel(
   const int c = t / kGroupsPerTile;
   const int tg = t % kGroupsPerTile;
   const int64_t ch = ch0 + c;
-  if (ch >= cols) return;
+  // channels in [cols, 128*ceil(cols/128)) are padding rows of the tiled scale layout: their
+  // (all-zero) blocks give scale 0, which is written; packed data exists only for ch < cols
+  const bool real_ch = ch < cols;
+  if (!real_ch && !tiled) return;
   const int64_t nblk_t = rows_pad / BLK;               // blocks per channel row
   const int64_t nG = ((rows_pad + 127) / 128) * (32 / BLK);
   const int64_t sf_group_bytes = tiled ? ((cols + 127) / 128) * nG * 512 : cols * nblk_t;
@@ -184,7 +187,7 @@ __global__ void __launch_bounds__(128) quant_outer_kernel(
     for (int k = 0; k < BLK; ++k) v[k] = tile[c][lt + k];
     uint32_t s;
     uint8_t* dst = packed + (gi * cols + ch) * (rows_pad / 2) + (tok0 + lt) / 2;
-    const bool inside = tok0 + lt < rows_pad;
+    const bool inside = real_ch && tok0 + lt < rows_pad;
     if constexpr (BLK == 16) {
       uint2 p;
       s = quant_block16_nvfp4(v, denom, g, p);
@@ -377,7 +380,8 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
     if (smooth_mul) return FA4Q_ERR_UNSUPPORTED;
     if (groups > 65535) return FA4Q_ERR_UNSUPPORTED;
     const int64_t rows_pad = (rows + 31) / 32 * 32;
-    dim3 grid((unsigned)((rows_pad + 127) / 128), (unsigned)((cols + 63) / 64), (unsigned)groups);
+    const int64_t ch_tiles = tiled ? (cols + 127) / 128 * 2 : (cols + 63) / 64;
+    dim3 grid((unsigned)((rows_pad + 127) / 128), (unsigned)ch_tiles, (unsigned)groups);
     if (grid.y > 65535) return FA4Q_ERR_UNSUPPORTED;
     if (blk == 16)
       quant_outer_kernel<16><<<grid, 128, 0, st>>>((const uint16_t*)x, rows, cols, row_stride,
