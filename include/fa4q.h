@@ -201,6 +201,38 @@ fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const uint8_t* k_
                         int num_splits, void* stream);
 
 /*
+ * fa4q_decode_noalloc - fa4q_decode for callers that cannot allocate device memory.
+ *
+ * The paper has no counterpart to this call; it is a deployment convenience.  Some callers
+ * cannot call cudaMalloc or hand the library a workspace: a plug-in whose host framework
+ * owns every byte of device memory and gives extensions no allocator, or a latency-critical
+ * serving loop where an allocation (which may synchronise the device) is not acceptable.
+ * This call takes the same inputs and output as fa4q_decode but no workspace: the split
+ * partials go to one static device array of 8 MiB inside the library, which every GPU that
+ * loads the library holds until the process exits.  Nothing is allocated per call.
+ *
+ * Limit: the partials take B*Hq*(d+2)*4 bytes per split.  With num_splits = 0 the split
+ * count is the automatic one, lowered as needed to fit 8 MiB; a request that does not fit
+ * even with one split, or an explicit num_splits that does not fit, returns
+ * FA4Q_ERR_UNSUPPORTED (use fa4q_decode with a caller workspace instead).
+ * The first call on each device looks up the array's device address (with that device
+ * current) and caches it; make that first call before any stream capture.
+ * All calls share the array and it keeps the last call's contents (every partial is
+ * rewritten before it is read, so nothing needs clearing); calls whose execution overlaps
+ * on the GPU (different streams, or different host threads) race on it and must be
+ * serialised by the caller.
+ */
+fa4q_status fa4q_decode_noalloc(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
+                                const uint8_t* vt_pages, const uint8_t* vt_sf,
+                                const int32_t* block_table, const int32_t* fp4_len,
+                                const uint64_t* excl_mask, const void* hp_k, const void* hp_v,
+                                const int32_t* hp_count, const void* win_k, const void* win_v,
+                                const int32_t* win_len, int B, int Hq, int Hkv, int d,
+                                int max_pages, int max_hp, int W, fa4q_format fmt, float g_k,
+                                float g_v, float sm_scale, void* out, int num_splits,
+                                void* stream);
+
+/*
  * fa4q_selftest_block_mma - diagnostic: one 128 x N x K block-scaled FP4 tensor-core
  * product D = A * B^T (FP32), the same MMA path the prefill kernel uses.
  * a packed [128][K/2], b packed [N][K/2] (K-major), a_sf / b_sf FA4Q_SF_TILED over

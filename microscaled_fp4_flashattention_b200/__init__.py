@@ -25,7 +25,7 @@ STATUS = {0: "FA4Q_OK", 1: "FA4Q_ERR_INVALID_ARG", 2: "FA4Q_ERR_UNSUPPORTED", 3:
 EXPORTED = [
     "fa4q_status_string", "fa4q_version", "fa4q_sf_tiled_bytes", "fa4q_quantize",
     "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_quantize_kv_pages",
-    "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_selftest_block_mma",
+    "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout",
 ]
 
@@ -65,6 +65,9 @@ def lib() -> ctypes.CDLL:
         L.fa4q_decode.restype = I
         L.fa4q_decode.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, F,
                                   F, P, P, Z, I, P]
+        L.fa4q_decode_noalloc.restype = I
+        L.fa4q_decode_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                          F, F, F, P, I, P]
         L.fa4q_selftest_block_mma.restype = I
         L.fa4q_selftest_block_mma.argtypes = [P, P, P, P, I, I, I, P, P]
         L.fa4q_device_status.restype = I
@@ -211,6 +214,27 @@ def decode(q, k_pages, k_sf, vt_pages, vt_sf, block_table, fp4_len, excl_mask, h
         _ptr(fp4_len), _ptr(excl_mask), _ptr(hp_k), _ptr(hp_v), _ptr(hp_count), _ptr(win_k),
         _ptr(win_v), _ptr(win_len), B, Hq, Hkv, d, max_pages, max_hp, W, _fmt(fmt), g_k, g_v, sm_scale,
         _ptr(out), _ptr(workspace), workspace.numel(), num_splits, _stream(stream)))
+    return out
+
+
+def decode_noalloc(q, k_pages, k_sf, vt_pages, vt_sf, block_table, fp4_len, excl_mask, hp_k, hp_v,
+                   hp_count, win_k, win_v, win_len, *, fmt="nvfp4", g_k=1.0, g_v=1.0, sm_scale=0.0,
+                   num_splits=0, out=None, stream=None):
+    """decode() without a workspace: the split partials live in the library's static device
+    array (for callers that cannot allocate device memory; see fa4q_decode_noalloc)."""
+    import torch
+    B, Hq, d = q.shape
+    Hkv = k_pages.shape[1] if k_pages is not None else hp_k.shape[1]
+    max_pages = block_table.shape[1] if block_table is not None else 0
+    max_hp = hp_k.shape[2] if hp_k is not None else 0
+    W = win_k.shape[2] if win_k is not None else 0
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    _check("fa4q_decode_noalloc", lib().fa4q_decode_noalloc(
+        _ptr(q), _ptr(k_pages), _ptr(k_sf), _ptr(vt_pages), _ptr(vt_sf), _ptr(block_table),
+        _ptr(fp4_len), _ptr(excl_mask), _ptr(hp_k), _ptr(hp_v), _ptr(hp_count), _ptr(win_k),
+        _ptr(win_v), _ptr(win_len), B, Hq, Hkv, d, max_pages, max_hp, W, _fmt(fmt), g_k, g_v, sm_scale,
+        _ptr(out), num_splits, _stream(stream)))
     return out
 
 

@@ -449,3 +449,70 @@ extern "C" fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const 
   decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(p.ws, rows, splits, p.out);
   return launch_status();
 }
+
+// =======================================================================================
+// fa4q_decode_noalloc: the same decode with its split partials in a static device array
+// =======================================================================================
+#include <mutex>
+
+namespace fa4q {
+
+// Upper bound of the static scratch: every GPU that loads the library holds these 8 MiB
+// until the process exits.  Enough for the split partials of B * Hq <= 1024 query heads at
+// the automatic split count of a 32768-key cache (about 3.7 MiB at d = 128).
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of g_decode_scratch, looked up once per device with that device current.
+// (In host code the symbol is only a host-side handle; passing it to a kernel directly
+// would address the wrong memory.)
+constexpr int kMaxDevices = 64;
+static std::mutex g_scratch_mu;
+static void* g_scratch_addr[kMaxDevices] = {};
+
+static fa4q_status scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA4Q_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return FA4Q_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || p == nullptr) return FA4Q_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return FA4Q_OK;
+}
+
+}  // namespace fa4q
+
+extern "C" fa4q_status fa4q_decode_noalloc(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
+                                           const uint8_t* vt_pages, const uint8_t* vt_sf,
+                                           const int32_t* block_table, const int32_t* fp4_len,
+                                           const uint64_t* excl_mask, const void* hp_k,
+                                           const void* hp_v, const int32_t* hp_count,
+                                           const void* win_k, const void* win_v,
+                                           const int32_t* win_len, int B, int Hq, int Hkv, int d,
+                                           int max_pages, int max_hp, int W, fa4q_format fmt,
+                                           float g_k, float g_v, float sm_scale, void* out,
+                                           int num_splits, void* stream) {
+  if (d != kDecD) return FA4Q_ERR_UNSUPPORTED;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_pages < 0 || max_hp < 0 || W < 0 || num_splits < 0)
+    return FA4Q_ERR_INVALID_ARG;
+  const size_t per_split = (size_t)B * Hq * (kDecD + 2) * sizeof(float);
+  int splits = num_splits;
+  if (splits == 0) {
+    splits = decode_auto_splits(B, Hkv, decode_chunks(max_pages, max_hp, W));
+    const size_t cap = kNoAllocScratchBytes / per_split;
+    if (cap < 1) return FA4Q_ERR_UNSUPPORTED;  // even one split's partials exceed the array
+    if ((size_t)splits > cap) splits = (int)cap;
+  } else if (per_split * (size_t)splits > kNoAllocScratchBytes) {
+    return FA4Q_ERR_UNSUPPORTED;               // the requested splits need more than 8 MiB
+  }
+  void* scratch = nullptr;
+  const fa4q_status st = scratch_address(&scratch);
+  if (st != FA4Q_OK) return st;
+  return fa4q_decode(q, k_pages, k_sf, vt_pages, vt_sf, block_table, fp4_len, excl_mask, hp_k, hp_v,
+                     hp_count, win_k, win_v, win_len, B, Hq, Hkv, d, max_pages, max_hp, W, fmt, g_k,
+                     g_v, sm_scale, out, scratch, kNoAllocScratchBytes, splits, stream);
+}
