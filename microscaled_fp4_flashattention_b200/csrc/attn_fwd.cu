@@ -15,16 +15,18 @@
 // "System-Level Optimization" - transposed softmax: P blocks run along the MMA reduction
 // (key) axis so P is quantised in registers and never leaves the SM.
 //
-// Kernel structure (one CTA per query tile, 256 threads, one CTA per SM):
+// Kernel structure (one CTA per query tile, 384 threads, one CTA per SM):
 //   warp 0      TMA producer: Q tile once, then K, V^T tiles and their scale atoms through
 //               an NST-deep shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
 //   warp 1      TMEM owner and MMA issuer (one elected thread): tcgen05.cp of the scale
 //               atoms into TMEM, tcgen05.mma kind::mxf4nvf4 (NVFP4) or kind::mxf4 (MXFP4).
-//   warps 4-7   softmax: one query row per thread; tcgen05.ld of S, mask, running max,
+//   warps 2-3   idle (they complete warpgroup 0 for the register split)
+//   warps 4-11  softmax: two groups of four warps take alternate key tiles, one query row
+//               per thread; tcgen05.ld of S, mask, running max (passed between the groups),
 //               exp2, block scales, cvt to E2M1, P^ to shared memory (the A operand of the
-//               PV MMA), rescale of O and l in TMEM when the maximum moves, epilogue.
-// TMEM (512 columns): S double buffer [0,256), O [256,256+D), l [384,400), scale factors
-// [400,464).  Every mbarrier wait is bounded; on expiry the CTA records a status bit,
+//               PV MMA), rescale of the group's O and l in TMEM, epilogue.
+// TMEM (512 columns): S [0,128), O even/odd tiles [128,256) and [256,384), l even/odd
+// [384,400) and [400,416), scale factors [416,480).  Every mbarrier wait is bounded; on expiry the CTA records a status bit,
 // skips the remaining waits, drains its own copies and MMAs and exits.
 #include <math.h>
 
@@ -37,14 +39,18 @@ static __device__ uint32_t g_attn_status;
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
+// Register split (setmaxnreg): launched at 168 per thread (3 warps per scheduler x 168 x 32 =
+// 16128 of the scheduler's 16384); warpgroup 0 (TMA, MMA, 2 idle warps) drops to 56 and the
+// two softmax warpgroups rise to 224: 56*32 + 2*224*32 = 16128, the launch total exactly.
+constexpr int kRegsIssue = 56, kRegsSoftmax = 224;
 constexpr int kStages = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGpNvfp4 = 1.0f / 2688.0f;  // g_P = 1/(6*448), rounded to FP32
 
-// TMEM column map
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColL = 384;
-constexpr uint32_t kColSfQ = 400, kColSfK = 408, kColSfP = 424, kColSfV = 440, kColSfOne = 456;
+// TMEM column map: one S buffer, two O and l accumulators (even / odd key tiles), scales
+constexpr uint32_t kColS = 0, kColO0 = 128, kColO1 = 256, kColL0 = 384, kColL1 = 400;
+constexpr uint32_t kColSfQ = 416, kColSfK = 424, kColSfP = 440, kColSfV = 456, kColSfOne = 472;
 
 template <int D, bool MX>
 struct Cfg {
@@ -77,11 +83,13 @@ struct __align__(1024) Smem {
   uint64_t bar_q;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_full[2];
-  uint64_t s_free[2];
+  uint64_t s_full[2];        // S of an even / odd key tile ready (one per softmax group)
+  uint64_t s_free;
   uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t o_done[2];
   uint64_t drain;
+  float m_xchg[2][kBM];       // running maximum after tile j, slot j%2, per row
+  float m_last[2][kBM];       // per group: the maximum its accumulator is relative to
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -124,6 +132,53 @@ FA4Q_DEVINL float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+FA4Q_DEVINL float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1) in one packed FP32 instruction
+FA4Q_DEVINL void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}\n"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// maximum of N consecutive values, as a tree of 3-input maxima
+template <int N>
+FA4Q_DEVINL float block_max(const float* v) {
+  float a[(N + 2) / 3];
+#pragma unroll
+  for (int i = 0; i < N / 3; ++i) a[i] = fmax3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+  if constexpr (N % 3 == 1) a[N / 3] = v[N - 1];
+  if constexpr (N % 3 == 2) a[N / 3] = fmaxf(v[N - 2], v[N - 1]);
+  if constexpr ((N + 2) / 3 == 1) {
+    return a[0];
+  } else {
+    return block_max<(N + 2) / 3>(a);
+  }
+}
+
+template <int N>
+FA4Q_DEVINL void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+FA4Q_DEVINL void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+FA4Q_DEVINL void named_bar_arrive(int id, int count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+FA4Q_DEVINL void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 FA4Q_DEVINL void tmem_ld1(uint32_t taddr, uint32_t& r) {
@@ -184,12 +239,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
+    mbar_init(&sm.s_free, 4);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_free[s], 4);
       mbar_init(&sm.p_full[s], 4);
+      mbar_init(&sm.o_done[s], 1);
     }
-    mbar_init(&sm.o_done, 1);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
@@ -212,6 +267,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
+  if (warp < 4) {
+  setmaxnreg_dec<kRegsIssue>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
@@ -257,24 +314,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_cp_sf_atom(tmem + kColSfOne + 4 * a, smem_u32(sm.sfone + 512 * a));
       for (int j = 0; ok && j <= n_tiles; ++j) {
         if (j < n_tiles) {
-          const int s = j % kStages, sb = j & 1;
+          // S_j = Q K_j^T into the single S buffer once the softmax holds S_{j-1} in registers
+          const int s = j % kStages, kb = j & 1;
           if (!cta_wait(&sm.kv_full[s], (j / kStages) & 1, abort_flag, kStatusTimeoutMma)) break;
-          if (j >= 2 && !cta_wait(&sm.s_free[sb], ((j - 2) >> 1) & 1, abort_flag, kStatusTimeoutMma))
-            break;
+          if (j >= 1 && !cta_wait(&sm.s_free, (j - 1) & 1, abort_flag, kStatusTimeoutMma)) break;
           tc_fence_after();
           for (int a = 0; a < C::kSfQAtoms; ++a)
-            tmem_cp_sf_atom(tmem + kColSfK + 8 * sb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
+            tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
           const uint32_t k_addr = smem_u32(sm.k[s]);
 #pragma unroll
           for (int ks = 0; ks < C::kKStepsQK; ++ks) {
             const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
             const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-            mma_step<MX>(tmem + (sb ? kColS1 : kColS0), ad, bd, kBN, ks, tmem + kColSfQ,
-                         tmem + kColSfK + 8 * sb, ks > 0);
+            mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ, tmem + kColSfK + 8 * kb, ks > 0);
           }
-          tc_commit(&sm.s_full[sb]);
+          tc_commit(&sm.s_full[j & 1]);
         }
         if (j >= 1) {
+          // [O | l]_{jp%2} (+)= P^_jp [V_jp | 1]
           const int jp = j - 1, s = jp % kStages, pb = jp & 1;
           if (!cta_wait(&sm.p_full[pb], (jp >> 1) & 1, abort_flag, kStatusTimeoutMma)) break;
           tc_fence_after();
@@ -284,16 +341,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t p_addr = smem_u32(sm.p[pb]);
           const uint32_t v_addr = smem_u32(sm.v[s]);
+          const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
             const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
             const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint32_t acc = (jp > 0 || ks > 0) ? 1u : 0u;
-            mma_step<MX>(tmem + kColO, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
-            mma_step<MX>(tmem + kColL, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
+            const uint32_t acc = (jp >= 2 || ks > 0) ? 1u : 0u;
+            mma_step<MX>(tmem + o_col, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
+            mma_step<MX>(tmem + l_col, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
           }
-          tc_commit(&sm.o_done);
+          tc_commit(&sm.o_done[pb]);
           tc_commit(&sm.kv_empty[s]);
         }
       }
@@ -301,32 +359,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, &g_attn_status, kStatusTimeoutDrain);
     }
-  } else if (warp >= 4) {
+  }
+  } else {
+    setmaxnreg_inc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax / PNQ / epilogue
-    const int wq = warp - 4;                       // TMEM lane quadrant
+    // Two softmax groups of four warps: group A (warps 4-7) takes the even key tiles, group B
+    // (warps 8-11) the odd ones; each thread owns one full query row of its tiles, and the TMEM
+    // lane quadrant of a warp is warp % 4.  Only the running maximum passes from one tile to
+    // the next: the group finishing tile j publishes m_j in shared memory and arrives on a
+    // named barrier the other group synchronises on.  Each group accumulates its own O and l,
+    // so the rescale before a tile's PV product waits on the group's previous PV product,
+    // issued two tiles earlier.  The loops never leave early (after an abort every wait
+    // returns at once), so arrivals and synchronisations on the named barriers always pair.
+    const int g = (warp - 4) >> 2;                 // softmax group: 0 = even tiles, 1 = odd
+    const int wq = warp & 3;                       // TMEM lane quadrant
     const int r = wq * 32 + lane;                  // row within the query tile
     const int row = qt * kBM + r;                  // query index
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const int bar_send = 1 + 4 * g + wq, bar_recv = 1 + 4 * (g ^ 1) + wq, bar_epi = 9 + wq;
     const float sc = p.score_scale_log2;
+    constexpr int kNB = kBN / C::kBlk;             // P blocks per row: 8 (NVFP4) / 4 (MXFP4)
     // Running maximum kept in the raw MMA-score domain.  Block maxima are taken from the
     // exact difference (bmax - m) * sc, so the block holding the row maximum gets amax = 1
     // exactly: the MX OCP exponent floor(log2 amax) - 2 jumps at every power of two, and a
     // fused s*sc - round(m*sc) that lands 1 ulp below 0 would move that block's scale.
-    float m = -INFINITY;
+    float m_acc = -INFINITY;                       // maximum of this group's last tile
     bool ok = true;
-    for (int j = 0; j < n_tiles && ok; ++j) {
-      const int sb = j & 1;
-      // warp-uniform outcome: every lane waits, all lanes take the same branch
-      if (!__all_sync(0xffffffffu, cta_wait(&sm.s_full[sb], (j >> 1) & 1, abort_flag, kStatusTimeoutSoftmax))) {
-        ok = false;
-        break;
-      }
+    for (int j = g; j < n_tiles; j += 2) {
+      ok = __all_sync(0xffffffffu, cta_wait(&sm.s_full[g], (j >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) && ok;
       tc_fence_after();
       float s[kBN];
       {
         uint32_t raw[kBN / 32][32];
 #pragma unroll
-        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + (sb ? kColS1 : kColS0) + 32 * c, raw[c]);
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + kColS + 32 * c, raw[c]);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < kBN / 32; ++c)
@@ -335,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.s_free[sb]);
+      if (lane == 0) mbar_arrive(&sm.s_free);
       // masking: keys beyond S_k, and (causal) keys after this query
       const int key0 = j * kBN;
       const bool edge = (key0 + kBN > p.S_k) || (CAUSAL && key0 + kBN - 1 > qt * kBM);
@@ -345,133 +411,157 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < kBN; ++i)
           if (i >= lim) s[i] = -INFINITY;
       }
-      // block maxima of the raw scores (the scale is positive), then the tile maximum
-      constexpr int kNB = kBN / C::kBlk;
+      // block maxima of the raw scores (the scale is positive), tree-shaped for ILP
       float bmax[kNB];
 #pragma unroll
-      for (int bi = 0; bi < kNB; ++bi) {
-        float mx = s[bi * C::kBlk];
-#pragma unroll
-        for (int i = 1; i < C::kBlk; ++i) mx = fmaxf(mx, s[bi * C::kBlk + i]);
-        bmax[bi] = mx;
-      }
+      for (int bi = 0; bi < kNB; ++bi) bmax[bi] = block_max<C::kBlk>(s + bi * C::kBlk);
       float tmax = bmax[0];
 #pragma unroll
       for (int bi = 1; bi < kNB; ++bi) tmax = fmaxf(tmax, bmax[bi]);
-      const float m_new = fmaxf(m, tmax);
-      const float alpha = ex2_approx((m - m_new) * sc);   // 0 on the first tile
+      // running maximum: take m_{j-1} from the other group, publish m_j
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        named_bar_sync(bar_recv, 64);
+        m_prev = sm.m_xchg[(j - 1) & 1][r];
+      }
+      const float m_new = fmaxf(m_prev, tmax);
+      sm.m_xchg[j & 1][r] = m_new;
+      named_bar_arrive(bar_send, 64);
       const float mref = m_new * sc;
       // per block: amax = exp2((bmax - m)*sc); scale; y_i = exp2(s_i*sc - m*sc - log2(scale))
-      uint32_t packed[kBN / 8];
-      uint32_t sfw[kNB / 4 > 0 ? kNB / 4 : 1];
+      float off[kNB];
+      uint32_t sfw[kNB / 4];
 #pragma unroll
-      for (int w = 0; w < (kNB / 4 > 0 ? kNB / 4 : 1); ++w) sfw[w] = 0;
+      for (int w = 0; w < kNB / 4; ++w) sfw[w] = 0;
 #pragma unroll
       for (int bi = 0; bi < kNB; ++bi) {
         const float amax = ex2_approx((bmax[bi] - m_new) * sc);
-        float off;
         uint32_t code;
         if constexpr (MX) {
           const int e = mx_exponent(amax, p.qmax_p);
           code = static_cast<uint32_t>(e + 127);
-          off = mref + static_cast<float>(e);
-          if (!(amax > 0.0f)) off = INFINITY;
+          off[bi] = amax > 0.0f ? mref + static_cast<float>(e) : INFINITY;
         } else {
           const float t = __fdiv_rn(amax, 6.0f * kGpNvfp4);       // amax / (6 * g_P)
           code = ue4m3_encode(t);
           const float sf = ue4m3_decode(code);
-          off = sf > 0.0f ? mref + lg2_approx(sf * kGpNvfp4) : INFINITY;
+          off[bi] = sf > 0.0f ? mref + lg2_approx(sf * kGpNvfp4) : INFINITY;
         }
         sfw[bi >> 2] |= code << (8 * (bi & 3));
-#pragma unroll
-        for (int g8 = 0; g8 < C::kBlk / 8; ++g8) {
-          const int base = bi * C::kBlk + g8 * 8;
-          float y[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) y[i] = ex2_approx(fmaf(s[base + i], sc, -off));
-          packed[base / 8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-        }
       }
-      // P^ (64 bytes of this row) and its scales into the shared-memory A operand
-      uint8_t* pbuf = sm.p[sb];
+      uint32_t packed[kBN / 8];
+#pragma unroll
+      for (int g8 = 0; g8 < kBN / 8; ++g8) {
+        const float o8 = off[(g8 * 8) / C::kBlk];
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) ffma2(y[i], y[i + 1], s[8 * g8 + i], s[8 * g8 + i + 1], sc, sc, -o8, -o8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = ex2_approx(y[i]);
+        packed[g8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+      }
+      // accumulator g and P buffer g were last used by this group's previous PV product
+      if (j >= 2)
+        ok = __all_sync(0xffffffffu, cta_wait(&sm.o_done[g], ((j - 2) >> 1) & 1, abort_flag,
+                                              kStatusTimeoutSoftmax)) && ok;
+      uint8_t* pbuf = sm.p[g];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
         *reinterpret_cast<uint4*>(pbuf + swz64_offset(r, c)) =
             make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
 #pragma unroll
       for (int a = 0; a < C::kSfTileAtoms; ++a)
-        *reinterpret_cast<uint32_t*>(sm.sfp[sb] + 512 * a + (r & 31) * 16 + (r >> 5) * 4) = sfw[a];
+        *reinterpret_cast<uint32_t*>(sm.sfp[g] + 512 * a + (r & 31) * 16 + (r >> 5) * 4) = sfw[a];
       fence_proxy_async_smem();
-      // rescale O and l once the previous PV product has landed
-      if (j >= 1) {
-        if (!__all_sync(0xffffffffu, cta_wait(&sm.o_done, (j - 1) & 1, abort_flag, kStatusTimeoutSoftmax))) {
-          ok = false;
-          break;
-        }
+      // bring accumulator g from the maximum it holds (tile j-2) to m_j
+      if (j >= 2) {
         tc_fence_after();
+        const float alpha = ex2_approx((m_acc - m_new) * sc);
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          const uint32_t o_col = g ? kColO1 : kColO0, l_col = g ? kColL1 : kColL0;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t raw[32];
-            tmem_ld32(lane_base + kColO + 32 * c, raw);
+            tmem_ld32(lane_base + o_col + 32 * c, raw);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
-            tmem_st32(lane_base + kColO + 32 * c, raw);
+            tmem_st32(lane_base + o_col + 32 * c, raw);
           }
           uint32_t lr;
-          tmem_ld1(lane_base + kColL, lr);
+          tmem_ld1(lane_base + l_col, lr);
           tmem_wait_ld();
-          tmem_st1(lane_base + kColL, __float_as_uint(__uint_as_float(lr) * alpha));
+          tmem_st1(lane_base + l_col, __float_as_uint(__uint_as_float(lr) * alpha));
           tmem_wait_st();
         }
       }
-      m = m_new;
+      m_acc = m_new;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[sb]);
+      if (lane == 0) mbar_arrive(&sm.p_full[g]);
     }
+    // the group that did not process the last tile consumes its maximum (keeps the named
+    // barrier arrivals and synchronisations paired)
+    if (((n_tiles - 1) & 1) != g) named_bar_sync(bar_recv, 64);
     // ---------------------------------------------------------------- epilogue
-    if (ok && __all_sync(0xffffffffu, cta_wait(&sm.o_done, (n_tiles - 1) & 1, abort_flag, kStatusTimeoutSoftmax))) {
+    // out = (O_A 2^((mA - m) sc) + O_B 2^((mB - m) sc)) / (l_A ... + l_B ...) * g_v with m the
+    // final maximum; group A writes output columns [0, D/2), group B [D/2, D)
+    sm.m_last[g][r] = m_acc;
+    named_bar_sync(bar_epi, 64);
+    const float mA = sm.m_last[0][r], mB = sm.m_last[1][r];
+    const float m = fmaxf(mA, mB);
+    const int last0 = (n_tiles - 1) & ~1, last1 = n_tiles >= 2 ? ((n_tiles - 2) | 1) : -1;
+    ok = __all_sync(0xffffffffu, cta_wait(&sm.o_done[0], (last0 >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) && ok;
+    if (last1 >= 0)
+      ok = __all_sync(0xffffffffu, cta_wait(&sm.o_done[1], (last1 >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) && ok;
+    if (ok) {
       tc_fence_after();
-      uint32_t lr;
-      tmem_ld1(lane_base + kColL, lr);
+      const bool has_b = last1 >= 0;
+      const float wa = ex2_approx((mA - m) * sc), wb = has_b ? ex2_approx((mB - m) * sc) : 0.0f;
+      uint32_t lra, lrb = 0;
+      tmem_ld1(lane_base + kColL0, lra);
+      if (has_b) tmem_ld1(lane_base + kColL1, lrb);
+      uint32_t rawa[D / 64][32], rawb[D / 64][32];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tmem_ld32(lane_base + kColO0 + g * (D / 2) + 32 * c, rawa[c]);
+        tmem_ld32(lane_base + kColO1 + g * (D / 2) + 32 * c, rawb[c]);
+      }
       tmem_wait_ld();
-      const float l = __uint_as_float(lr);
-      const float inv = p.g_v / l;
+      const float l = __uint_as_float(lra) * wa + (has_b ? __uint_as_float(lrb) * wb : 0.0f);
+      const float inva = p.g_v / l * wa, invb = p.g_v / l * wb;
       const bool store = row < p.S_q;
       const int64_t orow = (int64_t)bh_q * p.S_q + row;
+      if (store) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t raw[32];
-        tmem_ld32(lane_base + kColO + 32 * c, raw);
-        tmem_wait_ld();
-        if (store) {
+        for (int c = 0; c < D / 64; ++c) {
+          const int ocol = g * (D / 2) + 32 * c;
+          float o[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            o[i] = __uint_as_float(rawa[c][i]) * inva + (has_b ? __uint_as_float(rawb[c][i]) * invb : 0.0f);
           if (p.out_fp32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * D + 32 * c);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow * D + ocol);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(raw[4 * i]) * inv, __uint_as_float(raw[4 * i + 1]) * inv,
-                                   __uint_as_float(raw[4 * i + 2]) * inv, __uint_as_float(raw[4 * i + 3]) * inv);
+            for (int i = 0; i < 8; ++i) dst[i] = make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * D + 32 * c);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow * D + ocol);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
               uint32_t w[4];
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                __nv_bfloat162 pr = __floats2bfloat162_rn(__uint_as_float(raw[8 * i + 2 * q]) * inv,
-                                                          __uint_as_float(raw[8 * i + 2 * q + 1]) * inv);
+                __nv_bfloat162 pr = __floats2bfloat162_rn(o[8 * i + 2 * q], o[8 * i + 2 * q + 1]);
                 w[q] = *reinterpret_cast<uint32_t*>(&pr);
               }
               dst[i] = make_uint4(w[0], w[1], w[2], w[3]);
             }
           }
         }
-      }
-      if (store && p.lse != nullptr) {
-        const float lscale = MX ? 1.0f : kGpNvfp4;
-        p.lse[orow] = m * sc * 0.69314718055994531f + logf(l * lscale);
+        if (g == 0 && p.lse != nullptr) {
+          const float lscale = MX ? 1.0f : kGpNvfp4;
+          p.lse[orow] = m * sc * 0.69314718055994531f + logf(l * lscale);
+        }
       }
     }
   }
