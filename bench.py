@@ -204,6 +204,38 @@ class DecodeRun:
                            workspace=self.ws)
 
 
+def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
+    """Time the decode over the paged hybrid cache; adds line["decode"]."""
+    import torch
+    dw = synth.WORKLOADS[4]
+    drun = DecodeRun(dw, dev, fa4q)
+    for _ in range(max(3, args.warmup)):
+        drun.step()
+    barrier()
+    dsteps = max(20, args.steps)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dsampler = ClockSampler(dev.index)
+    with dsampler:
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            for _ in range(20):
+                drun.step()
+            torch.cuda.synchronize()
+        d0.record()
+        for _ in range(dsteps):
+            drun.step()
+        d1.record()
+        barrier()
+    d_ms = d0.elapsed_time(d1) / dsteps
+    gbs = drun.bytes / (d_ms * 1e-3) / 1e9
+    line["decode"] = {"workload": dw.name, "us_per_step": d_ms * 1e3, "higher_is_better": False,
+                      "GBps": gbs, "bytes_per_step": drun.bytes, "gpu_launches": 2 * dsteps,
+                      "roofline": {"kernel": "decode_split_kernel+decode_combine_kernel", "bound": "hbm",
+                                   "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                                   "traffic": None, "peak_source": f"{peak_kind} hbm copy"},
+                      "l2": "working set 1.4 GB > L2", "clocks": dsampler.summary()}
+
+
 # ------------------------------------------------------------------------------ CPU oracle timing
 def oracle_prefill_sample(w, budget_s: float, host=None):
     """Time the oracle on sampled (head, row) work of workload w for about budget_s seconds;
@@ -242,6 +274,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true", help="time only the decode path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--soak-s", type=float, default=2.0)
     args = ap.parse_args()
@@ -285,6 +318,11 @@ def main():
     torch.cuda.set_device(dev)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = load_peaks()
 
+    if args.decode_only:
+        line = {"metric": METRIC, "n_gpus": world}
+        decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier=lambda: torch.cuda.synchronize())
+        print(json.dumps(line))
+        return
     run = PrefillRun(w, dev, fa4q, seed_offset=rank)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
 
@@ -378,33 +416,7 @@ def main():
     if not args.no_decode:
         del run, flush
         torch.cuda.empty_cache()
-        dw = synth.WORKLOADS[4]
-        drun = DecodeRun(dw, dev, fa4q)
-        for _ in range(max(3, args.warmup)):
-            drun.step()
-        barrier()
-        dsteps = max(20, args.steps)
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        dsampler = ClockSampler(dev.index)
-        with dsampler:
-            t_end = time.time() + 1.0
-            while time.time() < t_end:
-                for _ in range(20):
-                    drun.step()
-                torch.cuda.synchronize()
-            d0.record()
-            for _ in range(dsteps):
-                drun.step()
-            d1.record()
-            barrier()
-        d_ms = d0.elapsed_time(d1) / dsteps
-        gbs = drun.bytes / (d_ms * 1e-3) / 1e9
-        line["decode"] = {"workload": dw.name, "us_per_step": d_ms * 1e3, "higher_is_better": False,
-                          "GBps": gbs, "bytes_per_step": drun.bytes, "gpu_launches": 2 * dsteps,
-                          "roofline": {"kernel": "decode_split_kernel+decode_combine_kernel", "bound": "hbm",
-                                       "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                                       "traffic": None, "peak_source": f"{peak_kind} hbm copy"},
-                          "l2": "working set 1.4 GB > L2", "clocks": dsampler.summary()}
+        decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, _ = oracle_prefill_sample(w, 12.0)

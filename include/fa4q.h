@@ -252,10 +252,11 @@ fa4q_status fa4q_device_status(void* stream, uint32_t* detail);
 /*
  * fa4q_selftest_wait_timeout - diagnostic: launch one kernel that waits, with the same
  * bounded-wait helper every pipelined kernel uses, on a barrier nothing will complete, for
- * `polls` polls.  The wait expires, the kernel records FA4Q_ERR_TIMEOUT in the device status
- * word and returns; no GPU hang or fault is involved.  Read it with fa4q_device_status.
+ * `wait_us` microseconds.  The wait expires, the kernel records FA4Q_ERR_TIMEOUT in the
+ * device status word and returns; no GPU hang or fault is involved.  Read it with
+ * fa4q_device_status.  (Every pipelined kernel's waits give up after 2 s the same way.)
  */
-fa4q_status fa4q_selftest_wait_timeout(uint32_t polls, void* stream);
+fa4q_status fa4q_selftest_wait_timeout(uint32_t wait_us, void* stream);
 
 #ifdef __cplusplus
 }

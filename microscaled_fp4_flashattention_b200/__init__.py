@@ -253,8 +253,8 @@ def device_status(stream=None):
     return code, detail.value
 
 
-def selftest_wait_timeout(polls: int, stream=None):
-    _check("fa4q_selftest_wait_timeout", lib().fa4q_selftest_wait_timeout(polls, _stream(stream)))
+def selftest_wait_timeout(wait_us: int, stream=None):
+    _check("fa4q_selftest_wait_timeout", lib().fa4q_selftest_wait_timeout(wait_us, _stream(stream)))
 
 
 def default_sm_scale(d: int) -> float:

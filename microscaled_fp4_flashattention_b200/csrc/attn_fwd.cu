@@ -113,9 +113,12 @@ struct AttnParams {
 FA4Q_DEVINL bool cta_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag,
                           uint32_t code) {
   if (*abort_flag) return false;
-  for (uint32_t i = 0; i < kWaitPolls; ++i) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023) == 1023 && *abort_flag) return false;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitNs) break;
   }
   atomicOr(&g_attn_status, code);
   *abort_flag = 1;
@@ -665,15 +668,15 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
-// bounded-wait probe: waits on a barrier nothing will complete, for `polls` polls
-__global__ void wait_probe_kernel(uint32_t polls) {
+// bounded-wait probe: waits on a barrier nothing will complete, for `wait_us` microseconds
+__global__ void wait_probe_kernel(uint32_t wait_us) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(&bar, 0, &g_attn_status, kStatusTimeoutProbe, polls);
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &g_attn_status, kStatusTimeoutProbe, uint64_t(wait_us) * 1000);
 }
 
 cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word) {
@@ -810,7 +813,7 @@ extern "C" fa4q_status fa4q_selftest_block_mma(const uint8_t* a, const uint8_t* 
   return launch_status();
 }
 
-extern "C" fa4q_status fa4q_selftest_wait_timeout(uint32_t polls, void* stream) {
-  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(polls);
+extern "C" fa4q_status fa4q_selftest_wait_timeout(uint32_t wait_us, void* stream) {
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(wait_us);
   return launch_status();
 }

@@ -71,6 +71,14 @@ FA4Q_DEVINL uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   return out;
 }
 
+// four E2M1 codes (the low 16 bits of w, low nibble first) -> two f16x2 (codes 0,1 and 2,3)
+FA4Q_DEVINL void e2m1x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 // two E4M3 bytes (low byte first) -> f16x2
 FA4Q_DEVINL uint32_t e4m3x2_to_f16x2(uint32_t two) {
   uint32_t out;
@@ -101,17 +109,81 @@ FA4Q_DEVINL float ex2f(float x) {
   return y;
 }
 
-__global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const DecParams p) {
-  __shared__ float s_o[kDecWarps][8][kDecD];
-  __shared__ float s_m[kDecWarps][8];
-  __shared__ float s_l[kDecWarps][8];
+// Work units of one (sequence, kv-head): FP4 pages (64 tokens) first, then 16-token slices
+// of the BF16 vertical-line set, then 16-token slices of the BF16 window.
+constexpr int kStageBytes = 9216;          // K page 4096 + K scales 512 + V^T page 4096 + scales 512
+constexpr int kDecStages = 3;              // per-warp shared-memory ring depth
+
+struct UnitInfo {
+  int kind;        // 0 FP4 page, 1 vertical-line slice, 2 window slice
+  int base;        // first token of the unit within its class
+  int nvalid;      // tokens of the unit that exist (<= 64 or 16)
+};
+
+FA4Q_DEVINL UnitInfo unit_info(const DecParams& p, int u, int n_fp4, int n_hp, int n_win) {
+  UnitInfo x;
+  if (u < p.n_ch_fp4) {
+    x.kind = 0; x.base = u * 64; x.nvalid = min(64, n_fp4 - x.base);
+  } else if (u < p.n_ch_fp4 + p.n_ch_hp) {
+    x.kind = 1; x.base = (u - p.n_ch_fp4) * 16; x.nvalid = min(16, n_hp - x.base);
+  } else {
+    x.kind = 2; x.base = (u - p.n_ch_fp4 - p.n_ch_hp) * 16; x.nvalid = min(16, n_win - x.base);
+  }
+  return x;
+}
+
+FA4Q_DEVINL void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// Issue the copies of unit `u` into one ring stage (lane 0 only).
+FA4Q_DEVINL void issue_unit(const DecParams& p, const UnitInfo& x, int b, int hk, int bh, int u,
+                            uint8_t* stage, uint64_t* bar) {
+  if (x.kind == 0) {
+    const int64_t phys = p.table[(int64_t)b * p.max_pages + u];
+    const int64_t ph = phys * p.Hkv + hk;
+    mbar_arrive_expect_tx(bar, kStageBytes);
+    bulk_load(stage, p.kp + ph * 64 * (kDecD / 2), 4096, bar);
+    bulk_load(stage + 4096, p.ksf + ph * 64 * (kDecD / 16), 512, bar);
+    bulk_load(stage + 4608, p.vp + ph * kDecD * 32, 4096, bar);
+    bulk_load(stage + 8704, p.vsf + ph * kDecD * 4, 512, bar);
+  } else {
+    const uint16_t* kb = x.kind == 1 ? p.hp_k + ((int64_t)bh * p.max_hp + x.base) * kDecD
+                                     : p.win_k + ((int64_t)bh * p.W + x.base) * kDecD;
+    const uint16_t* vb = x.kind == 1 ? p.hp_v + ((int64_t)bh * p.max_hp + x.base) * kDecD
+                                     : p.win_v + ((int64_t)bh * p.W + x.base) * kDecD;
+    const uint32_t bytes = static_cast<uint32_t>(x.nvalid) * kDecD * 2;
+    mbar_arrive_expect_tx(bar, 2 * bytes);
+    bulk_load(stage, kb, bytes, bar);
+    bulk_load(stage + 4608, vb, bytes, bar);
+  }
+}
+
+__global__ void __launch_bounds__(kDecWarps * 32, 2) decode_split_kernel(const DecParams p) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  // [rings of all warps][mbarriers]; after the scan the rings are reused for the warp merge
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dsm + kDecWarps * kDecStages * kStageBytes);
+  float* s_o = reinterpret_cast<float*>(dsm);                  // [warps][8][128]  (aliases rings)
+  float* s_m = s_o + kDecWarps * 8 * kDecD;                    // [warps][8]
+  float* s_l = s_m + kDecWarps * 8;                            // [warps][8]
   const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int G = p.G;
   const int bh = b * p.Hkv + hk;
+  uint8_t* ring = dsm + warp * kDecStages * kStageBytes;
+  uint64_t* full = bars + warp * kDecStages;
+  if (lane == 0) {
+    for (int st = 0; st < kDecStages; ++st) mbar_init(&full[st], 1);
+    fence_barrier_init();
+  }
+  __syncwarp();
 
-  // ---- query fragments: row g = GQA head g of this kv-head (rows >= G are zero)
+  // ---- query fragments: row g = GQA head g of this kv-head (rows >= G are zero).  The
+  // reduction order of the score MMA is permuted: logical k = 2t+e / 2t+8+e of chunk kc is
+  // head dim 32t + 4kc + e / 32t + 4kc + 2 + e, so a thread's B operand is 32 consecutive dims.
   uint32_t qa[8][2];
   {
     const bool real = g < G;
@@ -133,160 +205,191 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
   const int n_fp4 = min(p.fp4_len[b], p.max_pages * 64);
   const int n_hp = p.hp_count ? min(p.hp_count[bh], p.max_hp) : 0;
   const int n_win = p.win_len ? min(p.win_len[b], p.W) : 0;
-  const int total_chunks = p.n_ch_fp4 + p.n_ch_hp + p.n_ch_win;
+  const int total = p.n_ch_fp4 + p.n_ch_hp + p.n_ch_win;
   const int c_begin = split * p.chunks_per_split;
-  const int c_end = min(total_chunks, c_begin + p.chunks_per_split);
-
-  for (int ch = c_begin + warp; ch < c_end; ch += kDecWarps) {
-    // ---- classify the chunk; skip chunks with no valid key
-    int kind, base, nvalid;
-    if (ch < p.n_ch_fp4) {
-      kind = 0; base = ch * 64; nvalid = n_fp4 - base;
-    } else if (ch < p.n_ch_fp4 + p.n_ch_hp) {
-      kind = 1; base = (ch - p.n_ch_fp4) * 64; nvalid = n_hp - base;
-    } else {
-      kind = 2; base = (ch - p.n_ch_fp4 - p.n_ch_hp) * 64; nvalid = n_win - base;
+  const int c_end = min(total, c_begin + p.chunks_per_split);
+  // this warp's units: c_begin + warp, + kDecWarps, ... skipping units without a valid token
+  auto next_valid = [&](int u) {
+    while (u < c_end && unit_info(p, u, n_fp4, n_hp, n_win).nvalid <= 0) u += kDecWarps;
+    return u;
+  };
+  int u_issue = next_valid(c_begin + warp);
+  int n_issued = 0;
+  if (lane == 0) {
+    for (int k = 0; k < kDecStages - 1 && u_issue < c_end; ++k) {
+      issue_unit(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
+                 ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
+      ++n_issued;
+      u_issue = next_valid(u_issue + kDecWarps);
     }
-    if (nvalid <= 0) continue;
-    uint64_t vmask = nvalid >= 64 ? ~0ull : ((1ull << nvalid) - 1ull);
-    const uint8_t* kpage = nullptr;
-    const uint8_t* ksfp = nullptr;
-    const uint8_t* vpage = nullptr;
-    const uint8_t* vsfp = nullptr;
-    const uint16_t* kb16 = nullptr;
-    const uint16_t* vb16 = nullptr;
-    if (kind == 0) {
-      const int64_t phys = p.table[(int64_t)b * p.max_pages + ch];
-      if (p.excl) vmask &= ~p.excl[(int64_t)bh * p.max_pages + ch];
-      kpage = p.kp + (phys * p.Hkv + hk) * 64 * (kDecD / 2);
-      ksfp = p.ksf + (phys * p.Hkv + hk) * 64 * (kDecD / 16);
-      vpage = p.vp + (phys * p.Hkv + hk) * kDecD * 32;
-      vsfp = p.vsf + (phys * p.Hkv + hk) * kDecD * 4;
-    } else if (kind == 1) {
-      kb16 = p.hp_k + ((int64_t)bh * p.max_hp + base) * kDecD;
-      vb16 = p.hp_v + ((int64_t)bh * p.max_hp + base) * kDecD;
-    } else {
-      kb16 = p.win_k + ((int64_t)bh * p.W + base) * kDecD;
-      vb16 = p.win_v + ((int64_t)bh * p.W + base) * kDecD;
+  } else {
+    for (int k = 0; k < kDecStages - 1 && u_issue < c_end; ++k) {
+      ++n_issued;
+      u_issue = next_valid(u_issue + kDecWarps);
     }
+  }
+  int n_done = 0;
+  bool ok = true;
+  for (int u = next_valid(c_begin + warp); u < c_end; u = next_valid(u + kDecWarps)) {
+    // keep the ring full: the stage refilled now was consumed in the previous iteration
+    // (after a failed wait nothing new is issued; copies already in flight are still awaited)
+    __syncwarp();
+    if (ok && u_issue < c_end) {
+      if (lane == 0)
+        issue_unit(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
+                   ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
+      ++n_issued;
+      u_issue = next_valid(u_issue + kDecWarps);
+    }
+    const UnitInfo x = unit_info(p, u, n_fp4, n_hp, n_win);
+    const int stg = n_done % kDecStages;
+    if (n_done >= n_issued) break;                  // stopped issuing after a failed wait
+    ok = __all_sync(0xffffffffu, mbar_wait(&full[stg], (n_done / kDecStages) & 1, &g_decode_status,
+                                           kStatusTimeoutDecode)) && ok;
+    const uint8_t* st8 = ring + stg * kStageBytes;
+    ++n_done;
+    if (!ok) continue;
+    uint64_t vmask = x.nvalid >= 64 ? ~0ull : ((1ull << x.nvalid) - 1ull);
+    if (x.kind == 0 && p.excl) vmask &= ~p.excl[(int64_t)bh * p.max_pages + u];
     if (vmask == 0ull) continue;
-    const float sc = kind == 0 ? p.sc_fp4 : p.sc_bf16;
 
-    // ---- scores for 8 groups (c, sigma): thread's own token in group = 16(g>>1)+4c+2sigma+(g&1)
-    float s[8][2];
+    if (x.kind == 0) {
+      // ================= FP4 page: 64 tokens, permuted order (see the file header)
+      const float sc = p.sc_fp4;
+      float s[8][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int c = i >> 1, sg = i & 1;
-      const int tok = 16 * (g >> 1) + 4 * c + 2 * sg + (g & 1);
-      uint32_t bfr[8][2];
-      if (kind == 0) {
-        const uint4 kw = *reinterpret_cast<const uint4*>(kpage + tok * 64 + 16 * t);
-        const uint32_t sfw = *reinterpret_cast<const uint16_t*>(ksfp + tok * 8 + 2 * t);
+      for (int i = 0; i < 8; ++i) {
+        const int c = i >> 1, sg = i & 1;
+        const int tok = 16 * (g >> 1) + 4 * c + 2 * sg + (g & 1);
+        const uint4 kw = *reinterpret_cast<const uint4*>(st8 + tok * 64 + 16 * t);
+        const uint32_t sfw = *reinterpret_cast<const uint16_t*>(st8 + 4096 + tok * 8 + 2 * t);
         const uint32_t sf2 = e4m3x2_to_f16x2(sfw);
         const uint32_t sfa = __byte_perm(sf2, 0, 0x1010), sfb = __byte_perm(sf2, 0, 0x3232);
         const uint32_t words[4] = {kw.x, kw.y, kw.z, kw.w};
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
-          const uint32_t wd = words[kc >> 1];
-          const int sh = (kc & 1) * 16;
+          uint32_t f0, f1;
+          e2m1x4_to_f16x2x2(words[kc >> 1] >> ((kc & 1) * 16), f0, f1);
           const uint32_t scl = kc < 4 ? sfa : sfb;
-          bfr[kc][0] = hmul2(e2m1x2_to_f16x2((wd >> sh) & 0xFF), scl);
-          bfr[kc][1] = hmul2(e2m1x2_to_f16x2((wd >> (sh + 8)) & 0xFF), scl);
+          mma_f16(acc, qa[kc][0], qa[kc][1], hmul2(f0, scl), hmul2(f1, scl));
         }
-      } else {
-        const uint16_t* kr = kb16 + (int64_t)tok * kDecD + 32 * t;
-        if (tok < nvalid) {
 #pragma unroll
-          for (int kc = 0; kc < 8; ++kc) {
-            const uint2 w = *reinterpret_cast<const uint2*>(kr + 4 * kc);
-            bfr[kc][0] = bf16x2_to_f16x2(w.x);
-            bfr[kc][1] = bf16x2_to_f16x2(w.y);
-          }
-        } else {
-#pragma unroll
-          for (int kc = 0; kc < 8; ++kc) bfr[kc][0] = bfr[kc][1] = 0u;
+        for (int e = 0; e < 2; ++e) {
+          const int tk = 16 * t + 4 * c + 2 * sg + e;
+          s[i][e] = ((vmask >> tk) & 1ull) ? acc[e] * sc : -INFINITY;
         }
       }
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      float cmax = s[0][0];
 #pragma unroll
-      for (int kc = 0; kc < 8; ++kc) mma_f16(acc, qa[kc][0], qa[kc][1], bfr[kc][0], bfr[kc][1]);
-      // accumulator (row g, columns 2t, 2t+1) = tokens 16t + 4c + 2sigma + {0, 1}
+      for (int i = 0; i < 8; ++i) cmax = fmaxf(cmax, fmaxf(s[i][0], s[i][1]));
+      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
+      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
+      const float m_new = fmaxf(m, cmax);
+      const float alpha = ex2f(m - m_new);
+      uint32_t pa[8];
+      float psum = 0.0f;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tk = 16 * t + 4 * c + 2 * sg + e;
-        s[i][e] = ((vmask >> tk) & 1ull) ? acc[e] * sc : -INFINITY;
+      for (int i = 0; i < 8; ++i) {
+        const float p0 = ex2f(s[i][0] - m_new), p1 = ex2f(s[i][1] - m_new);
+        psum += p0 + p1;
+        pa[i] = f32x2_to_f16x2(p0 * p.g_v, p1 * p.g_v);
       }
-    }
-    // ---- online softmax update (row g; the 4 threads of a group share the row)
-    float cmax = s[0][0];
+      l = l * alpha + psum;
+      m = m_new;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) cmax = fmaxf(cmax, fmaxf(s[i][0], s[i][1]));
-    cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
-    cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
-    const float m_new = fmaxf(m, cmax);
-    const float alpha = ex2f(m - m_new);
-    const float gv = kind == 0 ? p.g_v : 1.0f;
-    uint32_t pa[8];
-    float psum = 0.0f;
+      for (int i = 0; i < 16; ++i) {
+        o[i][0] *= alpha;
+        o[i][1] *= alpha;
+      }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float p0 = ex2f(s[i][0] - m_new), p1 = ex2f(s[i][1] - m_new);
-      psum += p0 + p1;
-      pa[i] = f32x2_to_f16x2(p0 * gv, p1 * gv);
-    }
-    l = l * alpha + psum;
-    m = m_new;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      o[i][0] *= alpha;
-      o[i][1] *= alpha;
-    }
-    // ---- O += P V: channel 8*nt + g, tokens 16t + 4c + {0..3}
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int chn = 8 * nt + g;
-      uint32_t vb[4][2];
-      if (kind == 0) {
-        const uint2 vw = *reinterpret_cast<const uint2*>(vpage + chn * 32 + 8 * t);
-        const uint32_t sfv = vsfp[chn * 4 + t];
+      for (int nt = 0; nt < 16; ++nt) {
+        const int chn = 8 * nt + g;
+        const uint2 vw = *reinterpret_cast<const uint2*>(st8 + 4608 + chn * 32 + 8 * t);
+        const uint32_t sfv = st8[8704 + chn * 4 + t];
         const uint32_t s2 = e4m3x2_to_f16x2(sfv | (sfv << 8));
-        const uint32_t words[2] = {vw.x, vw.y};
+        uint32_t v0, v1, v2, v3;
+        e2m1x4_to_f16x2x2(vw.x, v0, v1);
+        mma_f16(o[nt], pa[0], pa[1], hmul2(v0, s2), hmul2(v1, s2));
+        e2m1x4_to_f16x2x2(vw.x >> 16, v2, v3);
+        mma_f16(o[nt], pa[2], pa[3], hmul2(v2, s2), hmul2(v3, s2));
+        e2m1x4_to_f16x2x2(vw.y, v0, v1);
+        mma_f16(o[nt], pa[4], pa[5], hmul2(v0, s2), hmul2(v1, s2));
+        e2m1x4_to_f16x2x2(vw.y >> 16, v2, v3);
+        mma_f16(o[nt], pa[6], pa[7], hmul2(v2, s2), hmul2(v3, s2));
+      }
+    } else {
+      // ================= BF16 slice: 16 tokens, natural order; K rows 256 B, V rows 256 B
+      const float sc = p.sc_bf16;
+      float s[2][2];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t wd = words[c >> 1];
-          const int sh = (c & 1) * 16;
-          vb[c][0] = hmul2(e2m1x2_to_f16x2((wd >> sh) & 0xFF), s2);
-          vb[c][1] = hmul2(e2m1x2_to_f16x2((wd >> (sh + 8)) & 0xFF), s2);
+      for (int sg = 0; sg < 2; ++sg) {
+        const int tok = 8 * sg + g;
+        const uint8_t* kr = st8 + tok * 256 + 64 * t;
+        // rows past nvalid are not loaded (zeros); the MMAs stay outside the branch because
+        // mma.sync.aligned must be executed by all lanes of the warp together
+        const bool have = tok < x.nvalid;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint4 w = have ? *reinterpret_cast<const uint4*>(kr + 16 * q4) : make_uint4(0u, 0u, 0u, 0u);
+          mma_f16(acc, qa[2 * q4][0], qa[2 * q4][1], bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y));
+          mma_f16(acc, qa[2 * q4 + 1][0], qa[2 * q4 + 1][1], bf16x2_to_f16x2(w.z), bf16x2_to_f16x2(w.w));
         }
-      } else {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t hv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int tk = 16 * t + 4 * c + e;
-            hv[e] = tk < nvalid ? static_cast<uint32_t>(vb16[(int64_t)tk * kDecD + chn]) : 0u;
-          }
-          vb[c][0] = bf16x2_to_f16x2(hv[0] | (hv[1] << 16));
-          vb[c][1] = bf16x2_to_f16x2(hv[2] | (hv[3] << 16));
+        for (int e = 0; e < 2; ++e) {
+          const int tk = 8 * sg + 2 * t + e;
+          s[sg][e] = ((vmask >> tk) & 1ull) ? acc[e] * sc : -INFINITY;
         }
       }
+      float cmax = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
+      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
+      const float m_new = fmaxf(m, cmax);
+      const float alpha = ex2f(m - m_new);
+      const float p00 = ex2f(s[0][0] - m_new), p01 = ex2f(s[0][1] - m_new);
+      const float p10 = ex2f(s[1][0] - m_new), p11 = ex2f(s[1][1] - m_new);
+      l = l * alpha + (p00 + p01) + (p10 + p11);
+      m = m_new;
+      const uint32_t a0 = f32x2_to_f16x2(p00, p01), a2 = f32x2_to_f16x2(p10, p11);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) mma_f16(o[nt], pa[2 * c], pa[2 * c + 1], vb[c][0], vb[c][1]);
+      for (int i = 0; i < 16; ++i) {
+        o[i][0] *= alpha;
+        o[i][1] *= alpha;
+      }
+      // V^T fragments by ldmatrix.trans of [16 tokens][8 channels] tiles; rows past nvalid
+      // may hold stale bytes, so their halves are zeroed (P is zero there, but 0 * NaN is not)
+      const uint32_t vbase = smem_u32(st8 + 4608);
+      const int r_ld = lane & 15, c_ld = (lane >> 4) * 8;   // row / column block of this lane
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_trans(vbase + r_ld * 256 + (16 * np + c_ld) * 2, b0, b1, b2, b3);
+        uint32_t v00 = bf16x2_to_f16x2(b0), v01 = bf16x2_to_f16x2(b1);
+        uint32_t v10 = bf16x2_to_f16x2(b2), v11 = bf16x2_to_f16x2(b3);
+        if (x.nvalid < 16) {
+          const uint32_t k0 = (2 * t < x.nvalid ? 0xFFFFu : 0u) | (2 * t + 1 < x.nvalid ? 0xFFFF0000u : 0u);
+          const uint32_t k1 = (2 * t + 8 < x.nvalid ? 0xFFFFu : 0u) | (2 * t + 9 < x.nvalid ? 0xFFFF0000u : 0u);
+          v00 &= k0; v01 &= k1; v10 &= k0; v11 &= k1;
+        }
+        mma_f16(o[2 * np], a0, a2, v00, v01);
+        mma_f16(o[2 * np + 1], a0, a2, v10, v11);
+      }
     }
   }
-  // ---- merge the 4 warps of the CTA
+  // ---- merge the warps of the CTA (the rings are free once every warp has left the scan)
+  __syncthreads();
   l += __shfl_xor_sync(0xffffffffu, l, 1);
   l += __shfl_xor_sync(0xffffffffu, l, 2);
   if (g < G) {
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {
-      s_o[warp][g][8 * nt + 2 * t] = o[nt][0];
-      s_o[warp][g][8 * nt + 2 * t + 1] = o[nt][1];
+      s_o[(warp * 8 + g) * kDecD + 8 * nt + 2 * t] = o[nt][0];
+      s_o[(warp * 8 + g) * kDecD + 8 * nt + 2 * t + 1] = o[nt][1];
     }
     if (t == 0) {
-      s_m[warp][g] = m;
-      s_l[warp][g] = l;
+      s_m[warp * 8 + g] = m;
+      s_l[warp * 8 + g] = l;
     }
   }
   __syncthreads();
@@ -295,14 +398,14 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
     const int hh = idx / kDecD, c = idx % kDecD;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, s_m[w][hh]);
+    for (int w = 0; w < kDecWarps; ++w) M = fmaxf(M, s_m[w * 8 + hh]);
     float acc = 0.0f, lsum = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kDecWarps; ++w) {
-        const float wt = ex2f(s_m[w][hh] - M);
-        acc += wt * s_o[w][hh][c];
-        lsum += wt * s_l[w][hh];
+        const float wt = ex2f(s_m[w * 8 + hh] - M);
+        acc += wt * s_o[(w * 8 + hh) * kDecD + c];
+        lsum += wt * s_l[w * 8 + hh];
       }
     }
     float* dst = p.ws + (((int64_t)b * p.Hq + hk * G + hh) * p.splits + split) * stride;
@@ -313,6 +416,10 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
     }
   }
 }
+
+constexpr size_t kDecSmem = (size_t)kDecWarps * kDecStages * kStageBytes + kDecWarps * kDecStages * 8;
+static_assert(kDecWarps * 8 * kDecD * 4 + 2 * kDecWarps * 8 * 4 <= kDecWarps * kDecStages * kStageBytes,
+              "merge buffers must fit in the rings they alias");
 
 // one warp per (sequence, q-head): log-sum-exp merge of the split partials
 __global__ void decode_combine_kernel(const float* __restrict__ ws, int n_rows, int splits,
@@ -356,11 +463,11 @@ cudaError_t decode_status_fetch(cudaStream_t st, uint32_t* host_word) {
 }
 
 static int decode_chunks(int max_pages, int max_hp, int W) {
-  return max_pages + (max_hp + 63) / 64 + (W + 63) / 64;
+  return max_pages + (max_hp + 15) / 16 + (W + 15) / 16;
 }
 
 static int decode_auto_splits(int B, int Hkv, int chunks) {
-  const int target_ctas = 148 * 3 * 4;                    // ~4 waves of 3 CTAs per SM
+  const int target_ctas = 148 * 2 * 4;                    // ~4 waves of 2 CTAs per SM
   int s = (target_ctas + B * Hkv - 1) / (B * Hkv);
   s = s < 1 ? 1 : s;
   const int max_s = (chunks + kDecWarps - 1) / kDecWarps;  // at least a chunk per warp
@@ -373,8 +480,9 @@ using namespace fa4q;
 
 extern "C" size_t fa4q_decode_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int num_splits) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || d != kDecD || max_pages < 0) return 0;
-  // the hp set and window sizes only enter through the split count; size for the worst case
-  const int splits = num_splits > 0 ? num_splits : decode_auto_splits(B, Hkv, max_pages + 64);
+  // the automatic split count is capped by the number of work units; size for the uncapped
+  // value, an upper bound for any cache shape
+  const int splits = num_splits > 0 ? num_splits : decode_auto_splits(B, Hkv, 1 << 30);
   return (size_t)B * Hq * splits * (kDecD + 2) * sizeof(float);
 }
 
@@ -436,15 +544,18 @@ extern "C" fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const 
   p.sc_bf16 = sms * kDecLog2e;
   p.g_v = g_v;
   p.n_ch_fp4 = max_pages;
-  p.n_ch_hp = (max_hp + 63) / 64;
-  p.n_ch_win = (W + 63) / 64;
+  p.n_ch_hp = (max_hp + 15) / 16;
+  p.n_ch_win = (W + 15) / 16;
   p.splits = splits;
   p.chunks_per_split = (chunks + splits - 1) / splits;
   p.ws = static_cast<float*>(workspace);
   p.out = static_cast<uint16_t*>(out);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, Hkv, B);
-  decode_split_kernel<<<grid, kDecWarps * 32, 0, st>>>(p);
+  if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kDecSmem) != cudaSuccess)
+    return FA4Q_ERR_CUDA;
+  decode_split_kernel<<<grid, kDecWarps * 32, kDecSmem, st>>>(p);
   const int rows = B * Hq;
   decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(p.ws, rows, splits, p.out);
   return launch_status();

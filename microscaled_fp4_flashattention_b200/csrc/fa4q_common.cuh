@@ -34,9 +34,15 @@ enum : uint32_t {
   kStatusTimeoutDecode = 1u << 5,
 };
 
-// Default cap on the polls of a bounded wait: far above any legitimate wait (each poll
-// is a try_wait with a hardware time hint), small enough to end in seconds.
-constexpr uint32_t kWaitPolls = 1u << 26;
+// Time limit of a bounded wait (global timer nanoseconds): far above any legitimate wait,
+// short enough that a wait nothing will satisfy ends in seconds.
+constexpr uint64_t kWaitNs = 2000000000ull;
+
+FA4Q_DEVINL uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 // ---------------------------------------------------------------------------------------
 // basic address helpers
@@ -84,7 +90,7 @@ FA4Q_DEVINL bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 0x989680;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 0xF4240;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}\n"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
@@ -92,11 +98,15 @@ FA4Q_DEVINL bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait on phase `parity`; returns false (and records `code` in *status) on expiry.
+// Bounded wait on phase `parity` (each try_wait suspends at most 1 ms); returns false, and
+// records `code` in *status, once `limit_ns` have passed without the phase completing.
 FA4Q_DEVINL bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status, uint32_t code,
-                           uint32_t polls = kWaitPolls) {
-  for (uint32_t i = 0; i < polls; ++i) {
+                           uint64_t limit_ns = kWaitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) break;
   }
   atomicOr(status, code);
   return false;
