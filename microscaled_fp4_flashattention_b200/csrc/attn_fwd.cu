@@ -44,7 +44,7 @@ constexpr int kThreads = 384;
 // 16128 of the scheduler's 16384); warpgroup 0 (TMA, MMA, 2 idle warps) drops to 56 and the
 // two softmax warpgroups rise to 224: 56*32 + 2*224*32 = 16128, the launch total exactly.
 constexpr int kRegsIssue = 56, kRegsSoftmax = 224;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGpNvfp4 = 1.0f / 2688.0f;  // g_P = 1/(6*448), rounded to FP32
 
@@ -315,48 +315,57 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int a = 0; a < C::kSfQAtoms; ++a) tmem_cp_sf_atom(tmem + kColSfQ + 4 * a, smem_u32(sm.sfq + 512 * a));
       for (int a = 0; a < C::kSfTileAtoms; ++a)
         tmem_cp_sf_atom(tmem + kColSfOne + 4 * a, smem_u32(sm.sfone + 512 * a));
+      // S_j = Q K_j^T into the single S buffer once the softmax group of tile j-1 holds
+      // S_{j-1} in registers
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % kStages, kb = j & 1;
+        if (!cta_wait(&sm.kv_full[s], (j / kStages) & 1, abort_flag, kStatusTimeoutMma)) return false;
+        if (j >= 1 && !cta_wait(&sm.s_free, (j - 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
+        tc_fence_after();
+        for (int a = 0; a < C::kSfQAtoms; ++a)
+          tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
+        const uint32_t k_addr = smem_u32(sm.k[s]);
+#pragma unroll
+        for (int ks = 0; ks < C::kKStepsQK; ++ks) {
+          const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+          const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+          mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ, tmem + kColSfK + 8 * kb, ks > 0);
+        }
+        tc_commit(&sm.s_full[j & 1]);
+        return true;
+      };
+      // [O | l]_{j%2} (+)= P^_j [V_j | 1] once the softmax group has written P^_j
+      auto issue_pv = [&](int jp) -> bool {
+        const int s = jp % kStages, pb = jp & 1;
+        if (!cta_wait(&sm.p_full[pb], (jp >> 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
+        tc_fence_after();
+        for (int a = 0; a < C::kSfTileAtoms; ++a) {
+          tmem_cp_sf_atom(tmem + kColSfP + 8 * pb + 4 * a, smem_u32(sm.sfp[pb] + 512 * a));
+          tmem_cp_sf_atom(tmem + kColSfV + 8 * pb + 4 * a, smem_u32(sm.sfv[s] + 512 * a));
+        }
+        const uint32_t p_addr = smem_u32(sm.p[pb]);
+        const uint32_t v_addr = smem_u32(sm.v[s]);
+        const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
+          const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
+          const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
+          const uint32_t acc = (jp >= 2 || ks > 0) ? 1u : 0u;
+          mma_step<MX>(tmem + o_col, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
+          mma_step<MX>(tmem + l_col, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
+        }
+        tc_commit(&sm.o_done[pb]);
+        tc_commit(&sm.kv_empty[s]);
+        return true;
+      };
+      // Issue order S_0, S_1, PV_0, S_2, PV_1, ...: S runs two products ahead of PV, so the
+      // next S is computed as soon as the S buffer is free (the other group has loaded its
+      // scores, early in its tile) instead of waiting behind the previous tile's P^.
+      ok = ok && issue_s(0);
       for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j < n_tiles) {
-          // S_j = Q K_j^T into the single S buffer once the softmax holds S_{j-1} in registers
-          const int s = j % kStages, kb = j & 1;
-          if (!cta_wait(&sm.kv_full[s], (j / kStages) & 1, abort_flag, kStatusTimeoutMma)) break;
-          if (j >= 1 && !cta_wait(&sm.s_free, (j - 1) & 1, abort_flag, kStatusTimeoutMma)) break;
-          tc_fence_after();
-          for (int a = 0; a < C::kSfQAtoms; ++a)
-            tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
-          const uint32_t k_addr = smem_u32(sm.k[s]);
-#pragma unroll
-          for (int ks = 0; ks < C::kKStepsQK; ++ks) {
-            const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-            const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-            mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ, tmem + kColSfK + 8 * kb, ks > 0);
-          }
-          tc_commit(&sm.s_full[j & 1]);
-        }
-        if (j >= 1) {
-          // [O | l]_{jp%2} (+)= P^_jp [V_jp | 1]
-          const int jp = j - 1, s = jp % kStages, pb = jp & 1;
-          if (!cta_wait(&sm.p_full[pb], (jp >> 1) & 1, abort_flag, kStatusTimeoutMma)) break;
-          tc_fence_after();
-          for (int a = 0; a < C::kSfTileAtoms; ++a) {
-            tmem_cp_sf_atom(tmem + kColSfP + 8 * pb + 4 * a, smem_u32(sm.sfp[pb] + 512 * a));
-            tmem_cp_sf_atom(tmem + kColSfV + 8 * pb + 4 * a, smem_u32(sm.sfv[s] + 512 * a));
-          }
-          const uint32_t p_addr = smem_u32(sm.p[pb]);
-          const uint32_t v_addr = smem_u32(sm.v[s]);
-          const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint32_t acc = (jp >= 2 || ks > 0) ? 1u : 0u;
-            mma_step<MX>(tmem + o_col, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
-            mma_step<MX>(tmem + l_col, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
-          }
-          tc_commit(&sm.o_done[pb]);
-          tc_commit(&sm.kv_empty[s]);
-        }
+        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
+        if (j >= 1 && !issue_pv(j - 1)) break;
       }
       // drain: all MMAs this thread issued complete before TMEM is released
       tc_commit(&sm.drain);
@@ -482,18 +491,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = ex2_approx((m_acc - m_new) * sc);
         if (__any_sync(0xffffffffu, alpha != 1.0f)) {
           const uint32_t o_col = g ? kColO1 : kColO0, l_col = g ? kColL1 : kColL0;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t raw[32];
-            tmem_ld32(lane_base + o_col + 32 * c, raw);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
-            tmem_st32(lane_base + o_col + 32 * c, raw);
-          }
+          uint32_t raw[D / 32][32];
           uint32_t lr;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + o_col + 32 * c, raw[c]);
           tmem_ld1(lane_base + l_col, lr);
           tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) raw[c][i] = __float_as_uint(__uint_as_float(raw[c][i]) * alpha);
+            tmem_st32(lane_base + o_col + 32 * c, raw[c]);
+          }
           tmem_st1(lane_base + l_col, __float_as_uint(__uint_as_float(lr) * alpha));
           tmem_wait_st();
         }
