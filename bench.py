@@ -208,6 +208,9 @@ def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
     """Time the decode over the paged hybrid cache; adds line["decode"]."""
     import torch
     dw = synth.WORKLOADS[4]
+    if args.decode_batch:
+        import dataclasses
+        dw = dataclasses.replace(dw, B=args.decode_batch)
     drun = DecodeRun(dw, dev, fa4q)
     for _ in range(max(3, args.warmup)):
         drun.step()
@@ -275,6 +278,8 @@ def main():
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode path")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="decode batch (0 = the workload's 32); smaller batches are for profiling")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--soak-s", type=float, default=2.0)
     args = ap.parse_args()

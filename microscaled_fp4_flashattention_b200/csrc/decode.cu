@@ -10,17 +10,18 @@
 // Optimization" - paged cache behind a block table, query MMAs stacked over the pages.
 //
 // Design: the scan is HBM-bound (1 byte of cache feeds ~4 multiply-adds per GQA head), so
-// the kernel streams each 64-token page once with coalesced 16-byte loads, dequantises in
-// registers (E2M1 x E4M3 products are exact in FP16) straight into mma.sync m16n8k16
-// fragments (FP32 accumulate), and never stages dequantised data in shared memory.
-//   scores  D[16 x 8] = Q[16 heads x 16 dims] * K^T[16 dims x 8 tokens]
-//   output  O[16 x 8] += P[16 heads x 16 tokens] * V[16 tokens x 8 channels]
-// The token order inside a page is permuted so that the score accumulators of a thread are
-// exactly its P fragment for the output MMA (no shuffles), and every V^T fragment is one
+// each warp streams its work units (64-token FP4 pages, 16-token BF16 slices) once through a
+// private ring of cp.async.bulk copies, dequantises in registers (E2M1 x E4M3 products are
+// exact in FP16) straight into mma.sync m16n8k16 fragments (FP32 accumulate), and never
+// stages dequantised data.  Swap-AB form, tokens / channels in M and the GQA heads in N:
+//   scores  S^T[16 tokens x 8 heads]   = K[16 tokens x 16 dims] * q^T[16 dims x 8 heads]
+//   output  O^T[16 chans x 8 heads]   += V^T[16 chans x 16 tokens] * P^T[16 tokens x 8 heads]
+// The score accumulators, packed to f16 and transposed by movmatrix, are the P^T operand.
+// The token order inside a page is permuted so that every V^T fragment of a thread is one
 // 8-byte load covering a whole 16-token scale block.
 // Grid: (split, kv-head, sequence); each warp runs its own online softmax over a strided
-// subset of the split's 64-token chunks; warps merge in shared memory, splits merge in the
-// combine kernel (log-sum-exp weighted).
+// subset of the split's units; warps merge in shared memory, splits merge in the combine
+// kernel (log-sum-exp weighted).
 #include <math.h>
 
 #include "fa4q_common.cuh"
@@ -62,6 +63,23 @@ FA4Q_DEVINL void mma_f16(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, u
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// D[16x8] += A[16x16] * B[16x8] with all four A registers (rows g, g+8; k halves)
+FA4Q_DEVINL void mma_f16x4(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                           uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// transpose of an 8x8 b16 matrix held one row pair per thread (the mma accumulator layout)
+FA4Q_DEVINL uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
 }
 
 // two E2M1 codes (one byte, low nibble first) -> f16x2 (low half = low nibble)
@@ -197,10 +215,11 @@ __global__ void __launch_bounds__(kDecWarps * 32, 2) decode_split_kernel(const D
       qa[kc][1] = bf16x2_to_f16x2(w23);
     }
   }
-  float o[16][4];
+  // swap-AB accumulators: O^T tile ct holds channels 16ct+g / 16ct+g+8 for heads 2t / 2t+1
+  float o[8][4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-  float m = -INFINITY, l = 0.0f;
+  for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;   // heads 2t, 2t+1
 
   const int n_fp4 = min(p.fp4_len[b], p.max_pages * 64);
   const int n_hp = p.hp_count ? min(p.hp_count[bh], p.max_hp) : 0;
@@ -253,144 +272,166 @@ __global__ void __launch_bounds__(kDecWarps * 32, 2) decode_split_kernel(const D
     if (x.kind == 0 && p.excl) vmask &= ~p.excl[(int64_t)bh * p.max_pages + u];
     if (vmask == 0ull) continue;
 
+    // Both unit kinds use the swap-AB form: score rows = tokens (M = 16), columns = the GQA
+    // heads (N = 8; rows of q past G are zero), so half as many MMAs as with heads in M.  The
+    // score accumulators, packed to f16 and transposed with movmatrix, are the B operand of
+    // O^T[channels x heads] += V^T[channels x tokens] * P^T.
+    float s4[4][4];     // [chunk][(T_lo,h0) (T_lo,h1) (T_hi,h0) (T_hi,h1)]
+    int nchunk;
     if (x.kind == 0) {
-      // ================= FP4 page: 64 tokens, permuted order (see the file header)
+      // FP4 page, chunk c of 16 tokens: score row r (0..7) = token 16(r>>1) + 4c + (r&1), row
+      // r+8 = that + 2; the PV reduction index k = 2t+e is token 16t + 4c + e and k = 2t+8+e
+      // is 16t + 4c + 2 + e, so one 8-byte V^T load per channel covers all four chunks.
+      nchunk = 4;
       const float sc = p.sc_fp4;
-      float s[8][2];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int c = i >> 1, sg = i & 1;
-        const int tok = 16 * (g >> 1) + 4 * c + 2 * sg + (g & 1);
-        const uint4 kw = *reinterpret_cast<const uint4*>(st8 + tok * 64 + 16 * t);
-        const uint32_t sfw = *reinterpret_cast<const uint16_t*>(st8 + 4096 + tok * 8 + 2 * t);
-        const uint32_t sf2 = e4m3x2_to_f16x2(sfw);
-        const uint32_t sfa = __byte_perm(sf2, 0, 0x1010), sfb = __byte_perm(sf2, 0, 0x3232);
-        const uint32_t words[4] = {kw.x, kw.y, kw.z, kw.w};
+      for (int c = 0; c < 4; ++c) {
+        const int tlo = 16 * (g >> 1) + 4 * c + (g & 1), thi = tlo + 2;
+        const uint4 klo = *reinterpret_cast<const uint4*>(st8 + tlo * 64 + 16 * t);
+        const uint4 khi = *reinterpret_cast<const uint4*>(st8 + thi * 64 + 16 * t);
+        const uint32_t flo = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(st8 + 4096 + tlo * 8 + 2 * t));
+        const uint32_t fhi = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(st8 + 4096 + thi * 8 + 2 * t));
+        const uint32_t sla = __byte_perm(flo, 0, 0x1010), slb = __byte_perm(flo, 0, 0x3232);
+        const uint32_t sha = __byte_perm(fhi, 0, 0x1010), shb = __byte_perm(fhi, 0, 0x3232);
+        const uint32_t wl[4] = {klo.x, klo.y, klo.z, klo.w}, wh[4] = {khi.x, khi.y, khi.z, khi.w};
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int kc = 0; kc < 8; ++kc) {
-          uint32_t f0, f1;
-          e2m1x4_to_f16x2x2(words[kc >> 1] >> ((kc & 1) * 16), f0, f1);
-          const uint32_t scl = kc < 4 ? sfa : sfb;
-          mma_f16(acc, qa[kc][0], qa[kc][1], hmul2(f0, scl), hmul2(f1, scl));
+          uint32_t la, lb, ha, hb;
+          e2m1x4_to_f16x2x2(wl[kc >> 1] >> ((kc & 1) * 16), la, lb);
+          e2m1x4_to_f16x2x2(wh[kc >> 1] >> ((kc & 1) * 16), ha, hb);
+          const uint32_t sl = kc < 4 ? sla : slb, sh = kc < 4 ? sha : shb;
+          mma_f16x4(acc, hmul2(la, sl), hmul2(ha, sh), hmul2(lb, sl), hmul2(hb, sh), qa[kc][0], qa[kc][1]);
         }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tk = 16 * t + 4 * c + 2 * sg + e;
-          s[i][e] = ((vmask >> tk) & 1ull) ? acc[e] * sc : -INFINITY;
-        }
-      }
-      float cmax = s[0][0];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) cmax = fmaxf(cmax, fmaxf(s[i][0], s[i][1]));
-      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
-      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
-      const float m_new = fmaxf(m, cmax);
-      const float alpha = ex2f(m - m_new);
-      uint32_t pa[8];
-      float psum = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float p0 = ex2f(s[i][0] - m_new), p1 = ex2f(s[i][1] - m_new);
-        psum += p0 + p1;
-        pa[i] = f32x2_to_f16x2(p0 * p.g_v, p1 * p.g_v);
-      }
-      l = l * alpha + psum;
-      m = m_new;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        o[i][0] *= alpha;
-        o[i][1] *= alpha;
-      }
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        const int chn = 8 * nt + g;
-        const uint2 vw = *reinterpret_cast<const uint2*>(st8 + 4608 + chn * 32 + 8 * t);
-        const uint32_t sfv = st8[8704 + chn * 4 + t];
-        const uint32_t s2 = e4m3x2_to_f16x2(sfv | (sfv << 8));
-        uint32_t v0, v1, v2, v3;
-        e2m1x4_to_f16x2x2(vw.x, v0, v1);
-        mma_f16(o[nt], pa[0], pa[1], hmul2(v0, s2), hmul2(v1, s2));
-        e2m1x4_to_f16x2x2(vw.x >> 16, v2, v3);
-        mma_f16(o[nt], pa[2], pa[3], hmul2(v2, s2), hmul2(v3, s2));
-        e2m1x4_to_f16x2x2(vw.y, v0, v1);
-        mma_f16(o[nt], pa[4], pa[5], hmul2(v0, s2), hmul2(v1, s2));
-        e2m1x4_to_f16x2x2(vw.y >> 16, v2, v3);
-        mma_f16(o[nt], pa[6], pa[7], hmul2(v2, s2), hmul2(v3, s2));
+        const bool vl = (vmask >> tlo) & 1ull, vh = (vmask >> thi) & 1ull;
+        s4[c][0] = vl ? acc[0] * sc : -INFINITY;
+        s4[c][1] = vl ? acc[1] * sc : -INFINITY;
+        s4[c][2] = vh ? acc[2] * sc : -INFINITY;
+        s4[c][3] = vh ? acc[3] * sc : -INFINITY;
       }
     } else {
-      // ================= BF16 slice: 16 tokens, natural order; K rows 256 B, V rows 256 B
+      // BF16 slice of 16 tokens in natural order: score rows g and g+8 are tokens g and g+8;
+      // rows past nvalid are not loaded (zeros) and the MMAs stay outside the per-lane test,
+      // because mma.sync.aligned must be executed by all lanes of the warp together
+      nchunk = 1;
       const float sc = p.sc_bf16;
-      float s[2][2];
+      const bool hl = g < x.nvalid, hh = g + 8 < x.nvalid;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int sg = 0; sg < 2; ++sg) {
-        const int tok = 8 * sg + g;
-        const uint8_t* kr = st8 + tok * 256 + 64 * t;
-        // rows past nvalid are not loaded (zeros); the MMAs stay outside the branch because
-        // mma.sync.aligned must be executed by all lanes of the warp together
-        const bool have = tok < x.nvalid;
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const uint4 zl = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 wl = hl ? *reinterpret_cast<const uint4*>(st8 + g * 256 + 64 * t + 16 * q4) : zl;
+        const uint4 wh = hh ? *reinterpret_cast<const uint4*>(st8 + (g + 8) * 256 + 64 * t + 16 * q4) : zl;
+        mma_f16x4(acc, bf16x2_to_f16x2(wl.x), bf16x2_to_f16x2(wh.x), bf16x2_to_f16x2(wl.y),
+                  bf16x2_to_f16x2(wh.y), qa[2 * q4][0], qa[2 * q4][1]);
+        mma_f16x4(acc, bf16x2_to_f16x2(wl.z), bf16x2_to_f16x2(wh.z), bf16x2_to_f16x2(wl.w),
+                  bf16x2_to_f16x2(wh.w), qa[2 * q4 + 1][0], qa[2 * q4 + 1][1]);
+      }
+      const bool vl = (vmask >> g) & 1ull, vh = (vmask >> (g + 8)) & 1ull;
+      s4[0][0] = vl ? acc[0] * sc : -INFINITY;
+      s4[0][1] = vl ? acc[1] * sc : -INFINITY;
+      s4[0][2] = vh ? acc[2] * sc : -INFINITY;
+      s4[0][3] = vh ? acc[3] * sc : -INFINITY;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const uint4 w = have ? *reinterpret_cast<const uint4*>(kr + 16 * q4) : make_uint4(0u, 0u, 0u, 0u);
-          mma_f16(acc, qa[2 * q4][0], qa[2 * q4][1], bf16x2_to_f16x2(w.x), bf16x2_to_f16x2(w.y));
-          mma_f16(acc, qa[2 * q4 + 1][0], qa[2 * q4 + 1][1], bf16x2_to_f16x2(w.z), bf16x2_to_f16x2(w.w));
-        }
+      for (int c = 1; c < 4; ++c) s4[c][0] = s4[c][1] = s4[c][2] = s4[c][3] = -INFINITY;
+    }
+    // ---- online softmax per head (the 8 lanes sharing t hold one head pair)
+    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int tk = 8 * sg + 2 * t + e;
-          s[sg][e] = ((vmask >> tk) & 1ull) ? acc[e] * sc : -INFINITY;
+    for (int c = 0; c < 4; ++c) {
+      mx0 = fmaxf(mx0, fmaxf(s4[c][0], s4[c][2]));
+      mx1 = fmaxf(mx1, fmaxf(s4[c][1], s4[c][3]));
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+    }
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float al0 = ex2f(m0 - mn0), al1 = ex2f(m1 - mn1);
+    const float gv = x.kind == 0 ? p.g_v : 1.0f;
+    uint32_t pb0[4], pb1[4];
+    float ps0 = 0.0f, ps1 = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c < nchunk) {
+        const float q0 = ex2f(s4[c][0] - mn0), q1 = ex2f(s4[c][1] - mn1);
+        const float q2 = ex2f(s4[c][2] - mn0), q3 = ex2f(s4[c][3] - mn1);
+        ps0 += q0 + q2;
+        ps1 += q1 + q3;
+        pb0[c] = movmatrix_t(f32x2_to_f16x2(q0 * gv, q1 * gv));
+        pb1[c] = movmatrix_t(f32x2_to_f16x2(q2 * gv, q3 * gv));
+      }
+    }
+    l0 = l0 * al0 + ps0;
+    l1 = l1 * al1 + ps1;
+    m0 = mn0;
+    m1 = mn1;
+#pragma unroll
+    for (int ct = 0; ct < 8; ++ct) {
+      o[ct][0] *= al0;
+      o[ct][1] *= al1;
+      o[ct][2] *= al0;
+      o[ct][3] *= al1;
+    }
+    // ---- O^T += V^T P^T, channel tiles of 16
+    if (x.kind == 0) {
+#pragma unroll
+      for (int ct = 0; ct < 8; ++ct) {
+        const int cha = 16 * ct + g, chb = cha + 8;
+        const uint2 va = *reinterpret_cast<const uint2*>(st8 + 4608 + cha * 32 + 8 * t);
+        const uint2 vb = *reinterpret_cast<const uint2*>(st8 + 4608 + chb * 32 + 8 * t);
+        const uint32_t fa = st8[8704 + cha * 4 + t], fb = st8[8704 + chb * 4 + t];
+        const uint32_t sa = e4m3x2_to_f16x2(fa | (fa << 8)), sb = e4m3x2_to_f16x2(fb | (fb << 8));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t la, ha, lb, hb;
+          e2m1x4_to_f16x2x2((c >> 1 ? va.y : va.x) >> ((c & 1) * 16), la, ha);
+          e2m1x4_to_f16x2x2((c >> 1 ? vb.y : vb.x) >> ((c & 1) * 16), lb, hb);
+          mma_f16x4(o[ct], hmul2(la, sa), hmul2(lb, sb), hmul2(ha, sa), hmul2(hb, sb), pb0[c], pb1[c]);
         }
       }
-      float cmax = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
-      cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
-      const float m_new = fmaxf(m, cmax);
-      const float alpha = ex2f(m - m_new);
-      const float p00 = ex2f(s[0][0] - m_new), p01 = ex2f(s[0][1] - m_new);
-      const float p10 = ex2f(s[1][0] - m_new), p11 = ex2f(s[1][1] - m_new);
-      l = l * alpha + (p00 + p01) + (p10 + p11);
-      m = m_new;
-      const uint32_t a0 = f32x2_to_f16x2(p00, p01), a2 = f32x2_to_f16x2(p10, p11);
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        o[i][0] *= alpha;
-        o[i][1] *= alpha;
-      }
-      // V^T fragments by ldmatrix.trans of [16 tokens][8 channels] tiles; rows past nvalid
-      // may hold stale bytes, so their halves are zeroed (P is zero there, but 0 * NaN is not)
+    } else {
+      // V rows [token][channel] -> A fragments by ldmatrix.trans; halves of rows past nvalid
+      // are zeroed (P is zero there, but 0 * NaN is not)
       const uint32_t vbase = smem_u32(st8 + 4608);
-      const int r_ld = lane & 15, c_ld = (lane >> 4) * 8;   // row / column block of this lane
+      const int tok_ld = (lane & 7) + ((lane >> 4) & 1) * 8, ch_ld = ((lane >> 3) & 1) * 8;
+      const uint32_t k0 = x.nvalid >= 16 ? 0xFFFFFFFFu
+                          : ((2 * t < x.nvalid ? 0xFFFFu : 0u) | (2 * t + 1 < x.nvalid ? 0xFFFF0000u : 0u));
+      const uint32_t k1 = x.nvalid >= 16 ? 0xFFFFFFFFu
+                          : ((2 * t + 8 < x.nvalid ? 0xFFFFu : 0u) | (2 * t + 9 < x.nvalid ? 0xFFFF0000u : 0u));
 #pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_trans(vbase + r_ld * 256 + (16 * np + c_ld) * 2, b0, b1, b2, b3);
-        uint32_t v00 = bf16x2_to_f16x2(b0), v01 = bf16x2_to_f16x2(b1);
-        uint32_t v10 = bf16x2_to_f16x2(b2), v11 = bf16x2_to_f16x2(b3);
-        if (x.nvalid < 16) {
-          const uint32_t k0 = (2 * t < x.nvalid ? 0xFFFFu : 0u) | (2 * t + 1 < x.nvalid ? 0xFFFF0000u : 0u);
-          const uint32_t k1 = (2 * t + 8 < x.nvalid ? 0xFFFFu : 0u) | (2 * t + 9 < x.nvalid ? 0xFFFF0000u : 0u);
-          v00 &= k0; v01 &= k1; v10 &= k0; v11 &= k1;
-        }
-        mma_f16(o[2 * np], a0, a2, v00, v01);
-        mma_f16(o[2 * np + 1], a0, a2, v10, v11);
+      for (int ct = 0; ct < 8; ++ct) {
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_trans(vbase + tok_ld * 256 + (16 * ct + ch_ld) * 2, r0, r1, r2, r3);
+        mma_f16x4(o[ct], bf16x2_to_f16x2(r0) & k0, bf16x2_to_f16x2(r1) & k0, bf16x2_to_f16x2(r2) & k1,
+                  bf16x2_to_f16x2(r3) & k1, pb0[0], pb1[0]);
       }
     }
   }
   // ---- merge the warps of the CTA (the rings are free once every warp has left the scan)
   __syncthreads();
-  l += __shfl_xor_sync(0xffffffffu, l, 1);
-  l += __shfl_xor_sync(0xffffffffu, l, 2);
-  if (g < G) {
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      s_o[(warp * 8 + g) * kDecD + 8 * nt + 2 * t] = o[nt][0];
-      s_o[(warp * 8 + g) * kDecD + 8 * nt + 2 * t + 1] = o[nt][1];
+  for (int off = 4; off < 32; off <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
+  }
+  const int h0 = 2 * t, h1 = 2 * t + 1;
+#pragma unroll
+  for (int ct = 0; ct < 8; ++ct) {
+    const int cha = 16 * ct + g, chb = cha + 8;
+    if (h0 < G) {
+      s_o[(warp * 8 + h0) * kDecD + cha] = o[ct][0];
+      s_o[(warp * 8 + h0) * kDecD + chb] = o[ct][2];
     }
-    if (t == 0) {
-      s_m[warp * 8 + g] = m;
-      s_l[warp * 8 + g] = l;
+    if (h1 < G) {
+      s_o[(warp * 8 + h1) * kDecD + cha] = o[ct][1];
+      s_o[(warp * 8 + h1) * kDecD + chb] = o[ct][3];
     }
+  }
+  if (g == 0) {
+    if (h0 < G) { s_m[warp * 8 + h0] = m0; s_l[warp * 8 + h0] = l0; }
+    if (h1 < G) { s_m[warp * 8 + h1] = m1; s_l[warp * 8 + h1] = l1; }
   }
   __syncthreads();
   const int stride = kDecD + 2;
