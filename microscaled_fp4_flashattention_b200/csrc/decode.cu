@@ -130,7 +130,7 @@ FA4Q_DEVINL float ex2f(float x) {
 // Work units of one (sequence, kv-head): FP4 pages (64 tokens) first, then 16-token slices
 // of the BF16 vertical-line set, then 16-token slices of the BF16 window.
 constexpr int kStageBytes = 9216;          // K page 4096 + K scales 512 + V^T page 4096 + scales 512
-constexpr int kDecStages = 3;              // per-warp shared-memory ring depth
+constexpr int kDecStages = 2;              // per-warp ring depth (2 x 9 KB: 3 CTAs per SM fit)
 
 struct UnitInfo {
   int kind;        // 0 FP4 page, 1 vertical-line slice, 2 window slice
@@ -179,7 +179,7 @@ FA4Q_DEVINL void issue_unit(const DecParams& p, const UnitInfo& x, int b, int hk
   }
 }
 
-__global__ void __launch_bounds__(kDecWarps * 32, 2) decode_split_kernel(const DecParams p) {
+__global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const DecParams p) {
   extern __shared__ __align__(128) uint8_t dsm[];
   // [rings of all warps][mbarriers]; after the scan the rings are reused for the warp merge
   uint64_t* bars = reinterpret_cast<uint64_t*>(dsm + kDecWarps * kDecStages * kStageBytes);
@@ -508,7 +508,7 @@ static int decode_chunks(int max_pages, int max_hp, int W) {
 }
 
 static int decode_auto_splits(int B, int Hkv, int chunks) {
-  const int target_ctas = 148 * 2 * 4;                    // ~4 waves of 2 CTAs per SM
+  const int target_ctas = 148 * 8;                        // 1184: ~2.9 waves of 3 CTAs per SM at B*Hkv = 256
   int s = (target_ctas + B * Hkv - 1) / (B * Hkv);
   s = s < 1 ? 1 : s;
   const int max_s = (chunks + kDecWarps - 1) / kDecWarps;  // at least a chunk per warp
