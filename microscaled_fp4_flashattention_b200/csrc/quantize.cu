@@ -81,56 +81,55 @@ FA4Q_DEVINL int64_t sf_tiled_offset(int64_t r, int64_t k, int64_t nG) {
 // ---------------------------------------------------------------------------------------
 template <int BLK>
 __global__ void __launch_bounds__(256) quant_inner_kernel(
-    const uint16_t* __restrict__ x, int64_t groups, int64_t rows, int64_t cols,
-    int64_t row_stride, float qmax, float g, const float* __restrict__ mul, int64_t mheads,
-    int64_t mratio, int tiled, uint8_t* __restrict__ packed, uint8_t* __restrict__ sf) {
-  const int64_t nblk = cols / BLK;
-  const int64_t rows_sp = tiled ? ((rows + 127) / 128) * 128 : rows;   // rows in SF space
-  const int64_t nG = tiled ? ((cols + 127) / 128) * (32 / BLK) : 0;
-  const int64_t ncol_sp = tiled ? nG * 4 : nblk;                        // scale columns in SF space
-  const int64_t per_group = rows_sp * ncol_sp;
-  const int64_t total = groups * per_group;
-  const int64_t sf_group_bytes = tiled ? ((rows + 127) / 128) * nG * 512 : rows * nblk;
-  const float denom = __fmul_rn(qmax, g);
-  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
-       idx += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t gi = idx / per_group;
-    const int64_t rem = idx - gi * per_group;
-    const int64_t r = rem / ncol_sp;
-    const int64_t kb = rem - r * ncol_sp;
-    uint32_t s = 0;
-    if (r < rows && kb < nblk) {
-      const uint16_t* src = x + (gi * rows + r) * row_stride + kb * BLK;
-      float v[BLK];
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t row_stride, float qmax,
+    float g, const float* __restrict__ mul, int64_t mheads, int64_t mratio, int tiled,
+    uint8_t* __restrict__ packed, uint8_t* __restrict__ sf) {
+  // grid: x over the (row, block) slots of one group's scale space, y = group; 32-bit
+  // in-group indices (no 64-bit divisions per 32-element block)
+  const int nblk = static_cast<int>(cols / BLK);
+  const int rows_i = static_cast<int>(rows);
+  const int rows_sp = tiled ? ((rows_i + 127) / 128) * 128 : rows_i;
+  const int nG = tiled ? static_cast<int>((cols + 127) / 128) * (32 / BLK) : 0;
+  const int ncol_sp = tiled ? nG * 4 : nblk;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows_sp * ncol_sp) return;
+  const int64_t gi = blockIdx.y;
+  const int r = idx / ncol_sp;
+  const int kb = idx - r * ncol_sp;
+  const int64_t sf_group_bytes = tiled ? (int64_t)((rows_i + 127) / 128) * nG * 512 : (int64_t)rows_i * nblk;
+  uint32_t s = 0;
+  if (r < rows_i && kb < nblk) {
+    const uint16_t* src = x + (gi * rows + r) * row_stride + kb * BLK;
+    float v[BLK];
 #pragma unroll
-      for (int c = 0; c < BLK; c += 8) load_bf16x8(src + c, v + c);
-      if (mul != nullptr) {
-        const float* m = mul + ((gi % mheads) / mratio) * cols + kb * BLK;
+    for (int c = 0; c < BLK; c += 8) load_bf16x8(src + c, v + c);
+    if (mul != nullptr) {
+      const int mrow = (static_cast<int>(gi) % static_cast<int>(mheads)) / static_cast<int>(mratio);
+      const float* m = mul + (int64_t)mrow * cols + kb * BLK;
 #pragma unroll
-        for (int c = 0; c < BLK; c += 4) {
-          const float4 mm = *reinterpret_cast<const float4*>(m + c);
-          v[c] = __fmul_rn(v[c], mm.x);
-          v[c + 1] = __fmul_rn(v[c + 1], mm.y);
-          v[c + 2] = __fmul_rn(v[c + 2], mm.z);
-          v[c + 3] = __fmul_rn(v[c + 3], mm.w);
-        }
-      }
-      uint8_t* dst = packed + (gi * rows + r) * (cols / 2) + kb * (BLK / 2);
-      if constexpr (BLK == 16) {
-        uint2 p;
-        s = quant_block16_nvfp4(v, denom, g, p);
-        *reinterpret_cast<uint2*>(dst) = p;
-      } else {
-        uint4 p;
-        s = quant_block32_mxfp4(v, qmax, p);
-        *reinterpret_cast<uint4*>(dst) = p;
+      for (int c = 0; c < BLK; c += 4) {
+        const float4 mm = *reinterpret_cast<const float4*>(m + c);
+        v[c] = __fmul_rn(v[c], mm.x);
+        v[c + 1] = __fmul_rn(v[c + 1], mm.y);
+        v[c + 2] = __fmul_rn(v[c + 2], mm.z);
+        v[c + 3] = __fmul_rn(v[c + 3], mm.w);
       }
     }
-    if (tiled)
-      sf[gi * sf_group_bytes + sf_tiled_offset(r, kb, nG)] = (uint8_t)s;
-    else
-      sf[gi * sf_group_bytes + r * nblk + kb] = (uint8_t)s;
+    uint8_t* dst = packed + (gi * rows + r) * (cols / 2) + kb * (BLK / 2);
+    if constexpr (BLK == 16) {
+      uint2 p;
+      s = quant_block16_nvfp4(v, __fmul_rn(qmax, g), g, p);
+      *reinterpret_cast<uint2*>(dst) = p;
+    } else {
+      uint4 p;
+      s = quant_block32_mxfp4(v, qmax, p);
+      *reinterpret_cast<uint4*>(dst) = p;
+    }
   }
+  if (tiled)
+    sf[gi * sf_group_bytes + sf_tiled_offset(r, kb, nG)] = (uint8_t)s;
+  else
+    sf[gi * sf_group_bytes + (int64_t)r * nblk + kb] = (uint8_t)s;
 }
 
 // ---------------------------------------------------------------------------------------
@@ -360,18 +359,16 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
     const int64_t nblk = cols / blk;
     const int64_t rows_sp = tiled ? (rows + 127) / 128 * 128 : rows;
     const int64_t ncol_sp = tiled ? (cols + 127) / 128 * (32 / blk) * 4 : nblk;
-    const int64_t total = groups * rows_sp * ncol_sp;
-    const int64_t nblocks = std::min<int64_t>((total + 255) / 256, 148LL * 32);
+    const int64_t per_group = rows_sp * ncol_sp;
+    if (groups > 65535 || per_group > (int64_t)1 << 30 || rows > ((int64_t)1 << 30)) return FA4Q_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)((per_group + 255) / 256), (unsigned)groups);
+    const int64_t mh = smooth_heads > 0 ? smooth_heads : 1, mr = smooth_ratio > 0 ? smooth_ratio : 1;
     if (blk == 16)
-      quant_inner_kernel<16><<<(unsigned)nblocks, 256, 0, st>>>(
-          (const uint16_t*)x, groups, rows, cols, row_stride, qm, g, smooth_mul,
-          smooth_heads > 0 ? smooth_heads : 1, smooth_ratio > 0 ? smooth_ratio : 1, tiled,
-          packed_out, scales_out);
+      quant_inner_kernel<16><<<grid, 256, 0, st>>>((const uint16_t*)x, rows, cols, row_stride, qm, g,
+                                                   smooth_mul, mh, mr, tiled, packed_out, scales_out);
     else
-      quant_inner_kernel<32><<<(unsigned)nblocks, 256, 0, st>>>(
-          (const uint16_t*)x, groups, rows, cols, row_stride, qm, g, smooth_mul,
-          smooth_heads > 0 ? smooth_heads : 1, smooth_ratio > 0 ? smooth_ratio : 1, tiled,
-          packed_out, scales_out);
+      quant_inner_kernel<32><<<grid, 256, 0, st>>>((const uint16_t*)x, rows, cols, row_stride, qm, g,
+                                                   smooth_mul, mh, mr, tiled, packed_out, scales_out);
   } else {
     if (smooth_mul) return FA4Q_ERR_UNSUPPORTED;
     if (groups > 65535) return FA4Q_ERR_UNSUPPORTED;
