@@ -243,6 +243,18 @@ fa4q_status fa4q_selftest_block_mma(const uint8_t* a, const uint8_t* a_sf, const
                                     float* d_out, void* stream);
 
 /*
+ * fa4q_selftest_exp2 - diagnostic: y[i] = 2^x[i] through the FMA-pipe polynomial that the
+ * prefill kernel uses for part of the unnormalised exponentials P~ = exp(S - m).  Source:
+ * FLAMIA (FLAsh MIcroscaling Attention ... on Blackwell), Abstract - its FlashAttention-4
+ * account lists a software-emulated exponential among the ways to relieve the exponential
+ * units on B200; written here as range reduction plus a cubic minimax fit of 2^f on [0, 1)
+ * (coefficients from fit_exp2_poly.py).  Relative error <= 1.6e-4 for x in [-126, 128);
+ * inputs below -126 (and -inf) give a non-negative value below 2^-126.  x, y: device FP32 arrays of n
+ * elements (caller-owned; n even).  Returns FA4Q_ERR_INVALID_ARG for null pointers or odd n.
+ */
+fa4q_status fa4q_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
+
+/*
  * fa4q_device_status - synchronise `stream`, then read and clear the device status word.
  * Returns FA4Q_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call
  * (*detail, if non-null, receives the kernel-specific code), FA4Q_OK otherwise.

@@ -26,7 +26,7 @@ EXPORTED = [
     "fa4q_status_string", "fa4q_version", "fa4q_sf_tiled_bytes", "fa4q_quantize",
     "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_quantize_kv_pages",
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
-    "fa4q_device_status", "fa4q_selftest_wait_timeout",
+    "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
 ]
 
 _LIB = None
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.fa4q_device_status.argtypes = [P, ctypes.POINTER(U32)]
         L.fa4q_selftest_wait_timeout.restype = I
         L.fa4q_selftest_wait_timeout.argtypes = [U32, P]
+        L.fa4q_selftest_exp2.restype = I
+        L.fa4q_selftest_exp2.argtypes = [P, P, I64, P]
         _LIB = L
     return _LIB
 
@@ -255,6 +257,15 @@ def device_status(stream=None):
 
 def selftest_wait_timeout(wait_us: int, stream=None):
     _check("fa4q_selftest_wait_timeout", lib().fa4q_selftest_wait_timeout(wait_us, _stream(stream)))
+
+
+def selftest_exp2(x, stream=None):
+    """2^x through the prefill kernel's FMA-pipe exponential (x: CUDA float32, even length)."""
+    import torch
+    x = x.contiguous()
+    y = torch.empty_like(x)
+    _check("fa4q_selftest_exp2", lib().fa4q_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+    return y
 
 
 def default_sm_scale(d: int) -> float:

@@ -23,8 +23,9 @@
 //   warps 2-3   idle (they complete warpgroup 0 for the register split)
 //   warps 4-11  softmax: two groups of four warps take alternate key tiles, one query row
 //               per thread; tcgen05.ld of S, mask, running max (passed between the groups),
-//               exp2, block scales, cvt to E2M1, P^ to shared memory (the A operand of the
-//               PV MMA), rescale of the group's O and l in TMEM, epilogue.
+//               exp2 (two of every eight on the FMA pipe by a polynomial, the rest on MUFU),
+//               block scales, cvt to E2M1, P^ to shared memory (the A operand of the PV MMA),
+//               rescale of the group's O and l in TMEM, epilogue.
 // TMEM (512 columns): S [0,128), O even/odd tiles [128,256) and [256,384), l even/odd
 // [384,400) and [400,416), scale factors [416,480).  Every mbarrier wait is bounded; on expiry the CTA records a status bit,
 // skips the remaining waits, drains its own copies and MMAs and exits.
@@ -47,6 +48,11 @@ constexpr int kRegsIssue = 56, kRegsSoftmax = 224;
 constexpr int kStages = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGpNvfp4 = 1.0f / 2688.0f;  // g_P = 1/(6*448), rounded to FP32
+// polynomial 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [0, 1) (see ex2_poly2)
+constexpr float kExp2C0 = 0.9999252557754517f, kExp2C1 = 0.6958334445953369f;
+constexpr float kExp2C2 = 0.22606724500656128f, kExp2C3 = 0.07802451401948929f;
+constexpr int kEmulPer8 = 2;  // exponentials of every 8 computed by ex2_poly2 (the rest on MUFU)
+
 
 // TMEM column map: one S buffer, two O and l accumulators (even / odd key tiles), scales
 constexpr uint32_t kColS = 0, kColO0 = 128, kColO1 = 256, kColL0 = 384, kColL1 = 400;
@@ -125,6 +131,25 @@ FA4Q_DEVINL bool cta_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abo
   return false;
 }
 
+FA4Q_DEVINL bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Warp-uniform bounded wait for the softmax warps: a non-blocking test first (the phase has
+// usually completed long before), the suspending bounded wait only when it has not.
+FA4Q_DEVINL bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag, uint32_t code) {
+  if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+  return __all_sync(0xffffffffu, cta_wait(bar, parity, abort_flag, code));
+}
+
 FA4Q_DEVINL float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -150,6 +175,35 @@ FA4Q_DEVINL void ffma2(float& d0, float& d1, float a0, float a1, float b0, float
       "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}\n"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// 2^x for two values on the FMA pipe (Cody-Waite style range reduction and a polynomial),
+// used for part of the exponentials so that the MUFU and FMA pipes share the work (FLAMIA,
+// Abstract: FlashAttention-4's software-emulated exponential on Blackwell):
+//   x := max(x, -126)                        (2^-126 and below quantise to 0 anyway; p(0)
+//                                            is just below 1, so -126 is the lowest floor
+//                                            whose exponent sum stays non-negative)
+//   t  = x + 1.5*2^23 rounded toward -inf    -> the low mantissa bits of t hold floor(x)
+//   f  = x - (t - 1.5*2^23)                  in [0, 1), exact
+//   p  = c0 + f (c1 + f (c2 + f c3))         2^f, minimax (relative) fit on [0, 1),
+//                                            max relative error 7.5e-5
+//   2^x = p * 2^floor(x): floor(x) added to the exponent field of p (bits of t << 23)
+// The coefficients come from an iteratively reweighted least-squares fit of 2^f on [0, 1)
+// (fit_exp2_poly.py beside this file).  The result feeds E2M1 rounding (3 significant bits).
+FA4Q_DEVINL void ex2_poly2(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  uint32_t t0, t1, p0, p1;
+  asm("{\n\t.reg .b64 rx, rt, rj, rf, rp, rm, c0, c1, c2, c3;\n\t"
+      "mov.b64 rx, {%4, %5};\n\tmov.b64 rm, {%6, %6};\n\t"
+      "add.rm.f32x2 rt, rx, rm;\n\tsub.rn.f32x2 rj, rt, rm;\n\tsub.rn.f32x2 rf, rx, rj;\n\t"
+      "mov.b64 c3, {%10, %10};\n\tmov.b64 c2, {%9, %9};\n\tmov.b64 c1, {%8, %8};\n\tmov.b64 c0, {%7, %7};\n\t"
+      "fma.rn.f32x2 rp, c3, rf, c2;\n\tfma.rn.f32x2 rp, rp, rf, c1;\n\tfma.rn.f32x2 rp, rp, rf, c0;\n\t"
+      "mov.b64 {%0, %1}, rt;\n\tmov.b64 {%2, %3}, rp;\n\t}"
+      : "=r"(t0), "=r"(t1), "=r"(p0), "=r"(p1)
+      : "f"(x0), "f"(x1), "f"(12582912.0f), "f"(kExp2C0), "f"(kExp2C1), "f"(kExp2C2), "f"(kExp2C3));
+  y0 = __uint_as_float(p0 + (t0 << 23));
+  y1 = __uint_as_float(p1 + (t1 << 23));
 }
 
 // maximum of N consecutive values, as a tree of 3-input maxima
@@ -398,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_acc = -INFINITY;                       // maximum of this group's last tile
     bool ok = true;
     for (int j = g; j < n_tiles; j += 2) {
-      ok = __all_sync(0xffffffffu, cta_wait(&sm.s_full[g], (j >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) && ok;
+      ok = warp_wait(&sm.s_full[g], (j >> 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       tc_fence_after();
       float s[kBN];
       {
@@ -469,13 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; i += 2) ffma2(y[i], y[i + 1], s[8 * g8 + i], s[8 * g8 + i + 1], sc, sc, -o8, -o8);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = ex2_approx(y[i]);
+        for (int i = 0; i < kEmulPer8; i += 2) ex2_poly2(y[i], y[i + 1], y[i], y[i + 1]);
+#pragma unroll
+        for (int i = kEmulPer8; i < 8; ++i) y[i] = ex2_approx(y[i]);
         packed[g8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
       }
       // accumulator g and P buffer g were last used by this group's previous PV product
       if (j >= 2)
-        ok = __all_sync(0xffffffffu, cta_wait(&sm.o_done[g], ((j - 2) >> 1) & 1, abort_flag,
-                                              kStatusTimeoutSoftmax)) && ok;
+        ok = warp_wait(&sm.o_done[g], ((j - 2) >> 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       uint8_t* pbuf = sm.p[g];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -677,6 +732,16 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// elementwise 2^x through ex2_poly2 (two values per thread)
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t npairs) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= npairs) return;
+  const float2 v = reinterpret_cast<const float2*>(x)[i];
+  float a, b;
+  ex2_poly2(a, b, v.x, v.y);
+  reinterpret_cast<float2*>(y)[i] = make_float2(a, b);
+}
+
 // bounded-wait probe: waits on a barrier nothing will complete, for `wait_us` microseconds
 __global__ void wait_probe_kernel(uint32_t wait_us) {
   __shared__ uint64_t bar;
@@ -819,6 +884,17 @@ extern "C" fa4q_status fa4q_selftest_block_mma(const uint8_t* a, const uint8_t* 
     selftest_mma_kernel<false><<<1, 128, 0, st>>>(a, a_sf, b, b_sf, N, K, d_out);
   else
     return FA4Q_ERR_INVALID_ARG;
+  return launch_status();
+}
+
+extern "C" fa4q_status fa4q_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (!x || !y || n < 0 || (n & 1)) return FA4Q_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 7) return FA4Q_ERR_INVALID_ARG;
+  if (n == 0) return FA4Q_OK;
+  const int64_t npairs = n / 2;
+  const int64_t blocks = (npairs + 255) / 256;
+  if (blocks > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
+  selftest_exp2_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, npairs);
   return launch_status();
 }
 
