@@ -39,6 +39,39 @@ FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PF
 FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 
 
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture
+# of each roofline kernel (summaries and commands in profiles/).  A figure is reported only
+# while the kernel's sources hash to the ones it was taken on; any change makes it null.
+# The decode capture ran 8 of the 32 sequences: its traffic is per sequence (it grows with the
+# number of sequences) and is scaled to the timed batch.
+NCU_TRAFFIC = {
+    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,419,264 + 22,784 B (bench workload)
+    "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
+                 "sha256": "7662871aa128626e7287f00aa3c7afcedd674d5510ec41f5508b2b8a312a8ed8",
+                 "bytes_per_launch": 13419264 + 22784},
+    # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,900,224 + 5,366,016 B for 8 sequences
+    "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
+               "sha256": "3fae0c63206939932514f70e30ad22e4b951a7a02beed961c9a384b935120fdc",
+               "bytes_per_sequence": 364266240 // 8},
+}
+
+
+def sources_sha256(names) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "microscaled_fp4_flashattention_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic(kernel: str, sequences: int = 0):
+    e = NCU_TRAFFIC[kernel]
+    if e["sha256"] is None or sources_sha256(e["sources"]) != e["sha256"]:
+        return None
+    return e["bytes_per_launch"] if kernel == "attn_fwd" else e["bytes_per_sequence"] * sequences
+
+
 # ------------------------------------------------------------------------------ helpers
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -235,7 +268,7 @@ def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
                       "GBps": gbs, "bytes_per_step": drun.bytes, "gpu_launches": 2 * dsteps,
                       "roofline": {"kernel": "decode_split_kernel+decode_combine_kernel", "bound": "hbm",
                                    "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                                   "traffic": None, "peak_source": f"{peak_kind} hbm copy"},
+                                   "traffic": ncu_traffic("decode", dw.B), "peak_source": f"{peak_kind} hbm copy"},
                       "l2": "working set 1.4 GB > L2", "clocks": dsampler.summary()}
 
 
@@ -412,7 +445,8 @@ def main():
         "e2e": {"value": world * run.flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
         "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
-                     "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                     "traffic": ncu_traffic("attn_fwd") if w.name == synth.WORKLOADS[2].name else None,
                      "peak_source": f"{peak_kind} bf16 burst {bf16_tf:.1f} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4/BF16)",
                      "ms_per_launch": a_ms},
         "clocks": sampler.summary(),
