@@ -8,9 +8,11 @@ attention probability it receives, summed over later queries); the top-rho
 fraction of the non-window prefix (5% by default) is kept in full precision.
 
 Reading: the mass is summed over a set of observation queries and over the
-q-heads of a GQA group, with an exact softmax over the non-window prefix.
-Parity unpinned in value (no worked example on the pages); the test checks
-that planted heavy-hitter positions are recovered.
+q-heads of a GQA group, with an exact softmax over the non-window prefix; the
+selection keeps ceil(rho * N) positions, equal masses lowest position first.
+Pins (no worked example on the pages): masses sum to the number of queries,
+all-zero queries give the uniform mass, a scalar math.exp loop agrees on a tiny
+case, planted heavy-hitter positions are recovered, count and tie rules.
 """
 from __future__ import annotations
 

@@ -214,6 +214,12 @@ def decode_kv_slice(w: DecodeWorkload, which: str, b: int, h: int, L: int | None
     return round_to_bf16(normal(w.wid, stream, (L, w.d), b, h))
 
 
+def decode_observation_queries(w: DecodeWorkload, b: int, n_obs: int = 64) -> np.ndarray:
+    """[Hq, n_obs, d] bf16-valued observation queries (stream 6) from which the vertical-line
+    tokens of sequence b are identified by accumulated column mass."""
+    return round_to_bf16(normal(w.wid, STREAM_OBS, (w.Hq, n_obs, w.d), b))
+
+
 def decode_hp_positions(w: DecodeWorkload, b: int, h: int, fp4_len: int | None = None, n_hp: int | None = None) -> np.ndarray:
     """Sorted positions of the full-precision vertical-line tokens, drawn without replacement
     from the non-window prefix [0, fp4_len)."""

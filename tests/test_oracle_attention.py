@@ -240,3 +240,40 @@ def test_vertical_lines_recover_planted_positions():
     sel = H.select_vertical_lines(q, k, 0.05)
     assert len(sel) == 100
     assert len(np.intersect1d(sel, planted)) >= 95
+
+
+def test_column_mass_invariants_and_brute_force():
+    """Each observation query's probabilities sum to 1, so the masses sum to Nq; all-zero
+    queries give the uniform mass Nq/N; a scalar loop with math.exp agrees on a tiny case."""
+    import math
+    rng = np.random.default_rng(37)
+    q = rng.normal(size=(48, 32))
+    k = rng.normal(size=(300, 32)) * 1.7
+    m = H.column_mass(q, k)
+    assert np.all(m >= 0.0)
+    assert abs(m.sum() - 48.0) < 1e-10
+    mz = H.column_mass(np.zeros((7, 32)), k)
+    assert np.max(np.abs(mz - 7.0 / 300.0)) < 1e-15
+    qs, ks = rng.normal(size=(3, 4)), rng.normal(size=(5, 4))
+    ref = [0.0] * 5
+    for i in range(3):
+        sc = [sum(qs[i][c] * ks[j][c] for c in range(4)) / 2.0 for j in range(5)]
+        mx = max(sc)
+        e = [math.exp(x - mx) for x in sc]
+        tot = sum(e)
+        for j in range(5):
+            ref[j] += e[j] / tot
+    assert np.max(np.abs(H.column_mass(qs, ks) - np.array(ref))) < 1e-13
+
+
+def test_vertical_line_count_and_ties():
+    """n = ceil(rho * N) (0.05 * 32640 -> 1632 exactly, 0.05 * 101 -> 6); equal masses are
+    taken lowest position first; the result is sorted."""
+    k = np.random.default_rng(38).normal(size=(32640, 8))
+    sel = H.select_vertical_lines(np.zeros((4, 8)), k, 0.05)
+    assert len(sel) == 1632 and np.array_equal(sel, np.arange(1632))
+    k2 = np.random.default_rng(39).normal(size=(101, 8))
+    sel2 = H.select_vertical_lines(np.random.default_rng(40).normal(size=(5, 8)), k2, 0.05)
+    assert len(sel2) == 6 and np.all(np.diff(sel2) > 0)
+    mass = H.column_mass(np.random.default_rng(40).normal(size=(5, 8)), k2)
+    assert mass[sel2].min() >= np.sort(mass)[-6]
