@@ -233,6 +233,49 @@ fa4q_status fa4q_decode_noalloc(const void* q, const uint8_t* k_pages, const uin
                                 void* stream);
 
 /*
+ * fa4q_select_vertical_lines - identify the full-precision ("vertical line") tokens of the
+ * hybrid cache by accumulated column mass, and write everything the cache and the decode
+ * need about them.
+ * Source: HyQuant (Hybrid-Precision Quantization for LLM Attention): tokens that receive a
+ * large accumulated attention mass from later queries stay in full precision (the top 5%
+ * of the non-window prefix by default), the rest is stored in 4 bits; the mass comes from a
+ * set of observation queries.
+ *
+ * Per (sequence b, kv-head h), over the candidate prefix [0, n_prefix[b]) (clamped to L):
+ *   s_ij = (q_i . k_j) * sm_scale for the R = (Hq/Hkv) * n_obs observation rows q_i of the
+ *          group's q-heads (row g * n_obs + t = observation t of q-head h*Hq/Hkv + g)
+ *   mass_j = sum_i softmax_j(s_ij)            exact softmax over the whole prefix
+ *   kept   = the ceil(rho * n_prefix[b]) largest masses, equal masses lowest position first
+ *
+ * q_obs      bf16 [B][Hq][n_obs][d]; R must be a multiple of 32 and at most 256.
+ * k, v       bf16 [B][Hkv][L][d] (v may be null when hp_v is null).
+ * n_prefix   device int32 [B].
+ * rho        (0, 1], double (the count ceil(rho * n) is taken in double precision, less
+ *            1e-9, so 0.05 * 32640 gives 1632); sm_scale 0 -> 1/sqrt(d).  d in {64, 128}.
+ * mass       out, FP32 [B][Hkv][L] (0 outside the prefix).
+ * positions  out, int32 [B][Hkv][max_select], the kept positions ascending (entries past
+ *            counts[b][h] are not written); counts out, int32 [B][Hkv].
+ *            max_select >= ceil(rho * L).
+ * excl_mask  nullable out, uint64 [B][Hkv][max_pages] in the paged-cache layout (bit t of
+ *            word j = position 64 j + t is kept); max_pages * 64 >= L.  Pass it to
+ *            fa4q_quantize_kv_pages and fa4q_decode.
+ * hp_k, hp_v nullable out, bf16 [B][Hkv][max_select][d]: the kept rows of k and v in
+ *            position order (the decode's full-precision set; rows past counts not written).
+ * workspace  device, >= fa4q_vlines_workspace_size(B, Hq, Hkv, n_obs, L) bytes, 8-aligned.
+ * The candidates of one (sequence, kv-head) are selected in shared memory: L up to ~55,000
+ * keys (4 L + 4 max_select + 8 max_pages bytes <= 227 KB), else FA4Q_ERR_UNSUPPORTED.
+ * Errors: null required pointers, bad sizes, short workspace or misaligned (16-byte) bf16
+ * pointers -> FA4Q_ERR_INVALID_ARG.  Asynchronous on `stream`.
+ */
+size_t fa4q_vlines_workspace_size(int B, int Hq, int Hkv, int n_obs, int L);
+fa4q_status fa4q_select_vertical_lines(const void* q_obs, const void* k, const void* v,
+                                       const int32_t* n_prefix, int B, int Hq, int Hkv, int n_obs,
+                                       int L, int d, double rho, float sm_scale, float* mass,
+                                       int32_t* positions, int32_t* counts, int max_select,
+                                       uint64_t* excl_mask, int max_pages, void* hp_k, void* hp_v,
+                                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa4q_selftest_block_mma - diagnostic: one 128 x N x K block-scaled FP4 tensor-core
  * product D = A * B^T (FP32), the same MMA path the prefill kernel uses.
  * a packed [128][K/2], b packed [N][K/2] (K-major), a_sf / b_sf FA4Q_SF_TILED over

@@ -27,6 +27,7 @@ EXPORTED = [
     "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_quantize_kv_pages",
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
+    "fa4q_vlines_workspace_size", "fa4q_select_vertical_lines",
 ]
 
 _LIB = None
@@ -76,6 +77,11 @@ def lib() -> ctypes.CDLL:
         L.fa4q_selftest_wait_timeout.argtypes = [U32, P]
         L.fa4q_selftest_exp2.restype = I
         L.fa4q_selftest_exp2.argtypes = [P, P, I64, P]
+        L.fa4q_vlines_workspace_size.restype = Z
+        L.fa4q_vlines_workspace_size.argtypes = [I, I, I, I, I]
+        L.fa4q_select_vertical_lines.restype = I
+        L.fa4q_select_vertical_lines.argtypes = [P, P, P, P, I, I, I, I, I, I, ctypes.c_double, F, P, P, P, I, P, I, P, P,
+                                                 P, Z, P]
         _LIB = L
     return _LIB
 
@@ -190,6 +196,43 @@ def quantize_kv_pages(k, v, fp4_len, excl_mask, block_table, n_phys_pages: int, 
         _ptr(k), _ptr(v), B, Hkv, L, d, _ptr(fp4_len), _ptr(excl_mask), _ptr(block_table), max_pages,
         f, g_k, g_v, _ptr(kp), _ptr(ks), _ptr(vp), _ptr(vs), _stream(stream)))
     return kp, ks, vp, vs
+
+
+def vlines_workspace_size(B, Hq, Hkv, n_obs, L) -> int:
+    return int(lib().fa4q_vlines_workspace_size(B, Hq, Hkv, n_obs, L))
+
+
+def select_vertical_lines(q_obs, k, v, n_prefix, *, rho=0.05, sm_scale=0.0, max_select=None,
+                          max_pages=None, with_rows=True, workspace=None, stream=None):
+    """Vertical-line tokens by accumulated column mass.
+
+    q_obs bf16 [B, Hq, n_obs, d]; k, v bf16 [B, Hkv, L, d]; n_prefix int32 [B] (device).
+    Returns a dict: mass [B, Hkv, L] fp32, positions [B, Hkv, max_select] int32 (ascending,
+    valid up to counts), counts [B, Hkv] int32, excl (uint64 words as int64 [B, Hkv, max_pages]),
+    hp_k / hp_v [B, Hkv, max_select, d] bf16 (when with_rows)."""
+    import math
+    import torch
+    B, Hq, n_obs, d = q_obs.shape
+    _, Hkv, L, _ = k.shape
+    dev = k.device
+    if max_select is None:
+        max_select = max(1, int(math.ceil(rho * L - 1e-9)))
+    if max_pages is None:
+        max_pages = -(-L // 64)
+    mass = torch.empty((B, Hkv, L), dtype=torch.float32, device=dev)
+    positions = torch.empty((B, Hkv, max_select), dtype=torch.int32, device=dev)
+    counts = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+    excl = torch.empty((B, Hkv, max_pages), dtype=torch.int64, device=dev)
+    hp_k = torch.zeros((B, Hkv, max_select, d), dtype=torch.bfloat16, device=dev) if with_rows else None
+    hp_v = torch.zeros((B, Hkv, max_select, d), dtype=torch.bfloat16, device=dev) if with_rows else None
+    ws_bytes = vlines_workspace_size(B, Hq, Hkv, n_obs, L)
+    if workspace is None:
+        workspace = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
+    _check("fa4q_select_vertical_lines", lib().fa4q_select_vertical_lines(
+        _ptr(q_obs), _ptr(k), _ptr(v) if with_rows else None, _ptr(n_prefix), B, Hq, Hkv, n_obs, L, d,
+        rho, sm_scale, _ptr(mass), _ptr(positions), _ptr(counts), max_select, _ptr(excl), max_pages,
+        _ptr(hp_k), _ptr(hp_v), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return {"mass": mass, "positions": positions, "counts": counts, "excl": excl, "hp_k": hp_k, "hp_v": hp_v}
 
 
 def decode_workspace_size(B, Hq, Hkv, d, max_pages, num_splits=0) -> int:
