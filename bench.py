@@ -202,25 +202,22 @@ class DecodeRun:
                 tK[b, h] = torch.from_numpy(synth.decode_kv_slice(dw, "k", b, h)).to(dev).to(torch.bfloat16)
                 tV[b, h] = torch.from_numpy(synth.decode_kv_slice(dw, "v", b, h)).to(dev).to(torch.bfloat16)
         Q = np.stack([synth.decode_query(dw, b) for b in range(B)])
-        hp = np.stack([np.stack([synth.decode_hp_positions(dw, b, h) for h in range(Hkv)]) for b in range(B)])
-        excl = np.zeros((B, Hkv, P), dtype=np.uint64)
-        bb, hh, jj = np.meshgrid(np.arange(B), np.arange(Hkv), np.arange(n_hp), indexing="ij")
-        np.bitwise_or.at(excl, (bb.ravel(), hh.ravel(), hp.ravel() // 64),
-                         np.left_shift(np.uint64(1), (hp.ravel() % 64).astype(np.uint64)))
         i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a).astype(np.int32)).to(dev)
         self.table = i32(synth.decode_block_table(dw))
         self.fp4_len = i32(np.full(B, n_fp4))
-        self.excl = torch.from_numpy(excl.view(np.int64)).to(dev)
+        # vertical-line tokens: top 5% of the non-window prefix by column mass from 64
+        # observation queries per q-head (GPU identification), then the FP4 pages without them
+        self.q_obs = torch.from_numpy(np.stack([synth.decode_observation_queries(dw, b) for b in range(B)])
+                                      ).to(dev).to(torch.bfloat16)
+        self.tK, self.tV = tK, tV
+        sel = fa4q.select_vertical_lines(self.q_obs, tK, tV, self.fp4_len, rho=dw.hp_frac)
+        assert int(sel["counts"].min()) == int(sel["counts"].max()) == n_hp
+        self.excl = sel["excl"][:, :, :P].contiguous()
         self.kp, self.ks, self.vp, self.vs = fa4q.quantize_kv_pages(tK, tV, self.fp4_len, self.excl,
                                                                     self.table, B * P)
-        idx = torch.from_numpy(hp).to(dev)
-        self.hpk = torch.gather(tK[:, :, :n_fp4], 2, idx[..., None].expand(-1, -1, -1, d)).contiguous()
-        self.hpv = torch.gather(tV[:, :, :n_fp4], 2, idx[..., None].expand(-1, -1, -1, d)).contiguous()
-        self.hpc = i32(np.full((B, Hkv), n_hp))
+        self.hpk, self.hpv, self.hpc = sel["hp_k"], sel["hp_v"], sel["counts"]
         self.wk, self.wv = tK[:, :, n_fp4:].contiguous(), tV[:, :, n_fp4:].contiguous()
         self.wl = i32(np.full(B, W))
-        del tK, tV
-        torch.cuda.empty_cache()
         self.q = torch.from_numpy(Q).to(dev).to(torch.bfloat16)
         self.out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
         self.ws = torch.empty(fa4q.decode_workspace_size(B, Hq, Hkv, d, P), dtype=torch.uint8, device=dev)
@@ -264,11 +261,29 @@ def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
         barrier()
     d_ms = d0.elapsed_time(d1) / dsteps
     gbs = drun.bytes / (d_ms * 1e-3) / 1e9
+    # vertical-line identification (column mass + selection + mask + row gather); the method
+    # refreshes it every 64 decoded tokens, so it is reported beside the step, not in it
+    ws = torch.empty(fa4q.vlines_workspace_size(dw.B, dw.Hq, dw.Hkv, drun.q_obs.shape[2], dw.L),
+                     dtype=torch.uint8, device=dev)
+    ident = lambda: fa4q.select_vertical_lines(drun.q_obs, drun.tK, drun.tV, drun.fp4_len, rho=dw.hp_frac,
+                                                workspace=ws)
+    for _ in range(2):
+        ident()
+    i0, i1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    i0.record()
+    for _ in range(5):
+        ident()
+    i1.record()
+    torch.cuda.synchronize()
+    id_ms = i0.elapsed_time(i1) / 5
     line["decode"] = {"workload": dw.name, "us_per_step": d_ms * 1e3, "higher_is_better": False,
                       "GBps": gbs, "bytes_per_step": drun.bytes, "gpu_launches": 2 * dsteps,
                       "roofline": {"kernel": "decode_split_kernel+decode_combine_kernel", "bound": "hbm",
                                    "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
                                    "traffic": ncu_traffic("decode", dw.B), "peak_source": f"{peak_kind} hbm copy"},
+                      "identify": {"ms": id_ms, "every_tokens": 64, "us_per_step_amortized": id_ms * 1e3 / 64,
+                                   "what": "column mass of 64 observation queries x 4 q-heads over the 32640-token "
+                                           "prefix, top-5% selection, exclusion mask, BF16 row gather (all 32 x 8 groups)"},
                       "l2": "working set 1.4 GB > L2", "clocks": dsampler.summary()}
 
 

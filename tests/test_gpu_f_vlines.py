@@ -109,3 +109,44 @@ def test_select_vertical_lines_decode_workload_sampled():
     overlaps = [_check_group(res, b, h, q_obs, k, v, w.fp4_len, w.hp_frac, Hq // Hkv)
                 for (b, h) in [(0, 0), (17, 5), (31, 7)]]
     assert min(overlaps) >= 0.9, overlaps
+
+
+def test_identify_quantize_decode_pipeline():
+    """Identification -> page quantisation with its exclusion mask -> decode with its BF16
+    rows, against the oracle's hybrid decode over the positions the GPU selected (the
+    selection itself is checked above; here every later step must agree on it)."""
+    import dataclasses
+    import torch
+    import microscaled_fp4_flashattention_b200 as fa4q
+    from oracle import decode as OD
+    from fa4q_testlib import assert_close
+    w = dataclasses.replace(synth.WORKLOADS[4], B=3, L=2200)
+    dev = torch.device("cuda:0")
+    B, Hq, Hkv, d, L, W, P = w.B, w.Hq, w.Hkv, w.d, w.L, w.window, w.n_pages
+    host = {(b, h): (synth.decode_kv_slice(w, "k", b, h), synth.decode_kv_slice(w, "v", b, h))
+            for b in range(B) for h in range(Hkv)}
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(dev).to(torch.bfloat16)
+    tK = bf(np.stack([np.stack([host[(b, h)][0] for h in range(Hkv)]) for b in range(B)]))
+    tV = bf(np.stack([np.stack([host[(b, h)][1] for h in range(Hkv)]) for b in range(B)]))
+    Q = np.stack([synth.decode_query(w, b) for b in range(B)])
+    q_obs = bf(np.stack([synth.decode_observation_queries(w, b) for b in range(B)]))
+    fp4_len = torch.full((B,), w.fp4_len, dtype=torch.int32, device=dev)
+    sel = fa4q.select_vertical_lines(q_obs, tK, tV, fp4_len, rho=w.hp_frac)
+    excl = sel["excl"][:, :, :P].contiguous()           # the cache's pages only
+    table = torch.from_numpy(synth.decode_block_table(w).astype(np.int32)).to(dev)
+    kp, ks, vp, vs = fa4q.quantize_kv_pages(tK, tV, fp4_len, excl, table, B * P)
+    wl = torch.full((B,), W, dtype=torch.int32, device=dev)
+    out = fa4q.decode(bf(Q), kp, ks, vp, vs, table, fp4_len, excl, sel["hp_k"], sel["hp_v"], sel["counts"],
+                      tK[:, :, w.fp4_len:].contiguous(), tV[:, :, w.fp4_len:].contiguous(), wl)
+    out = out.float().cpu().numpy()
+    assert fa4q.device_status()[0] == 0
+    pos, cnt = sel["positions"].cpu().numpy(), sel["counts"].cpu().numpy()
+    G = Hq // Hkv
+    gs, rs = [], []
+    for b in range(B):
+        for h in range(Hkv):
+            kk, vv = host[(b, h)]
+            ref = OD.decode_group(Q[b, h * G:(h + 1) * G], kk, vv, pos[b, h, :cnt[b, h]], W, "nvfp4")
+            gs.append(out[b, h * G:(h + 1) * G])
+            rs.append(synth.round_to_bf16(np.asarray(ref, dtype=np.float32)))
+    assert_close(np.stack(gs), np.stack(rs), mean_rel=5e-3, what="identify+decode")
