@@ -281,9 +281,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* abort_flag = &sm.abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // causal: heaviest query tiles first
-  const int qt = CAUSAL ? (p.n_qtiles - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-  const int h = blockIdx.y, b = blockIdx.z;
+  // Causal: the grid is linearised query-tile-major with the heaviest (last) query tiles of
+  // every head first, so the block scheduler hands out work longest-first across the whole
+  // launch and the light tiles fill the tail.  Non-causal tiles are all equal: head-major
+  // order keeps the CTAs in flight on few heads, whose K/V tiles then stay in L2.
+  const int qt = CAUSAL ? (p.n_qtiles - 1 - (int)(blockIdx.x / p.Hq)) : (int)blockIdx.x;
+  const int h = CAUSAL ? (int)(blockIdx.x % p.Hq) : (int)blockIdx.y, b = blockIdx.z;
   const int hk = h / (p.Hq / p.Hkv);
   const int bh_q = b * p.Hq + h, bh_k = b * p.Hkv + hk;
   const int n_ktiles_all = (p.S_k + kBN - 1) / kBN;
@@ -811,7 +814,7 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
   auto kern = attn_fwd_kernel<D, MX, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return FA4Q_ERR_CUDA;
-  dim3 grid(prm.n_qtiles, prm.Hq, prm.B);
+  const dim3 grid = CAUSAL ? dim3(prm.n_qtiles * prm.Hq, 1, prm.B) : dim3(prm.n_qtiles, prm.Hq, prm.B);
   kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
   return launch_status();
 }
@@ -841,7 +844,7 @@ extern "C" fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, cons
   if (B == 0 || S_q == 0) return FA4Q_OK;
   if (S_k == 0) return FA4Q_ERR_INVALID_ARG;
   const int n_qtiles = (S_q + kBM - 1) / kBM;
-  if (B > 65535 || Hq > 65535) return FA4Q_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535 || static_cast<int64_t>(n_qtiles) * Hq > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
   AttnParams prm;
   prm.q_sf = q_sf;
   prm.k_sf = k_sf;
