@@ -15,9 +15,13 @@
 // "System-Level Optimization" - transposed softmax: P blocks run along the MMA reduction
 // (key) axis so P is quantised in registers and never leaves the SM.
 //
-// Kernel structure (one CTA per query tile, 384 threads, one CTA per SM):
-//   warp 0      TMA producer: Q tile once, then K, V^T tiles and their scale atoms through
-//               an NST-deep shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
+// Kernel structure (384 threads, one CTA per SM).  A work item is one 128-row query tile of
+// one (batch, q-head).  Launches whose items are short (causal attention over a few thousand
+// keys) run persistently, one CTA per SM walking a longest-first item list; the others run
+// one CTA per item.  Roles:
+//   warp 0      TMA producer: each item's Q tile (two slots, so the next item's Q loads
+//               during this one), then K, V^T tiles and their scale atoms through an
+//               NST-deep shared-memory ring (cp.async.bulk.tensor / cp.async.bulk).
 //   warp 1      TMEM owner and MMA issuer (one elected thread): tcgen05.cp of the scale
 //               atoms into TMEM, tcgen05.mma kind::mxf4nvf4 (NVFP4) or kind::mxf4 (MXFP4).
 //   warps 2-3   idle (they complete warpgroup 0 for the register split)
@@ -27,7 +31,7 @@
 //               block scales, cvt to E2M1, P^ to shared memory (the A operand of the PV MMA),
 //               rescale of the group's O and l in TMEM, epilogue.
 // TMEM (512 columns): S [0,128), O even/odd tiles [128,256) and [256,384), l even/odd
-// [384,400) and [400,416), scale factors [416,480).  Every mbarrier wait is bounded; on expiry the CTA records a status bit,
+// [384,400) and [400,416), scale factors [416,488).  Every mbarrier wait is bounded; on expiry the CTA records a status bit,
 // skips the remaining waits, drains its own copies and MMAs and exits.
 #include <math.h>
 
@@ -56,7 +60,8 @@ constexpr int kEmulPer8 = 2;  // exponentials of every 8 computed by ex2_poly2 (
 
 // TMEM column map: one S buffer, two O and l accumulators (even / odd key tiles), scales
 constexpr uint32_t kColS = 0, kColO0 = 128, kColO1 = 256, kColL0 = 384, kColL1 = 400;
-constexpr uint32_t kColSfQ = 416, kColSfK = 424, kColSfP = 440, kColSfV = 456, kColSfOne = 472;
+// (Q scales double-buffered by work item, K scales by key tile, P and V scales by group)
+constexpr uint32_t kColSfQ = 416, kColSfK = 432, kColSfP = 448, kColSfV = 464, kColSfOne = 480;
 
 template <int D, bool MX>
 struct Cfg {
@@ -76,17 +81,19 @@ struct Cfg {
 template <int D, bool MX>
 struct __align__(1024) Smem {
   using C = Cfg<D, MX>;
-  uint8_t q[C::kQBytes];
+  uint8_t q[2][C::kQBytes];                 // double-buffered by work item
   uint8_t k[kStages][C::kKBytes];
   uint8_t v[kStages][C::kVBytes];
   uint8_t p[2][C::kPBytes];
   uint8_t ones[1024];
-  uint8_t sfq[2 * 512];
+  uint8_t sfq[2][2 * 512];
   uint8_t sfk[kStages][2 * 512];
   uint8_t sfv[kStages][2 * 512];
   uint8_t sfp[2][2 * 512];
   uint8_t sfone[2 * 512];
-  uint64_t bar_q;
+  uint64_t bar_q[2];         // Q tile (and its scales) of work item k landed, slot k % 2
+  uint64_t q_free[2];        // all S products of work item k issued and complete
+  uint64_t o_free;           // all eight softmax warps have read O and l in the epilogue
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
   uint64_t s_full[2];        // S of an even / odd key tile ready (one per softmax group)
@@ -108,6 +115,7 @@ struct AttnParams {
   float* lse;
   int B, Hq, Hkv, S_q, S_k, S_kpad;
   int n_qtiles;
+  int n_items;             // B * Hq * n_qtiles work items
   float score_scale_log2;  // sm_scale * g_q * g_k * log2(e)
   float g_v;
   float qmax_p;
@@ -270,7 +278,7 @@ FA4Q_DEVINL void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, int N
   }
 }
 
-template <int D, bool MX, bool CAUSAL>
+template <int D, bool MX, bool CAUSAL, bool PERSIST>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -281,20 +289,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* abort_flag = &sm.abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // Causal: the grid is linearised query-tile-major with the heaviest (last) query tiles of
-  // every head first, so the block scheduler hands out work longest-first across the whole
-  // launch and the light tiles fill the tail.  Non-causal tiles are all equal: head-major
-  // order keeps the CTAs in flight on few heads, whose K/V tiles then stay in L2.
-  const int qt = CAUSAL ? (p.n_qtiles - 1 - (int)(blockIdx.x / p.Hq)) : (int)blockIdx.x;
-  const int h = CAUSAL ? (int)(blockIdx.x % p.Hq) : (int)blockIdx.y, b = blockIdx.z;
-  const int hk = h / (p.Hq / p.Hkv);
-  const int bh_q = b * p.Hq + h, bh_k = b * p.Hkv + hk;
+  // Persistent CTAs (one per SM) walk one list of work items (batch, q-head, query tile).
+  // Causal lists are query-tile-major with the heaviest (last) query tiles of every head
+  // first; non-causal lists are head-major, so the items in flight share few heads whose
+  // K/V tiles stay in L2.  CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... (G CTAs): a snake
+  // over the longest-first list that evens out the work.  Every role walks the same items,
+  // so the barrier phases below follow from counters each role keeps itself.
+  struct Item {
+    int b, h, qt, n_tiles;
+  };
   const int n_ktiles_all = (p.S_k + kBN - 1) / kBN;
-  const int n_tiles = CAUSAL ? min(qt + 1, n_ktiles_all) : n_ktiles_all;
+  auto item_index = [&](int k) -> int {
+    if constexpr (!PERSIST) return k == 0 ? static_cast<int>(blockIdx.x) : -1;   // one item per CTA
+    const int G = gridDim.x, c = blockIdx.x;
+    const int64_t u = static_cast<int64_t>(k) * G + ((k & 1) ? (G - 1 - c) : c);
+    return u < p.n_items ? static_cast<int>(u) : -1;
+  };
+  auto decode_item = [&](int u) -> Item {
+    Item it;
+    if (CAUSAL) {
+      const int per = p.B * p.Hq, rem = u % per;
+      it.qt = p.n_qtiles - 1 - u / per;
+      it.b = rem / p.Hq;
+      it.h = rem % p.Hq;
+      it.n_tiles = min(it.qt + 1, n_ktiles_all);
+    } else {
+      const int per = p.Hq * p.n_qtiles, rem = u % per;
+      it.b = u / per;
+      it.h = rem / p.n_qtiles;
+      it.qt = rem % p.n_qtiles;
+      it.n_tiles = n_ktiles_all;
+    }
+    return it;
+  };
 
   // ---------------------------------------------------------------- setup
   if (threadIdx.x == 0) {
-    mbar_init(&sm.bar_q, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.bar_q[s], 1);
+      mbar_init(&sm.q_free[s], 1);
+    }
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
@@ -305,6 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.p_full[s], 4);
       mbar_init(&sm.o_done[s], 1);
     }
+    mbar_init(&sm.o_free, 8);
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
@@ -337,92 +372,124 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_v);
       const int nrt_q = (p.S_q + 127) / 128, nrt_k = (p.S_k + 127) / 128;
       const int ng_v = ((p.S_kpad + 127) / 128) * C::kSfGroups;
-      mbar_arrive_expect_tx(&sm.bar_q, C::kQBytes + C::kSfQAtoms * 512);
-      tma_load_3d(sm.q, &tm_q, 0, qt * kBM, bh_q, &sm.bar_q);
-      bulk_load(sm.sfq, p.q_sf + ((int64_t)bh_q * nrt_q + qt) * C::kSfGroups * 512,
-                C::kSfQAtoms * 512, &sm.bar_q);
-      int issued = 0;
-      for (int j = 0; j < n_tiles; ++j) {
-        const int s = j % kStages;
-        if (j >= kStages && !cta_wait(&sm.kv_empty[s], ((j / kStages) - 1) & 1, abort_flag,
-                                      kStatusTimeoutTmaFull))
-          break;
-        mbar_arrive_expect_tx(&sm.kv_full[s], C::kKBytes + C::kVBytes + C::kSfQAtoms * 512 +
-                                                  C::kSfTileAtoms * 512);
-        tma_load_3d(sm.k[s], &tm_k, 0, j * kBN, bh_k, &sm.kv_full[s]);
-        bulk_load(sm.sfk[s], p.k_sf + ((int64_t)bh_k * nrt_k + j) * C::kSfGroups * 512,
-                  C::kSfQAtoms * 512, &sm.kv_full[s]);
-        tma_load_3d(sm.v[s], &tm_v, j * (kBN / 2), 0, bh_k, &sm.kv_full[s]);
-        bulk_load(sm.sfv[s], p.vt_sf + (int64_t)bh_k * ng_v * 512 + (int64_t)j * C::kSfTileAtoms * 512,
-                  C::kSfTileAtoms * 512, &sm.kv_full[s]);
-        issued = j + 1;
+      int T = 0, q_issued = 0;                     // key tiles / Q tiles issued so far
+      bool go = true;
+      for (int k = 0; go && (PERSIST || k < 1); ++k) {
+        const int u = item_index(k);
+        if (u < 0) break;
+        const Item it = decode_item(u);
+        const int bh_q = it.b * p.Hq + it.h, bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
+        const int qs = k & 1;
+        // Q slot qs was last read by the S products of item k-2
+        if (k >= 2 && !cta_wait(&sm.q_free[qs], ((k - 2) >> 1) & 1, abort_flag, kStatusTimeoutTmaFull)) break;
+        mbar_arrive_expect_tx(&sm.bar_q[qs], C::kQBytes + C::kSfQAtoms * 512);
+        tma_load_3d(sm.q[qs], &tm_q, 0, it.qt * kBM, bh_q, &sm.bar_q[qs]);
+        bulk_load(sm.sfq[qs], p.q_sf + ((int64_t)bh_q * nrt_q + it.qt) * C::kSfGroups * 512,
+                  C::kSfQAtoms * 512, &sm.bar_q[qs]);
+        q_issued = k + 1;
+        for (int j = 0; j < it.n_tiles; ++j, ++T) {
+          const int s = T % kStages;
+          if (T >= kStages && !cta_wait(&sm.kv_empty[s], ((T / kStages) - 1) & 1, abort_flag,
+                                        kStatusTimeoutTmaFull)) {
+            go = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.kv_full[s], C::kKBytes + C::kVBytes + C::kSfQAtoms * 512 +
+                                                    C::kSfTileAtoms * 512);
+          tma_load_3d(sm.k[s], &tm_k, 0, j * kBN, bh_k, &sm.kv_full[s]);
+          bulk_load(sm.sfk[s], p.k_sf + ((int64_t)bh_k * nrt_k + j) * C::kSfGroups * 512,
+                    C::kSfQAtoms * 512, &sm.kv_full[s]);
+          tma_load_3d(sm.v[s], &tm_v, j * (kBN / 2), 0, bh_k, &sm.kv_full[s]);
+          bulk_load(sm.sfv[s], p.vt_sf + (int64_t)bh_k * ng_v * 512 + (int64_t)j * C::kSfTileAtoms * 512,
+                    C::kSfTileAtoms * 512, &sm.kv_full[s]);
+        }
       }
-      // drain: every issued stage must have landed before the CTA may exit
-      for (int j = max(0, issued - kStages); j < issued; ++j)
-        mbar_wait(&sm.kv_full[j % kStages], (j / kStages) & 1, &g_attn_status, kStatusTimeoutDrain);
-      if (!(*abort_flag)) mbar_wait(&sm.bar_q, 0, &g_attn_status, kStatusTimeoutDrain);
+      // drain: every issued copy must have landed before the CTA may exit
+      for (int t = max(0, T - kStages); t < T; ++t)
+        mbar_wait(&sm.kv_full[t % kStages], (t / kStages) & 1, &g_attn_status, kStatusTimeoutDrain);
+      for (int k = max(0, q_issued - 2); k < q_issued; ++k)
+        mbar_wait(&sm.bar_q[k & 1], (k >> 1) & 1, &g_attn_status, kStatusTimeoutDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      const uint32_t q_addr = smem_u32(sm.q);
       const uint32_t ones_addr = smem_u32(sm.ones);
-      bool ok = cta_wait(&sm.bar_q, 0, abort_flag, kStatusTimeoutMma);
-      tc_fence_after();
-      for (int a = 0; a < C::kSfQAtoms; ++a) tmem_cp_sf_atom(tmem + kColSfQ + 4 * a, smem_u32(sm.sfq + 512 * a));
       for (int a = 0; a < C::kSfTileAtoms; ++a)
         tmem_cp_sf_atom(tmem + kColSfOne + 4 * a, smem_u32(sm.sfone + 512 * a));
-      // S_j = Q K_j^T into the single S buffer once the softmax group of tile j-1 holds
-      // S_{j-1} in registers
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % kStages, kb = j & 1;
-        if (!cta_wait(&sm.kv_full[s], (j / kStages) & 1, abort_flag, kStatusTimeoutMma)) return false;
-        if (j >= 1 && !cta_wait(&sm.s_free, (j - 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
+      bool ok = true;
+      int T = 0;                                   // key tiles of all earlier items
+      int n_pv0 = 0, n_pv1 = 0;                    // PV products issued per softmax group
+      for (int k = 0; ok && (PERSIST || k < 1); ++k) {
+        const int u = item_index(k);
+        if (u < 0) break;
+        const Item it = decode_item(u);
+        const int qs = k & 1, T0 = T, n_tiles = it.n_tiles;
+        if (!cta_wait(&sm.bar_q[qs], (k >> 1) & 1, abort_flag, kStatusTimeoutMma)) break;
         tc_fence_after();
+        // item k-2 used this scale slot; all of its products completed before item k-1 ended
         for (int a = 0; a < C::kSfQAtoms; ++a)
-          tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
-        const uint32_t k_addr = smem_u32(sm.k[s]);
+          tmem_cp_sf_atom(tmem + kColSfQ + 8 * qs + 4 * a, smem_u32(sm.sfq[qs] + 512 * a));
+        const uint32_t q_addr = smem_u32(sm.q[qs]);
+        // S_j = Q K_j^T into the single S buffer once the softmax group of the previous key
+        // tile (of this item or the last) holds its scores in registers
+        auto issue_s = [&](int j) -> bool {
+          const int t = T0 + j, s = t % kStages, kb = t & 1;
+          if (!cta_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag, kStatusTimeoutMma)) return false;
+          if (t >= 1 && !cta_wait(&sm.s_free, (t - 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
+          tc_fence_after();
+          for (int a = 0; a < C::kSfQAtoms; ++a)
+            tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
+          const uint32_t k_addr = smem_u32(sm.k[s]);
 #pragma unroll
-        for (int ks = 0; ks < C::kKStepsQK; ++ks) {
-          const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-          const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-          mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ, tmem + kColSfK + 8 * kb, ks > 0);
-        }
-        tc_commit(&sm.s_full[j & 1]);
-        return true;
-      };
-      // [O | l]_{j%2} (+)= P^_j [V_j | 1] once the softmax group has written P^_j
-      auto issue_pv = [&](int jp) -> bool {
-        const int s = jp % kStages, pb = jp & 1;
-        if (!cta_wait(&sm.p_full[pb], (jp >> 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
-        tc_fence_after();
-        for (int a = 0; a < C::kSfTileAtoms; ++a) {
-          tmem_cp_sf_atom(tmem + kColSfP + 8 * pb + 4 * a, smem_u32(sm.sfp[pb] + 512 * a));
-          tmem_cp_sf_atom(tmem + kColSfV + 8 * pb + 4 * a, smem_u32(sm.sfv[s] + 512 * a));
-        }
-        const uint32_t p_addr = smem_u32(sm.p[pb]);
-        const uint32_t v_addr = smem_u32(sm.v[s]);
-        const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
+          for (int ks = 0; ks < C::kKStepsQK; ++ks) {
+            const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+            const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+            mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ + 8 * qs, tmem + kColSfK + 8 * kb, ks > 0);
+          }
+          tc_commit(&sm.s_full[j & 1]);
+          return true;
+        };
+        // [O | l]_{j%2} (+)= P^_j [V_j | 1] once the softmax group has written P^_j; the first
+        // product of an item waits until the previous item's epilogue has read O and l
+        auto issue_pv = [&](int jp) -> bool {
+          const int t = T0 + jp, s = t % kStages, pb = jp & 1;
+          if (jp == 0 && k >= 1 && !cta_wait(&sm.o_free, (k - 1) & 1, abort_flag, kStatusTimeoutMma))
+            return false;
+          int& n_pv = pb ? n_pv1 : n_pv0;
+          if (!cta_wait(&sm.p_full[pb], n_pv & 1, abort_flag, kStatusTimeoutMma)) return false;
+          ++n_pv;
+          tc_fence_after();
+          for (int a = 0; a < C::kSfTileAtoms; ++a) {
+            tmem_cp_sf_atom(tmem + kColSfP + 8 * pb + 4 * a, smem_u32(sm.sfp[pb] + 512 * a));
+            tmem_cp_sf_atom(tmem + kColSfV + 8 * pb + 4 * a, smem_u32(sm.sfv[s] + 512 * a));
+          }
+          const uint32_t p_addr = smem_u32(sm.p[pb]);
+          const uint32_t v_addr = smem_u32(sm.v[s]);
+          const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
 #pragma unroll
-        for (int ks = 0; ks < 2; ++ks) {
-          const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
-          const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
-          const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
-          const uint32_t acc = (jp >= 2 || ks > 0) ? 1u : 0u;
-          mma_step<MX>(tmem + o_col, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
-          mma_step<MX>(tmem + l_col, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
+          for (int ks = 0; ks < 2; ++ks) {
+            const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
+            const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
+            const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
+            const uint32_t acc = (jp >= 2 || ks > 0) ? 1u : 0u;
+            mma_step<MX>(tmem + o_col, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
+            mma_step<MX>(tmem + l_col, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
+          }
+          tc_commit(&sm.o_done[pb]);
+          tc_commit(&sm.kv_empty[s]);
+          return true;
+        };
+        // Issue order S_0, S_1, PV_0, S_2, PV_1, ...: S runs two products ahead of PV, so the
+        // next S is computed as soon as the S buffer is free (the other group has loaded its
+        // scores, early in its tile) instead of waiting behind the previous tile's P^.  The
+        // first scores of the next item are computed while this item's epilogue runs.
+        ok = issue_s(0);
+        for (int j = 0; ok && j <= n_tiles; ++j) {
+          if (j + 1 < n_tiles && !issue_s(j + 1)) ok = false;
+          else if (j >= 1 && !issue_pv(j - 1)) ok = false;
         }
-        tc_commit(&sm.o_done[pb]);
-        tc_commit(&sm.kv_empty[s]);
-        return true;
-      };
-      // Issue order S_0, S_1, PV_0, S_2, PV_1, ...: S runs two products ahead of PV, so the
-      // next S is computed as soon as the S buffer is free (the other group has loaded its
-      // scores, early in its tile) instead of waiting behind the previous tile's P^.
-      ok = ok && issue_s(0);
-      for (int j = 0; ok && j <= n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
-        if (j >= 1 && !issue_pv(j - 1)) break;
+        tc_commit(&sm.q_free[qs]);                 // every product that read Q slot qs
+        T += n_tiles;
       }
       // drain: all MMAs this thread issued complete before TMEM is released
       tc_commit(&sm.drain);
@@ -443,7 +510,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = (warp - 4) >> 2;                 // softmax group: 0 = even tiles, 1 = odd
     const int wq = warp & 3;                       // TMEM lane quadrant
     const int r = wq * 32 + lane;                  // row within the query tile
-    const int row = qt * kBM + r;                  // query index
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const int bar_send = 1 + 4 * g + wq, bar_recv = 1 + 4 * (g ^ 1) + wq, bar_epi = 9 + wq;
     const float sc = p.score_scale_log2;
@@ -452,10 +518,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // exact difference (bmax - m) * sc, so the block holding the row maximum gets amax = 1
     // exactly: the MX OCP exponent floor(log2 amax) - 2 jumps at every power of two, and a
     // fused s*sc - round(m*sc) that lands 1 ulp below 0 would move that block's scale.
-    float m_acc = -INFINITY;                       // maximum of this group's last tile
     bool ok = true;
+    int done_a = 0, done_b = 0;                    // key tiles each group processed in earlier items
+    for (int k = 0; PERSIST || k < 1; ++k) {
+    const int u = item_index(k);
+    if (u < 0) break;
+    const Item it = decode_item(u);
+    const int qt = it.qt, n_tiles = it.n_tiles;
+    const int bh_q = it.b * p.Hq + it.h;
+    const int row = qt * kBM + r;                  // query index
+    const int done_g = g ? done_b : done_a;
+    float m_acc = -INFINITY;                       // maximum of this group's last tile
     for (int j = g; j < n_tiles; j += 2) {
-      ok = warp_wait(&sm.s_full[g], (j >> 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
+      ok = warp_wait(&sm.s_full[g], (done_g + (j >> 1)) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       tc_fence_after();
       float s[kBN];
       {
@@ -533,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // accumulator g and P buffer g were last used by this group's previous PV product
       if (j >= 2)
-        ok = warp_wait(&sm.o_done[g], ((j - 2) >> 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
+        ok = warp_wait(&sm.o_done[g], (done_g + (j >> 1) - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       uint8_t* pbuf = sm.p[g];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -580,13 +655,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     named_bar_sync(bar_epi, 64);
     const float mA = sm.m_last[0][r], mB = sm.m_last[1][r];
     const float m = fmaxf(mA, mB);
-    const int last0 = (n_tiles - 1) & ~1, last1 = n_tiles >= 2 ? ((n_tiles - 2) | 1) : -1;
-    ok = __all_sync(0xffffffffu, cta_wait(&sm.o_done[0], (last0 >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) && ok;
-    if (last1 >= 0)
-      ok = __all_sync(0xffffffffu, cta_wait(&sm.o_done[1], (last1 >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) && ok;
+    // the last PV product of each group in this item is the most recent phase of its o_done
+    // barrier (the next item's products wait on o_free, which needs this epilogue)
+    const int cnt_a = (n_tiles + 1) / 2, cnt_b = n_tiles / 2;   // key tiles of each group
+    ok = warp_wait(&sm.o_done[0], (done_a + cnt_a - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
+    if (cnt_b > 0)
+      ok = warp_wait(&sm.o_done[1], (done_b + cnt_b - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
     if (ok) {
       tc_fence_after();
-      const bool has_b = last1 >= 0;
+      const bool has_b = cnt_b > 0;
       const float wa = ex2_approx((mA - m) * sc), wb = has_b ? ex2_approx((mB - m) * sc) : 0.0f;
       uint32_t lra, lrb = 0;
       tmem_ld1(lane_base + kColL0, lra);
@@ -633,6 +710,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           p.lse[orow] = m * sc * 0.69314718055994531f + logf(l * lscale);
         }
       }
+    }
+    done_a += cnt_a;
+    done_b += cnt_b;
+    // O and l have been read: the next item's first PV product may overwrite them
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.o_free);
     }
   }
   // ---------------------------------------------------------------- teardown
@@ -811,10 +895,18 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
                    CU_TENSOR_MAP_SWIZZLE_64B))
     return FA4Q_ERR_CUDA;
   const size_t smem = sizeof(Smem<D, MX>) + 1024;
-  auto kern = attn_fwd_kernel<D, MX, CAUSAL>;
+  // Short items (few key tiles on average, as in causal attention over a few thousand keys)
+  // run persistently, one CTA per SM walking the item list, so the per-CTA setup and the
+  // pipeline fill and drain of an item overlap the neighbouring items.  Long items run one
+  // CTA per item: the block scheduler then balances them dynamically across the SMs, and the
+  // kernel is compiled without the item loop.
+  const int n_ktiles = (prm.S_k + kBN - 1) / kBN;
+  const double avg_tiles = CAUSAL ? 0.5 * (std::min(prm.n_qtiles, n_ktiles) + 1) : n_ktiles;
+  const bool persist = avg_tiles <= 48.0 && prm.n_items > num_sms();
+  auto kern = persist ? attn_fwd_kernel<D, MX, CAUSAL, true> : attn_fwd_kernel<D, MX, CAUSAL, false>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return FA4Q_ERR_CUDA;
-  const dim3 grid = CAUSAL ? dim3(prm.n_qtiles * prm.Hq, 1, prm.B) : dim3(prm.n_qtiles, prm.Hq, prm.B);
+  const dim3 grid(static_cast<unsigned>(persist ? num_sms() : prm.n_items));
   kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
   return launch_status();
 }
@@ -844,7 +936,7 @@ extern "C" fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, cons
   if (B == 0 || S_q == 0) return FA4Q_OK;
   if (S_k == 0) return FA4Q_ERR_INVALID_ARG;
   const int n_qtiles = (S_q + kBM - 1) / kBM;
-  if (B > 65535 || Hq > 65535 || static_cast<int64_t>(n_qtiles) * Hq > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * Hq * n_qtiles > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
   AttnParams prm;
   prm.q_sf = q_sf;
   prm.k_sf = k_sf;
@@ -858,6 +950,7 @@ extern "C" fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, cons
   prm.S_k = S_k;
   prm.S_kpad = (S_k + 31) / 32 * 32;
   prm.n_qtiles = n_qtiles;
+  prm.n_items = B * Hq * n_qtiles;
   const float sms = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)d);
   prm.score_scale_log2 = sms * g_q * g_k * kLog2e;
   prm.g_v = g_v;

@@ -18,6 +18,19 @@ inline fa4q_status launch_status() {
   return e == cudaSuccess ? FA4Q_OK : FA4Q_ERR_CUDA;
 }
 
+// Streaming multiprocessors of the current device (cached per device; 148 on B200).
+inline int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cached[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = n > 0 ? n : 148;
+  }
+  return cached[dev];
+}
+
 // Each translation unit with bounded device waits owns one status word; these host
 // functions read-and-clear them (stream-ordered, then synchronised by the caller).
 cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word);

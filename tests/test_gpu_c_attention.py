@@ -104,6 +104,22 @@ def test_smoothed_mxfp4_gqa_recipe():
     check(q, k, v, "mxfp4", True, lam=lam, what="smoothed")
 
 
+@pytest.mark.parametrize("fmt,causal,S,Hq,Hkv,B", [
+    ("mxfp4", True, 1000, 40, 8, 1),     # 320 items of 1..8 key tiles, several per CTA
+    ("nvfp4", False, 200, 80, 16, 2),    # 320 items of 2 key tiles (ragged last tile)
+])
+def test_prefill_persistent_many_short_items(fmt, causal, S, Hq, Hkv, B):
+    """More work items than SMs, all short: the kernel runs persistently (one CTA per SM
+    walking the longest-first item list), so CTAs carry their barrier phases, Q slots and
+    accumulators from one item to the next; heads spread over the list are checked."""
+    d = 128
+    q = _rand((B, Hq, S, d), S + 7, 1.5)
+    k = _rand((B, Hkv, S, d), S + 8, 1.5)
+    v = _rand((B, Hkv, S, d), S + 9)
+    heads = [(0, 0), (0, 1), (B - 1, Hq // 2), (B - 1, Hq - 3), (B - 1, Hq - 1)]
+    check(q, k, v, fmt, causal, heads=heads, what=f"persistent {fmt} causal={causal}")
+
+
 def _rows(S, n_rand, seed):
     base = [0, 1, 127, 128, 129, S // 2, S - 129, S - 128, S - 1]
     rnd = np.random.default_rng(seed).choice(S, n_rand, replace=False)
