@@ -163,7 +163,8 @@ class PrefillRun:
             self.mq, self.mk = fa4q.smooth_calibrate(torch.from_numpy(qc).to(dev).to(torch.bfloat16),
                                                      torch.from_numpy(kc).to(dev).to(torch.bfloat16))
         self.out = torch.empty((w.B, w.Hq, w.S, w.d), dtype=torch.bfloat16, device=dev)
-        self.launches_per_step = 4
+        self.qkv = fa4q.quantize_qkv(self.q, self.k, self.v, w.fmt, w.qmax, mul_q=self.mq, mul_k=self.mk)
+        self.launches_per_step = 2
 
     @staticmethod
     def _shifted(w, off):
@@ -176,9 +177,9 @@ class PrefillRun:
         q = self.q if q is None else q
         k = self.k if k is None else k
         v = self.v if v is None else v
-        pq, sq = fa4q.quantize(q, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax, 1.0, self.mq, w.Hq, w.Hq // w.Hkv)
-        pk, sk = fa4q.quantize(k, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax, 1.0, self.mk, w.Hkv, 1)
-        pv, sv = fa4q.quantize(v, w.fmt, fa4q.FA4Q_AXIS_OUTER, w.qmax)
+        # quantise Q, K (with the smoothing multipliers) and V in one launch, then attention
+        pq, sq, pk, sk, pv, sv = fa4q.quantize_qkv(q, k, v, w.fmt, w.qmax, mul_q=self.mq, mul_k=self.mk,
+                                                   out=self.qkv)
         if attn_events is not None:
             attn_events[0].record()
         fa4q.attn_fwd(pq, sq, pk, sk, pv, sv, B=w.B, Hq=w.Hq, Hkv=w.Hkv, S_q=w.S, S_k=w.S, d=w.d,

@@ -101,6 +101,25 @@ fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows, int64_t c
                           uint8_t* scales_out, void* stream);
 
 /*
+ * fa4q_quantize_qkv - the three quantisations of a prefill in one launch, bit-identical to
+ *   fa4q_quantize(q, B*Hq,  S_q, d, d, fmt, INNER, qmax, g_q, mul_q, Hq,  Hq/Hkv, TILED, ...)
+ *   fa4q_quantize(k, B*Hkv, S_k, d, d, fmt, INNER, qmax, g_k, mul_k, Hkv, 1,      TILED, ...)
+ *   fa4q_quantize(v, B*Hkv, S_k, d, d, fmt, OUTER, qmax, g_v, NULL,  0,   0,      TILED, ...)
+ * i.e. exactly the operands fa4q_attn_fwd reads.  Same sources as fa4q_quantize (block
+ * quantisation of Q, K along d with the optional Smooth-QK multipliers, of V along tokens,
+ * stored transposed).  The CTAs of one launch are split between the three tensors, so the
+ * small K and V parts run beside Q instead of as two more launches.
+ * q bf16 [B][Hq][S_q][d], k, v bf16 [B][Hkv][S_k][d] (contiguous); mul_q / mul_k nullable
+ * FP32 [Hkv][d] (lambda and 1/lambda); outputs as fa4q_quantize's (tiled scales).  d in
+ * {64, 128}; the NVFP4 tensor scales g_* are ignored for MXFP4.  Errors as fa4q_quantize.
+ */
+fa4q_status fa4q_quantize_qkv(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                              int S_q, int S_k, int d, fa4q_format fmt, float qmax, float g_q,
+                              float g_k, float g_v, const float* mul_q, const float* mul_k,
+                              uint8_t* q_packed, uint8_t* q_sf, uint8_t* k_packed, uint8_t* k_sf,
+                              uint8_t* vt_packed, uint8_t* vt_sf, void* stream);
+
+/*
  * fa4q_smooth_calibrate - static per-channel Smooth-QK multipliers from a calibration draw.
  *
  * Source: HiFA4, Abstract (calibration-static per-channel equivalent rescaling of Q and K

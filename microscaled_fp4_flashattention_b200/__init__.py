@@ -27,7 +27,7 @@ EXPORTED = [
     "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_quantize_kv_pages",
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
-    "fa4q_vlines_workspace_size", "fa4q_select_vertical_lines",
+    "fa4q_vlines_workspace_size", "fa4q_select_vertical_lines", "fa4q_quantize_qkv",
 ]
 
 _LIB = None
@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.fa4q_selftest_wait_timeout.argtypes = [U32, P]
         L.fa4q_selftest_exp2.restype = I
         L.fa4q_selftest_exp2.argtypes = [P, P, I64, P]
+        L.fa4q_quantize_qkv.restype = I
+        L.fa4q_quantize_qkv.argtypes = [P, P, P, I, I, I, I, I, I, I, F, F, F, F, P, P, P, P, P, P, P, P, P]
         L.fa4q_vlines_workspace_size.restype = Z
         L.fa4q_vlines_workspace_size.argtypes = [I, I, I, I, I]
         L.fa4q_select_vertical_lines.restype = I
@@ -175,6 +177,29 @@ def attn_fwd(q, q_sf, k, k_sf, vt, vt_sf, *, B, Hq, Hkv, S_q, S_k, d, fmt, causa
         _ptr(q), _ptr(q_sf), _ptr(k), _ptr(k_sf), _ptr(vt), _ptr(vt_sf), g_q, g_k, g_v, B, Hq, Hkv,
         S_q, S_k, d, _fmt(fmt), qmax_p, int(causal), sm_scale, _ptr(out), int(out_fp32), _ptr(lse),
         _stream(stream)))
+    return out
+
+
+def quantize_qkv(q, k, v, fmt, qmax: float = 0.0, g_q=1.0, g_k=1.0, g_v=1.0, mul_q=None, mul_k=None,
+                 out=None, stream=None):
+    """Q, K (blocks along d, optional smoothing multipliers) and V (transposed) in one launch.
+    q bf16 [B, Hq, S_q, d]; k, v bf16 [B, Hkv, S_k, d].  Returns (pq, sq, pk, sk, pv, sv) as
+    quantize() gives them with the tiled scale layout; `out` may pass those six tensors."""
+    import torch
+    B, Hq, S_q, d = q.shape
+    _, Hkv, S_k, _ = k.shape
+    f = _fmt(fmt)
+    if out is None:
+        dev = q.device
+        u8 = lambda *s: torch.empty(s, dtype=torch.uint8, device=dev)
+        rp = (S_k + 31) // 32 * 32
+        out = (u8(B, Hq, S_q, d // 2), u8(B, Hq, sf_tiled_bytes(S_q, d, f)),
+               u8(B, Hkv, S_k, d // 2), u8(B, Hkv, sf_tiled_bytes(S_k, d, f)),
+               u8(B, Hkv, d, rp // 2), u8(B, Hkv, sf_tiled_bytes(d, rp, f)))
+    pq, sq, pk, sk, pv, sv = out
+    _check("fa4q_quantize_qkv", lib().fa4q_quantize_qkv(
+        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, S_q, S_k, d, f, qmax, g_q, g_k, g_v, _ptr(mul_q), _ptr(mul_k),
+        _ptr(pq), _ptr(sq), _ptr(pk), _ptr(sk), _ptr(pv), _ptr(sv), _stream(stream)))
     return out
 
 

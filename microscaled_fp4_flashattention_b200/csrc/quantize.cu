@@ -79,33 +79,38 @@ FA4Q_DEVINL int64_t sf_tiled_offset(int64_t r, int64_t k, int64_t nG) {
 // rate); in the tiled layout the index space also covers the padding rows and scale columns,
 // whose bytes are written as the scale of an all-zero block (0)
 // ---------------------------------------------------------------------------------------
+struct InnerArgs {
+  const uint16_t* x;
+  int64_t rows, cols, row_stride;
+  float qmax, g;
+  const float* mul;
+  int64_t mheads, mratio;
+  int tiled;
+  uint8_t* packed;
+  uint8_t* sf;
+};
+
+// slot idx of group gi's scale space (32-bit in-group indices: no 64-bit divisions per block)
 template <int BLK>
-__global__ void __launch_bounds__(256) quant_inner_kernel(
-    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t row_stride, float qmax,
-    float g, const float* __restrict__ mul, int64_t mheads, int64_t mratio, int tiled,
-    uint8_t* __restrict__ packed, uint8_t* __restrict__ sf) {
-  // grid: x over the (row, block) slots of one group's scale space, y = group; 32-bit
-  // in-group indices (no 64-bit divisions per 32-element block)
-  const int nblk = static_cast<int>(cols / BLK);
-  const int rows_i = static_cast<int>(rows);
-  const int rows_sp = tiled ? ((rows_i + 127) / 128) * 128 : rows_i;
-  const int nG = tiled ? static_cast<int>((cols + 127) / 128) * (32 / BLK) : 0;
-  const int ncol_sp = tiled ? nG * 4 : nblk;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+FA4Q_DEVINL void quant_inner_slot(const InnerArgs& a, int64_t gi, int idx) {
+  const int nblk = static_cast<int>(a.cols / BLK);
+  const int rows_i = static_cast<int>(a.rows);
+  const int rows_sp = a.tiled ? ((rows_i + 127) / 128) * 128 : rows_i;
+  const int nG = a.tiled ? static_cast<int>((a.cols + 127) / 128) * (32 / BLK) : 0;
+  const int ncol_sp = a.tiled ? nG * 4 : nblk;
   if (idx >= rows_sp * ncol_sp) return;
-  const int64_t gi = blockIdx.y;
   const int r = idx / ncol_sp;
   const int kb = idx - r * ncol_sp;
-  const int64_t sf_group_bytes = tiled ? (int64_t)((rows_i + 127) / 128) * nG * 512 : (int64_t)rows_i * nblk;
+  const int64_t sf_group_bytes = a.tiled ? (int64_t)((rows_i + 127) / 128) * nG * 512 : (int64_t)rows_i * nblk;
   uint32_t s = 0;
   if (r < rows_i && kb < nblk) {
-    const uint16_t* src = x + (gi * rows + r) * row_stride + kb * BLK;
+    const uint16_t* src = a.x + (gi * a.rows + r) * a.row_stride + kb * BLK;
     float v[BLK];
 #pragma unroll
     for (int c = 0; c < BLK; c += 8) load_bf16x8(src + c, v + c);
-    if (mul != nullptr) {
-      const int mrow = (static_cast<int>(gi) % static_cast<int>(mheads)) / static_cast<int>(mratio);
-      const float* m = mul + (int64_t)mrow * cols + kb * BLK;
+    if (a.mul != nullptr) {
+      const int mrow = (static_cast<int>(gi) % static_cast<int>(a.mheads)) / static_cast<int>(a.mratio);
+      const float* m = a.mul + (int64_t)mrow * a.cols + kb * BLK;
 #pragma unroll
       for (int c = 0; c < BLK; c += 4) {
         const float4 mm = *reinterpret_cast<const float4*>(m + c);
@@ -115,49 +120,66 @@ __global__ void __launch_bounds__(256) quant_inner_kernel(
         v[c + 3] = __fmul_rn(v[c + 3], mm.w);
       }
     }
-    uint8_t* dst = packed + (gi * rows + r) * (cols / 2) + kb * (BLK / 2);
+    uint8_t* dst = a.packed + (gi * a.rows + r) * (a.cols / 2) + kb * (BLK / 2);
     if constexpr (BLK == 16) {
       uint2 p;
-      s = quant_block16_nvfp4(v, __fmul_rn(qmax, g), g, p);
+      s = quant_block16_nvfp4(v, __fmul_rn(a.qmax, a.g), a.g, p);
       *reinterpret_cast<uint2*>(dst) = p;
     } else {
       uint4 p;
-      s = quant_block32_mxfp4(v, qmax, p);
+      s = quant_block32_mxfp4(v, a.qmax, p);
       *reinterpret_cast<uint4*>(dst) = p;
     }
   }
-  if (tiled)
-    sf[gi * sf_group_bytes + sf_tiled_offset(r, kb, nG)] = (uint8_t)s;
+  if (a.tiled)
+    a.sf[gi * sf_group_bytes + sf_tiled_offset(r, kb, nG)] = (uint8_t)s;
   else
-    sf[gi * sf_group_bytes + (int64_t)r * nblk + kb] = (uint8_t)s;
+    a.sf[gi * sf_group_bytes + (int64_t)r * nblk + kb] = (uint8_t)s;
+}
+
+template <int BLK>
+__global__ void __launch_bounds__(256) quant_inner_kernel(const InnerArgs a) {
+  // grid: x over the (row, block) slots of one group's scale space, y = group
+  quant_inner_slot<BLK>(a, blockIdx.y, blockIdx.x * blockDim.x + threadIdx.x);
 }
 
 // ---------------------------------------------------------------------------------------
-// AXIS_OUTER: blocks along tokens, transposed output.  CTA = (group, 128 tokens, 64 ch).
+// AXIS_OUTER: blocks along tokens, transposed output.  One tile = (group, 128 tokens,
+// 64 channels) handled by 128 threads t (t = 0..127) through a shared-memory transpose.
 // ---------------------------------------------------------------------------------------
+struct OuterArgs {
+  const uint16_t* x;
+  int64_t rows, cols, row_stride;
+  float qmax, g;
+  int tiled;
+  uint8_t* packed;
+  uint8_t* sf;
+};
+
+// every thread of the CTA calls this (it synchronises the CTA once); `valid` false makes the
+// thread's half a no-op that still takes part in the synchronisation
 template <int BLK>
-__global__ void __launch_bounds__(128) quant_outer_kernel(
-    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t row_stride, float qmax,
-    float g, int tiled, uint8_t* __restrict__ packed, uint8_t* __restrict__ sf) {
-  __shared__ float tile[64][129];
-  const int64_t gi = blockIdx.z;
-  const int64_t tok0 = (int64_t)blockIdx.x * 128;
-  const int64_t ch0 = (int64_t)blockIdx.y * 64;
-  const int64_t rows_pad = (rows + 31) / 32 * 32;
-  const int t = threadIdx.x;
+FA4Q_DEVINL void quant_outer_tile(const OuterArgs& a, int64_t gi, int64_t tok_tile, int64_t ch_tile, int t,
+                                  float (*tile)[129], bool valid) {
+  const int64_t tok0 = tok_tile * 128;
+  const int64_t ch0 = ch_tile * 64;
+  const int64_t rows_pad = (a.rows + 31) / 32 * 32;
   // load [128 tokens][64 channels] -> tile[ch][tok]
+  if (valid) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int u = t + 128 * i;
-    const int tr = u >> 3, c8 = (u & 7) * 8;
-    float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    if (tok0 + tr < rows && ch0 + c8 < cols)
-      load_bf16x8(x + (gi * rows + tok0 + tr) * row_stride + ch0 + c8, v);
+    for (int i = 0; i < 8; ++i) {
+      const int u = t + 128 * i;
+      const int tr = u >> 3, c8 = (u & 7) * 8;
+      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (tok0 + tr < a.rows && ch0 + c8 < a.cols)
+        load_bf16x8(a.x + (gi * a.rows + tok0 + tr) * a.row_stride + ch0 + c8, v);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) tile[c8 + k][tr] = v[k];
+      for (int k = 0; k < 8; ++k) tile[c8 + k][tr] = v[k];
+    }
   }
   __syncthreads();
-  const float denom = __fmul_rn(qmax, g);
+  if (!valid) return;
+  const float denom = __fmul_rn(a.qmax, a.g);
   // thread -> (channel, 4 consecutive blocks of tokens)
   constexpr int kGroupTok = 4 * BLK;                  // 64 (NVFP4) or 128 (MXFP4)
   constexpr int kGroupsPerTile = 128 / kGroupTok;     // 2 or 1
@@ -167,11 +189,11 @@ __global__ void __launch_bounds__(128) quant_outer_kernel(
   const int64_t ch = ch0 + c;
   // channels in [cols, 128*ceil(cols/128)) are padding rows of the tiled scale layout: their
   // (all-zero) blocks give scale 0, which is written; packed data exists only for ch < cols
-  const bool real_ch = ch < cols;
-  if (!real_ch && !tiled) return;
+  const bool real_ch = ch < a.cols;
+  if (!real_ch && !a.tiled) return;
   const int64_t nblk_t = rows_pad / BLK;               // blocks per channel row
   const int64_t nG = ((rows_pad + 127) / 128) * (32 / BLK);
-  const int64_t sf_group_bytes = tiled ? ((cols + 127) / 128) * nG * 512 : cols * nblk_t;
+  const int64_t sf_group_bytes = a.tiled ? ((a.cols + 127) / 128) * nG * 512 : a.cols * nblk_t;
   uint32_t sword = 0;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -181,24 +203,64 @@ __global__ void __launch_bounds__(128) quant_outer_kernel(
 #pragma unroll
     for (int k = 0; k < BLK; ++k) v[k] = tile[c][lt + k];
     uint32_t s;
-    uint8_t* dst = packed + (gi * cols + ch) * (rows_pad / 2) + (tok0 + lt) / 2;
+    uint8_t* dst = a.packed + (gi * a.cols + ch) * (rows_pad / 2) + (tok0 + lt) / 2;
     const bool inside = real_ch && tok0 + lt < rows_pad;
     if constexpr (BLK == 16) {
       uint2 p;
-      s = quant_block16_nvfp4(v, denom, g, p);
+      s = quant_block16_nvfp4(v, denom, a.g, p);
       if (inside) *reinterpret_cast<uint2*>(dst) = p;
     } else {
       uint4 p;
-      s = quant_block32_mxfp4(v, qmax, p);
+      s = quant_block32_mxfp4(v, a.qmax, p);
       if (inside) *reinterpret_cast<uint4*>(dst) = p;
     }
     sword |= s << (8 * i);
-    if (!tiled && inside) sf[gi * sf_group_bytes + ch * nblk_t + kb] = (uint8_t)s;
+    if (!a.tiled && inside) a.sf[gi * sf_group_bytes + ch * nblk_t + kb] = (uint8_t)s;
   }
-  if (tiled) {
+  if (a.tiled) {
     const int64_t k0 = (tok0 + tg * kGroupTok) / BLK;
-    *reinterpret_cast<uint32_t*>(sf + gi * sf_group_bytes + sf_tiled_offset(ch, k0, nG)) = sword;
+    *reinterpret_cast<uint32_t*>(a.sf + gi * sf_group_bytes + sf_tiled_offset(ch, k0, nG)) = sword;
   }
+}
+
+template <int BLK>
+__global__ void __launch_bounds__(128) quant_outer_kernel(const OuterArgs a) {
+  __shared__ float tile[64][129];
+  quant_outer_tile<BLK>(a, blockIdx.z, blockIdx.x, blockIdx.y, threadIdx.x, tile, true);
+}
+
+// ---------------------------------------------------------------------------------------
+// Q, K (blocks along d) and V (blocks along tokens, transposed) in one launch: CTAs
+// [0, n_q) take Q slots, [n_q, n_q + n_k) K slots, the rest two V tiles each (one per 128
+// threads), so the small K and V work runs in the same wave as Q instead of two more launches.
+// ---------------------------------------------------------------------------------------
+struct QkvGrid {
+  int64_t per_group_q, per_group_k;       // inner slots per group
+  int64_t groups_q, groups_k, groups_v;
+  int64_t n_q, n_k;                       // CTAs of the Q and K parts
+  int64_t tok_tiles, ch_tiles, n_vtiles;  // V tiles: groups_v * tok_tiles * ch_tiles
+};
+
+template <int BLK>
+__global__ void __launch_bounds__(256) quant_qkv_kernel(const InnerArgs aq, const InnerArgs ak,
+                                                        const OuterArgs av, const QkvGrid gr) {
+  extern __shared__ __align__(16) float qkv_tile[];   // [2][64][129]
+  const int64_t cta = blockIdx.x;
+  if (cta < gr.n_q + gr.n_k) {
+    const bool is_q = cta < gr.n_q;
+    const int64_t flat = (is_q ? cta : cta - gr.n_q) * 256 + threadIdx.x;
+    const int64_t per = is_q ? gr.per_group_q : gr.per_group_k;
+    const int64_t gi = flat / per;
+    if (gi < (is_q ? gr.groups_q : gr.groups_k)) quant_inner_slot<BLK>(is_q ? aq : ak, gi, (int)(flat - gi * per));
+    return;
+  }
+  const int half = threadIdx.x >> 7;
+  const int64_t ti = 2 * (cta - gr.n_q - gr.n_k) + half;
+  const bool valid = ti < gr.n_vtiles;
+  const int64_t per_g = gr.tok_tiles * gr.ch_tiles;
+  const int64_t gi = valid ? ti / per_g : 0, rem = valid ? ti - gi * per_g : 0;
+  float(*tile)[129] = reinterpret_cast<float(*)[129]>(qkv_tile + half * 64 * 129);
+  quant_outer_tile<BLK>(av, gi, rem / gr.ch_tiles, rem % gr.ch_tiles, threadIdx.x & 127, tile, valid);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -363,12 +425,12 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
     if (groups > 65535 || per_group > (int64_t)1 << 30 || rows > ((int64_t)1 << 30)) return FA4Q_ERR_UNSUPPORTED;
     dim3 grid((unsigned)((per_group + 255) / 256), (unsigned)groups);
     const int64_t mh = smooth_heads > 0 ? smooth_heads : 1, mr = smooth_ratio > 0 ? smooth_ratio : 1;
+    const InnerArgs ia{(const uint16_t*)x, rows, cols, row_stride, qm, g, smooth_mul, mh, mr, tiled,
+                       packed_out, scales_out};
     if (blk == 16)
-      quant_inner_kernel<16><<<grid, 256, 0, st>>>((const uint16_t*)x, rows, cols, row_stride, qm, g,
-                                                   smooth_mul, mh, mr, tiled, packed_out, scales_out);
+      quant_inner_kernel<16><<<grid, 256, 0, st>>>(ia);
     else
-      quant_inner_kernel<32><<<grid, 256, 0, st>>>((const uint16_t*)x, rows, cols, row_stride, qm, g,
-                                                   smooth_mul, mh, mr, tiled, packed_out, scales_out);
+      quant_inner_kernel<32><<<grid, 256, 0, st>>>(ia);
   } else {
     if (smooth_mul) return FA4Q_ERR_UNSUPPORTED;
     if (groups > 65535) return FA4Q_ERR_UNSUPPORTED;
@@ -376,12 +438,68 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
     const int64_t ch_tiles = tiled ? (cols + 127) / 128 * 2 : (cols + 63) / 64;
     dim3 grid((unsigned)((rows_pad + 127) / 128), (unsigned)ch_tiles, (unsigned)groups);
     if (grid.y > 65535) return FA4Q_ERR_UNSUPPORTED;
+    const OuterArgs oa{(const uint16_t*)x, rows, cols, row_stride, qm, g, tiled, packed_out, scales_out};
     if (blk == 16)
-      quant_outer_kernel<16><<<grid, 128, 0, st>>>((const uint16_t*)x, rows, cols, row_stride,
-                                                   qm, g, tiled, packed_out, scales_out);
+      quant_outer_kernel<16><<<grid, 128, 0, st>>>(oa);
     else
-      quant_outer_kernel<32><<<grid, 128, 0, st>>>((const uint16_t*)x, rows, cols, row_stride,
-                                                   qm, g, tiled, packed_out, scales_out);
+      quant_outer_kernel<32><<<grid, 128, 0, st>>>(oa);
+  }
+  return launch_status();
+}
+
+extern "C" fa4q_status fa4q_quantize_qkv(const void* q, const void* k, const void* v, int B, int Hq,
+                                         int Hkv, int S_q, int S_k, int d, fa4q_format fmt, float qmax,
+                                         float g_q, float g_k, float g_v, const float* mul_q,
+                                         const float* mul_k, uint8_t* q_packed, uint8_t* q_sf,
+                                         uint8_t* k_packed, uint8_t* k_sf, uint8_t* vt_packed,
+                                         uint8_t* vt_sf, void* stream) {
+  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (!q || !k || !v || !q_packed || !q_sf || !k_packed || !k_sf || !vt_packed || !vt_sf)
+    return FA4Q_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || S_q < 0 || S_k < 0) return FA4Q_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA4Q_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_packed) || !aligned16(k_packed) ||
+      !aligned16(vt_packed) || !aligned16(q_sf) || !aligned16(k_sf) || !aligned16(vt_sf) ||
+      (mul_q && !aligned16(mul_q)) || (mul_k && !aligned16(mul_k)))
+    return FA4Q_ERR_INVALID_ARG;
+  if (!(qmax >= 0.0f) || !isfinite(qmax)) return FA4Q_ERR_INVALID_ARG;
+  const bool nv = fmt == FA4Q_NVFP4;
+  if (!nv) g_q = g_k = g_v = 1.0f;
+  if (!(g_q > 0.0f) || !(g_k > 0.0f) || !(g_v > 0.0f) || !isfinite(g_q) || !isfinite(g_k) || !isfinite(g_v))
+    return FA4Q_ERR_INVALID_ARG;
+  if (B == 0 || (S_q == 0 && S_k == 0)) return FA4Q_OK;
+  const int blk = nv ? 16 : 32;
+  const float qm = (nv && qmax == 0.0f) ? 6.0f : qmax;
+  // inner (Q, K) slot spaces of the tiled layout, V tiles of 128 tokens x 64 channels
+  const int64_t ncol_sp = (d + 127) / 128 * (32 / blk) * 4;
+  QkvGrid gr;
+  gr.per_group_q = (static_cast<int64_t>(S_q) + 127) / 128 * 128 * ncol_sp;
+  gr.per_group_k = (static_cast<int64_t>(S_k) + 127) / 128 * 128 * ncol_sp;
+  gr.groups_q = static_cast<int64_t>(B) * Hq;
+  gr.groups_k = gr.groups_v = static_cast<int64_t>(B) * Hkv;
+  gr.n_q = S_q > 0 ? (gr.groups_q * gr.per_group_q + 255) / 256 : 0;
+  gr.n_k = S_k > 0 ? (gr.groups_k * gr.per_group_k + 255) / 256 : 0;
+  const int64_t rows_pad_v = (static_cast<int64_t>(S_k) + 31) / 32 * 32;
+  gr.tok_tiles = S_k > 0 ? (rows_pad_v + 127) / 128 : 0;
+  gr.ch_tiles = (d + 127) / 128 * 2;                  // tiled layout: channels padded to 128
+  gr.n_vtiles = gr.groups_v * gr.tok_tiles * gr.ch_tiles;
+  const int64_t n_ctas = gr.n_q + gr.n_k + (gr.n_vtiles + 1) / 2;
+  if (gr.per_group_q > ((int64_t)1 << 30) || gr.per_group_k > ((int64_t)1 << 30) || n_ctas > 0x7fffffff)
+    return FA4Q_ERR_UNSUPPORTED;
+  if (n_ctas == 0) return FA4Q_OK;
+  const InnerArgs aq{(const uint16_t*)q, S_q, d, d, qm, g_q, mul_q, Hq, Hq / Hkv, 1, q_packed, q_sf};
+  const InnerArgs ak{(const uint16_t*)k, S_k, d, d, qm, g_k, mul_k, Hkv, 1, 1, k_packed, k_sf};
+  const OuterArgs av{(const uint16_t*)v, S_k, d, d, qm, g_v, 1, vt_packed, vt_sf};
+  const int smem = 2 * 64 * 129 * static_cast<int>(sizeof(float));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (blk == 16) {
+    if (cudaFuncSetAttribute(quant_qkv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return FA4Q_ERR_CUDA;
+    quant_qkv_kernel<16><<<static_cast<unsigned>(n_ctas), 256, smem, st>>>(aq, ak, av, gr);
+  } else {
+    if (cudaFuncSetAttribute(quant_qkv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return FA4Q_ERR_CUDA;
+    quant_qkv_kernel<32><<<static_cast<unsigned>(n_ctas), 256, smem, st>>>(aq, ak, av, gr);
   }
   return launch_status();
 }

@@ -128,3 +128,35 @@ def test_full_size_long_prefill_tensors_bit_exact():
         rp, rs = F.quantize_cols_transposed(v, "nvfp4")
         assert np.array_equal(pv.cpu().numpy()[0], rp)
         assert np.array_equal(untile_sf(sv.cpu().numpy()[0], w.d, w.S, 16), rs)
+
+
+@pytest.mark.parametrize("fmt,d,S_q,S_k,Hq,Hkv,B,qmax,smooth,gs", [
+    ("mxfp4", 128, 300, 300, 8, 2, 1, 0.0, True, (1.0, 1.0, 1.0)),
+    ("nvfp4", 64, 129, 129, 4, 4, 2, 0.0, False, (0.5, 2.0, 0.25)),
+    ("mxfp4", 128, 200, 333, 4, 1, 1, 7.25, False, (1.0, 1.0, 1.0)),
+    ("nvfp4", 128, 4096, 4096, 32, 8, 1, 0.0, True, (1.0, 1.0, 1.0)),
+])
+def test_quantize_qkv_matches_separate_calls(fmt, d, S_q, S_k, Hq, Hkv, B, qmax, smooth, gs):
+    """The one-launch Q/K/V quantisation writes exactly the bytes of the three separate calls
+    (which the tests above pin bit-exactly to the oracle), padding bytes included."""
+    import torch
+    import microscaled_fp4_flashattention_b200 as fa4q
+    dev = torch.device("cuda:0")
+    rng = np.random.default_rng(S_q + S_k + d)
+    t = lambda shape: torch.from_numpy(synth.round_to_bf16(rng.normal(size=shape).astype(np.float32) * 2)
+                                       ).to(dev).to(torch.bfloat16)
+    q, k, v = t((B, Hq, S_q, d)), t((B, Hkv, S_k, d)), t((B, Hkv, S_k, d))
+    mq = mk = None
+    if smooth:
+        lam = np.exp2(rng.integers(-3, 4, size=(Hkv, d))).astype(np.float32)
+        mq = torch.from_numpy(lam).to(dev)
+        mk = torch.from_numpy((1.0 / lam).astype(np.float32)).to(dev)
+    g_q, g_k, g_v = gs
+    sep = (*fa4q.quantize(q, fmt, fa4q.FA4Q_AXIS_INNER, qmax, g_q, mq, Hq, Hq // Hkv),
+           *fa4q.quantize(k, fmt, fa4q.FA4Q_AXIS_INNER, qmax, g_k, mk, Hkv, 1),
+           *fa4q.quantize(v, fmt, fa4q.FA4Q_AXIS_OUTER, qmax, g_v))
+    fused = fa4q.quantize_qkv(q, k, v, fmt, qmax, g_q, g_k, g_v, mq, mk)
+    torch.cuda.synchronize()
+    for name, a, b in zip(("q", "q_sf", "k", "k_sf", "vt", "vt_sf"), sep, fused):
+        assert a.shape == b.shape, (name, a.shape, b.shape)
+        assert torch.equal(a, b), f"{name} differs"
