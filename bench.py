@@ -45,11 +45,12 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # The decode capture ran 8 of the 32 sequences: its traffic is per sequence (it grows with the
 # number of sequences) and is scaled to the timed batch.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,419,264 + 22,784 B (bench workload)
+    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,470,976 + 73,472 B (bench workload)
     "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
-                 "sha256": "7662871aa128626e7287f00aa3c7afcedd674d5510ec41f5508b2b8a312a8ed8",
-                 "bytes_per_launch": 13419264 + 22784},
+                 "sha256": "239aa1f4f1b754683e82aa1ceb156ee0272726ec94497101a6313bf6ad3cbe7c",
+                 "bytes_per_launch": 13470976 + 73472},
     # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,900,224 + 5,366,016 B for 8 sequences
+    # (taken before the MXFP4 page path was added to decode.cu: null until recaptured)
     "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
                "sha256": "3fae0c63206939932514f70e30ad22e4b951a7a02beed961c9a384b935120fdc",
                "bytes_per_sequence": 364266240 // 8},

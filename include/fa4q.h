@@ -206,8 +206,14 @@ size_t fa4q_decode_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, 
  * q        bf16 [B][Hq][d]; out bf16 [B][Hq][d].  d == 128, Hq % Hkv == 0, Hq/Hkv <= 8.
  * hp_k, hp_v  nullable bf16 [B][Hkv][max_hp][d]; hp_count int32 [B][Hkv] (<= max_hp).
  * win_k, win_v nullable bf16 [B][Hkv][W][d]; win_len int32 [B] (<= W).
- * g_k, g_v NVFP4 tensor scales of the pages (1 for MXFP4).  sm_scale 0 -> 1/sqrt(d).
+ * fmt      format of the pages, as written by fa4q_quantize_kv_pages: NVFP4 (K scales
+ *          [P][Hkv][64][8], V^T scales [P][Hkv][d][4]) or MXFP4 ([P][Hkv][64][4], [P][Hkv][d][2]).
+ * g_k, g_v NVFP4 tensor scales of the pages (ignored for MXFP4).  sm_scale 0 -> 1/sqrt(d).
  * workspace  device scratch of fa4q_decode_workspace_size bytes (caller-owned).
+ * Numerics: dequantised page values, q, the probabilities and the BF16 rows enter FP16
+ * tensor-core tiles (FP32 accumulation).  FP4 page values are exact there for any scale
+ * (MXFP4 block exponents are applied in FP32); q and the BF16 rows must lie within FP16's
+ * range (|x| <= 65504; magnitudes below 2^-14 lose precision).
  */
 fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
                         const uint8_t* vt_pages, const uint8_t* vt_sf,

@@ -52,6 +52,9 @@ constexpr int kRegsIssue = 56, kRegsSoftmax = 224;
 constexpr int kStages = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGpNvfp4 = 1.0f / 2688.0f;  // g_P = 1/(6*448), rounded to FP32
+// 1 / (6 g_P) in FP32: the P scale t = amax / (6 g_P) is taken as one multiply (t may differ
+// from the IEEE quotient by one ulp; amax itself comes from an approximate exponential)
+constexpr float kInvSixGp = 1.0f / (6.0f * kGpNvfp4);
 // polynomial 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [0, 1) (see ex2_poly2)
 constexpr float kExp2C0 = 0.9999252557754517f, kExp2C1 = 0.6958334445953369f;
 constexpr float kExp2C2 = 0.22606724500656128f, kExp2C3 = 0.07802451401948929f;
@@ -174,6 +177,15 @@ FA4Q_DEVINL float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// (x0, x1) *= (a, a) in one packed FP32 instruction
+FA4Q_DEVINL void fmul2_inplace(uint32_t& x0, uint32_t& x1, float a) {
+  asm("{\n\t.reg .b64 rx, ra;\n\t"
+      "mov.b64 rx, {%0, %1};\n\tmov.b64 ra, {%2, %2};\n\t"
+      "mul.rn.f32x2 rx, rx, ra;\n\tmov.b64 {%0, %1}, rx;\n\t}\n"
+      : "+r"(x0), "+r"(x1)
+      : "f"(a));
 }
 
 // (d0, d1) = (a0 * b0 + c0, a1 * b1 + c1) in one packed FP32 instruction
@@ -586,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           code = static_cast<uint32_t>(e + 127);
           off[bi] = amax > 0.0f ? mref + static_cast<float>(e) : INFINITY;
         } else {
-          const float t = __fdiv_rn(amax, 6.0f * kGpNvfp4);       // amax / (6 * g_P)
+          const float t = amax * kInvSixGp;                        // amax / (6 * g_P)
           code = ue4m3_encode(t);
           const float sf = ue4m3_decode(code);
           off[bi] = sf > 0.0f ? mref + lg2_approx(sf * kGpNvfp4) : INFINITY;
@@ -633,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) raw[c][i] = __float_as_uint(__uint_as_float(raw[c][i]) * alpha);
+            for (int i = 0; i < 32; i += 2) fmul2_inplace(raw[c][i], raw[c][i + 1], alpha);
             tmem_st32(lane_base + o_col + 32 * c, raw[c]);
           }
           tmem_st1(lane_base + l_col, __float_as_uint(__uint_as_float(lr) * alpha));

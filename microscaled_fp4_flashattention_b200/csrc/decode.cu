@@ -130,6 +130,10 @@ FA4Q_DEVINL float ex2f(float x) {
 // Work units of one (sequence, kv-head): FP4 pages (64 tokens) first, then 16-token slices
 // of the BF16 vertical-line set, then 16-token slices of the BF16 window.
 constexpr int kStageBytes = 9216;          // K page 4096 + K scales 512 + V^T page 4096 + scales 512
+// scale bytes of one page piece: 64 tokens x 8 (NVFP4) / 4 (MXFP4) blocks of K; 128 channels x
+// 4 / 2 blocks of V^T
+template <bool MX>
+__host__ __device__ constexpr uint32_t page_sf_bytes() { return MX ? 256u : 512u; }
 constexpr int kDecStages = 2;              // per-warp ring depth (2 x 9 KB: 3 CTAs per SM fit)
 
 struct UnitInfo {
@@ -157,16 +161,18 @@ FA4Q_DEVINL void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32
 }
 
 // Issue the copies of unit `u` into one ring stage (lane 0 only).
+template <bool MX>
 FA4Q_DEVINL void issue_unit(const DecParams& p, const UnitInfo& x, int b, int hk, int bh, int u,
                             uint8_t* stage, uint64_t* bar) {
   if (x.kind == 0) {
+    constexpr uint32_t sf = page_sf_bytes<MX>();
     const int64_t phys = p.table[(int64_t)b * p.max_pages + u];
     const int64_t ph = phys * p.Hkv + hk;
-    mbar_arrive_expect_tx(bar, kStageBytes);
+    mbar_arrive_expect_tx(bar, 2 * (4096 + sf));
     bulk_load(stage, p.kp + ph * 64 * (kDecD / 2), 4096, bar);
-    bulk_load(stage + 4096, p.ksf + ph * 64 * (kDecD / 16), 512, bar);
+    bulk_load(stage + 4096, p.ksf + ph * sf, sf, bar);
     bulk_load(stage + 4608, p.vp + ph * kDecD * 32, 4096, bar);
-    bulk_load(stage + 8704, p.vsf + ph * kDecD * 4, 512, bar);
+    bulk_load(stage + 8704, p.vsf + ph * sf, sf, bar);
   } else {
     const uint16_t* kb = x.kind == 1 ? p.hp_k + ((int64_t)bh * p.max_hp + x.base) * kDecD
                                      : p.win_k + ((int64_t)bh * p.W + x.base) * kDecD;
@@ -179,6 +185,20 @@ FA4Q_DEVINL void issue_unit(const DecParams& p, const UnitInfo& x, int b, int hk
   }
 }
 
+// f16x2 holding 2^rel twice (rel <= 0): exact down to the smallest subnormal 2^-24, zero below
+FA4Q_DEVINL uint32_t f16x2_pow2(int rel) {
+  const uint32_t h = rel >= -14 ? static_cast<uint32_t>(rel + 15) << 10 : (rel >= -24 ? 1u << (rel + 24) : 0u);
+  return h | (h << 16);
+}
+
+// largest of the four bytes of w
+FA4Q_DEVINL int max_byte4(uint32_t w) {
+  uint32_t m = __vmaxu4(w, w >> 16);
+  m = __vmaxu4(m, m >> 8);
+  return static_cast<int>(m & 0xFFu);
+}
+
+template <bool MX>
 __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const DecParams p) {
   extern __shared__ __align__(128) uint8_t dsm[];
   // [rings of all warps][mbarriers]; after the scan the rings are reused for the warp merge
@@ -236,8 +256,8 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
   int n_issued = 0;
   if (lane == 0) {
     for (int k = 0; k < kDecStages - 1 && u_issue < c_end; ++k) {
-      issue_unit(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
-                 ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
+      issue_unit<MX>(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
+                     ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
       ++n_issued;
       u_issue = next_valid(u_issue + kDecWarps);
     }
@@ -255,8 +275,8 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
     __syncwarp();
     if (ok && u_issue < c_end) {
       if (lane == 0)
-        issue_unit(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
-                   ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
+        issue_unit<MX>(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
+                       ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
       ++n_issued;
       u_issue = next_valid(u_issue + kDecWarps);
     }
@@ -283,16 +303,33 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
       // r+8 = that + 2; the PV reduction index k = 2t+e is token 16t + 4c + e and k = 2t+8+e
       // is 16t + 4c + 2 + e, so one 8-byte V^T load per channel covers all four chunks.
       nchunk = 4;
-      const float sc = p.sc_fp4;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int tlo = 16 * (g >> 1) + 4 * c + (g & 1), thi = tlo + 2;
         const uint4 klo = *reinterpret_cast<const uint4*>(st8 + tlo * 64 + 16 * t);
         const uint4 khi = *reinterpret_cast<const uint4*>(st8 + thi * 64 + 16 * t);
-        const uint32_t flo = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(st8 + 4096 + tlo * 8 + 2 * t));
-        const uint32_t fhi = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(st8 + 4096 + thi * 8 + 2 * t));
-        const uint32_t sla = __byte_perm(flo, 0, 0x1010), slb = __byte_perm(flo, 0, 0x3232);
-        const uint32_t sha = __byte_perm(fhi, 0, 0x1010), shb = __byte_perm(fhi, 0, 0x3232);
+        // Scales of this thread's dims 32t..32t+31.  NVFP4: two UE4M3 blocks, exact in FP16.
+        // MXFP4: one E8M0 block 2^(e-127); FP16 cannot hold every power of two, so the codes
+        // are scaled by 2^(e - E) with E the token's largest block exponent (exact down to
+        // 2^-24 below it) and the score by 2^(E-127) in FP32.
+        uint32_t sla, slb, sha, shb;
+        float sc_lo = p.sc_fp4, sc_hi = p.sc_fp4;
+        if constexpr (MX) {
+          const uint32_t wlo = *reinterpret_cast<const uint32_t*>(st8 + 4096 + tlo * 4);
+          const uint32_t whi = *reinterpret_cast<const uint32_t*>(st8 + 4096 + thi * 4);
+          const int elo = max_byte4(wlo), ehi = max_byte4(whi);
+          sla = slb = f16x2_pow2(static_cast<int>((wlo >> (8 * t)) & 0xFFu) - elo);
+          sha = shb = f16x2_pow2(static_cast<int>((whi >> (8 * t)) & 0xFFu) - ehi);
+          sc_lo *= exp2i(elo - 127);
+          sc_hi *= exp2i(ehi - 127);
+        } else {
+          const uint32_t flo = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(st8 + 4096 + tlo * 8 + 2 * t));
+          const uint32_t fhi = e4m3x2_to_f16x2(*reinterpret_cast<const uint16_t*>(st8 + 4096 + thi * 8 + 2 * t));
+          sla = __byte_perm(flo, 0, 0x1010);
+          slb = __byte_perm(flo, 0, 0x3232);
+          sha = __byte_perm(fhi, 0, 0x1010);
+          shb = __byte_perm(fhi, 0, 0x3232);
+        }
         const uint32_t wl[4] = {klo.x, klo.y, klo.z, klo.w}, wh[4] = {khi.x, khi.y, khi.z, khi.w};
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -304,10 +341,10 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
           mma_f16x4(acc, hmul2(la, sl), hmul2(ha, sh), hmul2(lb, sl), hmul2(hb, sh), qa[kc][0], qa[kc][1]);
         }
         const bool vl = (vmask >> tlo) & 1ull, vh = (vmask >> thi) & 1ull;
-        s4[c][0] = vl ? acc[0] * sc : -INFINITY;
-        s4[c][1] = vl ? acc[1] * sc : -INFINITY;
-        s4[c][2] = vh ? acc[2] * sc : -INFINITY;
-        s4[c][3] = vh ? acc[3] * sc : -INFINITY;
+        s4[c][0] = vl ? acc[0] * sc_lo : -INFINITY;
+        s4[c][1] = vl ? acc[1] * sc_lo : -INFINITY;
+        s4[c][2] = vh ? acc[2] * sc_hi : -INFINITY;
+        s4[c][3] = vh ? acc[3] * sc_hi : -INFINITY;
       }
     } else {
       // BF16 slice of 16 tokens in natural order: score rows g and g+8 are tokens g and g+8;
@@ -381,14 +418,39 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
         const int cha = 16 * ct + g, chb = cha + 8;
         const uint2 va = *reinterpret_cast<const uint2*>(st8 + 4608 + cha * 32 + 8 * t);
         const uint2 vb = *reinterpret_cast<const uint2*>(st8 + 4608 + chb * 32 + 8 * t);
-        const uint32_t fa = st8[8704 + cha * 4 + t], fb = st8[8704 + chb * 4 + t];
-        const uint32_t sa = e4m3x2_to_f16x2(fa | (fa << 8)), sb = e4m3x2_to_f16x2(fb | (fb << 8));
+        if constexpr (MX) {
+          // this thread's tokens 16t..16t+15 lie in the channel's 32-token block t/2; the
+          // codes take 2^(e - F), F the larger of the page's two block exponents, and the
+          // page's products are added to O scaled by 2^(F-127) in FP32
+          const uint32_t ea = *reinterpret_cast<const uint16_t*>(st8 + 8704 + cha * 2);
+          const uint32_t eb = *reinterpret_cast<const uint16_t*>(st8 + 8704 + chb * 2);
+          const int Fa = max(static_cast<int>(ea & 0xFFu), static_cast<int>(ea >> 8));
+          const int Fb = max(static_cast<int>(eb & 0xFFu), static_cast<int>(eb >> 8));
+          const uint32_t sa = f16x2_pow2(static_cast<int>((ea >> (8 * (t >> 1))) & 0xFFu) - Fa);
+          const uint32_t sb = f16x2_pow2(static_cast<int>((eb >> (8 * (t >> 1))) & 0xFFu) - Fb);
+          float pg[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t la, ha, lb, hb;
-          e2m1x4_to_f16x2x2((c >> 1 ? va.y : va.x) >> ((c & 1) * 16), la, ha);
-          e2m1x4_to_f16x2x2((c >> 1 ? vb.y : vb.x) >> ((c & 1) * 16), lb, hb);
-          mma_f16x4(o[ct], hmul2(la, sa), hmul2(lb, sb), hmul2(ha, sa), hmul2(hb, sb), pb0[c], pb1[c]);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t la, ha, lb, hb;
+            e2m1x4_to_f16x2x2((c >> 1 ? va.y : va.x) >> ((c & 1) * 16), la, ha);
+            e2m1x4_to_f16x2x2((c >> 1 ? vb.y : vb.x) >> ((c & 1) * 16), lb, hb);
+            mma_f16x4(pg, hmul2(la, sa), hmul2(lb, sb), hmul2(ha, sa), hmul2(hb, sb), pb0[c], pb1[c]);
+          }
+          const float xa = exp2i(Fa - 127), xb = exp2i(Fb - 127);
+          o[ct][0] = fmaf(pg[0], xa, o[ct][0]);
+          o[ct][1] = fmaf(pg[1], xa, o[ct][1]);
+          o[ct][2] = fmaf(pg[2], xb, o[ct][2]);
+          o[ct][3] = fmaf(pg[3], xb, o[ct][3]);
+        } else {
+          const uint32_t fa = st8[8704 + cha * 4 + t], fb = st8[8704 + chb * 4 + t];
+          const uint32_t sa = e4m3x2_to_f16x2(fa | (fa << 8)), sb = e4m3x2_to_f16x2(fb | (fb << 8));
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t la, ha, lb, hb;
+            e2m1x4_to_f16x2x2((c >> 1 ? va.y : va.x) >> ((c & 1) * 16), la, ha);
+            e2m1x4_to_f16x2x2((c >> 1 ? vb.y : vb.x) >> ((c & 1) * 16), lb, hb);
+            mma_f16x4(o[ct], hmul2(la, sa), hmul2(lb, sb), hmul2(ha, sa), hmul2(hb, sb), pb0[c], pb1[c]);
+          }
         }
       }
     } else {
@@ -537,7 +599,6 @@ extern "C" fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const 
                                    float g_v, float sm_scale, void* out, void* workspace,
                                    size_t workspace_bytes, int num_splits, void* stream) {
   if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
-  if (fmt == FA4Q_MXFP4) return FA4Q_ERR_UNSUPPORTED;
   if (!q || !out || !fp4_len || !workspace) return FA4Q_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return FA4Q_ERR_INVALID_ARG;
   if (Hq / Hkv > 8) return FA4Q_ERR_UNSUPPORTED;
@@ -549,7 +610,8 @@ extern "C" fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const 
   if (W > 0 && (!win_k || !win_v || !win_len)) return FA4Q_ERR_INVALID_ARG;
   if (!(g_k > 0.0f) || !(g_v > 0.0f)) return FA4Q_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || (k_pages && !aligned16(k_pages)) ||
-      (vt_pages && !aligned16(vt_pages)) || (hp_k && !aligned16(hp_k)) ||
+      (vt_pages && !aligned16(vt_pages)) || (k_sf && !aligned16(k_sf)) ||
+      (vt_sf && !aligned16(vt_sf)) || (hp_k && !aligned16(hp_k)) ||
       (hp_v && !aligned16(hp_v)) || (win_k && !aligned16(win_k)) || (win_v && !aligned16(win_v)) ||
       !aligned16(workspace))
     return FA4Q_ERR_INVALID_ARG;
@@ -581,6 +643,8 @@ extern "C" fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const 
   p.max_hp = max_hp;
   p.W = W;
   const float sms = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)d);
+  const bool mx = fmt == FA4Q_MXFP4;
+  if (mx) g_k = g_v = 1.0f;                       // MXFP4 pages carry no tensor scale
   p.sc_fp4 = sms * g_k * kDecLog2e;
   p.sc_bf16 = sms * kDecLog2e;
   p.g_v = g_v;
@@ -593,10 +657,10 @@ extern "C" fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const 
   p.out = static_cast<uint16_t*>(out);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   dim3 grid(splits, Hkv, B);
-  if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kDecSmem) != cudaSuccess)
+  auto kern = mx ? decode_split_kernel<true> : decode_split_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecSmem) != cudaSuccess)
     return FA4Q_ERR_CUDA;
-  decode_split_kernel<<<grid, kDecWarps * 32, kDecSmem, st>>>(p);
+  kern<<<grid, kDecWarps * 32, kDecSmem, st>>>(p);
   const int rows = B * Hq;
   decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(p.ws, rows, splits, p.out);
   return launch_status();

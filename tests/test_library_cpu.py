@@ -68,10 +68,9 @@ def test_argument_errors_without_gpu(L):
     assert L.fa4q_attn_fwd(*args, 1, 4, 4, 128, 128, 96, 0, F(0), 0, F(0), fake, 1, None, None) == 2
     assert L.fa4q_attn_fwd(*args, 1, 6, 4, 128, 128, 128, 0, F(0), 0, F(0), fake, 1, None, None) == 1
     assert L.fa4q_attn_fwd(*args, 1, 4, 4, 128, 256, 128, 0, F(0), 1, F(0), fake, 1, None, None) == 1
-    # decode: group too large, MXFP4 not yet supported, workspace too small
+    # decode: group too large, workspace too small
     dargs = [fake] * 14
     assert L.fa4q_decode(*dargs, 1, 32, 2, 128, 4, 0, 0, 0, F(1), F(1), F(0), fake, fake, 1 << 30, 0, None) == 2
-    assert L.fa4q_decode(*dargs, 1, 8, 2, 128, 4, 0, 0, 1, F(1), F(1), F(0), fake, fake, 1 << 30, 0, None) == 2
     assert L.fa4q_decode(*dargs, 1, 8, 2, 128, 4, 0, 0, 0, F(1), F(1), F(0), fake, fake, 16, 0, None) == 1
     # selftest: bad shapes
     assert L.fa4q_selftest_block_mma(fake, fake, fake, fake, 24, 64, 0, fake, None) == 2
