@@ -164,6 +164,43 @@ fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, const uint8_t* 
                           float sm_scale, void* out, int out_is_fp32, float* lse, void* stream);
 
 /*
+ * fa4q_attn_fwd_ex - fa4q_attn_fwd with two ablations of the method (fa4q_attn_fwd is this
+ * call with rescale_tau = 0 and l_from_ptilde = 0).
+ *
+ * 1. Conditional rescaling (rescale_tau > 0).
+ * Source: the FlashAttention-4 abstract on the FLAMIA page names conditional softmax
+ * rescaling among its Blackwell techniques; the pages give no rule.  Here: the reference
+ * maximum m of a query row moves to a key tile's maximum only when that maximum exceeds m
+ * by more than rescale_tau binades, so the unnormalised exponentials P~ = exp(s - m) reach
+ * up to 2^rescale_tau and the O/l accumulators are rescaled only when m moves.  P~ is then
+ * quantised exactly as before (PNQ against the reference m; the MXFP4 block exponents absorb
+ * P~ > 1).  P_hat therefore differs from the exact-maximum result (the output stays a convex
+ * combination of V_hat).
+ *
+ * rescale_tau  integer in [0, 30]; anything else -> FA4Q_ERR_INVALID_ARG.  rescale_tau > 0
+ *              with NVFP4 -> FA4Q_ERR_UNSUPPORTED: a key whose score equals a kept
+ *              reference gets P~ = 1, i.e. y = 1/(s g_P 2^tau), an exact E2M1 tie for some
+ *              UE4M3 scales s that the kernel's exponential form cannot reproduce; with
+ *              MXFP4 that value is 2^-e, formed exactly from the score difference.
+ *
+ * 2. The inconsistent normaliser (l_from_ptilde = 1).  Source: HiFA4, Abstract - the
+ * normaliser accumulated from the unquantised exponentials while the numerator uses P_hat
+ * gives a coherent output-scaling error with net mass loss, which P-Reordering removes.
+ * Here the softmax threads sum P~ in FP32 (per tile, rescaled like O) and the epilogue divides
+ * by that sum; the PV product is unchanged, so each output row is the P-Reordering output
+ * times sum P_hat / sum P~ (the LSE, when asked for, uses the same sum).
+ * l_from_ptilde  0 or 1; anything else -> FA4Q_ERR_INVALID_ARG.
+ *
+ * All other arguments, layouts and errors as fa4q_attn_fwd.
+ */
+fa4q_status fa4q_attn_fwd_ex(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                             const uint8_t* k_sf, const uint8_t* vt, const uint8_t* vt_sf,
+                             float g_q, float g_k, float g_v, int B, int Hq, int Hkv, int S_q,
+                             int S_k, int d, fa4q_format fmt, float qmax_p, int causal,
+                             float sm_scale, int rescale_tau, int l_from_ptilde, void* out,
+                             int out_is_fp32, float* lse, void* stream);
+
+/*
  * Paged FP4 KV cache (BitDecoding-FP4, "System-Level Optimization": fixed-size token
  * blocks mapped to physical memory through a block table).  Page size 64 tokens.
  * For physical page p and kv-head h:

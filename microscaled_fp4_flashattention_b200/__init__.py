@@ -24,7 +24,7 @@ STATUS = {0: "FA4Q_OK", 1: "FA4Q_ERR_INVALID_ARG", 2: "FA4Q_ERR_UNSUPPORTED", 3:
 
 EXPORTED = [
     "fa4q_status_string", "fa4q_version", "fa4q_sf_tiled_bytes", "fa4q_quantize",
-    "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_quantize_kv_pages",
+    "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_attn_fwd_ex", "fa4q_quantize_kv_pages",
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
     "fa4q_vlines_workspace_size", "fa4q_select_vertical_lines", "fa4q_quantize_qkv",
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.fa4q_smooth_calibrate.argtypes = [P, P, I, I, I, I, P, P, P]
         L.fa4q_attn_fwd.restype = I
         L.fa4q_attn_fwd.argtypes = [P, P, P, P, P, P, F, F, F, I, I, I, I, I, I, I, F, I, F, P, I, P, P]
+        L.fa4q_attn_fwd_ex.restype = I
+        L.fa4q_attn_fwd_ex.argtypes = [P, P, P, P, P, P, F, F, F, I, I, I, I, I, I, I, F, I, F, I, I, P, I, P, P]
         L.fa4q_quantize_kv_pages.restype = I
         L.fa4q_quantize_kv_pages.argtypes = [P, P, I, I, I, I, P, P, P, I, I, F, F, P, P, P, P, P]
         L.fa4q_decode_workspace_size.restype = Z
@@ -167,12 +169,20 @@ def smooth_calibrate(q_cal, k_cal, stream=None):
 
 def attn_fwd(q, q_sf, k, k_sf, vt, vt_sf, *, B, Hq, Hkv, S_q, S_k, d, fmt, causal,
              g_q=1.0, g_k=1.0, g_v=1.0, qmax_p=0.0, sm_scale=0.0, out=None, out_fp32=False,
-             lse=None, stream=None):
-    """Prefill attention on quantised operands; returns out [B, Hq, S_q, d]."""
+             lse=None, rescale_tau=0, l_from_ptilde=False, stream=None):
+    """Prefill attention on quantised operands; returns out [B, Hq, S_q, d].
+    rescale_tau > 0 (conditional rescaling) or l_from_ptilde (the inconsistent normaliser)
+    select the ablations of fa4q_attn_fwd_ex."""
     import torch
     if out is None:
         out = torch.empty((B, Hq, S_q, d), dtype=torch.float32 if out_fp32 else torch.bfloat16,
                           device=q.device)
+    if rescale_tau or l_from_ptilde:
+        _check("fa4q_attn_fwd_ex", lib().fa4q_attn_fwd_ex(
+            _ptr(q), _ptr(q_sf), _ptr(k), _ptr(k_sf), _ptr(vt), _ptr(vt_sf), g_q, g_k, g_v, B, Hq, Hkv,
+            S_q, S_k, d, _fmt(fmt), qmax_p, int(causal), sm_scale, int(rescale_tau), int(l_from_ptilde),
+            _ptr(out), int(out_fp32), _ptr(lse), _stream(stream)))
+        return out
     _check("fa4q_attn_fwd", lib().fa4q_attn_fwd(
         _ptr(q), _ptr(q_sf), _ptr(k), _ptr(k_sf), _ptr(vt), _ptr(vt_sf), g_q, g_k, g_v, B, Hq, Hkv,
         S_q, S_k, d, _fmt(fmt), qmax_p, int(causal), sm_scale, _ptr(out), int(out_fp32), _ptr(lse),

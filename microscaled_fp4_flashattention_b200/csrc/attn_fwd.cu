@@ -106,6 +106,7 @@ struct __align__(1024) Smem {
   uint64_t drain;
   float m_xchg[2][kBM];       // running maximum after tile j, slot j%2, per row
   float m_last[2][kBM];       // per group: the maximum its accumulator is relative to
+  float l_last[2][kBM];       // per group: the normaliser summed from P~ (ablation only)
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -122,6 +123,20 @@ struct AttnParams {
   float score_scale_log2;  // sm_scale * g_q * g_k * log2(e)
   float g_v;
   float qmax_p;
+  // Conditional rescaling (FlashAttention-4, as named in the FLAMIA page's abstract): the
+  // reference maximum moves only when a tile's maximum exceeds it by more than tau binades
+  // (tau = 0: the exact running maximum).  NVFP4 P then takes the tensor scale
+  // gp = g_P * 2^tau, and the P scale t = amax / (6 gp) is one multiply by inv6gp (t may
+  // differ from the IEEE quotient by one ulp; amax itself comes from an approximate
+  // exponential).
+  float tau;
+  float gp;
+  float inv6gp;
+  // Ablation of P-Reordering (HiFA4, Abstract): 1 takes the normaliser from the unquantised
+  // exponentials P~ (summed in FP32 by the softmax threads) instead of from the P_hat that
+  // feeds the PV product; the numerator is unchanged, so each output row is scaled by
+  // sum P_hat / sum P~.
+  int l_from_ptilde;
   int causal;
   int out_fp32;
 };
@@ -290,7 +305,9 @@ FA4Q_DEVINL void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, int N
   }
 }
 
-template <int D, bool MX, bool CAUSAL, bool PERSIST>
+// ABL: the ablations of fa4q_attn_fwd_ex (conditional rescaling, normaliser from P~) are
+// compiled into separate instantiations so the default kernel carries none of their work.
+template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -541,6 +558,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = qt * kBM + r;                  // query index
     const int done_g = g ? done_b : done_a;
     float m_acc = -INFINITY;                       // maximum of this group's last tile
+    float lpt = 0.0f;                              // sum of P~ of this group (ABL), MMA units
+    const float gp_item = ABL ? p.gp : kGpNvfp4;
     for (int j = g; j < n_tiles; j += 2) {
       ok = warp_wait(&sm.s_full[g], (done_g + (j >> 1)) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       tc_fence_after();
@@ -580,12 +599,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         named_bar_sync(bar_recv, 64);
         m_prev = sm.m_xchg[(j - 1) & 1][r];
       }
-      const float m_new = fmaxf(m_prev, tmax);
+      float m_new = fmaxf(m_prev, tmax);
+      if constexpr (ABL) {
+        const bool grow = !(m_prev > -INFINITY) || (tmax - m_prev) * sc > p.tau;
+        if (!grow) m_new = m_prev;
+      }
       sm.m_xchg[j & 1][r] = m_new;
       named_bar_arrive(bar_send, 64);
       const float mref = m_new * sc;
       // per block: amax = exp2((bmax - m)*sc); scale; y_i = exp2(s_i*sc - m*sc - log2(scale))
-      float off[kNB];
+      float lsc[kNB];                              // log2 of each block's scale (+inf: zero block)
+      const float gp = ABL ? p.gp : kGpNvfp4, inv6gp = ABL ? p.inv6gp : kInvSixGp;
       uint32_t sfw[kNB / 4];
 #pragma unroll
       for (int w = 0; w < kNB / 4; ++w) sfw[w] = 0;
@@ -596,27 +620,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (MX) {
           const int e = mx_exponent(amax, p.qmax_p);
           code = static_cast<uint32_t>(e + 127);
-          off[bi] = amax > 0.0f ? mref + static_cast<float>(e) : INFINITY;
+          lsc[bi] = amax > 0.0f ? static_cast<float>(e) : INFINITY;
         } else {
-          const float t = amax * kInvSixGp;                        // amax / (6 * g_P)
+          const float t = amax * inv6gp;                           // amax / (6 * gp)
           code = ue4m3_encode(t);
           const float sf = ue4m3_decode(code);
-          off[bi] = sf > 0.0f ? mref + lg2_approx(sf * kGpNvfp4) : INFINITY;
+          lsc[bi] = sf > 0.0f ? lg2_approx(sf * gp) : INFINITY;
         }
         sfw[bi >> 2] |= code << (8 * (bi & 3));
       }
       uint32_t packed[kBN / 8];
+      auto quantise_row = [&](auto exponent_argument, auto observe) {
 #pragma unroll
-      for (int g8 = 0; g8 < kBN / 8; ++g8) {
-        const float o8 = off[(g8 * 8) / C::kBlk];
-        float y[8];
+        for (int g8 = 0; g8 < kBN / 8; ++g8) {
+          const float l8 = lsc[(g8 * 8) / C::kBlk];
+          float y[8];
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) ffma2(y[i], y[i + 1], s[8 * g8 + i], s[8 * g8 + i + 1], sc, sc, -o8, -o8);
+          for (int i = 0; i < 8; i += 2) exponent_argument(y[i], y[i + 1], s[8 * g8 + i], s[8 * g8 + i + 1], l8);
 #pragma unroll
-        for (int i = 0; i < kEmulPer8; i += 2) ex2_poly2(y[i], y[i + 1], y[i], y[i + 1]);
+          for (int i = 0; i < kEmulPer8; i += 2) ex2_poly2(y[i], y[i + 1], y[i], y[i + 1]);
 #pragma unroll
-        for (int i = kEmulPer8; i < 8; ++i) y[i] = ex2_approx(y[i]);
-        packed[g8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+          for (int i = kEmulPer8; i < 8; ++i) y[i] = ex2_approx(y[i]);
+          observe(g8, y);
+          packed[g8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+        }
+      };
+      auto no_observer = [](int, const float*) {};
+      auto standard_argument = [&](float& y0, float& y1, float s0, float s1, float l8) {
+        const float o8 = mref + l8;
+        ffma2(y0, y1, s0, s1, sc, sc, -o8, -o8);
+      };
+      float ysum[ABL ? kNB : 1];
+      if constexpr (!ABL) {
+        quantise_row(standard_argument, no_observer);
+      } else {
+        // scaled exponentials of the whole row for the P~ normaliser: per block, (sum of y)
+        // times the block's scale in MMA units (2^e for MXFP4, the UE4M3 value for NVFP4)
+#pragma unroll
+        for (int bi = 0; bi < kNB; ++bi) ysum[bi] = 0.0f;
+        auto sum_observer = [&](int g8, const float* y) {
+          ysum[(g8 * 8) / C::kBlk] += ((y[0] + y[1]) + (y[2] + y[3])) + ((y[4] + y[5]) + (y[6] + y[7]));
+        };
+        if (p.tau > 0.0f) {
+          // Reference kept from an earlier tile: a key whose score equals it has P~ = 1 in a
+          // block whose scale is 2^e, e possibly 2, so y = 2^-e may sit exactly on the E2M1
+          // tie 0.25.  The argument is formed from the exact difference s - m, so such a key
+          // gets exactly -e (2^-2 from MUFU, or just below from the polynomial: both round to
+          // 0 like the tie itself).
+          const float mn = m_new;
+          auto exact_argument = [&](float& y0, float& y1, float s0, float s1, float l8) {
+            ffma2(y0, y1, s0, s1, 1.0f, 1.0f, -mn, -mn);
+            ffma2(y0, y1, y0, y1, sc, sc, -l8, -l8);
+          };
+          if (p.l_from_ptilde) quantise_row(exact_argument, sum_observer);
+          else quantise_row(exact_argument, no_observer);
+        } else {
+          quantise_row(standard_argument, sum_observer);
+        }
       }
       // accumulator g and P buffer g were last used by this group's previous PV product
       if (j >= 2)
@@ -631,6 +691,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint32_t*>(sm.sfp[g] + 512 * a + (r & 31) * 16 + (r >> 5) * 4) = sfw[a];
       fence_proxy_async_smem();
       // bring accumulator g from the maximum it holds (tile j-2) to m_j
+      if (ABL && p.l_from_ptilde) {
+        float add = 0.0f;
+#pragma unroll
+        for (int bi = 0; bi < kNB; ++bi) {
+          const uint32_t code = (sfw[bi >> 2] >> (8 * (bi & 3))) & 0xFFu;
+          const float scale = MX ? exp2i(static_cast<int>(code) - 127) : ue4m3_decode(code);
+          add += ysum[bi] * scale;
+        }
+        lpt = (j >= 2 ? lpt * ex2_approx((m_acc - m_new) * sc) : 0.0f) + add;
+      }
       if (j >= 2) {
         tc_fence_after();
         const float alpha = ex2_approx((m_acc - m_new) * sc);
@@ -664,6 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // out = (O_A 2^((mA - m) sc) + O_B 2^((mB - m) sc)) / (l_A ... + l_B ...) * g_v with m the
     // final maximum; group A writes output columns [0, D/2), group B [D/2, D)
     sm.m_last[g][r] = m_acc;
+    if constexpr (ABL) sm.l_last[g][r] = lpt;
     named_bar_sync(bar_epi, 64);
     const float mA = sm.m_last[0][r], mB = sm.m_last[1][r];
     const float m = fmaxf(mA, mB);
@@ -687,7 +758,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(lane_base + kColO1 + g * (D / 2) + 32 * c, rawb[c]);
       }
       tmem_wait_ld();
-      const float l = __uint_as_float(lra) * wa + (has_b ? __uint_as_float(lrb) * wb : 0.0f);
+      const float la = (ABL && p.l_from_ptilde) ? sm.l_last[0][r] : __uint_as_float(lra);
+      const float lb = (ABL && p.l_from_ptilde) ? sm.l_last[1][r] : __uint_as_float(lrb);
+      const float l = la * wa + (has_b ? lb * wb : 0.0f);
       const float inva = p.g_v / l * wa, invb = p.g_v / l * wb;
       const bool store = row < p.S_q;
       const int64_t orow = (int64_t)bh_q * p.S_q + row;
@@ -718,7 +791,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (g == 0 && p.lse != nullptr) {
-          const float lscale = MX ? 1.0f : kGpNvfp4;
+          const float lscale = MX ? 1.0f : gp_item;
           p.lse[orow] = m * sc * 0.69314718055994531f + logf(l * lscale);
         }
       }
@@ -896,7 +969,7 @@ static bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool MX, bool CAUSAL>
+template <int D, bool MX, bool CAUSAL, bool ABL = false>
 static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t* vt,
                                const AttnParams& prm, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
@@ -915,7 +988,7 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
   const int n_ktiles = (prm.S_k + kBN - 1) / kBN;
   const double avg_tiles = CAUSAL ? 0.5 * (std::min(prm.n_qtiles, n_ktiles) + 1) : n_ktiles;
   const bool persist = avg_tiles <= 48.0 && prm.n_items > num_sms();
-  auto kern = persist ? attn_fwd_kernel<D, MX, CAUSAL, true> : attn_fwd_kernel<D, MX, CAUSAL, false>;
+  auto kern = persist ? attn_fwd_kernel<D, MX, CAUSAL, true, ABL> : attn_fwd_kernel<D, MX, CAUSAL, false, ABL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return FA4Q_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>(persist ? num_sms() : prm.n_items));
@@ -927,13 +1000,19 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
 
 using namespace fa4q;
 
-extern "C" fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
-                                     const uint8_t* k_sf, const uint8_t* vt, const uint8_t* vt_sf,
-                                     float g_q, float g_k, float g_v, int B, int Hq, int Hkv,
-                                     int S_q, int S_k, int d, fa4q_format fmt, float qmax_p,
-                                     int causal, float sm_scale, void* out, int out_is_fp32,
-                                     float* lse, void* stream) {
+extern "C" fa4q_status fa4q_attn_fwd_ex(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                        const uint8_t* k_sf, const uint8_t* vt, const uint8_t* vt_sf,
+                                        float g_q, float g_k, float g_v, int B, int Hq, int Hkv,
+                                        int S_q, int S_k, int d, fa4q_format fmt, float qmax_p,
+                                        int causal, float sm_scale, int rescale_tau,
+                                        int l_from_ptilde, void* out, int out_is_fp32, float* lse,
+                                        void* stream) {
   if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (rescale_tau < 0 || rescale_tau > 30) return FA4Q_ERR_INVALID_ARG;
+  if (l_from_ptilde != 0 && l_from_ptilde != 1) return FA4Q_ERR_INVALID_ARG;
+  // NVFP4 P under a kept reference: a key equal to the reference lands on 1/(s g_P 2^tau),
+  // an E2M1 tie for some UE4M3 s, which the exponential form cannot reproduce exactly
+  if (rescale_tau > 0 && fmt == FA4Q_NVFP4) return FA4Q_ERR_UNSUPPORTED;
   if (!q || !q_sf || !k || !k_sf || !vt || !vt_sf || !out) return FA4Q_ERR_INVALID_ARG;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || S_q < 0 || S_k < 0) return FA4Q_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FA4Q_ERR_INVALID_ARG;
@@ -967,16 +1046,35 @@ extern "C" fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, cons
   prm.score_scale_log2 = sms * g_q * g_k * kLog2e;
   prm.g_v = g_v;
   prm.qmax_p = qmax_p;
+  prm.tau = static_cast<float>(rescale_tau);
+  prm.gp = kGpNvfp4 * static_cast<float>(1u << rescale_tau);     // exact power-of-two multiple
+  prm.inv6gp = 1.0f / (6.0f * prm.gp);
+  prm.l_from_ptilde = l_from_ptilde;
   prm.causal = causal;
   prm.out_fp32 = out_is_fp32;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool mx = fmt == FA4Q_MXFP4;
+  if (rescale_tau > 0 || l_from_ptilde) {
+    if (d != 128) return FA4Q_ERR_UNSUPPORTED;   // the ablation kernels are built for d = 128
+    if (mx) return causal ? launch_attn<128, true, true, true>(q, k, vt, prm, st) : launch_attn<128, true, false, true>(q, k, vt, prm, st);
+    return causal ? launch_attn<128, false, true, true>(q, k, vt, prm, st) : launch_attn<128, false, false, true>(q, k, vt, prm, st);
+  }
   if (d == 128) {
     if (mx) return causal ? launch_attn<128, true, true>(q, k, vt, prm, st) : launch_attn<128, true, false>(q, k, vt, prm, st);
     return causal ? launch_attn<128, false, true>(q, k, vt, prm, st) : launch_attn<128, false, false>(q, k, vt, prm, st);
   }
   if (mx) return causal ? launch_attn<64, true, true>(q, k, vt, prm, st) : launch_attn<64, true, false>(q, k, vt, prm, st);
   return causal ? launch_attn<64, false, true>(q, k, vt, prm, st) : launch_attn<64, false, false>(q, k, vt, prm, st);
+}
+
+extern "C" fa4q_status fa4q_attn_fwd(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
+                                     const uint8_t* k_sf, const uint8_t* vt, const uint8_t* vt_sf,
+                                     float g_q, float g_k, float g_v, int B, int Hq, int Hkv,
+                                     int S_q, int S_k, int d, fa4q_format fmt, float qmax_p,
+                                     int causal, float sm_scale, void* out, int out_is_fp32,
+                                     float* lse, void* stream) {
+  return fa4q_attn_fwd_ex(q, q_sf, k, k_sf, vt, vt_sf, g_q, g_k, g_v, B, Hq, Hkv, S_q, S_k, d, fmt,
+                          qmax_p, causal, sm_scale, 0, 0, out, out_is_fp32, lse, stream);
 }
 
 extern "C" fa4q_status fa4q_selftest_block_mma(const uint8_t* a, const uint8_t* a_sf, const uint8_t* b,

@@ -35,6 +35,20 @@ exact at every tile (no conditional rescale); P is quantised against the
 current m_new; the P scale decision is taken in FP32 like the tensors';
 sm_scale = 1/sqrt(d); masked keys are exact zeros inside their P blocks;
 causal attention is top-left aligned (query i sees keys <= i).
+
+Variant (an ablation, off by default): conditional rescaling with a threshold tau
+(an integer number of binades), the FlashAttention-4 technique named in the
+FLAMIA page's FlashAttention-4 abstract.  The reference m is kept while a tile's
+maximum stays within tau binades above it, so p~ = exp(s - m) may reach 2^tau:
+
+        tmax = max_{j in T} s_j
+        if m = -inf or (tmax - m) * log2(e) > tau:  m_new = max(m, tmax)
+        else:                                       m_new = m
+        (then as above, against m_new)
+
+The MXFP4 P scale absorbs p~ > 1 unchanged; the NVFP4 P tensor scale becomes
+g_P * 2^tau so that UE4M3 still spans the block maxima.  tau = 0 is the exact
+running maximum above.
 """
 from __future__ import annotations
 
@@ -46,15 +60,17 @@ BC = 128
 G_P_NVFP4 = float(np.float32(1.0 / (6.0 * 448.0)))
 
 
-def p_tensor_scale(fmt: str) -> float:
-    return G_P_NVFP4 if fmt == "nvfp4" else 1.0
+def p_tensor_scale(fmt: str, tau: int = 0) -> float:
+    """Second-level FP32 scale of P: g_P = fl32(1/(6*448)) for NVFP4, times 2^tau under
+    conditional rescaling (exact: a power-of-two multiple); 1 for MXFP4."""
+    return G_P_NVFP4 * 2.0 ** int(tau) if fmt == "nvfp4" else 1.0
 
 
-def quantize_p(p32: np.ndarray, fmt: str, qmax_p: float = 0.0) -> np.ndarray:
+def quantize_p(p32: np.ndarray, fmt: str, qmax_p: float = 0.0, tau: int = 0) -> np.ndarray:
     """FP64 dequantised P_hat of FP32 exponentials p32 [R, BC], blocks along keys."""
     blk = formats.block_size(fmt)
     R, W = p32.shape
-    g = p_tensor_scale(fmt)
+    g = p_tensor_scale(fmt, tau)
     codes, s = formats.quantize_blocks(p32.reshape(R, W // blk, blk), fmt,
                                        qmax_p if fmt == "mxfp4" else 0.0, g)
     return formats.dequantize_blocks(codes, s, fmt, g).reshape(R, W)
@@ -63,7 +79,7 @@ def quantize_p(p32: np.ndarray, fmt: str, qmax_p: float = 0.0) -> np.ndarray:
 def attention_pnq(qhat, khat, vhat, *, causal: bool, fmt: str, qmax_p: float = 0.0,
                   sm_scale: float | None = None, rows=None, consistent: bool = True,
                   return_weights: bool = False, return_lse: bool = False, return_eps: bool = False,
-                  p_quantizer=None):
+                  p_quantizer=None, rescale_tau: int = 0):
     """Tiled PNQ attention for one (batch, head) on dequantised operands.
 
     qhat [Sq, d], khat/vhat [Sk, d] (FP64).  `rows` selects query rows (default all).
@@ -71,7 +87,11 @@ def attention_pnq(qhat, khat, vhat, *, causal: bool, fmt: str, qmax_p: float = 0
     (the HiFA4 'inconsistent' variant, a diagnostic).  Optional extras:
     the effective key weights (P_hat rescaled to the final maximum, divided by l),
     the log-sum-exp m + ln(l) and the per-tile mass ratio eps = sum p^ / sum p~ - 1.
-    `p_quantizer(p32) -> p_hat` replaces the P quantiser (tests use the identity)."""
+    `p_quantizer(p32) -> p_hat` replaces the P quantiser (tests use the identity).
+    `rescale_tau` > 0 selects conditional rescaling (see the module header)."""
+    tau = int(rescale_tau)
+    if tau < 0 or tau != rescale_tau:
+        raise ValueError("rescale_tau must be a non-negative integer")
     qhat = np.asarray(qhat, dtype=np.float64)
     khat = np.asarray(khat, dtype=np.float64)
     vhat = np.asarray(vhat, dtype=np.float64)
@@ -94,14 +114,19 @@ def attention_pnq(qhat, khat, vhat, *, causal: bool, fmt: str, qmax_p: float = 0
         act = np.isfinite(s).any(axis=1)
         if not act.any():
             continue
-        m_new = np.maximum(m, np.max(s, axis=1))          # masked keys are -inf
+        tmax = np.max(s, axis=1)                           # masked keys are -inf
+        m_new = np.maximum(m, tmax)
+        if tau > 0:
+            with np.errstate(invalid="ignore"):
+                grow = (tmax - m) * np.log2(np.e) > tau
+            m_new = np.where(np.isneginf(m) | grow, m_new, m)
         with np.errstate(invalid="ignore"):
             p = np.where(np.isfinite(s), np.exp(s - m_new[:, None]), 0.0)
             alpha = np.where(act, np.exp(m - m_new), 1.0)
         pad = np.zeros((R, BC))
         pad[:, : t1 - t0] = p
         if p_quantizer is None:
-            phat = quantize_p(pad.astype(np.float32), fmt, qmax_p)[:, : t1 - t0]
+            phat = quantize_p(pad.astype(np.float32), fmt, qmax_p, tau)[:, : t1 - t0]
         else:
             phat = np.asarray(p_quantizer(pad), dtype=np.float64)[:, : t1 - t0]
         phat[~act] = 0.0
@@ -159,7 +184,8 @@ def quantize_qkv(q, k, v, fmt: str, qmax: float = 0.0, g_q: float = 1.0, g_k: fl
 
 
 def prefill(q, k, v, *, causal: bool, fmt: str, qmax: float = 0.0, qmax_p: float = 0.0,
-            lam=None, sm_scale: float | None = None, rows=None, heads=None, return_lse: bool = False):
+            lam=None, sm_scale: float | None = None, rows=None, heads=None, return_lse: bool = False,
+            rescale_tau: int = 0, consistent: bool = True):
     """Oracle output of the library's prefill pipeline on bf16-valued inputs.
 
     q [B, Hq, Sq, d], k/v [B, Hkv, Sk, d]; `lam` [Hkv, d] Smooth-QK multipliers
@@ -181,5 +207,6 @@ def prefill(q, k, v, *, causal: bool, fmt: str, qmax: float = 0.0, qmax_p: float
         pq, sq = formats.quantize_rows(q[b, h], fmt, qmax, 1.0, mq)
         qh = formats.dequantize_rows(pq, sq, fmt)
         res[(b, h)] = attention_pnq(qh, kh, vh, causal=causal, fmt=fmt, qmax_p=qmax_p,
-                                    sm_scale=sm_scale, rows=rows, return_lse=return_lse)
+                                    sm_scale=sm_scale, rows=rows, return_lse=return_lse,
+                                    rescale_tau=rescale_tau, consistent=consistent)
     return res

@@ -13,7 +13,8 @@ from fa4q_testlib import assert_close, to_dev_bf16
 pytestmark = pytest.mark.gpu
 
 
-def run_prefill(q, k, v, fmt, causal, qmax=0.0, qmax_p=0.0, lam=None, out_fp32=True, want_lse=False):
+def run_prefill(q, k, v, fmt, causal, qmax=0.0, qmax_p=0.0, lam=None, out_fp32=True, want_lse=False,
+                tau=0, l_from_ptilde=False):
     import torch
     import microscaled_fp4_flashattention_b200 as fa4q
     dev = torch.device("cuda:0")
@@ -28,7 +29,8 @@ def run_prefill(q, k, v, fmt, causal, qmax=0.0, qmax_p=0.0, lam=None, out_fp32=T
     pv, sv = fa4q.quantize(to_dev_bf16(v, dev), fmt, fa4q.FA4Q_AXIS_OUTER, qmax)
     lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev) if want_lse else None
     out = fa4q.attn_fwd(pq, sq, pk, sk, pv, sv, B=B, Hq=Hq, Hkv=Hkv, S_q=S, S_k=Sk, d=d, fmt=fmt,
-                        causal=causal, qmax_p=qmax_p, out_fp32=out_fp32, lse=lse)
+                        causal=causal, qmax_p=qmax_p, out_fp32=out_fp32, lse=lse, rescale_tau=tau,
+                        l_from_ptilde=l_from_ptilde)
     torch.cuda.synchronize()
     code, detail = fa4q.device_status()
     assert code == 0, f"device status {code} detail {detail:#x}"
@@ -41,10 +43,11 @@ def _rand(shape, seed, scale=1.0):
                                * np.float32(scale))
 
 
-def check(q, k, v, fmt, causal, qmax=0.0, qmax_p=0.0, lam=None, rows=None, heads=None, what=""):
-    got = run_prefill(q, k, v, fmt, causal, qmax, qmax_p, lam)
+def check(q, k, v, fmt, causal, qmax=0.0, qmax_p=0.0, lam=None, rows=None, heads=None, what="",
+          tau=0):
+    got = run_prefill(q, k, v, fmt, causal, qmax, qmax_p, lam, tau=tau)
     ref = OA.prefill(q, k, v, causal=causal, fmt=fmt, qmax=qmax, qmax_p=qmax_p, lam=lam, rows=rows,
-                     heads=heads)
+                     heads=heads, rescale_tau=tau)
     gs, rs = [], []
     for (b, h), r in ref.items():
         gs.append(got[b, h] if rows is None else got[b, h][rows])
@@ -138,3 +141,56 @@ def test_full_size_workloads_sampled_rows(wid):
     rows = _rows(w.S, 23, wid)
     heads = [(0, 0), (0, w.Hq // 2 + 1), (0, w.Hq - 1)]
     check(q, k, v, w.fmt, w.causal, w.qmax, w.qmax_p, lam, rows=rows, heads=heads, what=w.name)
+
+
+@pytest.mark.parametrize("fmt,causal,S,Hq,Hkv,tau", [
+    ("mxfp4", True, 700, 4, 2, 8),       # holds keys equal to a kept reference (E2M1 tie 0.25)
+    ("mxfp4", False, 450, 2, 2, 4),
+    ("mxfp4", False, 300, 2, 1, 1),
+    ("mxfp4", True, 129, 2, 2, 8),
+])
+def test_conditional_rescale(fmt, causal, S, Hq, Hkv, tau):
+    """fa4q_attn_fwd_ex (reference maximum kept within tau binades) against the oracle's
+    conditional-rescale variant; keys grow along the sequence so the reference is often
+    kept while later tiles exceed it.  (NVFP4 with tau > 0 is refused on the host.)"""
+    d = 128
+    q = _rand((1, Hq, S, d), S + tau, 1.5)
+    k = _rand((1, Hkv, S, d), S + tau + 1, 1.5) * np.linspace(0.6, 1.4, S, dtype=np.float32)[:, None]
+    k = synth.round_to_bf16(k.astype(np.float32))
+    v = _rand((1, Hkv, S, d), S + tau + 2)
+    check(q, k, v, fmt, causal, tau=tau, what=f"rescale tau={tau} {fmt} causal={causal}")
+
+
+def test_conditional_rescale_full_size_sampled_rows():
+    """The causal GQA MXFP4 workload (the benchmark's) with tau = 8, sampled rows."""
+    w = synth.WORKLOADS[2]
+    q, k, v = synth.prefill_inputs(w)
+    lam = OS.calibrate(*synth.calibration_inputs(w))
+    rows = _rows(w.S, 23, 8)
+    heads = [(0, 0), (0, w.Hq - 1)]
+    check(q, k, v, w.fmt, w.causal, w.qmax, w.qmax_p, lam, rows=rows, heads=heads, what="tau=8 w2", tau=8)
+
+
+@pytest.mark.parametrize("fmt,causal,S,Hq,Hkv", [
+    ("nvfp4", False, 384, 2, 2),
+    ("mxfp4", True, 520, 4, 2),
+    ("nvfp4", True, 300, 2, 1),
+])
+def test_inconsistent_normaliser(fmt, causal, S, Hq, Hkv):
+    """l_from_ptilde: normaliser from the unquantised exponentials (the HiFA4 baseline)
+    against the oracle's inconsistent variant; and, from the two GPU outputs, the
+    coherent per-row scaling sum P_hat / sum P~ with net mass loss (median below 1)."""
+    d = 128
+    q = _rand((1, Hq, S, d), S + 31, 1.5)
+    k = _rand((1, Hkv, S, d), S + 32, 1.5)
+    v = _rand((1, Hkv, S, d), S + 33)
+    got = run_prefill(q, k, v, fmt, causal, l_from_ptilde=True)
+    ref = OA.prefill(q, k, v, causal=causal, fmt=fmt, consistent=False)
+    assert_close(np.stack([got[0, h] for h in range(Hq)]), np.stack([ref[(0, h)] for h in range(Hq)]),
+                 what=f"inconsistent normaliser {fmt}")
+    con = run_prefill(q, k, v, fmt, causal)
+    ratio = got / con                                   # per row: sum P_hat / sum P~
+    rows = np.abs(con).min(axis=-1) > 1e-3              # rows without near-zero entries
+    r = ratio[..., 0][rows]
+    assert np.max(np.abs(ratio[rows] - r[:, None])) <= 1e-4     # one factor per row
+    assert np.median(r) < 1.0                            # net mass loss

@@ -68,6 +68,12 @@ def test_argument_errors_without_gpu(L):
     assert L.fa4q_attn_fwd(*args, 1, 4, 4, 128, 128, 96, 0, F(0), 0, F(0), fake, 1, None, None) == 2
     assert L.fa4q_attn_fwd(*args, 1, 6, 4, 128, 128, 128, 0, F(0), 0, F(0), fake, 1, None, None) == 1
     assert L.fa4q_attn_fwd(*args, 1, 4, 4, 128, 256, 128, 0, F(0), 1, F(0), fake, 1, None, None) == 1
+    # conditional rescaling: threshold out of range; NVFP4 P with a kept reference
+    assert L.fa4q_attn_fwd_ex(*args, 1, 4, 4, 128, 128, 128, 1, F(0), 0, F(0), 31, 0, fake, 1, None, None) == 1
+    assert L.fa4q_attn_fwd_ex(*args, 1, 4, 4, 128, 128, 128, 1, F(0), 0, F(0), -1, 0, fake, 1, None, None) == 1
+    assert L.fa4q_attn_fwd_ex(*args, 1, 4, 4, 128, 128, 128, 0, F(0), 0, F(0), 8, 0, fake, 1, None, None) == 2
+    # inconsistent-normaliser flag must be 0 or 1
+    assert L.fa4q_attn_fwd_ex(*args, 1, 4, 4, 128, 128, 128, 1, F(0), 0, F(0), 0, 2, fake, 1, None, None) == 1
     # decode: group too large, workspace too small
     dargs = [fake] * 14
     assert L.fa4q_decode(*dargs, 1, 32, 2, 128, 4, 0, 0, 0, F(1), F(1), F(0), fake, fake, 1 << 30, 0, None) == 2

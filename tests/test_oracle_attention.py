@@ -30,13 +30,15 @@ def test_tiled_loop_identity_quantizer_is_softmax(causal, S):
     assert np.max(np.abs(out - ref)) <= 1e-12
 
 
-def _scalar_pnq(q, k, v, causal, fmt, qmax_p=0.0):
-    """Brute-force restatement with scalar Python loops (tiny inputs only)."""
+def _scalar_pnq(q, k, v, causal, fmt, qmax_p=0.0, tau=0, stats=None):
+    """Brute-force restatement with scalar Python loops (tiny inputs only).  tau > 0: the
+    reference maximum moves only when a tile's maximum exceeds it by more than tau binades
+    (then p~ may exceed 1, and NVFP4 P takes the tensor scale g_P * 2^tau)."""
     Sq, d = q.shape
     Sk = k.shape[0]
     sm = 1.0 / math.sqrt(d)
     blk = F.block_size(fmt)
-    g = A.p_tensor_scale(fmt)
+    g = np.float32(1.0 / (6.0 * 448.0)) * 2.0 ** tau if fmt == "nvfp4" else 1.0
     out = np.zeros((Sq, v.shape[1]))
     for i in range(Sq):
         m, l, o = -math.inf, 0.0, np.zeros(v.shape[1])
@@ -45,10 +47,16 @@ def _scalar_pnq(q, k, v, causal, fmt, qmax_p=0.0):
             if not keys:
                 continue
             s = {j: float(np.dot(q[i].astype(np.float64), k[j].astype(np.float64))) * sm for j in keys}
-            m_new = max(m, max(s.values()))
+            tmax = max(s.values())
+            if m == -math.inf or (tmax - m) / math.log(2.0) > tau:
+                m_new = max(m, tmax)
+            else:
+                m_new = m
             ptil = np.zeros(128, dtype=np.float32)
             for j in keys:
                 ptil[j - t0] = np.float32(math.exp(s[j] - m_new))
+            if stats is not None:
+                stats["max_ptilde"] = max(stats.get("max_ptilde", 0.0), float(ptil.max()))
             c, sb = F.quantize_blocks(ptil.reshape(128 // blk, blk), fmt, qmax_p if fmt == "mxfp4" else 0.0, g)
             phat = F.dequantize_blocks(c, sb, fmt, g).reshape(128)
             alpha = math.exp(m - m_new) if m != -math.inf else 0.0
@@ -277,3 +285,49 @@ def test_vertical_line_count_and_ties():
     assert len(sel2) == 6 and np.all(np.diff(sel2) > 0)
     mass = H.column_mass(np.random.default_rng(40).normal(size=(5, 8)), k2)
     assert mass[sel2].min() >= np.sort(mass)[-6]
+
+
+# ----------------------------------------------------------------------------- conditional rescale
+@pytest.mark.parametrize("causal", [False, True])
+def test_conditional_rescale_identity_quantizer_is_softmax(causal):
+    """A stale reference maximum only changes the bookkeeping: with an identity P quantiser
+    the result is still plain softmax attention."""
+    S = 520
+    q, k, v = _rand((S, 32), 41, 2.0), _rand((S, 32), 42, 2.0), _rand((S, 32), 43)
+    out = A.attention_pnq(q, k, v, causal=causal, fmt="mxfp4", p_quantizer=lambda p: p, rescale_tau=8)
+    ref = A.attention_plain(q, k, v, causal=causal)
+    assert np.max(np.abs(out - ref)) <= 1e-12
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_conditional_rescale_matches_scalar_bruteforce(fmt):
+    """Keys whose scores grow along the sequence: the second tile's maximum exceeds the
+    first's, by less than tau = 8 binades, so p~ above 1 is quantised (checked)."""
+    S, d = 256, 16
+    q = _rand((S, d), 44, 1.0)
+    k = _rand((S, d), 45, 1.0) * np.linspace(0.5, 1.5, S, dtype=np.float32)[:, None]
+    v = _rand((S, d), 46)
+    rows = np.array([5, 130, 200, 255])
+    out = A.attention_pnq(q, k, v, causal=False, fmt=fmt, rows=rows, rescale_tau=8)
+    st = {}
+    ref = _scalar_pnq(q[rows], k, v, False, fmt, tau=8, stats=st)
+    assert np.max(np.abs(out - ref)) <= 1e-12
+    assert st["max_ptilde"] > 1.0
+    exact = _scalar_pnq(q[rows], k, v, False, fmt, tau=0)
+    assert np.max(np.abs(exact - ref)) > 0.0        # the variant changes P_hat
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+def test_conditional_rescale_weights_are_convex(fmt):
+    S = 300
+    q, k, v = _rand((S, 64), 47, 1.5), _rand((S, 64), 48, 1.5), _rand((S, 64), 49)
+    out, w = A.attention_pnq(q, k, v, causal=True, fmt=fmt, return_weights=True, rescale_tau=8)
+    assert np.all(w >= 0)
+    assert np.max(np.abs(w.sum(axis=1) - 1.0)) <= 1e-12
+    assert np.max(np.abs(w @ v.astype(np.float64) - out)) <= 1e-12
+
+
+def test_conditional_rescale_rejects_fractional_tau():
+    q = _rand((8, 16), 50)
+    with pytest.raises(ValueError):
+        A.attention_pnq(q, q, q, causal=False, fmt="nvfp4", rescale_tau=2.5)
