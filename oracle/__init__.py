@@ -17,13 +17,15 @@ A plain, slow, obviously-correct numpy implementation, written from the pages:
 * `smooth`    - the calibration of the static per-channel Q/K multipliers.
 * `hyquant`   - vertical-line identification by accumulated column mass
                 (diagnostic; not on the timed path).
+* `rotate`    - Hadamard rotation of Q and K rows before quantisation (the
+                outlier-spreading alternative to Smooth-QK; an ablation).
 
 Every function states the passage it follows.  Floating point is FP64 except
 where the method fixes FP32 decisions (scale selection and element rounding),
 which are taken in IEEE FP32 exactly as specified in `formats`.
 
-Parity status: `formats`, `attention`, `decode` and `smooth` are pinned by the
+Parity status: `formats`, `attention`, `decode`, `smooth` and `rotate` are pinned by the
 `-m "not gpu"` tests in `tests/test_oracle_*.py`.  `hyquant` is a diagnostic
 pinned only qualitatively (planted vertical lines are recovered).
 """
-from . import formats, attention, decode, smooth, hyquant  # noqa: F401
+from . import formats, attention, decode, smooth, hyquant, rotate  # noqa: F401
