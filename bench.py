@@ -501,6 +501,29 @@ def main():
                                              f"{sm_mhz:.0f} MHz, 4*d FLOPs per score"}},
         "clocks": sampler.summary(),
     }
+    # ablation beside the headline: Hadamard-rotated Q and K (fa4q_quantize_rotated, the
+    # alternative to Smooth-QK) against the plain inner quantisation of the same tensors
+    def time_q(fn, reps=10):
+        for _ in range(2):
+            fn()
+        e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for i in range(reps):
+            flush.fill_(float(i))
+            e[i][0].record()
+            fn()
+            e[i][1].record()
+        barrier()
+        return float(np.mean([a.elapsed_time(b) for a, b in e]))
+    rot_ms = time_q(lambda: (fa4q.quantize_rotated(run.q, w.fmt, w.qmax), fa4q.quantize_rotated(run.k, w.fmt, w.qmax)))
+    inn_ms = time_q(lambda: (fa4q.quantize(run.q, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax),
+                             fa4q.quantize(run.k, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax)))
+    qk_elems = run.q.numel() + run.k.numel()
+    qk_bytes = qk_elems * 2 + qk_elems // 2 + qk_elems // (32 if w.fmt == "mxfp4" else 16)
+    line["ablation_hadamard"] = {
+        "kernel": "quant_rotated_kernel (Q and K, two launches)", "ms": rot_ms,
+        "GBps": qk_bytes / (rot_ms * 1e-3) / 1e9, "plain_inner_ms": inn_ms,
+        "plain_inner_GBps": qk_bytes / (inn_ms * 1e-3) / 1e9,
+        "note": "Walsh-Hadamard rotation of every Q/K row fused into the quantiser; not on the headline path"}
     if tau_ms is not None:
         line["ablation_rescale_tau8"] = {
             "kernel": "attn_fwd_kernel via fa4q_attn_fwd_ex(rescale_tau=8)", "ms_per_launch": tau_ms,

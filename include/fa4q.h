@@ -101,6 +101,28 @@ fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows, int64_t c
                           uint8_t* scales_out, void* stream);
 
 /*
+ * fa4q_quantize_rotated - fa4q_quantize (AXIS_INNER) of Hadamard-rotated rows, an ablation:
+ * the alternative to Smooth-QK for outlier channels of K.
+ *
+ * Source: BitDecoding-FP4, "Outlier-Aware Key Quantization" (an orthogonal Hadamard rotation
+ * of the keys spreads channel outliers across the head dimension; the same rotation on the
+ * query side leaves the scores unchanged).  The pages fix no normalisation or order.  Here
+ * every row (after the optional smooth_mul multiply) is replaced by its unnormalised
+ * Sylvester-order Walsh-Hadamard transform, computed in IEEE FP32 by butterflies in stages
+ * h = 1, 2, ..., cols/2 ((a, b) -> (a + b, a - b)), then quantised exactly as fa4q_quantize.
+ * Rotating both Q and K multiplies Q K^T by cols: pass sm_scale = 1/(cols*sqrt(cols)) to
+ * fa4q_attn_fwd (an exact power-of-two change of the default).  V is not rotated.
+ *
+ * cols 64 or 128 (else FA4Q_ERR_UNSUPPORTED); other arguments, layouts and errors as
+ * fa4q_quantize with axis = FA4Q_AXIS_INNER.
+ */
+fa4q_status fa4q_quantize_rotated(const void* x, int64_t groups, int64_t rows, int64_t cols,
+                                  int64_t row_stride, fa4q_format fmt, float qmax,
+                                  float tensor_scale, const float* smooth_mul, int64_t smooth_heads,
+                                  int64_t smooth_ratio, fa4q_sf_layout sf_layout,
+                                  uint8_t* packed_out, uint8_t* scales_out, void* stream);
+
+/*
  * fa4q_quantize_qkv - the three quantisations of a prefill in one launch, bit-identical to
  *   fa4q_quantize(q, B*Hq,  S_q, d, d, fmt, INNER, qmax, g_q, mul_q, Hq,  Hq/Hkv, TILED, ...)
  *   fa4q_quantize(k, B*Hkv, S_k, d, d, fmt, INNER, qmax, g_k, mul_k, Hkv, 1,      TILED, ...)

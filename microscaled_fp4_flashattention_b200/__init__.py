@@ -25,6 +25,7 @@ STATUS = {0: "FA4Q_OK", 1: "FA4Q_ERR_INVALID_ARG", 2: "FA4Q_ERR_UNSUPPORTED", 3:
 EXPORTED = [
     "fa4q_status_string", "fa4q_version", "fa4q_sf_tiled_bytes", "fa4q_quantize",
     "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_attn_fwd_ex", "fa4q_quantize_kv_pages",
+    "fa4q_quantize_rotated",
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
     "fa4q_vlines_workspace_size", "fa4q_select_vertical_lines", "fa4q_quantize_qkv",
@@ -55,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.fa4q_sf_tiled_bytes.argtypes = [I64, I64, I]
         L.fa4q_quantize.restype = I
         L.fa4q_quantize.argtypes = [P, I64, I64, I64, I64, I, I, F, F, P, I64, I64, I, P, P, P]
+        L.fa4q_quantize_rotated.restype = I
+        L.fa4q_quantize_rotated.argtypes = [P, I64, I64, I64, I64, I, F, F, P, I64, I64, I, P, P, P]
         L.fa4q_smooth_calibrate.restype = I
         L.fa4q_smooth_calibrate.argtypes = [P, P, I, I, I, I, P, P, P]
         L.fa4q_attn_fwd.restype = I
@@ -152,6 +155,29 @@ def quantize(x, fmt, axis: int = FA4Q_AXIS_INNER, qmax: float = 0.0, tensor_scal
     _check("fa4q_quantize", lib().fa4q_quantize(
         _ptr(x), groups, rows, cols, cols, f, axis, qmax, tensor_scale, _ptr(smooth_mul),
         smooth_heads, smooth_ratio, sf_layout, _ptr(packed), _ptr(sf), _stream(stream)))
+    return packed, sf
+
+
+def quantize_rotated(x, fmt, qmax: float = 0.0, tensor_scale: float = 1.0, smooth_mul=None,
+                     smooth_heads: int = 1, smooth_ratio: int = 1, sf_layout: int = FA4Q_SF_TILED,
+                     stream=None):
+    """Hadamard-rotated rows quantised along cols (fa4q_quantize_rotated); x bf16 CUDA
+    tensor [..., rows, cols], cols 64 or 128.  Returns (packed, scales) as quantize()."""
+    import torch
+    assert x.dtype == torch.bfloat16 and x.is_cuda and x.is_contiguous()
+    rows, cols = x.shape[-2], x.shape[-1]
+    groups = x.numel() // max(1, rows * cols)
+    f = _fmt(fmt)
+    blk = block_size(f)
+    lead = tuple(x.shape[:-2])
+    packed = torch.empty(lead + (rows, cols // 2), dtype=torch.uint8, device=x.device)
+    if sf_layout == FA4Q_SF_TILED:
+        sf = torch.empty(lead + (sf_tiled_bytes(rows, cols, f),), dtype=torch.uint8, device=x.device)
+    else:
+        sf = torch.empty(lead + (rows, cols // blk), dtype=torch.uint8, device=x.device)
+    _check("fa4q_quantize_rotated", lib().fa4q_quantize_rotated(
+        _ptr(x), groups, rows, cols, cols, f, qmax, tensor_scale, _ptr(smooth_mul), smooth_heads,
+        smooth_ratio, sf_layout, _ptr(packed), _ptr(sf), _stream(stream)))
     return packed, sf
 
 

@@ -90,36 +90,52 @@ struct InnerArgs {
   uint8_t* sf;
 };
 
-// slot idx of group gi's scale space (32-bit in-group indices: no 64-bit divisions per block)
+// Geometry of one group's scale space: `nblk` real blocks per row, `ncol_sp` scale slots per
+// row (the tiled layout pads the columns to whole 128-element tiles), `rows_sp` rows (padded
+// to 128 when tiled).
+struct InnerGeom {
+  int nblk, rows_i, rows_sp, nG, ncol_sp;
+  int64_t sf_group_bytes;
+};
+
 template <int BLK>
-FA4Q_DEVINL void quant_inner_slot(const InnerArgs& a, int64_t gi, int idx) {
-  const int nblk = static_cast<int>(a.cols / BLK);
-  const int rows_i = static_cast<int>(a.rows);
-  const int rows_sp = a.tiled ? ((rows_i + 127) / 128) * 128 : rows_i;
-  const int nG = a.tiled ? static_cast<int>((a.cols + 127) / 128) * (32 / BLK) : 0;
-  const int ncol_sp = a.tiled ? nG * 4 : nblk;
-  if (idx >= rows_sp * ncol_sp) return;
-  const int r = idx / ncol_sp;
-  const int kb = idx - r * ncol_sp;
-  const int64_t sf_group_bytes = a.tiled ? (int64_t)((rows_i + 127) / 128) * nG * 512 : (int64_t)rows_i * nblk;
-  uint32_t s = 0;
-  if (r < rows_i && kb < nblk) {
-    const uint16_t* src = a.x + (gi * a.rows + r) * a.row_stride + kb * BLK;
-    float v[BLK];
+FA4Q_DEVINL InnerGeom inner_geom(const InnerArgs& a) {
+  InnerGeom q;
+  q.nblk = static_cast<int>(a.cols / BLK);
+  q.rows_i = static_cast<int>(a.rows);
+  q.rows_sp = a.tiled ? ((q.rows_i + 127) / 128) * 128 : q.rows_i;
+  q.nG = a.tiled ? static_cast<int>((a.cols + 127) / 128) * (32 / BLK) : 0;
+  q.ncol_sp = a.tiled ? q.nG * 4 : q.nblk;
+  q.sf_group_bytes = a.tiled ? (int64_t)((q.rows_i + 127) / 128) * q.nG * 512 : (int64_t)q.rows_i * q.nblk;
+  return q;
+}
+
+// bf16 block (r, kb) of group gi -> FP32, times the Smooth-QK multiplier when given
+template <int BLK>
+FA4Q_DEVINL void inner_load(const InnerArgs& a, int64_t gi, int r, int kb, float* v) {
+  const uint16_t* src = a.x + (gi * a.rows + r) * a.row_stride + kb * BLK;
 #pragma unroll
-    for (int c = 0; c < BLK; c += 8) load_bf16x8(src + c, v + c);
-    if (a.mul != nullptr) {
-      const int mrow = (static_cast<int>(gi) % static_cast<int>(a.mheads)) / static_cast<int>(a.mratio);
-      const float* m = a.mul + (int64_t)mrow * a.cols + kb * BLK;
+  for (int c = 0; c < BLK; c += 8) load_bf16x8(src + c, v + c);
+  if (a.mul != nullptr) {
+    const int mrow = (static_cast<int>(gi) % static_cast<int>(a.mheads)) / static_cast<int>(a.mratio);
+    const float* m = a.mul + (int64_t)mrow * a.cols + kb * BLK;
 #pragma unroll
-      for (int c = 0; c < BLK; c += 4) {
-        const float4 mm = *reinterpret_cast<const float4*>(m + c);
-        v[c] = __fmul_rn(v[c], mm.x);
-        v[c + 1] = __fmul_rn(v[c + 1], mm.y);
-        v[c + 2] = __fmul_rn(v[c + 2], mm.z);
-        v[c + 3] = __fmul_rn(v[c + 3], mm.w);
-      }
+    for (int c = 0; c < BLK; c += 4) {
+      const float4 mm = *reinterpret_cast<const float4*>(m + c);
+      v[c] = __fmul_rn(v[c], mm.x);
+      v[c + 1] = __fmul_rn(v[c + 1], mm.y);
+      v[c + 2] = __fmul_rn(v[c + 2], mm.z);
+      v[c + 3] = __fmul_rn(v[c + 3], mm.w);
     }
+  }
+}
+
+// quantise block (r, kb) (when `real`) and write its scale slot (always)
+template <int BLK>
+FA4Q_DEVINL void inner_store(const InnerArgs& a, const InnerGeom& q, int64_t gi, int r, int kb, const float* v,
+                             bool real) {
+  uint32_t s = 0;
+  if (real) {
     uint8_t* dst = a.packed + (gi * a.rows + r) * (a.cols / 2) + kb * (BLK / 2);
     if constexpr (BLK == 16) {
       uint2 p;
@@ -132,15 +148,74 @@ FA4Q_DEVINL void quant_inner_slot(const InnerArgs& a, int64_t gi, int idx) {
     }
   }
   if (a.tiled)
-    a.sf[gi * sf_group_bytes + sf_tiled_offset(r, kb, nG)] = (uint8_t)s;
+    a.sf[gi * q.sf_group_bytes + sf_tiled_offset(r, kb, q.nG)] = (uint8_t)s;
   else
-    a.sf[gi * sf_group_bytes + (int64_t)r * nblk + kb] = (uint8_t)s;
+    a.sf[gi * q.sf_group_bytes + (int64_t)r * q.nblk + kb] = (uint8_t)s;
+}
+
+// slot idx of group gi's scale space (32-bit in-group indices: no 64-bit divisions per block)
+template <int BLK>
+FA4Q_DEVINL void quant_inner_slot(const InnerArgs& a, int64_t gi, int idx) {
+  const InnerGeom q = inner_geom<BLK>(a);
+  if (idx >= q.rows_sp * q.ncol_sp) return;
+  const int r = idx / q.ncol_sp;
+  const int kb = idx - r * q.ncol_sp;
+  const bool real = r < q.rows_i && kb < q.nblk;
+  float v[BLK];
+  if (real) inner_load<BLK>(a, gi, r, kb, v);
+  inner_store<BLK>(a, q, gi, r, kb, v, real);
 }
 
 template <int BLK>
 __global__ void __launch_bounds__(256) quant_inner_kernel(const InnerArgs a) {
   // grid: x over the (row, block) slots of one group's scale space, y = group
   quant_inner_slot<BLK>(a, blockIdx.y, blockIdx.x * blockDim.x + threadIdx.x);
+}
+
+// ---------------------------------------------------------------------------------------
+// AXIS_INNER with a Hadamard rotation of every row before quantisation (BitDecoding-FP4,
+// "Outlier-Aware Key Quantization": an orthogonal Hadamard transform of the keys spreads
+// channel outliers; the same transform of the queries keeps Q K^T up to the factor cols).
+// Unnormalised Sylvester order, FP32 butterflies in stages h = 1, 2, ..., cols/2: the stages
+// inside a block run in registers, the rest as warp shuffles between the lanes of one row
+// (slots idx = r * ncol_sp + kb, so a row's ncol_sp lanes are consecutive and aligned).
+// cols is 64 or 128.
+// ---------------------------------------------------------------------------------------
+template <int BLK>
+__global__ void __launch_bounds__(256) quant_rotated_kernel(const InnerArgs a) {
+  const InnerGeom q = inner_geom<BLK>(a);
+  const int64_t gi = blockIdx.y;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool in_space = idx < q.rows_sp * q.ncol_sp;
+  // warps wholly past the slot space leave; a partial warp holds whole rows (the space is a
+  // multiple of ncol_sp), so every lane left takes part in every shuffle below
+  if (__all_sync(0xffffffffu, !in_space)) return;
+  const int r = idx / q.ncol_sp;
+  const int kb = idx - r * q.ncol_sp;
+  const bool real = in_space && r < q.rows_i && kb < q.nblk;
+  float v[BLK];
+#pragma unroll
+  for (int i = 0; i < BLK; ++i) v[i] = 0.0f;
+  if (real) inner_load<BLK>(a, gi, r, kb, v);
+#pragma unroll
+  for (int h = 1; h < BLK; h *= 2)
+#pragma unroll
+    for (int i = 0; i < BLK; ++i)
+      if ((i & h) == 0) {
+        const float x0 = v[i], x1 = v[i + h];
+        v[i] = __fadd_rn(x0, x1);
+        v[i + h] = __fsub_rn(x0, x1);
+      }
+  for (int hb = 1; hb * BLK < static_cast<int>(a.cols); hb *= 2) {   // lane distance h / BLK
+    const bool upper = (kb & hb) != 0;
+#pragma unroll
+    for (int i = 0; i < BLK; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[i], hb);
+      v[i] = upper ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
+    }
+  }
+  if (!in_space) return;
+  inner_store<BLK>(a, q, gi, r, kb, v, real);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -444,6 +519,46 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
     else
       quant_outer_kernel<32><<<grid, 128, 0, st>>>(oa);
   }
+  return launch_status();
+}
+
+extern "C" fa4q_status fa4q_quantize_rotated(const void* x, int64_t groups, int64_t rows, int64_t cols,
+                                             int64_t row_stride, fa4q_format fmt, float qmax,
+                                             float tensor_scale, const float* smooth_mul,
+                                             int64_t smooth_heads, int64_t smooth_ratio,
+                                             fa4q_sf_layout sf_layout, uint8_t* packed_out,
+                                             uint8_t* scales_out, void* stream) {
+  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (sf_layout != FA4Q_SF_ROWMAJOR && sf_layout != FA4Q_SF_TILED) return FA4Q_ERR_INVALID_ARG;
+  if (groups < 0 || rows < 0 || cols < 0) return FA4Q_ERR_INVALID_ARG;
+  if (groups == 0 || rows == 0 || cols == 0) return FA4Q_OK;
+  if (cols != 64 && cols != 128) return FA4Q_ERR_UNSUPPORTED;
+  if (!x || !packed_out || !scales_out) return FA4Q_ERR_INVALID_ARG;
+  if (row_stride < cols || row_stride % 8 != 0) return FA4Q_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(packed_out)) return FA4Q_ERR_INVALID_ARG;
+  if (sf_layout == FA4Q_SF_TILED && !aligned16(scales_out)) return FA4Q_ERR_INVALID_ARG;
+  if (!(qmax >= 0.0f) || !isfinite(qmax)) return FA4Q_ERR_INVALID_ARG;
+  const float g = fmt == FA4Q_NVFP4 ? tensor_scale : 1.0f;
+  if (!(g > 0.0f) || !isfinite(g)) return FA4Q_ERR_INVALID_ARG;
+  if (smooth_mul && (smooth_heads <= 0 || smooth_ratio <= 0 || !aligned16(smooth_mul)))
+    return FA4Q_ERR_INVALID_ARG;
+  const int blk = fmt == FA4Q_MXFP4 ? 32 : 16;
+  const float qm = (fmt == FA4Q_NVFP4 && qmax == 0.0f) ? 6.0f : qmax;
+  const int tiled = sf_layout == FA4Q_SF_TILED;
+  const int64_t nblk = cols / blk;
+  const int64_t rows_sp = tiled ? (rows + 127) / 128 * 128 : rows;
+  const int64_t ncol_sp = tiled ? (cols + 127) / 128 * (32 / blk) * 4 : nblk;
+  const int64_t per_group = rows_sp * ncol_sp;
+  if (groups > 65535 || per_group > (int64_t)1 << 30 || rows > ((int64_t)1 << 30)) return FA4Q_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)((per_group + 255) / 256), (unsigned)groups);
+  const int64_t mh = smooth_heads > 0 ? smooth_heads : 1, mr = smooth_ratio > 0 ? smooth_ratio : 1;
+  const InnerArgs ia{(const uint16_t*)x, rows, cols, row_stride, qm, g, smooth_mul, mh, mr, tiled,
+                     packed_out, scales_out};
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (blk == 16)
+    quant_rotated_kernel<16><<<grid, 256, 0, st>>>(ia);
+  else
+    quant_rotated_kernel<32><<<grid, 256, 0, st>>>(ia);
   return launch_status();
 }
 

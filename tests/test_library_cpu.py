@@ -74,6 +74,9 @@ def test_argument_errors_without_gpu(L):
     assert L.fa4q_attn_fwd_ex(*args, 1, 4, 4, 128, 128, 128, 0, F(0), 0, F(0), 8, 0, fake, 1, None, None) == 2
     # inconsistent-normaliser flag must be 0 or 1
     assert L.fa4q_attn_fwd_ex(*args, 1, 4, 4, 128, 128, 128, 1, F(0), 0, F(0), 0, 2, fake, 1, None, None) == 1
+    # rotated quantisation: head dims other than 64 / 128
+    assert L.fa4q_quantize_rotated(fake, 1, 16, 96, 96, 0, F(0), F(1), None, 1, 1, 1, fake, fake, None) == 2
+    assert L.fa4q_quantize_rotated(None, 1, 16, 128, 128, 0, F(0), F(1), None, 1, 1, 1, fake, fake, None) == 1
     # decode: group too large, workspace too small
     dargs = [fake] * 14
     assert L.fa4q_decode(*dargs, 1, 32, 2, 128, 4, 0, 0, 0, F(1), F(1), F(0), fake, fake, 1 << 30, 0, None) == 2
