@@ -49,11 +49,10 @@ NCU_TRAFFIC = {
     "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
                  "sha256": "239aa1f4f1b754683e82aa1ceb156ee0272726ec94497101a6313bf6ad3cbe7c",
                  "bytes_per_launch": 13470976 + 73472},
-    # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,900,224 + 5,366,016 B for 8 sequences
-    # (taken before the MXFP4 page path was added to decode.cu: null until recaptured)
+    # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,891,008 + 4,980,480 B for 8 sequences
     "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
-               "sha256": "3fae0c63206939932514f70e30ad22e4b951a7a02beed961c9a384b935120fdc",
-               "bytes_per_sequence": 364266240 // 8},
+               "sha256": "8823e9bfcf14353afacabc2c8a977d045d5bc5088536c644f2f53732b444205f",
+               "bytes_per_sequence": (358891008 + 4980480) // 8},
 }
 
 
