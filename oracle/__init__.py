@@ -19,13 +19,15 @@ A plain, slow, obviously-correct numpy implementation, written from the pages:
                 (diagnostic; not on the timed path).
 * `rotate`    - Hadamard rotation of Q and K rows before quantisation (the
                 outlier-spreading alternative to Smooth-QK; an ablation).
+* `hybrid`    - hybrid-precision prefill: vertical-line and window keys in BF16,
+                the rest FP4, one online softmax.
 
 Every function states the passage it follows.  Floating point is FP64 except
 where the method fixes FP32 decisions (scale selection and element rounding),
 which are taken in IEEE FP32 exactly as specified in `formats`.
 
-Parity status: `formats`, `attention`, `decode`, `smooth` and `rotate` are pinned by the
+Parity status: `formats`, `attention`, `decode`, `smooth`, `rotate` and `hybrid` are pinned by the
 `-m "not gpu"` tests in `tests/test_oracle_*.py`.  `hyquant` is a diagnostic
 pinned only qualitatively (planted vertical lines are recovered).
 """
-from . import formats, attention, decode, smooth, hyquant, rotate  # noqa: F401
+from . import formats, attention, decode, smooth, hyquant, rotate, hybrid  # noqa: F401

@@ -79,7 +79,7 @@ def quantize_p(p32: np.ndarray, fmt: str, qmax_p: float = 0.0, tau: int = 0) -> 
 def attention_pnq(qhat, khat, vhat, *, causal: bool, fmt: str, qmax_p: float = 0.0,
                   sm_scale: float | None = None, rows=None, consistent: bool = True,
                   return_weights: bool = False, return_lse: bool = False, return_eps: bool = False,
-                  p_quantizer=None, rescale_tau: int = 0):
+                  p_quantizer=None, rescale_tau: int = 0, key_mask=None, init=None):
     """Tiled PNQ attention for one (batch, head) on dequantised operands.
 
     qhat [Sq, d], khat/vhat [Sk, d] (FP64).  `rows` selects query rows (default all).
@@ -88,7 +88,10 @@ def attention_pnq(qhat, khat, vhat, *, causal: bool, fmt: str, qmax_p: float = 0
     the effective key weights (P_hat rescaled to the final maximum, divided by l),
     the log-sum-exp m + ln(l) and the per-tile mass ratio eps = sum p^ / sum p~ - 1.
     `p_quantizer(p32) -> p_hat` replaces the P quantiser (tests use the identity).
-    `rescale_tau` > 0 selects conditional rescaling (see the module header)."""
+    `rescale_tau` > 0 selects conditional rescaling (see the module header).
+    `key_mask` (bool [R, Sk], True = the key takes part) removes keys beyond the causal
+    mask; `init` = (m, l, o) per row starts the online state from an earlier part of the
+    same softmax (the full-precision keys of the hybrid prefill)."""
     tau = int(rescale_tau)
     if tau < 0 or tau != rescale_tau:
         raise ValueError("rescale_tau must be a non-negative integer")
@@ -104,6 +107,10 @@ def attention_pnq(qhat, khat, vhat, *, causal: bool, fmt: str, qmax_p: float = 0
     m = np.full(R, -np.inf)
     l = np.zeros(R)
     o = np.zeros((R, vhat.shape[1]))
+    if init is not None:
+        m = np.array(init[0], dtype=np.float64, copy=True)
+        l = np.array(init[1], dtype=np.float64, copy=True)
+        o = np.array(init[2], dtype=np.float64, copy=True)
     W = np.zeros((R, Sk)) if return_weights else None
     eps = []
     for t0 in range(0, Sk, BC):
@@ -111,6 +118,8 @@ def attention_pnq(qhat, khat, vhat, *, causal: bool, fmt: str, qmax_p: float = 0
         s = S[:, t0:t1].copy()
         if causal:
             s[np.arange(t0, t1)[None, :] > rows[:, None]] = -np.inf
+        if key_mask is not None:
+            s[~np.asarray(key_mask)[:, t0:t1]] = -np.inf
         act = np.isfinite(s).any(axis=1)
         if not act.any():
             continue
