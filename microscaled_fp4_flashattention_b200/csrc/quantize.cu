@@ -21,6 +21,20 @@ namespace fa4q {
 // ---------------------------------------------------------------------------------------
 // per-block quantisation (FP32 values in registers)
 // ---------------------------------------------------------------------------------------
+// x / d rounded to nearest (IEEE), given r = 1/d rounded to nearest and d > 0: the product
+// q = RN(x r) is within an ulp of x/d, the remainder x - d q is exact in one FMA, and
+// RN(q + (x - d q) r) is the correctly rounded quotient (Markstein's theorem on FMA
+// division).  Quotients in the subnormal range may differ from IEEE division; they lie far
+// below the smallest E2M1 rounding threshold (0.25), so the codes do not.  The sign is
+// taken from x so that -0 stays -0; a product that overflows is returned as the infinity
+// IEEE division gives (the correction step would turn it into NaN).
+FA4Q_DEVINL float div_rn_recip(float x, float d, float r) {
+  const float q = __fmul_rn(x, r);
+  if (isinf(q)) return q;
+  const float e = __fmaf_rn(-q, d, x);
+  return copysignf(__fmaf_rn(e, r, q), x);
+}
+
 // NVFP4: s = UE4M3(amax / (qmax*g)); y = x / (float(s)*g); 16 elements -> 8 bytes.
 FA4Q_DEVINL uint32_t quant_block16_nvfp4(const float* v, float denom, float g, uint2& packed) {
   float amax = 0.0f;
@@ -31,8 +45,9 @@ FA4Q_DEVINL uint32_t quant_block16_nvfp4(const float* v, float denom, float g, u
   const float div = __fmul_rn(ue4m3_decode(s), g);
   float y[16];
   if (div > 0.0f) {
+    const float r = __frcp_rn(div);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = __fdiv_rn(v[i], div);
+    for (int i = 0; i < 16; ++i) y[i] = div_rn_recip(v[i], div, r);
   } else {
 #pragma unroll
     for (int i = 0; i < 16; ++i) y[i] = v[i] * 0.0f;
@@ -153,6 +168,31 @@ FA4Q_DEVINL void inner_store(const InnerArgs& a, const InnerGeom& q, int64_t gi,
     a.sf[gi * q.sf_group_bytes + (int64_t)r * q.nblk + kb] = (uint8_t)s;
 }
 
+// slots 2*pair and 2*pair + 1 (the same row: ncol_sp is even), both loads issued before
+// either block is quantised (NVFP4: twice the bytes in flight per thread at little register
+// cost; MXFP4 blocks are already 64 bytes and run one per thread)
+template <int BLK>
+FA4Q_DEVINL void quant_inner_pair(const InnerArgs& a, int64_t gi, int pair) {
+  const InnerGeom q = inner_geom<BLK>(a);
+  const int idx = 2 * pair;
+  if (idx >= q.rows_sp * q.ncol_sp) return;
+  const int r = idx / q.ncol_sp;
+  const int kb = idx - r * q.ncol_sp;
+  const bool real0 = r < q.rows_i && kb < q.nblk, real1 = r < q.rows_i && kb + 1 < q.nblk;
+  float v0[BLK], v1[BLK];
+  if (real0) inner_load<BLK>(a, gi, r, kb, v0);
+  if (real1) inner_load<BLK>(a, gi, r, kb + 1, v1);
+  inner_store<BLK>(a, q, gi, r, kb, v0, real0);
+  inner_store<BLK>(a, q, gi, r, kb + 1, v1, real1);
+}
+
+// slots handled by one thread of the inner quantiser
+template <int BLK>
+__host__ __device__ constexpr int inner_slots_per_thread() { return BLK == 16 ? 2 : 1; }
+
+template <int BLK>
+FA4Q_DEVINL void quant_inner_work(const InnerArgs& a, int64_t gi, int unit);
+
 // slot idx of group gi's scale space (32-bit in-group indices: no 64-bit divisions per block)
 template <int BLK>
 FA4Q_DEVINL void quant_inner_slot(const InnerArgs& a, int64_t gi, int idx) {
@@ -167,9 +207,15 @@ FA4Q_DEVINL void quant_inner_slot(const InnerArgs& a, int64_t gi, int idx) {
 }
 
 template <int BLK>
+FA4Q_DEVINL void quant_inner_work(const InnerArgs& a, int64_t gi, int unit) {
+  if constexpr (inner_slots_per_thread<BLK>() == 2) quant_inner_pair<BLK>(a, gi, unit);
+  else quant_inner_slot<BLK>(a, gi, unit);
+}
+
+template <int BLK>
 __global__ void __launch_bounds__(256) quant_inner_kernel(const InnerArgs a) {
-  // grid: x over the (row, block) slots of one group's scale space, y = group
-  quant_inner_slot<BLK>(a, blockIdx.y, blockIdx.x * blockDim.x + threadIdx.x);
+  // grid: x over the work units (one or two slots) of one group's scale space, y = group
+  quant_inner_work<BLK>(a, blockIdx.y, blockIdx.x * blockDim.x + threadIdx.x);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -233,9 +279,13 @@ struct OuterArgs {
 
 // every thread of the CTA calls this (it synchronises the CTA once); `valid` false makes the
 // thread's half a no-op that still takes part in the synchronisation
+// The tile holds the bf16 bit patterns (exact, half the shared memory of FP32): 64 channels
+// x 130 halves, an odd number of 32-bit words per row.
+constexpr int kOuterTileRow = 130;
+
 template <int BLK>
 FA4Q_DEVINL void quant_outer_tile(const OuterArgs& a, int64_t gi, int64_t tok_tile, int64_t ch_tile, int t,
-                                  float (*tile)[129], bool valid) {
+                                  uint16_t (*tile)[kOuterTileRow], bool valid) {
   const int64_t tok0 = tok_tile * 128;
   const int64_t ch0 = ch_tile * 64;
   const int64_t rows_pad = (a.rows + 31) / 32 * 32;
@@ -245,11 +295,15 @@ FA4Q_DEVINL void quant_outer_tile(const OuterArgs& a, int64_t gi, int64_t tok_ti
     for (int i = 0; i < 8; ++i) {
       const int u = t + 128 * i;
       const int tr = u >> 3, c8 = (u & 7) * 8;
-      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
       if (tok0 + tr < a.rows && ch0 + c8 < a.cols)
-        load_bf16x8(a.x + (gi * a.rows + tok0 + tr) * a.row_stride + ch0 + c8, v);
+        w = *reinterpret_cast<const uint4*>(a.x + (gi * a.rows + tok0 + tr) * a.row_stride + ch0 + c8);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) tile[c8 + k][tr] = v[k];
+      for (int k = 0; k < 4; ++k) {
+        tile[c8 + 2 * k][tr] = static_cast<uint16_t>(ww[k] & 0xFFFFu);
+        tile[c8 + 2 * k + 1][tr] = static_cast<uint16_t>(ww[k] >> 16);
+      }
     }
   }
   __syncthreads();
@@ -276,7 +330,7 @@ FA4Q_DEVINL void quant_outer_tile(const OuterArgs& a, int64_t gi, int64_t tok_ti
     const int64_t kb = (tok0 + lt) / BLK;              // block index along the channel row
     float v[BLK];
 #pragma unroll
-    for (int k = 0; k < BLK; ++k) v[k] = tile[c][lt + k];
+    for (int k = 0; k < BLK; ++k) v[k] = bf16_to_f32(tile[c][lt + k]);
     uint32_t s;
     uint8_t* dst = a.packed + (gi * a.cols + ch) * (rows_pad / 2) + (tok0 + lt) / 2;
     const bool inside = real_ch && tok0 + lt < rows_pad;
@@ -300,7 +354,7 @@ FA4Q_DEVINL void quant_outer_tile(const OuterArgs& a, int64_t gi, int64_t tok_ti
 
 template <int BLK>
 __global__ void __launch_bounds__(128) quant_outer_kernel(const OuterArgs a) {
-  __shared__ float tile[64][129];
+  __shared__ uint16_t tile[64][kOuterTileRow];
   quant_outer_tile<BLK>(a, blockIdx.z, blockIdx.x, blockIdx.y, threadIdx.x, tile, true);
 }
 
@@ -319,14 +373,14 @@ struct QkvGrid {
 template <int BLK>
 __global__ void __launch_bounds__(256) quant_qkv_kernel(const InnerArgs aq, const InnerArgs ak,
                                                         const OuterArgs av, const QkvGrid gr) {
-  extern __shared__ __align__(16) float qkv_tile[];   // [2][64][129]
+  extern __shared__ __align__(16) uint16_t qkv_tile[];   // [2][64][kOuterTileRow]
   const int64_t cta = blockIdx.x;
   if (cta < gr.n_q + gr.n_k) {
     const bool is_q = cta < gr.n_q;
     const int64_t flat = (is_q ? cta : cta - gr.n_q) * 256 + threadIdx.x;
-    const int64_t per = is_q ? gr.per_group_q : gr.per_group_k;
+    const int64_t per = (is_q ? gr.per_group_q : gr.per_group_k) / inner_slots_per_thread<BLK>();
     const int64_t gi = flat / per;
-    if (gi < (is_q ? gr.groups_q : gr.groups_k)) quant_inner_slot<BLK>(is_q ? aq : ak, gi, (int)(flat - gi * per));
+    if (gi < (is_q ? gr.groups_q : gr.groups_k)) quant_inner_work<BLK>(is_q ? aq : ak, gi, (int)(flat - gi * per));
     return;
   }
   const int half = threadIdx.x >> 7;
@@ -334,7 +388,8 @@ __global__ void __launch_bounds__(256) quant_qkv_kernel(const InnerArgs aq, cons
   const bool valid = ti < gr.n_vtiles;
   const int64_t per_g = gr.tok_tiles * gr.ch_tiles;
   const int64_t gi = valid ? ti / per_g : 0, rem = valid ? ti - gi * per_g : 0;
-  float(*tile)[129] = reinterpret_cast<float(*)[129]>(qkv_tile + half * 64 * 129);
+  uint16_t(*tile)[kOuterTileRow] =
+      reinterpret_cast<uint16_t(*)[kOuterTileRow]>(qkv_tile + half * 64 * kOuterTileRow);
   quant_outer_tile<BLK>(av, gi, rem / gr.ch_tiles, rem % gr.ch_tiles, threadIdx.x & 127, tile, valid);
 }
 
@@ -498,7 +553,8 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
     const int64_t ncol_sp = tiled ? (cols + 127) / 128 * (32 / blk) * 4 : nblk;
     const int64_t per_group = rows_sp * ncol_sp;
     if (groups > 65535 || per_group > (int64_t)1 << 30 || rows > ((int64_t)1 << 30)) return FA4Q_ERR_UNSUPPORTED;
-    dim3 grid((unsigned)((per_group + 255) / 256), (unsigned)groups);
+    const int64_t spt = blk == 16 ? inner_slots_per_thread<16>() : inner_slots_per_thread<32>();
+    dim3 grid((unsigned)((per_group / spt + 255) / 256), (unsigned)groups);
     const int64_t mh = smooth_heads > 0 ? smooth_heads : 1, mr = smooth_ratio > 0 ? smooth_ratio : 1;
     const InnerArgs ia{(const uint16_t*)x, rows, cols, row_stride, qm, g, smooth_mul, mh, mr, tiled,
                        packed_out, scales_out};
@@ -592,8 +648,9 @@ extern "C" fa4q_status fa4q_quantize_qkv(const void* q, const void* k, const voi
   gr.per_group_k = (static_cast<int64_t>(S_k) + 127) / 128 * 128 * ncol_sp;
   gr.groups_q = static_cast<int64_t>(B) * Hq;
   gr.groups_k = gr.groups_v = static_cast<int64_t>(B) * Hkv;
-  gr.n_q = S_q > 0 ? (gr.groups_q * gr.per_group_q + 255) / 256 : 0;
-  gr.n_k = S_k > 0 ? (gr.groups_k * gr.per_group_k + 255) / 256 : 0;
+  const int64_t spt = blk == 16 ? inner_slots_per_thread<16>() : inner_slots_per_thread<32>();
+  gr.n_q = S_q > 0 ? (gr.groups_q * gr.per_group_q / spt + 255) / 256 : 0;
+  gr.n_k = S_k > 0 ? (gr.groups_k * gr.per_group_k / spt + 255) / 256 : 0;
   const int64_t rows_pad_v = (static_cast<int64_t>(S_k) + 31) / 32 * 32;
   gr.tok_tiles = S_k > 0 ? (rows_pad_v + 127) / 128 : 0;
   gr.ch_tiles = (d + 127) / 128 * 2;                  // tiled layout: channels padded to 128
@@ -605,7 +662,7 @@ extern "C" fa4q_status fa4q_quantize_qkv(const void* q, const void* k, const voi
   const InnerArgs aq{(const uint16_t*)q, S_q, d, d, qm, g_q, mul_q, Hq, Hq / Hkv, 1, q_packed, q_sf};
   const InnerArgs ak{(const uint16_t*)k, S_k, d, d, qm, g_k, mul_k, Hkv, 1, 1, k_packed, k_sf};
   const OuterArgs av{(const uint16_t*)v, S_k, d, d, qm, g_v, 1, vt_packed, vt_sf};
-  const int smem = 2 * 64 * 129 * static_cast<int>(sizeof(float));
+  const int smem = 2 * 64 * kOuterTileRow * static_cast<int>(sizeof(uint16_t));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (blk == 16) {
     if (cudaFuncSetAttribute(quant_qkv_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
