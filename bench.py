@@ -45,10 +45,10 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # The decode capture ran 8 of the 32 sequences: its traffic is per sequence (it grows with the
 # number of sequences) and is scaled to the timed batch.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,470,976 + 73,472 B (bench workload)
+    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,485,568 + 70,400 B (bench workload)
     "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
-                 "sha256": "239aa1f4f1b754683e82aa1ceb156ee0272726ec94497101a6313bf6ad3cbe7c",
-                 "bytes_per_launch": 13470976 + 73472},
+                 "sha256": "1203cde5eceedf5b81f03d572a9a52248fe883d0cc35f765e4d60b509a95a276",
+                 "bytes_per_launch": 13485568 + 70400},
     # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,891,008 + 4,980,480 B for 8 sequences
     "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
                "sha256": "8823e9bfcf14353afacabc2c8a977d045d5bc5088536c644f2f53732b444205f",
@@ -194,6 +194,51 @@ class PrefillRun:
         if attn_events is not None:
             attn_events[1].record()
         return self.out
+
+
+def hybrid_bench(run, w, dev, fa4q, flush, barrier, steps):
+    """Time fa4q_attn_fwd_hybrid (two launches: the BF16 window / vertical-line part, then
+    the FP4 part from its state) on the prefill batch; FLOPs counted as the causal total."""
+    import torch
+    if not w.causal or w.d != 128:
+        return None
+    B, Hq, Hkv, S, d = w.B, w.Hq, w.Hkv, w.S, w.d
+    n_vl, W = int(0.05 * S), 128
+    rng = synth.generator(w.wid, 5, 7)
+    pos = np.stack([np.stack([np.sort(rng.choice(S, n_vl, replace=False)) for _ in range(Hkv)])
+                    for _ in range(B)]).astype(np.int32)
+    t_pos = torch.from_numpy(pos).to(dev)
+    t_cnt = torch.full((B, Hkv), n_vl, dtype=torch.int32, device=dev)
+    idx = t_pos.long()[..., None].expand(-1, -1, -1, d)
+    vk = torch.gather(run.k, 2, idx).contiguous()
+    vv = torch.gather(run.v, 2, idx).contiguous()
+    ex = np.zeros((B, Hkv, (S + 63) // 64), np.uint64)
+    for b in range(B):
+        for h in range(Hkv):
+            np.bitwise_or.at(ex[b, h], pos[b, h] // 64, np.uint64(1) << (pos[b, h] % 64).astype(np.uint64))
+    t_ex = torch.from_numpy(ex.view(np.int64)).to(dev)
+    kz, vz = run.k.clone(), run.v.clone()
+    kz.scatter_(2, idx, 0.0)
+    vz.scatter_(2, idx, 0.0)
+    pq, sq, pk, sk, pv, sv = fa4q.quantize_qkv(run.q, kz, vz, w.fmt, w.qmax, mul_q=run.mq, mul_k=run.mk)
+    ws = torch.empty(fa4q.lib().fa4q_attn_fwd_hybrid_workspace_size(B, Hq, S, d), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(run.out)
+    call = lambda: fa4q.attn_fwd_hybrid(pq, sq, pk, sk, pv, sv, run.q, run.k, run.v, t_pos, t_cnt, vk, vv, t_ex,
+                                        B=B, Hq=Hq, Hkv=Hkv, S=S, d=d, window=W, fmt=w.fmt, qmax_p=w.qmax_p,
+                                        out=out, workspace=ws)
+    for _ in range(3):
+        call()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(float(i))
+        ev[i][0].record()
+        call()
+        ev[i][1].record()
+    barrier()
+    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    return {"kernels": "hybrid_full_kernel (BF16 mma.sync) + attn_fwd_kernel<HYB> (tcgen05 FP4)",
+            "ms": ms, "TFLOP/s": run.flops / (ms * 1e-3) / 1e12, "window": W, "vertical_lines_per_kv_head": n_vl,
+            "note": "FLOPs of the whole causal attention (both parts); seeded random vertical-line positions"}
 
 
 # ------------------------------------------------------------------------------ decode workload
@@ -523,6 +568,9 @@ def main():
         "GBps": qk_bytes / (rot_ms * 1e-3) / 1e9, "plain_inner_ms": inn_ms,
         "plain_inner_GBps": qk_bytes / (inn_ms * 1e-3) / 1e9,
         "note": "Walsh-Hadamard rotation of every Q/K row fused into the quantiser; not on the headline path"}
+    # next row beside the headline: the hybrid-precision prefill (HyQuant) on the same
+    # inputs, 5% vertical lines per kv-head (seeded positions) and a 128-token window
+    line["hybrid_prefill"] = hybrid_bench(run, w, dev, fa4q, flush, barrier, args.steps)
     if tau_ms is not None:
         line["ablation_rescale_tau8"] = {
             "kernel": "attn_fwd_kernel via fa4q_attn_fwd_ex(rescale_tau=8)", "ms_per_launch": tau_ms,

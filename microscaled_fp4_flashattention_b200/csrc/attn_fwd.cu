@@ -137,6 +137,14 @@ struct AttnParams {
   // feeds the PV product; the numerator is unchanged, so each output row is scaled by
   // sum P_hat / sum P~.
   int l_from_ptilde;
+  // Hybrid-precision prefill (HyQuant): per row the full-precision part of the softmax,
+  // [m0 (log2 units), l0, o0[D]] in FP32, has already been computed over the window and
+  // vertical-line keys; this kernel starts from it and masks those keys out of its FP4
+  // tiles (window: key > row - hy_window; vertical lines: bit set in hy_excl).
+  const float* hy_part;      // [B][Hq][S_q][D + 4]: m0, l0, -, -, o0[D]
+  const uint64_t* hy_excl;   // [B][Hkv][hy_excl_words]
+  int hy_window;
+  int hy_excl_words;
   int causal;
   int out_fp32;
 };
@@ -307,7 +315,8 @@ FA4Q_DEVINL void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, int N
 
 // ABL: the ablations of fa4q_attn_fwd_ex (conditional rescaling, normaliser from P~) are
 // compiled into separate instantiations so the default kernel carries none of their work.
-template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL>
+// HYB: the FP4 part of the hybrid-precision prefill (causal only).
+template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL, bool HYB = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -342,6 +351,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       it.b = rem / p.Hq;
       it.h = rem % p.Hq;
       it.n_tiles = min(it.qt + 1, n_ktiles_all);
+      if constexpr (HYB) {
+        // the last FP4 key of the tile's last row is row - window; at least one (possibly
+        // fully masked) tile, so every item runs its epilogue
+        const int last = min(it.qt * kBM + kBM - 1, p.S_q - 1) - p.hy_window;
+        it.n_tiles = max(1, min(it.n_tiles, last >= 0 ? last / kBN + 1 : 0));
+      }
     } else {
       const int per = p.Hq * p.n_qtiles, rem = u % per;
       it.b = u / per;
@@ -500,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
             const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
             const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint32_t acc = (jp >= 2 || ks > 0) ? 1u : 0u;
+            // (hybrid: group A's accumulator starts from the full-precision part)
+            const uint32_t acc = (jp >= 2 || ks > 0 || (HYB && jp == 0)) ? 1u : 0u;
             mma_step<MX>(tmem + o_col, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
             mma_step<MX>(tmem + l_col, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
           }
@@ -579,12 +595,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&sm.s_free);
       // masking: keys beyond S_k, and (causal) keys after this query
       const int key0 = j * kBN;
-      const bool edge = (key0 + kBN > p.S_k) || (CAUSAL && key0 + kBN - 1 > qt * kBM);
-      if (edge) {
-        const int lim = CAUSAL ? min(p.S_k - key0, row - key0 + 1) : (p.S_k - key0);
+      if constexpr (HYB) {
+        // FP4 keys of row i: key <= i - window and not a vertical line
+        const int lim = min(p.S_k - key0, row - p.hy_window - key0 + 1);
+        const uint64_t* ex = p.hy_excl + (int64_t)(it.b * p.Hkv + it.h / (p.Hq / p.Hkv)) * p.hy_excl_words;
+        const int w0 = key0 >> 6;
+        const uint64_t e0 = w0 < p.hy_excl_words ? ex[w0] : 0ull;
+        const uint64_t e1 = w0 + 1 < p.hy_excl_words ? ex[w0 + 1] : 0ull;
 #pragma unroll
-        for (int i = 0; i < kBN; ++i)
-          if (i >= lim) s[i] = -INFINITY;
+        for (int i = 0; i < kBN; ++i) {
+          const uint64_t w = i < 64 ? e0 : e1;
+          if (i >= lim || ((w >> (i & 63)) & 1ull)) s[i] = -INFINITY;
+        }
+      } else {
+        const bool edge = (key0 + kBN > p.S_k) || (CAUSAL && key0 + kBN - 1 > qt * kBM);
+        if (edge) {
+          const int lim = CAUSAL ? min(p.S_k - key0, row - key0 + 1) : (p.S_k - key0);
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            if (i >= lim) s[i] = -INFINITY;
+        }
       }
       // block maxima of the raw scores (the scale is positive), tree-shaped for ILP
       float bmax[kNB];
@@ -595,6 +625,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int bi = 1; bi < kNB; ++bi) tmax = fmaxf(tmax, bmax[bi]);
       // running maximum: take m_{j-1} from the other group, publish m_j
       float m_prev = -INFINITY;
+      float hy_m0 = -INFINITY;                     // full-precision part, raw score units
+      if constexpr (HYB) {
+        if (j == 0 && row < p.S_q) hy_m0 = p.hy_part[((int64_t)bh_q * p.S_q + row) * (D + 4)] / sc;
+        if (j == 0) m_prev = hy_m0;
+      }
       if (j > 0) {
         named_bar_sync(bar_recv, 64);
         m_prev = sm.m_xchg[(j - 1) & 1][r];
@@ -700,6 +735,32 @@ __global__ void __launch_bounds__(kThreads, 1)
           add += ysum[bi] * scale;
         }
         lpt = (j >= 2 ? lpt * ex2_approx((m_acc - m_new) * sc) : 0.0f) + add;
+      }
+      if (HYB && j == 0) {
+        // group A's accumulator := the full-precision part, brought from m0 to m_new
+        // (O in MMA units: the PV products carry neither g_P nor g_v)
+        if (PERSIST && k >= 1)
+          ok = warp_wait(&sm.o_free, (k - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
+        tc_fence_after();
+        const float* src = p.hy_part + ((int64_t)bh_q * p.S_q + min(row, p.S_q - 1)) * (D + 4);
+        const float a0 = row < p.S_q ? ex2_approx((hy_m0 - m_new) * sc) : 0.0f;
+        const float gpl = MX ? 1.0f : kGpNvfp4;
+        const float so = a0 / (gpl * p.g_v), sl = a0 / gpl;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t raw[32];
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const float4 v4 = *reinterpret_cast<const float4*>(src + 4 + 32 * c + i);
+            raw[i] = __float_as_uint(v4.x * so);
+            raw[i + 1] = __float_as_uint(v4.y * so);
+            raw[i + 2] = __float_as_uint(v4.z * so);
+            raw[i + 3] = __float_as_uint(v4.w * so);
+          }
+          tmem_st32(lane_base + kColO0 + 32 * c, raw);
+        }
+        tmem_st1(lane_base + kColL0, __float_as_uint(src[1] * sl));
+        tmem_wait_st();
       }
       if (j >= 2) {
         tc_fence_after();
@@ -969,7 +1030,7 @@ static bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool MX, bool CAUSAL, bool ABL = false>
+template <int D, bool MX, bool CAUSAL, bool ABL = false, bool HYB = false>
 static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t* vt,
                                const AttnParams& prm, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
@@ -988,7 +1049,7 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
   const int n_ktiles = (prm.S_k + kBN - 1) / kBN;
   const double avg_tiles = CAUSAL ? 0.5 * (std::min(prm.n_qtiles, n_ktiles) + 1) : n_ktiles;
   const bool persist = avg_tiles <= 48.0 && prm.n_items > num_sms();
-  auto kern = persist ? attn_fwd_kernel<D, MX, CAUSAL, true, ABL> : attn_fwd_kernel<D, MX, CAUSAL, false, ABL>;
+  auto kern = persist ? attn_fwd_kernel<D, MX, CAUSAL, true, ABL, HYB> : attn_fwd_kernel<D, MX, CAUSAL, false, ABL, HYB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return FA4Q_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>(persist ? num_sms() : prm.n_items));
@@ -1028,7 +1089,7 @@ extern "C" fa4q_status fa4q_attn_fwd_ex(const uint8_t* q, const uint8_t* q_sf, c
   if (S_k == 0) return FA4Q_ERR_INVALID_ARG;
   const int n_qtiles = (S_q + kBM - 1) / kBM;
   if (static_cast<int64_t>(B) * Hq * n_qtiles > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
-  AttnParams prm;
+  AttnParams prm{};
   prm.q_sf = q_sf;
   prm.k_sf = k_sf;
   prm.vt_sf = vt_sf;
@@ -1107,4 +1168,86 @@ extern "C" fa4q_status fa4q_selftest_exp2(const float* x, float* y, int64_t n, v
 extern "C" fa4q_status fa4q_selftest_wait_timeout(uint32_t wait_us, void* stream) {
   wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(wait_us);
   return launch_status();
+}
+
+// =======================================================================================
+// hybrid-precision prefill: the full-precision part (hybrid.cu), then the FP4 part here
+// =======================================================================================
+extern "C" size_t fa4q_attn_fwd_hybrid_workspace_size(int B, int Hq, int S, int d) {
+  if (B <= 0 || Hq <= 0 || S <= 0 || d <= 0) return 0;
+  return (size_t)B * Hq * S * (d + 4) * sizeof(float);
+}
+
+extern "C" fa4q_status fa4q_attn_fwd_hybrid(
+    const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf, const uint8_t* vt,
+    const uint8_t* vt_sf, const void* q_bf16, const void* k_bf16, const void* v_bf16,
+    const int32_t* vl_pos, const int32_t* vl_count, const void* vl_k, const void* vl_v, int max_vl,
+    const uint64_t* vl_excl, float g_q, float g_k, float g_v, int B, int Hq, int Hkv, int S, int d,
+    int window, fa4q_format fmt, float qmax_p, float sm_scale, void* out, int out_is_fp32, float* lse,
+    void* workspace, size_t workspace_bytes, void* stream) {
+  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (!q || !q_sf || !k || !k_sf || !vt || !vt_sf || !q_bf16 || !k_bf16 || !v_bf16 || !out || !workspace)
+    return FA4Q_ERR_INVALID_ARG;
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || S < 0 || Hq % Hkv != 0 || window < 1 || max_vl < 0)
+    return FA4Q_ERR_INVALID_ARG;
+  if (max_vl > 0 && (!vl_pos || !vl_count || !vl_k || !vl_v || !vl_excl)) return FA4Q_ERR_INVALID_ARG;
+  if (d != 128) return FA4Q_ERR_UNSUPPORTED;
+  if (!(qmax_p >= 0.0f) || !isfinite(qmax_p)) return FA4Q_ERR_INVALID_ARG;
+  if (fmt == FA4Q_MXFP4) { g_q = g_k = g_v = 1.0f; }
+  if (!(g_q > 0.0f) || !(g_k > 0.0f) || !(g_v > 0.0f)) return FA4Q_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(q_sf) || !aligned16(k_sf) ||
+      !aligned16(vt_sf) || !aligned16(out) || !aligned16(q_bf16) || !aligned16(k_bf16) ||
+      !aligned16(v_bf16) || !aligned16(workspace) || (vl_k && !aligned16(vl_k)) || (vl_v && !aligned16(vl_v)))
+    return FA4Q_ERR_INVALID_ARG;
+  if (B == 0 || S == 0) return FA4Q_OK;
+  if (workspace_bytes < fa4q_attn_fwd_hybrid_workspace_size(B, Hq, S, d)) return FA4Q_ERR_INVALID_ARG;
+  const int n_qtiles = (S + kBM - 1) / kBM;
+  if (static_cast<int64_t>(B) * Hq * n_qtiles > 0x7fffffff || B > 65535 || Hq > 65535) return FA4Q_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float sms = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)d);
+  // 1. full-precision part: window and vertical-line keys, bf16, unquantised P
+  HyParams hp;
+  hp.q = static_cast<const uint16_t*>(q_bf16);
+  hp.k = static_cast<const uint16_t*>(k_bf16);
+  hp.v = static_cast<const uint16_t*>(v_bf16);
+  hp.vl_pos = max_vl > 0 ? vl_pos : nullptr;
+  hp.vl_count = max_vl > 0 ? vl_count : nullptr;
+  hp.vl_k = static_cast<const uint16_t*>(vl_k);
+  hp.vl_v = static_cast<const uint16_t*>(vl_v);
+  hp.part = static_cast<float*>(workspace);
+  hp.B = B;
+  hp.Hq = Hq;
+  hp.Hkv = Hkv;
+  hp.S = S;
+  hp.W = window;
+  hp.max_vl = max_vl;
+  hp.c2 = sms * kLog2e;
+  fa4q_status stt = launch_hybrid_full(hp, st);
+  if (stt != FA4Q_OK) return stt;
+  // 2. FP4 part, continuing each row's softmax from the full-precision state
+  AttnParams prm{};
+  prm.q_sf = q_sf;
+  prm.k_sf = k_sf;
+  prm.vt_sf = vt_sf;
+  prm.out = out;
+  prm.lse = lse;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.S_q = S;
+  prm.S_k = S;
+  prm.S_kpad = (S + 31) / 32 * 32;
+  prm.n_qtiles = n_qtiles;
+  prm.n_items = B * Hq * n_qtiles;
+  prm.score_scale_log2 = sms * g_q * g_k * kLog2e;
+  prm.g_v = g_v;
+  prm.qmax_p = qmax_p;
+  prm.causal = 1;
+  prm.out_fp32 = out_is_fp32;
+  prm.hy_part = static_cast<const float*>(workspace);
+  prm.hy_window = window;
+  prm.hy_excl_words = max_vl > 0 ? (S + 63) / 64 : 0;
+  prm.hy_excl = max_vl > 0 ? vl_excl : nullptr;     // read only while a word index is < hy_excl_words
+  if (fmt == FA4Q_MXFP4) return launch_attn<128, true, true, false, true>(q, k, vt, prm, st);
+  return launch_attn<128, false, true, false, true>(q, k, vt, prm, st);
 }

@@ -31,6 +31,23 @@ inline int num_sms() {
   return cached[dev];
 }
 
+// Full-precision part of the hybrid-precision prefill (hybrid.cu): per query row, the online
+// softmax state [m0 (log2 units), l0, -, -, o0[d]] (row stride d + 4) over the window and
+// vertical-line keys.
+struct HyParams {
+  const uint16_t* q;        // [B][Hq][S][d] bf16
+  const uint16_t* k;        // [B][Hkv][S][d] bf16
+  const uint16_t* v;        // [B][Hkv][S][d] bf16
+  const int32_t* vl_pos;    // [B][Hkv][max_vl] ascending positions (nullable: none)
+  const int32_t* vl_count;  // [B][Hkv]
+  const uint16_t* vl_k;     // [B][Hkv][max_vl][d] bf16 rows of the vertical lines
+  const uint16_t* vl_v;
+  float* part;              // [B][Hq][S][d + 4]
+  int B, Hq, Hkv, S, W, max_vl;
+  float c2;                 // sm_scale * log2(e)
+};
+fa4q_status launch_hybrid_full(const HyParams& p, cudaStream_t st);
+
 // Each translation unit with bounded device waits owns one status word; these host
 // functions read-and-clear them (stream-ordered, then synchronised by the caller).
 cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word);
