@@ -21,13 +21,16 @@ A plain, slow, obviously-correct numpy implementation, written from the pages:
                 outlier-spreading alternative to Smooth-QK; an ablation).
 * `hybrid`    - hybrid-precision prefill: vertical-line and window keys in BF16,
                 the rest FP4, one online softmax.
+* `bitdecode` - decode with a dual-residual FP4 query and FP4 probabilities against
+                the FP4 paged cache.
 
 Every function states the passage it follows.  Floating point is FP64 except
 where the method fixes FP32 decisions (scale selection and element rounding),
 which are taken in IEEE FP32 exactly as specified in `formats`.
 
-Parity status: `formats`, `attention`, `decode`, `smooth`, `rotate` and `hybrid` are pinned by the
+Parity status: `formats`, `attention`, `decode`, `smooth`, `rotate`, `hybrid` and `bitdecode`
+are pinned by the
 `-m "not gpu"` tests in `tests/test_oracle_*.py`.  `hyquant` is a diagnostic
 pinned only qualitatively (planted vertical lines are recovered).
 """
-from . import formats, attention, decode, smooth, hyquant, rotate, hybrid  # noqa: F401
+from . import formats, attention, decode, smooth, hyquant, rotate, hybrid, bitdecode  # noqa: F401
