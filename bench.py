@@ -9,7 +9,8 @@ MXFP4 workload (B=1, 32/8 heads, S=4096, d=128, Smooth-QK on): block quantisatio
 attention kernel.  Inputs are resident in HBM; L2 (126 MB) is flushed by a 256 MB write
 before every timed step.  The metric is prefill TFLOP/s (4*B*Hq*S^2*d, halved for causal).
 The decode path (batch 32, 32/8 heads, 32768 keys, NVFP4 pages + 5% BF16 vertical lines +
-128-token BF16 window) is timed in the same run and reported under "decode" (us/step, GB/s).
+128-token BF16 window) is timed in the same run and reported under "decode" (us/step, GB/s),
+and the FP4 tensor-core decode (dual-residual query) on the same shape under "decode_fp4q".
 
 N > 1 (torchrun): every rank runs its own independent batch (weak scaling, no collective on
 the data path); the step time is the max over ranks.  `--impl reference` times the CPU oracle
@@ -340,6 +341,77 @@ def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
                       "l2": "working set 1.4 GB > L2", "clocks": dsampler.summary()}
 
 
+def decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
+    """Time the FP4 tensor-core decode (dual-residual query, all-FP4 paged cache) on the
+    decode workload's shape; adds line["decode_fp4q"]."""
+    import torch
+    dw = synth.WORKLOADS[4]
+    if args.decode_batch:
+        import dataclasses
+        dw = dataclasses.replace(dw, B=args.decode_batch)
+    B, Hq, Hkv, d, L = dw.B, dw.Hq, dw.Hkv, dw.d, dw.L
+    P = (L + 63) // 64
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4242)
+    i32 = lambda a: torch.from_numpy(np.ascontiguousarray(a).astype(np.int32)).to(dev)
+    table = i32(np.random.default_rng(4242).permutation(B * P).reshape(B, P))
+    lens = i32(np.full(B, L))
+    # quantise the cache one sequence at a time (a BF16 copy of the whole cache is 4 GB)
+    kp = torch.empty((B * P, Hkv, 64, d // 2), dtype=torch.uint8, device=dev)
+    vp = torch.empty((B * P, Hkv, d, 32), dtype=torch.uint8, device=dev)
+    ks = vs = None
+    for b in range(B):
+        k = (torch.randn((1, Hkv, L, d), generator=gen, device=dev) * 1.5).to(torch.bfloat16)
+        v = torch.randn((1, Hkv, L, d), generator=gen, device=dev).to(torch.bfloat16)
+        tb = torch.arange(P, dtype=torch.int32, device=dev).view(1, P)
+        kpb, ksb, vpb, vsb = fa4q.quantize_kv_pages(k, v, lens[b:b + 1], None, tb, P)
+        if ks is None:
+            ks = torch.empty((B * P,) + tuple(ksb.shape[1:]), dtype=ksb.dtype, device=dev)
+            vs = torch.empty((B * P,) + tuple(vsb.shape[1:]), dtype=vsb.dtype, device=dev)
+        rows = table[b].long()
+        kp[rows], vp[rows], ks[rows], vs[rows] = kpb, vpb, ksb, vsb
+        del k, v
+    q = (torch.randn((B, Hq, d), generator=gen, device=dev) * 1.5).to(torch.bfloat16)
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(int(fa4q.lib().fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, d, P, 0)),
+                     dtype=torch.uint8, device=dev)
+    splits, tps = fa4q.decode_fp4q_plan(B, Hq, Hkv, P)
+    step = lambda: fa4q.decode_fp4q(q, kp, ks, vp, vs, table, lens, B * P, out=out, workspace=ws)
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    assert fa4q.device_status()[0] == 0
+    nbytes = (2 * B * Hkv * P * 64 * (d // 2 + d // 16)   # FP4 K and V^T pages + UE4M3 scales
+              + B * P * 4 + B * 4 + 2 * B * Hq * d * 2)   # block table, lengths, q, out
+    dsteps = max(20, args.steps)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        e0.record()
+        for _ in range(dsteps):
+            step()
+        e1.record()
+        barrier()
+    ms = e0.elapsed_time(e1) / dsteps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line["decode_fp4q"] = {
+        "workload": f"{dw.name} shape, all {L} keys FP4 (NVFP4 pages)", "us_per_step": ms * 1e3,
+        "higher_is_better": False, "GBps": gbs, "bytes_per_step": nbytes, "gpu_launches": 3 * dsteps,
+        "splits": splits, "tiles_per_split": tps,
+        "roofline": {"kernel": "attn_fwd_kernel<DEC>+dec_query_kernel+decode_combine_kernel", "bound": "hbm",
+                     "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                     "traffic": None, "peak_source": f"{peak_kind} hbm copy"},
+        "note": "dual-residual NVFP4 query and PNQ probabilities on the block-scaled tensor cores "
+                "(BitDecoding-FP4); seeded gaussian cache, not the hybrid cache of line['decode']",
+        "l2": "working set 1.2 GB > L2", "clocks": sampler.summary()}
+    del kp, vp, ks, vs, ws
+
+
 # ------------------------------------------------------------------------------ CPU oracle timing
 def oracle_prefill_sample(w, budget_s: float, host=None):
     """Time the oracle on sampled (head, row) work of workload w for about budget_s seconds;
@@ -379,6 +451,8 @@ def main():
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode path")
+    ap.add_argument("--decode-fp4q-only", action="store_true",
+                    help="time only the FP4 tensor-core decode (dual-residual query)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="decode batch (0 = the workload's 32); smaller batches are for profiling")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -424,9 +498,10 @@ def main():
     torch.cuda.set_device(dev)
     hbm_gbs, bf16_tf, bf16_tf_sus, peak_kind = load_peaks()
 
-    if args.decode_only:
+    if args.decode_only or args.decode_fp4q_only:
         line = {"metric": METRIC, "n_gpus": world}
-        decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier=lambda: torch.cuda.synchronize())
+        bench_fn = decode_fp4q_bench if args.decode_fp4q_only else decode_bench
+        bench_fn(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier=lambda: torch.cuda.synchronize())
         print(json.dumps(line))
         return
     run = PrefillRun(w, dev, fa4q, seed_offset=rank)
@@ -583,6 +658,8 @@ def main():
         del run, flush
         torch.cuda.empty_cache()
         decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier)
+        torch.cuda.empty_cache()
+        decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, desc, _ = oracle_prefill_sample(w, 12.0)

@@ -323,6 +323,40 @@ fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const uint8_t* k_
                         int num_splits, void* stream);
 
 /*
+ * fa4q_decode_fp4q - decode with FP4 tensor-core products on both sides over an all-FP4
+ * paged cache: a dual-residual NVFP4 query, and the probabilities quantised before PV.
+ *
+ * Source: BitDecoding-FP4, "Error Sources" (the query as the sum of two FP4 tensors, the
+ * second quantising the residual of the first, keeps the logits close) and "System-Level
+ * Optimization" (the softmax transposed so that P is quantised inside its reduction; query
+ * MMAs stacked over the paged cache).  Reading: q1 = NVFP4(q), r = q - deq(q1) in FP32,
+ * q2 = NVFP4(r); scores = (deq(q1) + deq(q2)) . k_hat; the keys of a sequence are scanned in
+ * tiles of 128 positions (page pairs, in position order) with pre-normalisation quantisation
+ * of P against the running maximum (NVFP4, g_P = 1/(6*448)) and the normaliser from P_hat,
+ * as the prefill; the scan is cut into splits of T = ceil(ceil(max_pages / 2) / S) tiles,
+ * S = num_splits or, for 0, ceil(1184 / (B * Hkv)), clamped to [1, ceil(max_pages / 2)];
+ * each split restarts the running state and the splits merge exactly (log-sum-exp), so T is
+ * part of the result.  The GQA heads of a kv-head share one 128-row query tile (rows
+ * 0..Hq/Hkv-1), both residuals in one accumulation.
+ *
+ * q           bf16 [B][Hq][d]; out bf16 [B][Hq][d].  d = 128, Hq % Hkv == 0.
+ * k_pages ... the NVFP4 paged cache of fa4q_quantize_kv_pages (every position 0..fp4_len-1
+ *             in FP4; no vertical-line set or window here); n_phys_pages = its page count.
+ * g_k, g_v    NVFP4 tensor scales of the pages.  sm_scale 0 -> 1/sqrt(d).
+ * workspace   device, >= fa4q_decode_fp4q_workspace_size(...) bytes, 16-byte aligned: the
+ *             query tiles and the split partials.
+ * MXFP4 pages -> FA4Q_ERR_UNSUPPORTED.  Other errors as fa4q_decode.  Three launches
+ * (query tiles, the tcgen05 scan, the combine), asynchronous on `stream`.
+ */
+size_t fa4q_decode_fp4q_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int num_splits);
+fa4q_status fa4q_decode_fp4q(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
+                             const uint8_t* vt_pages, const uint8_t* vt_sf, const int32_t* block_table,
+                             const int32_t* fp4_len, int n_phys_pages, int B, int Hq, int Hkv, int d,
+                             int max_pages, fa4q_format fmt, float g_k, float g_v, float sm_scale,
+                             void* out, void* workspace, size_t workspace_bytes, int num_splits,
+                             void* stream);
+
+/*
  * fa4q_decode_noalloc - fa4q_decode for callers that cannot allocate device memory.
  *
  * The paper has no counterpart to this call; it is a deployment convenience.  Some callers

@@ -26,6 +26,7 @@ EXPORTED = [
     "fa4q_status_string", "fa4q_version", "fa4q_sf_tiled_bytes", "fa4q_quantize",
     "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_attn_fwd_ex", "fa4q_quantize_kv_pages",
     "fa4q_quantize_rotated", "fa4q_attn_fwd_hybrid", "fa4q_attn_fwd_hybrid_workspace_size",
+    "fa4q_decode_fp4q", "fa4q_decode_fp4q_workspace_size",
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
     "fa4q_vlines_workspace_size", "fa4q_select_vertical_lines", "fa4q_quantize_qkv",
@@ -61,6 +62,10 @@ def lib() -> ctypes.CDLL:
         L.fa4q_attn_fwd_hybrid.restype = I
         L.fa4q_attn_fwd_hybrid.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, I, P, F, F, F, I, I, I, I, I,
                                            I, I, F, F, P, I, P, P, Z, P]
+        L.fa4q_decode_fp4q_workspace_size.restype = Z
+        L.fa4q_decode_fp4q_workspace_size.argtypes = [I, I, I, I, I, I]
+        L.fa4q_decode_fp4q.restype = I
+        L.fa4q_decode_fp4q.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, F, F, P, P, Z, I, P]
         L.fa4q_quantize_rotated.restype = I
         L.fa4q_quantize_rotated.argtypes = [P, I64, I64, I64, I64, I, F, F, P, I64, I64, I, P, P, P]
         L.fa4q_smooth_calibrate.restype = I
@@ -204,6 +209,34 @@ def attn_fwd_hybrid(q, q_sf, k, k_sf, vt, vt_sf, q_bf16, k_bf16, v_bf16, vl_pos,
         _ptr(v_bf16), _ptr(vl_pos), _ptr(vl_count), _ptr(vl_k), _ptr(vl_v), max_vl, _ptr(vl_excl), g_q, g_k,
         g_v, B, Hq, Hkv, S, d, window, _fmt(fmt), qmax_p, sm_scale, _ptr(out), int(out_fp32), _ptr(lse),
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return out
+
+
+def decode_fp4q_plan(B, Hq, Hkv, max_pages, num_splits=0):
+    """(splits, tiles per split) fa4q_decode_fp4q uses (the rule in fa4q.h)."""
+    tiles = (max_pages + 1) // 2
+    s = num_splits if num_splits > 0 else -(-148 * 8 // (B * Hkv))
+    s = max(1, min(s, max(1, tiles)))
+    tps = max(1, -(-tiles // s))
+    return max(1, -(-tiles // tps)), tps
+
+
+def decode_fp4q(q, k_pages, k_sf, vt_pages, vt_sf, block_table, fp4_len, n_phys_pages, *, fmt="nvfp4",
+                g_k=1.0, g_v=1.0, sm_scale=0.0, num_splits=0, out=None, workspace=None, stream=None):
+    """FP4 tensor-core decode with a dual-residual query (fa4q_decode_fp4q); out [B, Hq, d]."""
+    import torch
+    B, Hq, d = q.shape
+    Hkv = k_pages.shape[1]
+    max_pages = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
+    if workspace is None:
+        need = int(lib().fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, d, max_pages, num_splits))
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check("fa4q_decode_fp4q", lib().fa4q_decode_fp4q(
+        _ptr(q), _ptr(k_pages), _ptr(k_sf), _ptr(vt_pages), _ptr(vt_sf), _ptr(block_table), _ptr(fp4_len),
+        n_phys_pages, B, Hq, Hkv, d, max_pages, _fmt(fmt), g_k, g_v, sm_scale, _ptr(out), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), num_splits, _stream(stream)))
     return out
 
 

@@ -43,6 +43,7 @@ namespace fa4q {
 static __device__ uint32_t g_attn_status;
 
 constexpr int kBM = 128;
+constexpr int kDecHeadDim = 128;   // head dimension of the FP4 tensor-core decode
 constexpr int kBN = 128;
 constexpr int kThreads = 384;
 // Register split (setmaxnreg): launched at 168 per thread (3 warps per scheduler x 168 x 32 =
@@ -94,6 +95,7 @@ struct __align__(1024) Smem {
   uint8_t sfv[kStages][2 * 512];
   uint8_t sfp[2][2 * 512];
   uint8_t sfone[2 * 512];
+  uint8_t sfraw[kStages][4 * 512];   // decode: raw page scales (K of 2 pages, V^T of 2 pages)
   uint64_t bar_q[2];         // Q tile (and its scales) of work item k landed, slot k % 2
   uint64_t q_free[2];        // all S products of work item k issued and complete
   uint64_t o_free;           // all eight softmax warps have read O and l in the epilogue
@@ -104,6 +106,7 @@ struct __align__(1024) Smem {
   uint64_t p_full[2];
   uint64_t o_done[2];
   uint64_t drain;
+  uint64_t sf_ready[kStages];  // decode: the stage's scales permuted into atoms (warps 2, 3)
   float m_xchg[2][kBM];       // running maximum after tile j, slot j%2, per row
   float m_last[2][kBM];       // per group: the maximum its accumulator is relative to
   float l_last[2][kBM];       // per group: the normaliser summed from P~ (ablation only)
@@ -145,6 +148,16 @@ struct AttnParams {
   const uint64_t* hy_excl;   // [B][Hkv][hy_excl_words]
   int hy_window;
   int hy_excl_words;
+  // FP4 tensor-core decode (BitDecoding-FP4): items are (sequence, kv-head, split); the
+  // query tile holds the group's q-heads in rows 0..G-1 as two residual tiles (slots 0, 1);
+  // key tiles are page pairs of the paged cache through the block table; the epilogue
+  // writes split partials [m (log2 units), l, o[D]] for the combine kernel.
+  const int32_t* dec_table;  // [B][dec_max_pages]
+  const int32_t* dec_len;    // [B] cached tokens
+  const uint8_t* dec_ksf;    // page K scales [P][Hkv][64][D/16]
+  const uint8_t* dec_vsf;    // page V^T scales [P][Hkv][D][4]
+  float* dec_ws;             // [B*Hq][dec_splits][D + 2]
+  int dec_max_pages, dec_splits, dec_tiles_per_split;
   int causal;
   int out_fp32;
 };
@@ -316,7 +329,8 @@ FA4Q_DEVINL void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, int N
 // ABL: the ablations of fa4q_attn_fwd_ex (conditional rescaling, normaliser from P~) are
 // compiled into separate instantiations so the default kernel carries none of their work.
 // HYB: the FP4 part of the hybrid-precision prefill (causal only).
-template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL, bool HYB = false>
+// DEC: the FP4 tensor-core decode (non-causal, non-persistent, NVFP4, D = 128).
+template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL, bool HYB = false, bool DEC = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -345,7 +359,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   auto decode_item = [&](int u) -> Item {
     Item it;
-    if (CAUSAL) {
+    if constexpr (DEC) {
+      const int grp = u / p.dec_splits, split = u - grp * p.dec_splits;
+      it.b = grp / p.Hkv;
+      it.h = grp - it.b * p.Hkv;                 // the kv-head
+      it.qt = split;
+      const int L = max(0, min(p.dec_len[it.b], p.dec_max_pages * 64));
+      const int n_all = (L + kBN - 1) / kBN;
+      it.n_tiles = max(0, min(p.dec_tiles_per_split, n_all - split * p.dec_tiles_per_split));
+    } else if (CAUSAL) {
       const int per = p.B * p.Hq, rem = u % per;
       it.qt = p.n_qtiles - 1 - u / per;
       it.b = rem / p.Hq;
@@ -385,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.o_free, 8);
     mbar_init(&sm.drain, 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(&sm.sf_ready[s], 2);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -424,6 +447,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = decode_item(u);
         const int bh_q = it.b * p.Hq + it.h, bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
         const int qs = k & 1;
+        if constexpr (DEC) {
+          // both residual query tiles, then page pairs through the block table (a missing
+          // second page repeats the first: its keys are masked, its data finite)
+          if (it.n_tiles == 0) break;
+          const int grp = it.b * p.Hkv + it.h;
+          mbar_arrive_expect_tx(&sm.bar_q[0], 2 * (C::kQBytes + C::kSfQAtoms * 512));
+          for (int r = 0; r < 2; ++r) {
+            tma_load_3d(sm.q[r], &tm_q, 0, 0, grp * 2 + r, &sm.bar_q[0]);
+            bulk_load(sm.sfq[r], p.q_sf + ((int64_t)grp * 2 + r) * C::kSfQAtoms * 512, C::kSfQAtoms * 512,
+                      &sm.bar_q[0]);
+          }
+          q_issued = 1;
+          const int L = max(0, min(p.dec_len[it.b], p.dec_max_pages * 64));
+          const int n_pages = (L + 63) / 64, t0 = it.qt * p.dec_tiles_per_split;
+          for (int j = 0; j < it.n_tiles; ++j, ++T) {
+            const int s = T % kStages;
+            if (T >= kStages && !cta_wait(&sm.kv_empty[s], ((T / kStages) - 1) & 1, abort_flag,
+                                          kStatusTimeoutTmaFull)) {
+              go = false;
+              break;
+            }
+            const int lp0 = 2 * (t0 + j), lp1 = min(lp0 + 1, n_pages - 1);
+            const int ph0 = p.dec_table[(int64_t)it.b * p.dec_max_pages + lp0] * p.Hkv + it.h;
+            const int ph1 = p.dec_table[(int64_t)it.b * p.dec_max_pages + lp1] * p.Hkv + it.h;
+            mbar_arrive_expect_tx(&sm.kv_full[s], C::kKBytes + C::kVBytes + 4 * 512);
+            tma_load_3d(sm.k[s], &tm_k, 0, 0, ph0, &sm.kv_full[s]);
+            tma_load_3d(sm.k[s] + C::kKBytes / 2, &tm_k, 0, 0, ph1, &sm.kv_full[s]);
+            tma_load_3d(sm.v[s], &tm_v, 0, 0, ph0, &sm.kv_full[s]);
+            tma_load_3d(sm.v[s] + C::kVBytes / 2, &tm_v, 0, 0, ph1, &sm.kv_full[s]);
+            bulk_load(sm.sfraw[s], p.dec_ksf + (int64_t)ph0 * 512, 512, &sm.kv_full[s]);
+            bulk_load(sm.sfraw[s] + 512, p.dec_ksf + (int64_t)ph1 * 512, 512, &sm.kv_full[s]);
+            bulk_load(sm.sfraw[s] + 1024, p.dec_vsf + (int64_t)ph0 * 512, 512, &sm.kv_full[s]);
+            bulk_load(sm.sfraw[s] + 1536, p.dec_vsf + (int64_t)ph1 * 512, 512, &sm.kv_full[s]);
+          }
+          continue;
+        }
         // Q slot qs was last read by the S products of item k-2
         if (k >= 2 && !cta_wait(&sm.q_free[qs], ((k - 2) >> 1) & 1, abort_flag, kStatusTimeoutTmaFull)) break;
         mbar_arrive_expect_tx(&sm.bar_q[qs], C::kQBytes + C::kSfQAtoms * 512);
@@ -468,11 +527,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u < 0) break;
         const Item it = decode_item(u);
         const int qs = k & 1, T0 = T, n_tiles = it.n_tiles;
+        if (DEC && n_tiles == 0) break;            // empty split: the softmax threads write it
         if (!cta_wait(&sm.bar_q[qs], (k >> 1) & 1, abort_flag, kStatusTimeoutMma)) break;
         tc_fence_after();
         // item k-2 used this scale slot; all of its products completed before item k-1 ended
         for (int a = 0; a < C::kSfQAtoms; ++a)
           tmem_cp_sf_atom(tmem + kColSfQ + 8 * qs + 4 * a, smem_u32(sm.sfq[qs] + 512 * a));
+        if constexpr (DEC) {                       // second residual tile: slot 1
+          for (int a = 0; a < C::kSfQAtoms; ++a)
+            tmem_cp_sf_atom(tmem + kColSfQ + 8 + 4 * a, smem_u32(sm.sfq[1] + 512 * a));
+        }
         const uint32_t q_addr = smem_u32(sm.q[qs]);
         // S_j = Q K_j^T into the single S buffer once the softmax group of the previous key
         // tile (of this item or the last) holds its scores in registers
@@ -480,15 +544,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int t = T0 + j, s = t % kStages, kb = t & 1;
           if (!cta_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag, kStatusTimeoutMma)) return false;
           if (t >= 1 && !cta_wait(&sm.s_free, (t - 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
+          if (DEC && !cta_wait(&sm.sf_ready[s], (t / kStages) & 1, abort_flag, kStatusTimeoutMma)) return false;
           tc_fence_after();
           for (int a = 0; a < C::kSfQAtoms; ++a)
             tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
           const uint32_t k_addr = smem_u32(sm.k[s]);
+          if constexpr (DEC) {
+            // dual-residual query: S = Q1 K^T + Q2 K^T, K-steps 0,1 of each residual tile
+            const uint32_t q2_addr = smem_u32(sm.q[1]);
 #pragma unroll
-          for (int ks = 0; ks < C::kKStepsQK; ++ks) {
-            const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-            const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-            mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ + 8 * qs, tmem + kColSfK + 8 * kb, ks > 0);
+            for (int ks = 0; ks < 2 * C::kKStepsQK; ++ks) {
+              const int r = ks / C::kKStepsQK, st = ks % C::kKStepsQK;
+              const uint64_t ad = make_smem_desc((r ? q2_addr : q_addr) + 32 * st, 16, C::kQKSbo, C::kQKSwizzle);
+              const uint64_t bd = make_smem_desc(k_addr + 32 * st, 16, C::kQKSbo, C::kQKSwizzle);
+              mma_step<MX>(tmem + kColS, ad, bd, kBN, st, tmem + kColSfQ + 8 * r, tmem + kColSfK + 8 * kb, ks > 0);
+            }
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < C::kKStepsQK; ++ks) {
+              const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+              const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+              mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ + 8 * qs, tmem + kColSfK + 8 * kb, ks > 0);
+            }
           }
           tc_commit(&sm.s_full[j & 1]);
           return true;
@@ -513,7 +590,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
+            // decode: V^T of each page is its own [D][32 B] tile (32-byte swizzle), one K-step
+            const uint64_t vd = DEC ? make_smem_desc(v_addr + (C::kVBytes / 2) * ks, 16, 256, kSwiz32)
+                                    : make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
             const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
             // (hybrid: group A's accumulator starts from the full-precision part)
             const uint32_t acc = (jp >= 2 || ks > 0 || (HYB && jp == 0)) ? 1u : 0u;
@@ -539,6 +618,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: all MMAs this thread issued complete before TMEM is released
       tc_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, &g_attn_status, kStatusTimeoutDrain);
+    }
+  } else if (DEC) {
+    // ------------------------------------------------------------ decode: scale atoms
+    // Warps 2 and 3 move each tile's raw page scales into the scale-atom layout of the
+    // MMA (byte (r % 32) * 16 + (r / 32) * 4 + k of a 512-byte atom, row r, scale k of the
+    // K-step): K rows are the 128 tokens of the page pair (atoms = halves of d), V^T rows
+    // are the 128 channels (atom = page).  Stage s was last read by the tcgen05.cp of tile
+    // t - kStages, which completed before the producer refilled the stage.
+    const int u = item_index(0);
+    if (u >= 0) {
+      const Item it = decode_item(u);
+      const int t64 = (warp - 2) * 32 + lane;
+      for (int t = 0; t < it.n_tiles; ++t) {
+        const int s = t % kStages;
+        if (!warp_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag, kStatusTimeoutMma)) break;
+        const uint32_t* raw = reinterpret_cast<const uint32_t*>(sm.sfraw[s]);
+        for (int i = t64; i < 256; i += 64) {      // K: word i = page * 128 + token * 2 + half
+          const int rr = ((i >> 7) << 6) + ((i >> 1) & 63);
+          *reinterpret_cast<uint32_t*>(sm.sfk[s] + 512 * (i & 1) + (rr & 31) * 16 + (rr >> 5) * 4) = raw[i];
+        }
+        for (int i = t64; i < 256; i += 64) {      // V^T: word i = page * 128 + channel
+          const int ch = i & 127;
+          *reinterpret_cast<uint32_t*>(sm.sfv[s] + 512 * (i >> 7) + (ch & 31) * 16 + (ch >> 5) * 4) = raw[256 + i];
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.sf_ready[s]);
+      }
     }
   }
   } else {
@@ -576,6 +683,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_acc = -INFINITY;                       // maximum of this group's last tile
     float lpt = 0.0f;                              // sum of P~ of this group (ABL), MMA units
     const float gp_item = ABL ? p.gp : kGpNvfp4;
+    int dec_len = 0, dec_key0 = 0;                 // decode: cached tokens, first key of the split
+    if constexpr (DEC) {
+      dec_len = max(0, min(p.dec_len[it.b], p.dec_max_pages * 64));
+      dec_key0 = it.qt * p.dec_tiles_per_split * kBN;
+      if (n_tiles == 0) {
+        // a split with no key: partial (m, l, o) = (-inf, 0, 0); the other roles skip it too
+        const int G = p.Hq / p.Hkv;
+        if (r < G) {
+          float* dst = p.dec_ws + (((int64_t)it.b * p.Hq + it.h * G + r) * p.dec_splits + it.qt) * (D + 2);
+          if (g == 0) {
+            dst[0] = -INFINITY;
+            dst[1] = 0.0f;
+          }
+          for (int c = g * (D / 2); c < (g + 1) * (D / 2); ++c) dst[2 + c] = 0.0f;
+        }
+        continue;
+      }
+    }
     for (int j = g; j < n_tiles; j += 2) {
       ok = warp_wait(&sm.s_full[g], (done_g + (j >> 1)) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       tc_fence_after();
@@ -595,17 +720,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&sm.s_free);
       // masking: keys beyond S_k, and (causal) keys after this query
       const int key0 = j * kBN;
-      if constexpr (HYB) {
+      if constexpr (DEC) {
+        // decode: positions at or past the cached length
+        const int lim = dec_len - (dec_key0 + key0);
+        if (lim < kBN) {
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            if (i >= lim) s[i] = -INFINITY;
+        }
+      } else if constexpr (HYB) {
         // FP4 keys of row i: key <= i - window and not a vertical line
         const int lim = min(p.S_k - key0, row - p.hy_window - key0 + 1);
         const uint64_t* ex = p.hy_excl + (int64_t)(it.b * p.Hkv + it.h / (p.Hq / p.Hkv)) * p.hy_excl_words;
         const int w0 = key0 >> 6;
         const uint64_t e0 = w0 < p.hy_excl_words ? ex[w0] : 0ull;
         const uint64_t e1 = w0 + 1 < p.hy_excl_words ? ex[w0 + 1] : 0ull;
+        const uint32_t ew[4] = {static_cast<uint32_t>(e0), static_cast<uint32_t>(e0 >> 32),
+                                static_cast<uint32_t>(e1), static_cast<uint32_t>(e1 >> 32)};
 #pragma unroll
-        for (int i = 0; i < kBN; ++i) {
-          const uint64_t w = i < 64 ? e0 : e1;
-          if (i >= lim || ((w >> (i & 63)) & 1ull)) s[i] = -INFINITY;
+        for (int q4 = 0; q4 < 4; ++q4) {
+          if (ew[q4] == 0u) continue;              // no vertical line among these 32 keys
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (ew[q4] & (1u << i)) s[32 * q4 + i] = -INFINITY;
+        }
+        if (lim < kBN) {                           // the window band (the last FP4 tiles)
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
+            if (i >= lim) s[i] = -INFINITY;
         }
       } else {
         const bool edge = (key0 + kBN > p.S_k) || (CAUSAL && key0 + kBN - 1 > qt * kBM);
@@ -823,8 +965,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float lb = (ABL && p.l_from_ptilde) ? sm.l_last[1][r] : __uint_as_float(lrb);
       const float l = la * wa + (has_b ? lb * wb : 0.0f);
       const float inva = p.g_v / l * wa, invb = p.g_v / l * wb;
-      const bool store = row < p.S_q;
+      const bool store = !DEC && row < p.S_q;
       const int64_t orow = (int64_t)bh_q * p.S_q + row;
+      if constexpr (DEC) {
+        // split partial of q-head r of the group: m in log2 units, l and o in true units
+        // (the PV products carry neither g_P nor g_v)
+        const int G = p.Hq / p.Hkv;
+        if (r < G) {
+          float* dst = p.dec_ws + (((int64_t)it.b * p.Hq + it.h * G + r) * p.dec_splits + it.qt) * (D + 2);
+          const float so = kGpNvfp4 * p.g_v;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            const int ocol = g * (D / 2) + 32 * c;
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              dst[2 + ocol + i] = (__uint_as_float(rawa[c][i]) * wa + (has_b ? __uint_as_float(rawb[c][i]) * wb : 0.0f)) * so;
+          }
+          if (g == 0) {
+            dst[0] = m * sc;
+            dst[1] = l * kGpNvfp4;
+          }
+        }
+      }
       if (store) {
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -1250,4 +1412,107 @@ extern "C" fa4q_status fa4q_attn_fwd_hybrid(
   prm.hy_excl = max_vl > 0 ? vl_excl : nullptr;     // read only while a word index is < hy_excl_words
   if (fmt == FA4Q_MXFP4) return launch_attn<128, true, true, false, true>(q, k, vt, prm, st);
   return launch_attn<128, false, true, false, true>(q, k, vt, prm, st);
+}
+
+// =======================================================================================
+// FP4 tensor-core decode (BitDecoding-FP4): dual-residual FP4 query tiles, the prefill
+// kernel's tcgen05 pipeline over page pairs of the paged cache, split partials, combine
+// =======================================================================================
+namespace fa4q {
+
+struct DecPlan {
+  int splits, tiles_per_split;
+  size_t off_qt, off_qsf, total;
+};
+
+static DecPlan dec_plan(int B, int Hq, int Hkv, int max_pages, int num_splits) {
+  DecPlan pl;
+  const int tiles = (max_pages + 1) / 2;                       // page pairs of the longest sequence
+  int s = num_splits > 0 ? num_splits : (148 * 8 + B * Hkv - 1) / (B * Hkv);
+  s = std::max(1, std::min(s, std::max(1, tiles)));
+  pl.tiles_per_split = std::max(1, (tiles + s - 1) / s);
+  pl.splits = std::max(1, (tiles + pl.tiles_per_split - 1) / pl.tiles_per_split);
+  const size_t part = (size_t)B * Hq * pl.splits * (kDecHeadDim + 2) * sizeof(float);
+  pl.off_qt = (part + 1023) / 1024 * 1024;
+  pl.off_qsf = pl.off_qt + (size_t)B * Hkv * 2 * kBM * (kDecHeadDim / 2);
+  pl.total = pl.off_qsf + (size_t)B * Hkv * 2 * 2 * 512;
+  return pl;
+}
+
+}  // namespace fa4q
+
+extern "C" size_t fa4q_decode_fp4q_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int num_splits) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || d != kDecHeadDim || max_pages <= 0 || num_splits < 0) return 0;
+  return dec_plan(B, Hq, Hkv, max_pages, num_splits).total;
+}
+
+extern "C" fa4q_status fa4q_decode_fp4q(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
+                                        const uint8_t* vt_pages, const uint8_t* vt_sf,
+                                        const int32_t* block_table, const int32_t* fp4_len,
+                                        int n_phys_pages, int B, int Hq, int Hkv, int d, int max_pages,
+                                        fa4q_format fmt, float g_k, float g_v, float sm_scale, void* out,
+                                        void* workspace, size_t workspace_bytes, int num_splits,
+                                        void* stream) {
+  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
+  if (fmt == FA4Q_MXFP4) return FA4Q_ERR_UNSUPPORTED;          // the query residuals are NVFP4
+  if (!q || !k_pages || !k_sf || !vt_pages || !vt_sf || !block_table || !fp4_len || !out || !workspace)
+    return FA4Q_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_pages <= 0 || n_phys_pages <= 0 || num_splits < 0)
+    return FA4Q_ERR_INVALID_ARG;
+  if (d != kDecHeadDim || Hq / Hkv > kBM) return FA4Q_ERR_UNSUPPORTED;
+  if (!(g_k > 0.0f) || !(g_v > 0.0f)) return FA4Q_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(k_sf) || !aligned16(vt_pages) || !aligned16(vt_sf) ||
+      !aligned16(out) || !aligned16(workspace))
+    return FA4Q_ERR_INVALID_ARG;
+  if ((int64_t)n_phys_pages * Hkv > 0x7fffffff || (int64_t)B * Hkv * 2 > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
+  const DecPlan pl = dec_plan(B, Hq, Hkv, max_pages, num_splits);
+  if (workspace_bytes < pl.total) return FA4Q_ERR_INVALID_ARG;
+  if ((int64_t)B * Hkv * pl.splits > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* qt = ws + pl.off_qt;
+  uint8_t* qt_sf = ws + pl.off_qsf;
+  fa4q_status stt = launch_dec_query(static_cast<const uint16_t*>(q), B, Hq, Hkv, qt, qt_sf, st);
+  if (stt != FA4Q_OK) return stt;
+  CUtensorMap tq, tk, tv;
+  if (!make_map_3d(&tq, qt, kDecHeadDim / 2, kBM, (uint64_t)B * Hkv * 2, kDecHeadDim / 2, kBM,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_3d(&tk, k_pages, kDecHeadDim / 2, 64, (uint64_t)n_phys_pages * Hkv, kDecHeadDim / 2, 64,
+                   CU_TENSOR_MAP_SWIZZLE_64B) ||
+      !make_map_3d(&tv, vt_pages, 32, kDecHeadDim, (uint64_t)n_phys_pages * Hkv, 32, kDecHeadDim,
+                   CU_TENSOR_MAP_SWIZZLE_32B))
+    return FA4Q_ERR_CUDA;
+  const float sms = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)d);
+  AttnParams prm{};
+  prm.q_sf = qt_sf;
+  prm.k_sf = k_sf;
+  prm.vt_sf = vt_sf;
+  prm.out = out;
+  prm.B = B;
+  prm.Hq = Hq;
+  prm.Hkv = Hkv;
+  prm.S_q = kBM;
+  prm.S_k = kBN;
+  prm.S_kpad = kBN;
+  prm.n_qtiles = 1;
+  prm.n_items = B * Hkv * pl.splits;
+  prm.score_scale_log2 = sms * g_k * kLog2e;
+  prm.g_v = g_v;
+  prm.qmax_p = 0.0f;
+  prm.dec_table = block_table;
+  prm.dec_len = fp4_len;
+  prm.dec_ksf = k_sf;
+  prm.dec_vsf = vt_sf;
+  prm.dec_ws = reinterpret_cast<float*>(ws);
+  prm.dec_max_pages = max_pages;
+  prm.dec_splits = pl.splits;
+  prm.dec_tiles_per_split = pl.tiles_per_split;
+  auto kern = attn_fwd_kernel<kDecHeadDim, false, false, false, false, false, true>;
+  const size_t smem = sizeof(Smem<kDecHeadDim, false>) + 1024;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return FA4Q_ERR_CUDA;
+  kern<<<static_cast<unsigned>(prm.n_items), kThreads, smem, st>>>(tq, tk, tv, prm);
+  stt = launch_status();
+  if (stt != FA4Q_OK) return stt;
+  return launch_decode_combine(reinterpret_cast<const float*>(ws), B * Hq, pl.splits, static_cast<uint16_t*>(out), st);
 }

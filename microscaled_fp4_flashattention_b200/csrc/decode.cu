@@ -555,6 +555,11 @@ __global__ void decode_combine_kernel(const float* __restrict__ ws, int n_rows, 
   *reinterpret_cast<uint2*>(out + (int64_t)row * kDecD + lane * 4) = w;
 }
 
+fa4q_status launch_decode_combine(const float* ws, int rows, int splits, uint16_t* out, cudaStream_t st) {
+  decode_combine_kernel<<<(rows + 3) / 4, 128, 0, st>>>(ws, rows, splits, out);
+  return launch_status();
+}
+
 cudaError_t decode_status_fetch(cudaStream_t st, uint32_t* host_word) {
   cudaError_t e = cudaMemcpyFromSymbolAsync(host_word, g_decode_status, sizeof(uint32_t), 0,
                                             cudaMemcpyDeviceToHost, st);

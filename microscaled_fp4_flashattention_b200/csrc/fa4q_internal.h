@@ -48,6 +48,14 @@ struct HyParams {
 };
 fa4q_status launch_hybrid_full(const HyParams& p, cudaStream_t st);
 
+// Dual-residual NVFP4 query tiles of the FP4 tensor-core decode (quantize.cu): q bf16
+// [B][Hq][128] -> qt [B*Hkv][2][128][64] packed, qt_sf [B*Hkv][2][2][512] tiled atoms.
+fa4q_status launch_dec_query(const uint16_t* q, int B, int Hq, int Hkv, uint8_t* qt, uint8_t* qt_sf,
+                             cudaStream_t st);
+// log-sum-exp merge of decode split partials [rows][splits][d + 2] (m in log2 units, l, o)
+// into bf16 rows (decode.cu)
+fa4q_status launch_decode_combine(const float* ws, int rows, int splits, uint16_t* out, cudaStream_t st);
+
 // Each translation unit with bounded device waits owns one status word; these host
 // functions read-and-clear them (stream-ordered, then synchronised by the caller).
 cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word);

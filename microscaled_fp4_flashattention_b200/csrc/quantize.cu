@@ -578,6 +578,67 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
   return launch_status();
 }
 
+namespace fa4q {
+
+// ---------------------------------------------------------------------------------------
+// Dual-residual NVFP4 query tiles for the FP4 tensor-core decode (BitDecoding-FP4, "Error
+// Sources": the query as the sum of two FP4 tensors, the second quantising the residual of
+// the first).  Per (sequence, kv-head) group: two 128-row tiles (residual 0 and 1) whose
+// rows 0..G-1 are the group's q-heads and the rest zero, packed [128][d/2] with tiled scale
+// atoms, exactly the layout the prefill kernel reads for a query tile.
+//   q1 = NVFP4(q);  r = q - deq(q1) (FP32, deq exact);  q2 = NVFP4(r)
+// grid: groups; 128 threads, thread = tile row.
+// ---------------------------------------------------------------------------------------
+FA4Q_DEVINL float e2m1_value(uint32_t code) {
+  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  const float v = mag[code & 7u];
+  return (code & 8u) ? -v : v;
+}
+
+__global__ void __launch_bounds__(128) dec_query_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv,
+                                                        uint8_t* __restrict__ qt, uint8_t* __restrict__ qt_sf) {
+  constexpr int D = 128;
+  const int grp = blockIdx.x, r = threadIdx.x;
+  const int G = Hq / Hkv;
+  const int b = grp / Hkv, hk = grp % Hkv;
+  float x[D];
+  if (r < G) {
+    const uint16_t* src = q + ((int64_t)b * Hq + hk * G + r) * D;
+#pragma unroll
+    for (int c = 0; c < D; c += 8) load_bf16x8(src + c, x + c);
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; ++c) x[c] = 0.0f;
+  }
+  for (int res = 0; res < 2; ++res) {
+    uint8_t* dst = qt + ((int64_t)grp * 2 + res) * 128 * (D / 2) + r * (D / 2);
+    uint8_t* sdst = qt_sf + ((int64_t)grp * 2 + res) * 2 * 512;
+#pragma unroll
+    for (int kb = 0; kb < D / 16; ++kb) {
+      uint2 pk;
+      const uint32_t sc = quant_block16_nvfp4(x + 16 * kb, 6.0f, 1.0f, pk);
+      *reinterpret_cast<uint2*>(dst + 8 * kb) = pk;
+      sdst[sf_tiled_offset(r, kb, 2)] = static_cast<uint8_t>(sc);
+      if (res == 0) {
+        // residual of this block: x - code * scale (the product is exact in FP32)
+        const float s = ue4m3_decode(sc);
+        const uint32_t w[2] = {pk.x, pk.y};
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          x[16 * kb + i] = __fsub_rn(x[16 * kb + i], e2m1_value(w[i >> 3] >> (4 * (i & 7))) * s);
+      }
+    }
+  }
+}
+
+fa4q_status launch_dec_query(const uint16_t* q, int B, int Hq, int Hkv, uint8_t* qt, uint8_t* qt_sf,
+                             cudaStream_t st) {
+  dec_query_kernel<<<B * Hkv, 128, 0, st>>>(q, Hq, Hkv, qt, qt_sf);
+  return launch_status();
+}
+
+}  // namespace fa4q
+
 extern "C" fa4q_status fa4q_quantize_rotated(const void* x, int64_t groups, int64_t rows, int64_t cols,
                                              int64_t row_stride, fa4q_format fmt, float qmax,
                                              float tensor_scale, const float* smooth_mul,

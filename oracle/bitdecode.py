@@ -21,10 +21,10 @@ Readings (the pages give no formulas):
 * Keys are scanned in tiles of 128 positions (two 64-token pages) in position order; P is
   quantised exactly as in the prefill (pre-normalisation quantisation of exp(s - m) against
   the running maximum, 16-key NVFP4 blocks with g_P = 1/(6*448), normaliser from P_hat).
-* The scan of a sequence is split into `splits` contiguous ranges of whole tiles
-  (ceil(tiles / splits) tiles each, the last shorter); each range keeps its own running
-  state and the ranges are merged exactly (log-sum-exp).  The split count is part of the
-  definition, since each range restarts the running maximum.
+* The scan of a sequence is split into contiguous ranges of `tiles_per_split` whole tiles
+  (the last shorter); each range keeps its own running state and the ranges are merged
+  exactly (log-sum-exp).  The range length is part of the definition, since each range
+  restarts the running maximum.
 """
 from __future__ import annotations
 
@@ -43,13 +43,14 @@ def dual_residual_query(q):
     return d1 + formats.dequantize_rows(p2, s2, "nvfp4"), (p1, s1, p2, s2)
 
 
-def split_ranges(L: int, splits: int, tile: int = attention.BC):
+def split_ranges(L: int, tiles_per_split: int, tile: int = attention.BC):
+    """Key ranges [a, b) of the splits of an L-token scan."""
     n_tiles = -(-L // tile)
-    per = -(-n_tiles // max(1, splits))
+    per = max(1, int(tiles_per_split))
     return [(t0 * tile, min(L, (t0 + per) * tile)) for t0 in range(0, n_tiles, per)]
 
 
-def decode_group_fp4q(q, k, v, splits: int, sm_scale: float | None = None):
+def decode_group_fp4q(q, k, v, tiles_per_split: int, sm_scale: float | None = None):
     """Decode output for the G q-heads of one (sequence, kv-head): q [G, d], k, v [L, d] the
     bf16 values of the cached keys; returns [G, d] (FP64)."""
     L, d = k.shape
@@ -60,7 +61,7 @@ def decode_group_fp4q(q, k, v, splits: int, sm_scale: float | None = None):
     pv, sv = formats.quantize_cols_transposed(np.asarray(v, np.float32), "nvfp4")
     vh = formats.dequantize_rows(pv, sv, "nvfp4").T[:L]
     outs, lses = [], []
-    for a, b in split_ranges(L, splits):
+    for a, b in split_ranges(L, tiles_per_split):
         o, lse = attention.attention_pnq(qt, kh[a:b], vh[a:b], causal=False, fmt="nvfp4", sm_scale=sm,
                                          return_lse=True)
         outs.append(o)

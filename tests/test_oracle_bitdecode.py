@@ -45,10 +45,11 @@ def test_residual_cuts_the_logit_error():
 def test_split_ranges():
     assert BD.split_ranges(1000, 3) == [(0, 384), (384, 768), (768, 1000)]
     assert BD.split_ranges(128, 4) == [(0, 128)]
-    assert BD.split_ranges(300, 1) == [(0, 300)]
+    assert BD.split_ranges(300, 8) == [(0, 300)]
+    assert BD.split_ranges(300, 1) == [(0, 128), (128, 256), (256, 300)]
 
 
-def _scalar(q, k, v, splits):
+def _scalar(q, k, v, tps):
     G, d = q.shape
     L = k.shape[0]
     sm = 1.0 / math.sqrt(d)
@@ -61,7 +62,7 @@ def _scalar(q, k, v, splits):
     out = np.zeros((G, d))
     for gi in range(G):
         parts = []
-        for a, b in BD.split_ranges(L, splits):
+        for a, b in BD.split_ranges(L, tps):
             m, l, o = -math.inf, 0.0, np.zeros(d)
             for t0 in range(a, b, 128):
                 keys = list(range(t0, min(b, t0 + 128)))
@@ -83,17 +84,17 @@ def _scalar(q, k, v, splits):
     return out
 
 
-@pytest.mark.parametrize("L,splits", [(300, 2), (520, 3), (200, 1)])
-def test_matches_scalar_bruteforce(L, splits):
+@pytest.mark.parametrize("L,tps", [(300, 2), (520, 1), (200, 4)])
+def test_matches_scalar_bruteforce(L, tps):
     q, k, v = _rand((4, 128), 4, 1.5), _rand((L, 128), 5, 1.5), _rand((L, 128), 6)
-    got = BD.decode_group_fp4q(q, k, v, splits)
-    assert np.max(np.abs(got - _scalar(q, k, v, splits))) <= 1e-12
+    got = BD.decode_group_fp4q(q, k, v, tps)
+    assert np.max(np.abs(got - _scalar(q, k, v, tps))) <= 1e-12
 
 
 def test_one_split_is_the_prefill_loop_and_output_is_convex():
     L = 700
     q, k, v = _rand((4, 128), 7, 1.5), _rand((L, 128), 8, 1.5), _rand((L, 128), 9)
-    got = BD.decode_group_fp4q(q, k, v, 1)
+    got = BD.decode_group_fp4q(q, k, v, 100)
     qt, _ = BD.dual_residual_query(q)
     kh = F.dequantize_rows(*F.quantize_rows(k, "nvfp4"), "nvfp4")
     vh = F.dequantize_rows(*F.quantize_cols_transposed(v, "nvfp4"), "nvfp4").T[:L]
