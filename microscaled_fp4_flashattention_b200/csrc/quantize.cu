@@ -598,12 +598,14 @@ FA4Q_DEVINL float e2m1_value(uint32_t code) {
 __global__ void __launch_bounds__(128) dec_query_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv,
                                                         uint8_t* __restrict__ qt, uint8_t* __restrict__ qt_sf) {
   constexpr int D = 128;
+  // row r holds q-head r % 32 of the group: the G <= 32 heads repeat in every 32-row
+  // quadrant, each of which takes a quarter of every key tile
   const int grp = blockIdx.x, r = threadIdx.x;
   const int G = Hq / Hkv;
   const int b = grp / Hkv, hk = grp % Hkv;
   float x[D];
-  if (r < G) {
-    const uint16_t* src = q + ((int64_t)b * Hq + hk * G + r) * D;
+  if ((r & 31) < G) {
+    const uint16_t* src = q + ((int64_t)b * Hq + hk * G + (r & 31)) * D;
 #pragma unroll
     for (int c = 0; c < D; c += 8) load_bf16x8(src + c, x + c);
   } else {
