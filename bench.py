@@ -54,6 +54,10 @@ NCU_TRAFFIC = {
     "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
                "sha256": "8823e9bfcf14353afacabc2c8a977d045d5bc5088536c644f2f53732b444205f",
                "bytes_per_sequence": (358891008 + 4980480) // 8},
+    # profiles/decode_fp4q_paged_nvfp4_b32_l32k.md: 1,212,922,880 + 15,395,072 B (bench workload)
+    "decode_fp4q": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
+                    "sha256": "5052db0a146aa42476beef05e27ba27e1a7a2ace29031e36246b5bf23159ca63",
+                    "bytes_per_launch": 1212922880 + 15395072},
 }
 
 
@@ -70,7 +74,7 @@ def ncu_traffic(kernel: str, sequences: int = 0):
     e = NCU_TRAFFIC[kernel]
     if e["sha256"] is None or sources_sha256(e["sources"]) != e["sha256"]:
         return None
-    return e["bytes_per_launch"] if kernel == "attn_fwd" else e["bytes_per_sequence"] * sequences
+    return e["bytes_per_launch"] if "bytes_per_launch" in e else e["bytes_per_sequence"] * sequences
 
 
 # ------------------------------------------------------------------------------ helpers
@@ -405,7 +409,8 @@ def decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
         "splits": splits, "tiles_per_split": tps,
         "roofline": {"kernel": "attn_fwd_kernel<DEC>+dec_query_kernel+decode_combine_kernel", "bound": "hbm",
                      "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                     "traffic": None, "peak_source": f"{peak_kind} hbm copy"},
+                     "traffic": ncu_traffic("decode_fp4q") if not args.decode_batch else None,
+                     "peak_source": f"{peak_kind} hbm copy"},
         "note": "dual-residual NVFP4 query and PNQ probabilities on the block-scaled tensor cores "
                 "(BitDecoding-FP4); seeded gaussian cache, not the hybrid cache of line['decode']",
         "l2": "working set 1.2 GB > L2", "clocks": sampler.summary()}
