@@ -11,7 +11,7 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libfa4q.so")
-SOURCES = ["api.cu", "quantize.cu", "attn_fwd.cu", "decode.cu", "vlines.cu", "hybrid.cu"]
+SOURCES = ["api.cu", "quantize.cu", "attn_fwd.cu", "decode.cu", "decode_tc.cu", "vlines.cu", "hybrid.cu"]
 
 
 def nvcc_path() -> str:

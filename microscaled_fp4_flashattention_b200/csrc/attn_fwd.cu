@@ -1241,40 +1241,6 @@ cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word) {
   return cudaStreamSynchronize(st);
 }
 
-// ---------------------------------------------------------------------------------------
-// host: tensor maps
-// ---------------------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// 3-D byte tensor [d2][d1][d0 bytes] with box (box0 bytes, box1 rows, 1)
-static bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                        uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {d0, d0 * d1};
-  const cuuint32_t box[3] = {box0, box1, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int D, bool MX, bool CAUSAL, bool ABL = false, bool HYB = false>
 static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t* vt,
                                const AttnParams& prm, cudaStream_t st) {
@@ -1497,107 +1463,3 @@ extern "C" fa4q_status fa4q_attn_fwd_hybrid(
   return launch_attn<128, false, true, false, true>(q, k, vt, prm, st);
 }
 
-// =======================================================================================
-// FP4 tensor-core decode (BitDecoding-FP4): dual-residual FP4 query tiles, the prefill
-// kernel's tcgen05 pipeline over page pairs of the paged cache, split partials, combine
-// =======================================================================================
-namespace fa4q {
-
-struct DecPlan {
-  int splits, tiles_per_split;
-  size_t off_qt, off_qsf, total;
-};
-
-static DecPlan dec_plan(int B, int Hq, int Hkv, int max_pages, int num_splits) {
-  DecPlan pl;
-  const int tiles = (max_pages + 1) / 2;                       // page pairs of the longest sequence
-  int s = num_splits > 0 ? num_splits : (148 * 8 + B * Hkv - 1) / (B * Hkv);
-  s = std::max(1, std::min(s, std::max(1, tiles)));
-  pl.tiles_per_split = std::max(1, (tiles + s - 1) / s);
-  pl.splits = std::max(1, (tiles + pl.tiles_per_split - 1) / pl.tiles_per_split);
-  // one partial per q-head, split and TMEM lane quadrant (the quadrants split each tile's keys)
-  const size_t part = (size_t)B * Hq * pl.splits * 4 * (kDecHeadDim + 2) * sizeof(float);
-  pl.off_qt = (part + 1023) / 1024 * 1024;
-  pl.off_qsf = pl.off_qt + (size_t)B * Hkv * 2 * kBM * (kDecHeadDim / 2);
-  pl.total = pl.off_qsf + (size_t)B * Hkv * 2 * 2 * 512;
-  return pl;
-}
-
-}  // namespace fa4q
-
-extern "C" size_t fa4q_decode_fp4q_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int num_splits) {
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || d != kDecHeadDim || max_pages <= 0 || num_splits < 0) return 0;
-  return dec_plan(B, Hq, Hkv, max_pages, num_splits).total;
-}
-
-extern "C" fa4q_status fa4q_decode_fp4q(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
-                                        const uint8_t* vt_pages, const uint8_t* vt_sf,
-                                        const int32_t* block_table, const int32_t* fp4_len,
-                                        int n_phys_pages, int B, int Hq, int Hkv, int d, int max_pages,
-                                        fa4q_format fmt, float g_k, float g_v, float sm_scale, void* out,
-                                        void* workspace, size_t workspace_bytes, int num_splits,
-                                        void* stream) {
-  if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
-  if (fmt == FA4Q_MXFP4) return FA4Q_ERR_UNSUPPORTED;          // the query residuals are NVFP4
-  if (!q || !k_pages || !k_sf || !vt_pages || !vt_sf || !block_table || !fp4_len || !out || !workspace)
-    return FA4Q_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_pages <= 0 || n_phys_pages <= 0 || num_splits < 0)
-    return FA4Q_ERR_INVALID_ARG;
-  if (d != kDecHeadDim || Hq / Hkv > 32) return FA4Q_ERR_UNSUPPORTED;
-  if (!(g_k > 0.0f) || !(g_v > 0.0f)) return FA4Q_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(k_sf) || !aligned16(vt_pages) || !aligned16(vt_sf) ||
-      !aligned16(out) || !aligned16(workspace))
-    return FA4Q_ERR_INVALID_ARG;
-  if ((int64_t)n_phys_pages * Hkv > 0x7fffffff || (int64_t)B * Hkv * 2 > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
-  const DecPlan pl = dec_plan(B, Hq, Hkv, max_pages, num_splits);
-  if (workspace_bytes < pl.total) return FA4Q_ERR_INVALID_ARG;
-  if ((int64_t)B * Hkv * pl.splits * 4 > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* qt = ws + pl.off_qt;
-  uint8_t* qt_sf = ws + pl.off_qsf;
-  fa4q_status stt = launch_dec_query(static_cast<const uint16_t*>(q), B, Hq, Hkv, qt, qt_sf, st);
-  if (stt != FA4Q_OK) return stt;
-  CUtensorMap tq, tk, tv;
-  if (!make_map_3d(&tq, qt, kDecHeadDim / 2, kBM, (uint64_t)B * Hkv * 2, kDecHeadDim / 2, kBM,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_3d(&tk, k_pages, kDecHeadDim / 2, 64, (uint64_t)n_phys_pages * Hkv, kDecHeadDim / 2, 64,
-                   CU_TENSOR_MAP_SWIZZLE_64B) ||
-      !make_map_3d(&tv, vt_pages, 32, kDecHeadDim, (uint64_t)n_phys_pages * Hkv, 32, kDecHeadDim,
-                   CU_TENSOR_MAP_SWIZZLE_32B))
-    return FA4Q_ERR_CUDA;
-  const float sms = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)d);
-  AttnParams prm{};
-  prm.q_sf = qt_sf;
-  prm.k_sf = k_sf;
-  prm.vt_sf = vt_sf;
-  prm.out = out;
-  prm.B = B;
-  prm.Hq = Hq;
-  prm.Hkv = Hkv;
-  prm.S_q = kBM;
-  prm.S_k = kBN;
-  prm.S_kpad = kBN;
-  prm.n_qtiles = 1;
-  prm.n_items = B * Hkv * pl.splits;
-  prm.score_scale_log2 = sms * g_k * kLog2e;
-  prm.g_v = g_v;
-  prm.qmax_p = 0.0f;
-  prm.dec_table = block_table;
-  prm.dec_len = fp4_len;
-  prm.dec_ksf = k_sf;
-  prm.dec_vsf = vt_sf;
-  prm.dec_ws = reinterpret_cast<float*>(ws);
-  prm.dec_max_pages = max_pages;
-  prm.dec_splits = pl.splits;
-  prm.dec_tiles_per_split = pl.tiles_per_split;
-  auto kern = attn_fwd_kernel<kDecHeadDim, false, false, false, false, false, true>;
-  static_assert(sizeof(Smem<kDecHeadDim, false, kDecStages>) + 1024 <= 227 * 1024, "decode shared memory");
-  const size_t smem = sizeof(Smem<kDecHeadDim, false, kDecStages>) + 1024;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return FA4Q_ERR_CUDA;
-  kern<<<static_cast<unsigned>(prm.n_items), kThreads, smem, st>>>(tq, tk, tv, prm);
-  stt = launch_status();
-  if (stt != FA4Q_OK) return stt;
-  return launch_decode_combine(reinterpret_cast<const float*>(ws), B * Hq, pl.splits * 4, static_cast<uint16_t*>(out), st);
-}

@@ -1,6 +1,7 @@
 // fa4q_internal.h - host-side helpers shared by the fa4q translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -16,6 +17,38 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline fa4q_status launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? FA4Q_OK : FA4Q_ERR_CUDA;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link against libcuda)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D byte tensor [d2][d1][d0 bytes] with box (box0 bytes, box1 rows, 1)
+inline bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                        uint32_t box0, uint32_t box1, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0, d0 * d1};
+  const cuuint32_t box[3] = {box0, box1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Streaming multiprocessors of the current device (cached per device; 148 on B200).
@@ -49,7 +82,8 @@ struct HyParams {
 fa4q_status launch_hybrid_full(const HyParams& p, cudaStream_t st);
 
 // Dual-residual NVFP4 query tiles of the FP4 tensor-core decode (quantize.cu): q bf16
-// [B][Hq][128] -> qt [B*Hkv][2][128][64] packed, qt_sf [B*Hkv][2][2][512] tiled atoms.
+// [B][Hq][128] -> qt [B*Hkv][2][128][64] packed, qt_sf [B*Hkv][2][2][512] tiled atoms
+// (row r holds q-head r % 32 of the group, zero when r % 32 >= G).
 fa4q_status launch_dec_query(const uint16_t* q, int B, int Hq, int Hkv, uint8_t* qt, uint8_t* qt_sf,
                              cudaStream_t st);
 // log-sum-exp merge of decode split partials [rows][splits][d + 2] (m in log2 units, l, o)
@@ -60,5 +94,6 @@ fa4q_status launch_decode_combine(const float* ws, int rows, int splits, uint16_
 // functions read-and-clear them (stream-ordered, then synchronised by the caller).
 cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word);
 cudaError_t decode_status_fetch(cudaStream_t st, uint32_t* host_word);
+cudaError_t dectc_status_fetch(cudaStream_t st, uint32_t* host_word);
 
 }  // namespace fa4q

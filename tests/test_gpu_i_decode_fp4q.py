@@ -47,6 +47,8 @@ def _run(B, Hq, Hkv, L, seed, num_splits=0, lens=None, shuffle=True):
     (2, 8, 2, 1024, 3),
     (1, 4, 1, 4160, 0),
     (1, 8, 1, 300, 1),       # G = 8
+    (1, 16, 1, 520, 0),      # G = 16: every column of the 16-head MMA tile
+    (2, 6, 2, 1100, 2),      # G = 3: padded heads inside the 4-head instantiation
     (1, 2, 2, 130, 0),       # MHA; a last tile with 2 keys
 ])
 def test_decode_fp4q(B, Hq, Hkv, L, splits):
