@@ -54,10 +54,10 @@ NCU_TRAFFIC = {
     "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
                "sha256": "8823e9bfcf14353afacabc2c8a977d045d5bc5088536c644f2f53732b444205f",
                "bytes_per_sequence": (358891008 + 4980480) // 8},
-    # profiles/decode_fp4q_paged_nvfp4_b32_l32k.md: 1,212,922,880 + 15,395,072 B (bench workload)
-    "decode_fp4q": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
-                    "sha256": "5052db0a146aa42476beef05e27ba27e1a7a2ace29031e36246b5bf23159ca63",
-                    "bytes_per_launch": 1212922880 + 15395072},
+    # profiles/decode_fp4q_paged_nvfp4_b32_l32k.md (filled in from the capture of decode_tc_kernel)
+    "decode_fp4q": {"sources": ("decode_tc.cu", "fa4q_common.cuh"),
+                    "sha256": None,
+                    "bytes_per_launch": None},
 }
 
 
@@ -407,7 +407,7 @@ def decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
         "workload": f"{dw.name} shape, all {L} keys FP4 (NVFP4 pages)", "us_per_step": ms * 1e3,
         "higher_is_better": False, "GBps": gbs, "bytes_per_step": nbytes, "gpu_launches": 3 * dsteps,
         "splits": splits, "tiles_per_split": tps,
-        "roofline": {"kernel": "attn_fwd_kernel<DEC>+dec_query_kernel+decode_combine_kernel", "bound": "hbm",
+        "roofline": {"kernel": "decode_tc_kernel+dec_query_kernel+decode_combine_kernel", "bound": "hbm",
                      "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
                      "traffic": ncu_traffic("decode_fp4q") if not args.decode_batch else None,
                      "peak_source": f"{peak_kind} hbm copy"},

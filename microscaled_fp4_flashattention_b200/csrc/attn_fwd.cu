@@ -43,15 +43,13 @@ namespace fa4q {
 static __device__ uint32_t g_attn_status;
 
 constexpr int kBM = 128;
-constexpr int kDecHeadDim = 128;   // head dimension of the FP4 tensor-core decode
 constexpr int kBN = 128;
 constexpr int kThreads = 384;
 // Register split (setmaxnreg): launched at 168 per thread (3 warps per scheduler x 168 x 32 =
 // 16128 of the scheduler's 16384); warpgroup 0 (TMA, MMA, 2 idle warps) drops to 56 and the
 // two softmax warpgroups rise to 224: 56*32 + 2*224*32 = 16128, the launch total exactly.
 constexpr int kRegsIssue = 56, kRegsSoftmax = 224;
-constexpr int kStages = 4;      // K/V stages of the prefill (tiles mostly served from L2)
-constexpr int kDecStages = 8;   // decode: every page pair comes from HBM, so more bytes in flight
+constexpr int kStages = 4;      // K/V tile stages (tiles mostly served from L2)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGpNvfp4 = 1.0f / 2688.0f;  // g_P = 1/(6*448), rounded to FP32
 // 1 / (6 g_P) in FP32: the P scale t = amax / (6 g_P) is taken as one multiply (t may differ
@@ -83,35 +81,32 @@ struct Cfg {
   static constexpr int kQKSbo = D == 128 ? 512 : 256;
 };
 
-template <int D, bool MX, int NS>
+template <int D, bool MX>
 struct __align__(1024) Smem {
   using C = Cfg<D, MX>;
   uint8_t q[2][C::kQBytes];                 // double-buffered by work item
-  uint8_t k[NS][C::kKBytes];
-  uint8_t v[NS][C::kVBytes];
+  uint8_t k[kStages][C::kKBytes];
+  uint8_t v[kStages][C::kVBytes];
   uint8_t p[2][C::kPBytes];
   uint8_t ones[1024];
   uint8_t sfq[2][2 * 512];
-  uint8_t sfk[NS][2 * 512];
-  uint8_t sfv[NS][2 * 512];
+  uint8_t sfk[kStages][2 * 512];
+  uint8_t sfv[kStages][2 * 512];
   uint8_t sfp[2][2 * 512];
   uint8_t sfone[2 * 512];
-  uint8_t sfraw[NS][4 * 512];   // decode: raw page scales (K of 2 pages, V^T of 2 pages)
   uint64_t bar_q[2];         // Q tile (and its scales) of work item k landed, slot k % 2
   uint64_t q_free[2];        // all S products of work item k issued and complete
   uint64_t o_free;           // all eight softmax warps have read O and l in the epilogue
-  uint64_t kv_full[NS];
-  uint64_t kv_empty[NS];
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
   uint64_t s_full[2];        // S of an even / odd key tile ready (one per softmax group)
   uint64_t s_free;
   uint64_t p_full[2];
   uint64_t o_done[2];
   uint64_t drain;
-  uint64_t sf_ready[NS];  // decode: the stage's scales permuted into atoms (warps 2, 3)
   float m_xchg[2][kBM];       // running maximum after tile j, slot j%2, per row
   float m_last[2][kBM];       // per group: the maximum its accumulator is relative to
   float l_last[2][kBM];       // per group: the normaliser summed from P~ (ablation only)
-  float dec_qmax[2][2][kBM];  // decode: per group, slot (tile/2)%2, the quadrants' key maxima
   uint32_t tmem_base;
   uint32_t abort_flag;
 };
@@ -150,16 +145,6 @@ struct AttnParams {
   const uint64_t* hy_excl;   // [B][Hkv][hy_excl_words]
   int hy_window;
   int hy_excl_words;
-  // FP4 tensor-core decode (BitDecoding-FP4): items are (sequence, kv-head, split); the
-  // query tile holds the group's q-heads in rows 0..G-1 as two residual tiles (slots 0, 1);
-  // key tiles are page pairs of the paged cache through the block table; the epilogue
-  // writes split partials [m (log2 units), l, o[D]] for the combine kernel.
-  const int32_t* dec_table;  // [B][dec_max_pages]
-  const int32_t* dec_len;    // [B] cached tokens
-  const uint8_t* dec_ksf;    // page K scales [P][Hkv][64][D/16]
-  const uint8_t* dec_vsf;    // page V^T scales [P][Hkv][D][4]
-  float* dec_ws;             // [B*Hq][dec_splits][D + 2]
-  int dec_max_pages, dec_splits, dec_tiles_per_split;
   int causal;
   int out_fp32;
 };
@@ -331,15 +316,13 @@ FA4Q_DEVINL void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, int N
 // ABL: the ablations of fa4q_attn_fwd_ex (conditional rescaling, normaliser from P~) are
 // compiled into separate instantiations so the default kernel carries none of their work.
 // HYB: the FP4 part of the hybrid-precision prefill (causal only).
-// DEC: the FP4 tensor-core decode (non-causal, non-persistent, NVFP4, D = 128).
-template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL, bool HYB = false, bool DEC = false>
+template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL, bool HYB = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = Cfg<D, MX>;
-  constexpr int NS = DEC ? kDecStages : kStages;
   extern __shared__ uint8_t smem_raw[];
-  Smem<D, MX, NS>& sm = *reinterpret_cast<Smem<D, MX, NS>*>(
+  Smem<D, MX>& sm = *reinterpret_cast<Smem<D, MX>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   volatile uint32_t* abort_flag = &sm.abort_flag;
 
@@ -362,15 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   auto decode_item = [&](int u) -> Item {
     Item it;
-    if constexpr (DEC) {
-      const int grp = u / p.dec_splits, split = u - grp * p.dec_splits;
-      it.b = grp / p.Hkv;
-      it.h = grp - it.b * p.Hkv;                 // the kv-head
-      it.qt = split;
-      const int L = max(0, min(p.dec_len[it.b], p.dec_max_pages * 64));
-      const int n_all = (L + kBN - 1) / kBN;
-      it.n_tiles = max(0, min(p.dec_tiles_per_split, n_all - split * p.dec_tiles_per_split));
-    } else if (CAUSAL) {
+    if (CAUSAL) {
       const int per = p.B * p.Hq, rem = u % per;
       it.qt = p.n_qtiles - 1 - u / per;
       it.b = rem / p.Hq;
@@ -398,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.bar_q[s], 1);
       mbar_init(&sm.q_free[s], 1);
     }
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
     }
@@ -410,7 +385,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&sm.o_free, 8);
     mbar_init(&sm.drain, 1);
-    for (int s = 0; s < NS; ++s) mbar_init(&sm.sf_ready[s], 2);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
@@ -450,42 +424,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = decode_item(u);
         const int bh_q = it.b * p.Hq + it.h, bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
         const int qs = k & 1;
-        if constexpr (DEC) {
-          // both residual query tiles, then page pairs through the block table (a missing
-          // second page repeats the first: its keys are masked, its data finite)
-          if (it.n_tiles == 0) break;
-          const int grp = it.b * p.Hkv + it.h;
-          mbar_arrive_expect_tx(&sm.bar_q[0], 2 * (C::kQBytes + C::kSfQAtoms * 512));
-          for (int r = 0; r < 2; ++r) {
-            tma_load_3d(sm.q[r], &tm_q, 0, 0, grp * 2 + r, &sm.bar_q[0]);
-            bulk_load(sm.sfq[r], p.q_sf + ((int64_t)grp * 2 + r) * C::kSfQAtoms * 512, C::kSfQAtoms * 512,
-                      &sm.bar_q[0]);
-          }
-          q_issued = 1;
-          const int L = max(0, min(p.dec_len[it.b], p.dec_max_pages * 64));
-          const int n_pages = (L + 63) / 64, t0 = it.qt * p.dec_tiles_per_split;
-          for (int j = 0; j < it.n_tiles; ++j, ++T) {
-            const int s = T % NS;
-            if (T >= NS && !cta_wait(&sm.kv_empty[s], ((T / NS) - 1) & 1, abort_flag,
-                                          kStatusTimeoutTmaFull)) {
-              go = false;
-              break;
-            }
-            const int lp0 = 2 * (t0 + j), lp1 = min(lp0 + 1, n_pages - 1);
-            const int ph0 = p.dec_table[(int64_t)it.b * p.dec_max_pages + lp0] * p.Hkv + it.h;
-            const int ph1 = p.dec_table[(int64_t)it.b * p.dec_max_pages + lp1] * p.Hkv + it.h;
-            mbar_arrive_expect_tx(&sm.kv_full[s], C::kKBytes + C::kVBytes + 4 * 512);
-            tma_load_3d(sm.k[s], &tm_k, 0, 0, ph0, &sm.kv_full[s]);
-            tma_load_3d(sm.k[s] + C::kKBytes / 2, &tm_k, 0, 0, ph1, &sm.kv_full[s]);
-            tma_load_3d(sm.v[s], &tm_v, 0, 0, ph0, &sm.kv_full[s]);
-            tma_load_3d(sm.v[s] + C::kVBytes / 2, &tm_v, 0, 0, ph1, &sm.kv_full[s]);
-            bulk_load(sm.sfraw[s], p.dec_ksf + (int64_t)ph0 * 512, 512, &sm.kv_full[s]);
-            bulk_load(sm.sfraw[s] + 512, p.dec_ksf + (int64_t)ph1 * 512, 512, &sm.kv_full[s]);
-            bulk_load(sm.sfraw[s] + 1024, p.dec_vsf + (int64_t)ph0 * 512, 512, &sm.kv_full[s]);
-            bulk_load(sm.sfraw[s] + 1536, p.dec_vsf + (int64_t)ph1 * 512, 512, &sm.kv_full[s]);
-          }
-          continue;
-        }
         // Q slot qs was last read by the S products of item k-2
         if (k >= 2 && !cta_wait(&sm.q_free[qs], ((k - 2) >> 1) & 1, abort_flag, kStatusTimeoutTmaFull)) break;
         mbar_arrive_expect_tx(&sm.bar_q[qs], C::kQBytes + C::kSfQAtoms * 512);
@@ -494,8 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   C::kSfQAtoms * 512, &sm.bar_q[qs]);
         q_issued = k + 1;
         for (int j = 0; j < it.n_tiles; ++j, ++T) {
-          const int s = T % NS;
-          if (T >= NS && !cta_wait(&sm.kv_empty[s], ((T / NS) - 1) & 1, abort_flag,
+          const int s = T % kStages;
+          if (T >= kStages && !cta_wait(&sm.kv_empty[s], ((T / kStages) - 1) & 1, abort_flag,
                                         kStatusTimeoutTmaFull)) {
             go = false;
             break;
@@ -511,8 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: every issued copy must have landed before the CTA may exit
-      for (int t = max(0, T - NS); t < T; ++t)
-        mbar_wait(&sm.kv_full[t % NS], (t / NS) & 1, &g_attn_status, kStatusTimeoutDrain);
+      for (int t = max(0, T - kStages); t < T; ++t)
+        mbar_wait(&sm.kv_full[t % kStages], (t / kStages) & 1, &g_attn_status, kStatusTimeoutDrain);
       for (int k = max(0, q_issued - 2); k < q_issued; ++k)
         mbar_wait(&sm.bar_q[k & 1], (k >> 1) & 1, &g_attn_status, kStatusTimeoutDrain);
     }
@@ -530,45 +468,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u < 0) break;
         const Item it = decode_item(u);
         const int qs = k & 1, T0 = T, n_tiles = it.n_tiles;
-        if (DEC && n_tiles == 0) break;            // empty split: the softmax threads write it
         if (!cta_wait(&sm.bar_q[qs], (k >> 1) & 1, abort_flag, kStatusTimeoutMma)) break;
         tc_fence_after();
         // item k-2 used this scale slot; all of its products completed before item k-1 ended
         for (int a = 0; a < C::kSfQAtoms; ++a)
           tmem_cp_sf_atom(tmem + kColSfQ + 8 * qs + 4 * a, smem_u32(sm.sfq[qs] + 512 * a));
-        if constexpr (DEC) {                       // second residual tile: slot 1
-          for (int a = 0; a < C::kSfQAtoms; ++a)
-            tmem_cp_sf_atom(tmem + kColSfQ + 8 + 4 * a, smem_u32(sm.sfq[1] + 512 * a));
-        }
         const uint32_t q_addr = smem_u32(sm.q[qs]);
         // S_j = Q K_j^T into the single S buffer once the softmax group of the previous key
         // tile (of this item or the last) holds its scores in registers
         auto issue_s = [&](int j) -> bool {
-          const int t = T0 + j, s = t % NS, kb = t & 1;
-          if (!cta_wait(&sm.kv_full[s], (t / NS) & 1, abort_flag, kStatusTimeoutMma)) return false;
+          const int t = T0 + j, s = t % kStages, kb = t & 1;
+          if (!cta_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag, kStatusTimeoutMma)) return false;
           if (t >= 1 && !cta_wait(&sm.s_free, (t - 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
-          if (DEC && !cta_wait(&sm.sf_ready[s], (t / NS) & 1, abort_flag, kStatusTimeoutMma)) return false;
           tc_fence_after();
           for (int a = 0; a < C::kSfQAtoms; ++a)
             tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
           const uint32_t k_addr = smem_u32(sm.k[s]);
-          if constexpr (DEC) {
-            // dual-residual query: S = Q1 K^T + Q2 K^T, K-steps 0,1 of each residual tile
-            const uint32_t q2_addr = smem_u32(sm.q[1]);
 #pragma unroll
-            for (int ks = 0; ks < 2 * C::kKStepsQK; ++ks) {
-              const int r = ks / C::kKStepsQK, st = ks % C::kKStepsQK;
-              const uint64_t ad = make_smem_desc((r ? q2_addr : q_addr) + 32 * st, 16, C::kQKSbo, C::kQKSwizzle);
-              const uint64_t bd = make_smem_desc(k_addr + 32 * st, 16, C::kQKSbo, C::kQKSwizzle);
-              mma_step<MX>(tmem + kColS, ad, bd, kBN, st, tmem + kColSfQ + 8 * r, tmem + kColSfK + 8 * kb, ks > 0);
-            }
-          } else {
-#pragma unroll
-            for (int ks = 0; ks < C::kKStepsQK; ++ks) {
-              const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-              const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-              mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ + 8 * qs, tmem + kColSfK + 8 * kb, ks > 0);
-            }
+          for (int ks = 0; ks < C::kKStepsQK; ++ks) {
+            const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+            const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
+            mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ + 8 * qs, tmem + kColSfK + 8 * kb, ks > 0);
           }
           tc_commit(&sm.s_full[j & 1]);
           return true;
@@ -576,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // [O | l]_{j%2} (+)= P^_j [V_j | 1] once the softmax group has written P^_j; the first
         // product of an item waits until the previous item's epilogue has read O and l
         auto issue_pv = [&](int jp) -> bool {
-          const int t = T0 + jp, s = t % NS, pb = jp & 1;
+          const int t = T0 + jp, s = t % kStages, pb = jp & 1;
           if (jp == 0 && k >= 1 && !cta_wait(&sm.o_free, (k - 1) & 1, abort_flag, kStatusTimeoutMma))
             return false;
           int& n_pv = pb ? n_pv1 : n_pv0;
@@ -593,9 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
-            // decode: V^T of each page is its own [D][32 B] tile (32-byte swizzle), one K-step
-            const uint64_t vd = DEC ? make_smem_desc(v_addr + (C::kVBytes / 2) * ks, 16, 256, kSwiz32)
-                                    : make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
+            const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
             const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
             // (hybrid: group A's accumulator starts from the full-precision part)
             const uint32_t acc = (jp >= 2 || ks > 0 || (HYB && jp == 0)) ? 1u : 0u;
@@ -622,34 +540,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(&sm.drain);
       mbar_wait(&sm.drain, 0, &g_attn_status, kStatusTimeoutDrain);
     }
-  } else if (DEC) {
-    // ------------------------------------------------------------ decode: scale atoms
-    // Warps 2 and 3 move each tile's raw page scales into the scale-atom layout of the
-    // MMA (byte (r % 32) * 16 + (r / 32) * 4 + k of a 512-byte atom, row r, scale k of the
-    // K-step): K rows are the 128 tokens of the page pair (atoms = halves of d), V^T rows
-    // are the 128 channels (atom = page).  Stage s was last read by the tcgen05.cp of tile
-    // t - NS, which completed before the producer refilled the stage.
-    const int u = item_index(0);
-    if (u >= 0) {
-      const Item it = decode_item(u);
-      const int t64 = (warp - 2) * 32 + lane;
-      for (int t = 0; t < it.n_tiles; ++t) {
-        const int s = t % NS;
-        if (!warp_wait(&sm.kv_full[s], (t / NS) & 1, abort_flag, kStatusTimeoutMma)) break;
-        const uint32_t* raw = reinterpret_cast<const uint32_t*>(sm.sfraw[s]);
-        for (int i = t64; i < 256; i += 64) {      // K: word i = page * 128 + token * 2 + half
-          const int rr = ((i >> 7) << 6) + ((i >> 1) & 63);
-          *reinterpret_cast<uint32_t*>(sm.sfk[s] + 512 * (i & 1) + (rr & 31) * 16 + (rr >> 5) * 4) = raw[i];
-        }
-        for (int i = t64; i < 256; i += 64) {      // V^T: word i = page * 128 + channel
-          const int ch = i & 127;
-          *reinterpret_cast<uint32_t*>(sm.sfv[s] + 512 * (i >> 7) + (ch & 31) * 16 + (ch >> 5) * 4) = raw[256 + i];
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.sf_ready[s]);
-      }
-    }
   }
   } else {
     setmaxnreg_inc<kRegsSoftmax>();
@@ -675,14 +565,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // fused s*sc - round(m*sc) that lands 1 ulp below 0 would move that block's scale.
     bool ok = true;
     int done_a = 0, done_b = 0;                    // key tiles each group processed in earlier items
-    if constexpr (DEC) {
-      // decode: each thread clears its row of its group's P buffer and P scale atoms once
-#pragma unroll
-      for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(sm.p[g] + swz64_offset(r, c)) = make_uint4(0, 0, 0, 0);
-#pragma unroll
-      for (int a = 0; a < 2; ++a) *reinterpret_cast<uint32_t*>(sm.sfp[g] + 512 * a + (r & 31) * 16 + (r >> 5) * 4) = 0u;
-      fence_proxy_async_smem();
-    }
     for (int k = 0; PERSIST || k < 1; ++k) {
     const int u = item_index(k);
     if (u < 0) break;
@@ -694,262 +576,164 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_acc = -INFINITY;                       // maximum of this group's last tile
     float lpt = 0.0f;                              // sum of P~ of this group (ABL), MMA units
     const float gp_item = ABL ? p.gp : kGpNvfp4;
-    int dec_len = 0, dec_key0 = 0;                 // decode: cached tokens, first key of the split
-    if constexpr (DEC) {
-      dec_len = max(0, min(p.dec_len[it.b], p.dec_max_pages * 64));
-      dec_key0 = it.qt * p.dec_tiles_per_split * kBN;
-      if (n_tiles == 0) {
-        // a split with no key: partials (m, l, o) = (-inf, 0, 0); the other roles skip it too
-        const int G = p.Hq / p.Hkv;
-        if (lane < G) {
-          float* dst = p.dec_ws + ((((int64_t)it.b * p.Hq + it.h * G + lane) * p.dec_splits + it.qt) * 4 + wq) * (D + 2);
-          if (g == 0) {
-            dst[0] = -INFINITY;
-            dst[1] = 0.0f;
-          }
-          for (int c = g * (D / 2); c < (g + 1) * (D / 2); ++c) dst[2 + c] = 0.0f;
-        }
-        continue;
-      }
-    }
     for (int j = g; j < n_tiles; j += 2) {
       ok = warp_wait(&sm.s_full[g], (done_g + (j >> 1)) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       tc_fence_after();
-      float m_new;
-      uint32_t sfw[kNB / 4];
-      float ysum[ABL ? kNB : 1];
-      float hy_m0 = -INFINITY;                     // full-precision part, raw score units
-      if constexpr (DEC) {
-        // Quadrant wq holds the G heads of the group in its rows (the query tile repeats
-        // them in every quadrant) and quantises keys [32 wq, 32 wq + 32) of the tile.  The
-        // other 96 columns of its P row stay zero (cleared before the first tile), so the
-        // four quadrants' PV products and row sums are partial sums over disjoint keys that
-        // share one maximum: P^ is the one the whole-row quantisation gives.
-        float s[32];
-        {
-          uint32_t raw[32];
-          tmem_ld32(lane_base + kColS + 32 * wq, raw);
-          tmem_wait_ld();
+      float s[kBN];
+      {
+        uint32_t raw[kBN / 32][32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(raw[i]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_free);
-        const int lim = dec_len - (dec_key0 + j * kBN + 32 * wq);   // positions past the cache
-        if (lim < 32) {
+        for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + kColS + 32 * c, raw[c]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[c][i]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.s_free);
+      // masking: keys beyond S_k, and (causal) keys after this query
+      const int key0 = j * kBN;
+      if constexpr (HYB) {
+        // FP4 keys of row i: key <= i - window and not a vertical line
+        const int lim = min(p.S_k - key0, row - p.hy_window - key0 + 1);
+        const uint64_t* ex = p.hy_excl + (int64_t)(it.b * p.Hkv + it.h / (p.Hq / p.Hkv)) * p.hy_excl_words;
+        const int w0 = key0 >> 6;
+        const uint64_t e0 = w0 < p.hy_excl_words ? ex[w0] : 0ull;
+        const uint64_t e1 = w0 + 1 < p.hy_excl_words ? ex[w0 + 1] : 0ull;
+        const uint32_t ew[4] = {static_cast<uint32_t>(e0), static_cast<uint32_t>(e0 >> 32),
+                                static_cast<uint32_t>(e1), static_cast<uint32_t>(e1 >> 32)};
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          if (ew[q4] == 0u) continue;              // no vertical line among these 32 keys
 #pragma unroll
           for (int i = 0; i < 32; ++i)
+            if (ew[q4] & (1u << i)) s[32 * q4 + i] = -INFINITY;
+        }
+        if (lim < kBN) {                           // the window band (the last FP4 tiles)
+#pragma unroll
+          for (int i = 0; i < kBN; ++i)
             if (i >= lim) s[i] = -INFINITY;
         }
-        const float bm[2] = {block_max<16>(s), block_max<16>(s + 16)};
-        // the tile maximum from the four quadrants' maxima (slot (j / 2) % 2 of this group:
-        // a warp writes slot j/2+2 only after all four passed this barrier for tile j+2)
-        float* qx = sm.dec_qmax[g][(j >> 1) & 1];
-        qx[r] = fmaxf(bm[0], bm[1]);
-        named_bar_sync(13 + g, 128);
-        const float tmax = fmaxf(fmaxf(qx[lane], qx[32 + lane]), fmaxf(qx[64 + lane], qx[96 + lane]));
-        float m_prev = -INFINITY;
-        if (j > 0) {
-          named_bar_sync(bar_recv, 64);
-          m_prev = sm.m_xchg[(j - 1) & 1][r];
-        }
-        m_new = fmaxf(m_prev, tmax);
-        sm.m_xchg[j & 1][r] = m_new;
-        named_bar_arrive(bar_send, 64);
-        const float mref = m_new * sc;
-        uint32_t codes = 0;
-        float l2s[2];
+      } else {
+        const bool edge = (key0 + kBN > p.S_k) || (CAUSAL && key0 + kBN - 1 > qt * kBM);
+        if (edge) {
+          const int lim = CAUSAL ? min(p.S_k - key0, row - key0 + 1) : (p.S_k - key0);
 #pragma unroll
-        for (int bi = 0; bi < 2; ++bi) {
-          const float amax = ex2_approx((bm[bi] - m_new) * sc);
-          const uint32_t code = ue4m3_encode(amax * kInvSixGp);
+          for (int i = 0; i < kBN; ++i)
+            if (i >= lim) s[i] = -INFINITY;
+        }
+      }
+      // block maxima of the raw scores (the scale is positive), tree-shaped for ILP
+      float bmax[kNB];
+#pragma unroll
+      for (int bi = 0; bi < kNB; ++bi) bmax[bi] = block_max<C::kBlk>(s + bi * C::kBlk);
+      float tmax = bmax[0];
+#pragma unroll
+      for (int bi = 1; bi < kNB; ++bi) tmax = fmaxf(tmax, bmax[bi]);
+      // running maximum: take m_{j-1} from the other group, publish m_j
+      float m_prev = -INFINITY;
+      float hy_m0 = -INFINITY;                     // full-precision part, raw score units
+      if constexpr (HYB) {
+        if (j == 0 && row < p.S_q) hy_m0 = p.hy_part[((int64_t)bh_q * p.S_q + row) * (D + 4)] / sc;
+        if (j == 0) m_prev = hy_m0;
+      }
+      if (j > 0) {
+        named_bar_sync(bar_recv, 64);
+        m_prev = sm.m_xchg[(j - 1) & 1][r];
+      }
+      float m_new = fmaxf(m_prev, tmax);
+      if constexpr (ABL) {
+        const bool grow = !(m_prev > -INFINITY) || (tmax - m_prev) * sc > p.tau;
+        if (!grow) m_new = m_prev;
+      }
+      sm.m_xchg[j & 1][r] = m_new;
+      named_bar_arrive(bar_send, 64);
+      const float mref = m_new * sc;
+      // per block: amax = exp2((bmax - m)*sc); scale; y_i = exp2(s_i*sc - m*sc - log2(scale))
+      float lsc[kNB];                              // log2 of each block's scale (+inf: zero block)
+      const float gp = ABL ? p.gp : kGpNvfp4, inv6gp = ABL ? p.inv6gp : kInvSixGp;
+      uint32_t sfw[kNB / 4];
+#pragma unroll
+      for (int w = 0; w < kNB / 4; ++w) sfw[w] = 0;
+#pragma unroll
+      for (int bi = 0; bi < kNB; ++bi) {
+        const float amax = ex2_approx((bmax[bi] - m_new) * sc);
+        uint32_t code;
+        if constexpr (MX) {
+          const int e = mx_exponent(amax, p.qmax_p);
+          code = static_cast<uint32_t>(e + 127);
+          lsc[bi] = amax > 0.0f ? static_cast<float>(e) : INFINITY;
+        } else {
+          const float t = amax * inv6gp;                           // amax / (6 * gp)
+          code = ue4m3_encode(t);
           const float sf = ue4m3_decode(code);
-          l2s[bi] = sf > 0.0f ? lg2_approx(sf * kGpNvfp4) : INFINITY;
-          codes |= code << (8 * bi);
+          lsc[bi] = sf > 0.0f ? lg2_approx(sf * gp) : INFINITY;
         }
-        uint32_t packed[4];
+        sfw[bi >> 2] |= code << (8 * (bi & 3));
+      }
+      uint32_t packed[kBN / 8];
+      auto quantise_row = [&](auto exponent_argument, auto observe) {
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-          const float o8 = mref + l2s[g8 >> 1];
+        for (int g8 = 0; g8 < kBN / 8; ++g8) {
+          const float l8 = lsc[(g8 * 8) / C::kBlk];
           float y[8];
 #pragma unroll
-          for (int i = 0; i < 8; i += 2) ffma2(y[i], y[i + 1], s[8 * g8 + i], s[8 * g8 + i + 1], sc, sc, -o8, -o8);
+          for (int i = 0; i < 8; i += 2) exponent_argument(y[i], y[i + 1], s[8 * g8 + i], s[8 * g8 + i + 1], l8);
 #pragma unroll
           for (int i = 0; i < kEmulPer8; i += 2) ex2_poly2(y[i], y[i + 1], y[i], y[i + 1]);
 #pragma unroll
           for (int i = kEmulPer8; i < 8; ++i) y[i] = ex2_approx(y[i]);
+          observe(g8, y);
           packed[g8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
         }
-        // P buffer g was last read by this group's previous PV product
-        if (j >= 2)
-          ok = warp_wait(&sm.o_done[g], (done_g + (j >> 1) - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
-        *reinterpret_cast<uint4*>(sm.p[g] + swz64_offset(r, wq)) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        *reinterpret_cast<uint32_t*>(sm.sfp[g] + 512 * (wq >> 1) + (r & 31) * 16 + (r >> 5) * 4) =
-            codes << (16 * (wq & 1));
-        fence_proxy_async_smem();
+      };
+      auto no_observer = [](int, const float*) {};
+      auto standard_argument = [&](float& y0, float& y1, float s0, float s1, float l8) {
+        const float o8 = mref + l8;
+        ffma2(y0, y1, s0, s1, sc, sc, -o8, -o8);
+      };
+      float ysum[ABL ? kNB : 1];
+      if constexpr (!ABL) {
+        quantise_row(standard_argument, no_observer);
       } else {
-        float s[kBN];
-        {
-          uint32_t raw[kBN / 32][32];
-  #pragma unroll
-          for (int c = 0; c < kBN / 32; ++c) tmem_ld32(lane_base + kColS + 32 * c, raw[c]);
-          tmem_wait_ld();
-  #pragma unroll
-          for (int c = 0; c < kBN / 32; ++c)
-  #pragma unroll
-            for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(raw[c][i]);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_free);
-        // masking: keys beyond S_k, and (causal) keys after this query
-        const int key0 = j * kBN;
-        if constexpr (DEC) {
-          // decode: positions at or past the cached length
-          const int lim = dec_len - (dec_key0 + key0);
-          if (lim < kBN) {
-  #pragma unroll
-            for (int i = 0; i < kBN; ++i)
-              if (i >= lim) s[i] = -INFINITY;
-          }
-        } else if constexpr (HYB) {
-          // FP4 keys of row i: key <= i - window and not a vertical line
-          const int lim = min(p.S_k - key0, row - p.hy_window - key0 + 1);
-          const uint64_t* ex = p.hy_excl + (int64_t)(it.b * p.Hkv + it.h / (p.Hq / p.Hkv)) * p.hy_excl_words;
-          const int w0 = key0 >> 6;
-          const uint64_t e0 = w0 < p.hy_excl_words ? ex[w0] : 0ull;
-          const uint64_t e1 = w0 + 1 < p.hy_excl_words ? ex[w0 + 1] : 0ull;
-          const uint32_t ew[4] = {static_cast<uint32_t>(e0), static_cast<uint32_t>(e0 >> 32),
-                                  static_cast<uint32_t>(e1), static_cast<uint32_t>(e1 >> 32)};
-  #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            if (ew[q4] == 0u) continue;              // no vertical line among these 32 keys
-  #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (ew[q4] & (1u << i)) s[32 * q4 + i] = -INFINITY;
-          }
-          if (lim < kBN) {                           // the window band (the last FP4 tiles)
-  #pragma unroll
-            for (int i = 0; i < kBN; ++i)
-              if (i >= lim) s[i] = -INFINITY;
-          }
-        } else {
-          const bool edge = (key0 + kBN > p.S_k) || (CAUSAL && key0 + kBN - 1 > qt * kBM);
-          if (edge) {
-            const int lim = CAUSAL ? min(p.S_k - key0, row - key0 + 1) : (p.S_k - key0);
-  #pragma unroll
-            for (int i = 0; i < kBN; ++i)
-              if (i >= lim) s[i] = -INFINITY;
-          }
-        }
-        // block maxima of the raw scores (the scale is positive), tree-shaped for ILP
-        float bmax[kNB];
-  #pragma unroll
-        for (int bi = 0; bi < kNB; ++bi) bmax[bi] = block_max<C::kBlk>(s + bi * C::kBlk);
-        float tmax = bmax[0];
-  #pragma unroll
-        for (int bi = 1; bi < kNB; ++bi) tmax = fmaxf(tmax, bmax[bi]);
-        // running maximum: take m_{j-1} from the other group, publish m_j
-        float m_prev = -INFINITY;
-        if constexpr (HYB) {
-          if (j == 0 && row < p.S_q) hy_m0 = p.hy_part[((int64_t)bh_q * p.S_q + row) * (D + 4)] / sc;
-          if (j == 0) m_prev = hy_m0;
-        }
-        if (j > 0) {
-          named_bar_sync(bar_recv, 64);
-          m_prev = sm.m_xchg[(j - 1) & 1][r];
-        }
-        m_new = fmaxf(m_prev, tmax);
-        if constexpr (ABL) {
-          const bool grow = !(m_prev > -INFINITY) || (tmax - m_prev) * sc > p.tau;
-          if (!grow) m_new = m_prev;
-        }
-        sm.m_xchg[j & 1][r] = m_new;
-        named_bar_arrive(bar_send, 64);
-        const float mref = m_new * sc;
-        // per block: amax = exp2((bmax - m)*sc); scale; y_i = exp2(s_i*sc - m*sc - log2(scale))
-        float lsc[kNB];                              // log2 of each block's scale (+inf: zero block)
-        const float gp = ABL ? p.gp : kGpNvfp4, inv6gp = ABL ? p.inv6gp : kInvSixGp;
-  #pragma unroll
-        for (int w = 0; w < kNB / 4; ++w) sfw[w] = 0;
-  #pragma unroll
-        for (int bi = 0; bi < kNB; ++bi) {
-          const float amax = ex2_approx((bmax[bi] - m_new) * sc);
-          uint32_t code;
-          if constexpr (MX) {
-            const int e = mx_exponent(amax, p.qmax_p);
-            code = static_cast<uint32_t>(e + 127);
-            lsc[bi] = amax > 0.0f ? static_cast<float>(e) : INFINITY;
-          } else {
-            const float t = amax * inv6gp;                           // amax / (6 * gp)
-            code = ue4m3_encode(t);
-            const float sf = ue4m3_decode(code);
-            lsc[bi] = sf > 0.0f ? lg2_approx(sf * gp) : INFINITY;
-          }
-          sfw[bi >> 2] |= code << (8 * (bi & 3));
-        }
-        uint32_t packed[kBN / 8];
-        auto quantise_row = [&](auto exponent_argument, auto observe) {
-  #pragma unroll
-          for (int g8 = 0; g8 < kBN / 8; ++g8) {
-            const float l8 = lsc[(g8 * 8) / C::kBlk];
-            float y[8];
-  #pragma unroll
-            for (int i = 0; i < 8; i += 2) exponent_argument(y[i], y[i + 1], s[8 * g8 + i], s[8 * g8 + i + 1], l8);
-  #pragma unroll
-            for (int i = 0; i < kEmulPer8; i += 2) ex2_poly2(y[i], y[i + 1], y[i], y[i + 1]);
-  #pragma unroll
-            for (int i = kEmulPer8; i < 8; ++i) y[i] = ex2_approx(y[i]);
-            observe(g8, y);
-            packed[g8] = e2m1x8(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
-          }
+        // scaled exponentials of the whole row for the P~ normaliser: per block, (sum of y)
+        // times the block's scale in MMA units (2^e for MXFP4, the UE4M3 value for NVFP4)
+#pragma unroll
+        for (int bi = 0; bi < kNB; ++bi) ysum[bi] = 0.0f;
+        auto sum_observer = [&](int g8, const float* y) {
+          ysum[(g8 * 8) / C::kBlk] += ((y[0] + y[1]) + (y[2] + y[3])) + ((y[4] + y[5]) + (y[6] + y[7]));
         };
-        auto no_observer = [](int, const float*) {};
-        auto standard_argument = [&](float& y0, float& y1, float s0, float s1, float l8) {
-          const float o8 = mref + l8;
-          ffma2(y0, y1, s0, s1, sc, sc, -o8, -o8);
-        };
-        if constexpr (!ABL) {
-          quantise_row(standard_argument, no_observer);
-        } else {
-          // scaled exponentials of the whole row for the P~ normaliser: per block, (sum of y)
-          // times the block's scale in MMA units (2^e for MXFP4, the UE4M3 value for NVFP4)
-  #pragma unroll
-          for (int bi = 0; bi < kNB; ++bi) ysum[bi] = 0.0f;
-          auto sum_observer = [&](int g8, const float* y) {
-            ysum[(g8 * 8) / C::kBlk] += ((y[0] + y[1]) + (y[2] + y[3])) + ((y[4] + y[5]) + (y[6] + y[7]));
+        if (p.tau > 0.0f) {
+          // Reference kept from an earlier tile: a key whose score equals it has P~ = 1 in a
+          // block whose scale is 2^e, e possibly 2, so y = 2^-e may sit exactly on the E2M1
+          // tie 0.25.  The argument is formed from the exact difference s - m, so such a key
+          // gets exactly -e (2^-2 from MUFU, or just below from the polynomial: both round to
+          // 0 like the tie itself).
+          const float mn = m_new;
+          auto exact_argument = [&](float& y0, float& y1, float s0, float s1, float l8) {
+            ffma2(y0, y1, s0, s1, 1.0f, 1.0f, -mn, -mn);
+            ffma2(y0, y1, y0, y1, sc, sc, -l8, -l8);
           };
-          if (p.tau > 0.0f) {
-            // Reference kept from an earlier tile: a key whose score equals it has P~ = 1 in a
-            // block whose scale is 2^e, e possibly 2, so y = 2^-e may sit exactly on the E2M1
-            // tie 0.25.  The argument is formed from the exact difference s - m, so such a key
-            // gets exactly -e (2^-2 from MUFU, or just below from the polynomial: both round to
-            // 0 like the tie itself).
-            const float mn = m_new;
-            auto exact_argument = [&](float& y0, float& y1, float s0, float s1, float l8) {
-              ffma2(y0, y1, s0, s1, 1.0f, 1.0f, -mn, -mn);
-              ffma2(y0, y1, y0, y1, sc, sc, -l8, -l8);
-            };
-            if (p.l_from_ptilde) quantise_row(exact_argument, sum_observer);
-            else quantise_row(exact_argument, no_observer);
-          } else {
-            quantise_row(standard_argument, sum_observer);
-          }
+          if (p.l_from_ptilde) quantise_row(exact_argument, sum_observer);
+          else quantise_row(exact_argument, no_observer);
+        } else {
+          quantise_row(standard_argument, sum_observer);
         }
-        // accumulator g and P buffer g were last used by this group's previous PV product
-        if (j >= 2)
-          ok = warp_wait(&sm.o_done[g], (done_g + (j >> 1) - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
-        uint8_t* pbuf = sm.p[g];
-  #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(pbuf + swz64_offset(r, c)) =
-              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-  #pragma unroll
-        for (int a = 0; a < C::kSfTileAtoms; ++a)
-          *reinterpret_cast<uint32_t*>(sm.sfp[g] + 512 * a + (r & 31) * 16 + (r >> 5) * 4) = sfw[a];
-        fence_proxy_async_smem();
       }
+      // accumulator g and P buffer g were last used by this group's previous PV product
+      if (j >= 2)
+        ok = warp_wait(&sm.o_done[g], (done_g + (j >> 1) - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
+      uint8_t* pbuf = sm.p[g];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(pbuf + swz64_offset(r, c)) =
+            make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+#pragma unroll
+      for (int a = 0; a < C::kSfTileAtoms; ++a)
+        *reinterpret_cast<uint32_t*>(sm.sfp[g] + 512 * a + (r & 31) * 16 + (r >> 5) * 4) = sfw[a];
+      fence_proxy_async_smem();
       // bring accumulator g from the maximum it holds (tile j-2) to m_j
       if (ABL && p.l_from_ptilde) {
         float add = 0.0f;
@@ -1048,28 +832,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float lb = (ABL && p.l_from_ptilde) ? sm.l_last[1][r] : __uint_as_float(lrb);
       const float l = la * wa + (has_b ? lb * wb : 0.0f);
       const float inva = p.g_v / l * wa, invb = p.g_v / l * wb;
-      const bool store = !DEC && row < p.S_q;
+      const bool store = row < p.S_q;
       const int64_t orow = (int64_t)bh_q * p.S_q + row;
-      if constexpr (DEC) {
-        // partial of q-head `lane` of the group over quadrant wq's keys of the split: m in
-        // log2 units, l and o in true units (the PV products carry neither g_P nor g_v)
-        const int G = p.Hq / p.Hkv;
-        if (lane < G) {
-          float* dst = p.dec_ws + ((((int64_t)it.b * p.Hq + it.h * G + lane) * p.dec_splits + it.qt) * 4 + wq) * (D + 2);
-          const float so = kGpNvfp4 * p.g_v;
-#pragma unroll
-          for (int c = 0; c < D / 64; ++c) {
-            const int ocol = g * (D / 2) + 32 * c;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              dst[2 + ocol + i] = (__uint_as_float(rawa[c][i]) * wa + (has_b ? __uint_as_float(rawb[c][i]) * wb : 0.0f)) * so;
-          }
-          if (g == 0) {
-            dst[0] = m * sc;
-            dst[1] = l * kGpNvfp4;
-          }
-        }
-      }
       if (store) {
 #pragma unroll
         for (int c = 0; c < D / 64; ++c) {
@@ -1251,7 +1015,7 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
       !make_map_3d(&tv, vt, prm.S_kpad / 2, D, (uint64_t)prm.B * prm.Hkv, kBN / 2, D,
                    CU_TENSOR_MAP_SWIZZLE_64B))
     return FA4Q_ERR_CUDA;
-  const size_t smem = sizeof(Smem<D, MX, kStages>) + 1024;
+  const size_t smem = sizeof(Smem<D, MX>) + 1024;
   // Short items (few key tiles on average, as in causal attention over a few thousand keys)
   // run persistently, one CTA per SM walking the item list, so the per-CTA setup and the
   // pipeline fill and drain of an item overlap the neighbouring items.  Long items run one
@@ -1462,4 +1226,3 @@ extern "C" fa4q_status fa4q_attn_fwd_hybrid(
   if (fmt == FA4Q_MXFP4) return launch_attn<128, true, true, false, true>(q, k, vt, prm, st);
   return launch_attn<128, false, true, false, true>(q, k, vt, prm, st);
 }
-
