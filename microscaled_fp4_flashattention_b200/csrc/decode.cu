@@ -160,13 +160,19 @@ FA4Q_DEVINL void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32
                : "r"(addr));
 }
 
-// Issue the copies of unit `u` into one ring stage (lane 0 only).
+// Block-table entry of unit u (FP4 pages only; 0 otherwise).  Read one unit before the
+// unit is issued, so the lookup's latency is not on the path of the copy.
+FA4Q_DEVINL int64_t unit_page(const DecParams& p, int b, int u) {
+  return u < p.n_ch_fp4 ? static_cast<int64_t>(p.table[(int64_t)b * p.max_pages + u]) : 0;
+}
+
+// Issue the copies of unit `u` (physical page `phys` for an FP4 page) into one ring stage
+// (lane 0 only).
 template <bool MX>
-FA4Q_DEVINL void issue_unit(const DecParams& p, const UnitInfo& x, int b, int hk, int bh, int u,
+FA4Q_DEVINL void issue_unit(const DecParams& p, const UnitInfo& x, int hk, int bh, int64_t phys,
                             uint8_t* stage, uint64_t* bar) {
   if (x.kind == 0) {
     constexpr uint32_t sf = page_sf_bytes<MX>();
-    const int64_t phys = p.table[(int64_t)b * p.max_pages + u];
     const int64_t ph = phys * p.Hkv + hk;
     mbar_arrive_expect_tx(bar, 2 * (4096 + sf));
     bulk_load(stage, p.kp + ph * 64 * (kDecD / 2), 4096, bar);
@@ -254,12 +260,15 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
   };
   int u_issue = next_valid(c_begin + warp);
   int n_issued = 0;
+  int64_t page_next = 0;                          // lane 0: block-table entry of u_issue
   if (lane == 0) {
+    page_next = u_issue < c_end ? unit_page(p, b, u_issue) : 0;
     for (int k = 0; k < kDecStages - 1 && u_issue < c_end; ++k) {
-      issue_unit<MX>(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
+      issue_unit<MX>(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), hk, bh, page_next,
                      ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
       ++n_issued;
       u_issue = next_valid(u_issue + kDecWarps);
+      page_next = u_issue < c_end ? unit_page(p, b, u_issue) : 0;
     }
   } else {
     for (int k = 0; k < kDecStages - 1 && u_issue < c_end; ++k) {
@@ -274,22 +283,26 @@ __global__ void __launch_bounds__(kDecWarps * 32, 3) decode_split_kernel(const D
     // (after a failed wait nothing new is issued; copies already in flight are still awaited)
     __syncwarp();
     if (ok && u_issue < c_end) {
-      if (lane == 0)
-        issue_unit<MX>(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), b, hk, bh, u_issue,
+      if (lane == 0) {
+        issue_unit<MX>(p, unit_info(p, u_issue, n_fp4, n_hp, n_win), hk, bh, page_next,
                        ring + (n_issued % kDecStages) * kStageBytes, &full[n_issued % kDecStages]);
+      }
       ++n_issued;
       u_issue = next_valid(u_issue + kDecWarps);
+      if (lane == 0) page_next = u_issue < c_end ? unit_page(p, b, u_issue) : 0;
     }
     const UnitInfo x = unit_info(p, u, n_fp4, n_hp, n_win);
     const int stg = n_done % kDecStages;
     if (n_done >= n_issued) break;                  // stopped issuing after a failed wait
+    // the exclusion word is read before the wait, so its latency overlaps the copy's
+    const uint64_t excl_word = (x.kind == 0 && p.excl) ? p.excl[(int64_t)bh * p.max_pages + u] : 0ull;
     ok = __all_sync(0xffffffffu, mbar_wait(&full[stg], (n_done / kDecStages) & 1, &g_decode_status,
                                            kStatusTimeoutDecode)) && ok;
     const uint8_t* st8 = ring + stg * kStageBytes;
     ++n_done;
     if (!ok) continue;
     uint64_t vmask = x.nvalid >= 64 ? ~0ull : ((1ull << x.nvalid) - 1ull);
-    if (x.kind == 0 && p.excl) vmask &= ~p.excl[(int64_t)bh * p.max_pages + u];
+    vmask &= ~excl_word;
     if (vmask == 0ull) continue;
 
     // Both unit kinds use the swap-AB form: score rows = tokens (M = 16), columns = the GQA
