@@ -46,18 +46,18 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # The decode capture ran 8 of the 32 sequences: its traffic is per sequence (it grows with the
 # number of sequences) and is scaled to the timed batch.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,485,568 + 70,400 B (bench workload)
+    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,531,904 + 136,192 B (bench workload)
     "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
-                 "sha256": "1203cde5eceedf5b81f03d572a9a52248fe883d0cc35f765e4d60b509a95a276",
-                 "bytes_per_launch": 13485568 + 70400},
-    # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,891,008 + 4,980,480 B for 8 sequences
+                 "sha256": "db57444a96ac2c0fc3d32578247edcc5c9d91eb1e8a86729799f1ec73df0e70f",
+                 "bytes_per_launch": 13531904 + 136192},
+    # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,936,576 + 5,338,368 B for 8 sequences
     "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
-               "sha256": "8823e9bfcf14353afacabc2c8a977d045d5bc5088536c644f2f53732b444205f",
-               "bytes_per_sequence": (358891008 + 4980480) // 8},
-    # profiles/decode_fp4q_paged_nvfp4_b32_l32k.md (filled in from the capture of decode_tc_kernel)
+               "sha256": "30d1b993fd9dfb1d0f3e4d581d55f6a1d1ef7f27afa37ebdeb49f3c9b5fbb0c2",
+               "bytes_per_sequence": (358936576 + 5338368) // 8},
+    # profiles/decode_fp4q_paged_nvfp4_b32_l32k.md: 1,209,192,704 + 5,807,616 B (bench workload)
     "decode_fp4q": {"sources": ("decode_tc.cu", "fa4q_common.cuh"),
-                    "sha256": None,
-                    "bytes_per_launch": None},
+                    "sha256": "f71a491ab8410525e88baddbb8aba5a3043c66af813ea227d7bc4fd0891e9b6e",
+                    "bytes_per_launch": 1209192704 + 5807616},
 }
 
 

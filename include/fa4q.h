@@ -336,12 +336,12 @@ fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const uint8_t* k_
  * as the prefill; the scan is cut into splits of T = ceil(ceil(max_pages / 2) / S) tiles,
  * S = num_splits or, for 0, ceil(1184 / (B * Hkv)), clamped to [1, ceil(max_pages / 2)];
  * each split restarts the running state and the splits merge exactly (log-sum-exp), so T is
- * part of the result.  The GQA heads of a kv-head share one 128-row query tile, both
- * residuals in one accumulation; the heads repeat in each 32-row quadrant, and quadrant w
- * takes keys [32w, 32w+32) of every tile against the tile's common maximum, so the result
- * is the whole-tile one up to FP32 summation order.
+ * part of the result.  The GQA heads of a kv-head share one MMA operand: the kernel computes
+ * S^T = K_hat [Q_hat1 ; Q_hat2]^T and O^T += V_hat^T P_hat^T with the keys and channels on
+ * the MMA's M side and the heads on N, so the result is the definition's up to FP32
+ * summation order.
  *
- * q           bf16 [B][Hq][d]; out bf16 [B][Hq][d].  d = 128, Hq % Hkv == 0; Hq / Hkv > 32
+ * q           bf16 [B][Hq][d]; out bf16 [B][Hq][d].  d = 128, Hq % Hkv == 0; Hq / Hkv > 16
  *             -> FA4Q_ERR_UNSUPPORTED.
  * k_pages ... the NVFP4 paged cache of fa4q_quantize_kv_pages (every position 0..fp4_len-1
  *             in FP4; no vertical-line set or window here); n_phys_pages = its page count.
