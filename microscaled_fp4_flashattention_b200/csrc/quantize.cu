@@ -598,8 +598,8 @@ FA4Q_DEVINL float e2m1_value(uint32_t code) {
 __global__ void __launch_bounds__(128) dec_query_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv,
                                                         uint8_t* __restrict__ qt, uint8_t* __restrict__ qt_sf) {
   constexpr int D = 128;
-  // row r holds q-head r % 32 of the group: the G <= 32 heads repeat in every 32-row
-  // quadrant, each of which takes a quarter of every key tile
+  // row r holds q-head r % 32 of the group (zero when r % 32 >= G); the FP4 tensor-core
+  // decode reads rows 0..15 as the N side of its score products
   const int grp = blockIdx.x, r = threadIdx.x;
   const int G = Hq / Hkv;
   const int b = grp / Hkv, hk = grp % Hkv;
