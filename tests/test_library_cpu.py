@@ -93,3 +93,38 @@ def test_binding_refuses_without_device(L):
         pytest.skip("a device is present")
     with pytest.raises(RuntimeError):
         fa4q._stream()
+
+
+def test_decode_fp4q_plan_workspace_and_arguments(L):
+    """The FP4 tensor-core decode's split rule and workspace size as fa4q.h states them, and
+    its argument checks (all return before any device call)."""
+    import microscaled_fp4_flashattention_b200 as fa4q
+    for B, Hq, Hkv, P, ns in [(32, 32, 8, 512, 0), (2, 8, 2, 11, 0), (2, 8, 2, 16, 3), (1, 16, 1, 9, 0),
+                              (1, 4, 1, 1, 0), (3, 8, 2, 32, 4)]:
+        tiles = (P + 1) // 2
+        s = ns if ns > 0 else -(-1184 // (B * Hkv))
+        s = max(1, min(s, max(1, tiles)))
+        tps = max(1, -(-tiles // s))
+        splits = max(1, -(-tiles // tps))
+        assert fa4q.decode_fp4q_plan(B, Hq, Hkv, P, ns) == (splits, tps)
+        part = B * Hq * splits * (128 + 2) * 4
+        off_qt = -(-part // 1024) * 1024
+        total = off_qt + B * Hkv * 2 * 128 * 64 + B * Hkv * 2 * 2 * 512
+        assert L.fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, 128, P, ns) == total
+    assert L.fa4q_decode_fp4q_workspace_size(1, 4, 1, 64, 8, 0) == 0     # d != 128
+    assert L.fa4q_decode_fp4q_workspace_size(1, 4, 1, 128, 0, 0) == 0    # no pages
+    P_, F = ctypes.c_void_p, ctypes.c_float
+    fake = P_(0x1000)
+    ptrs = [fake] * 7
+    ws = L.fa4q_decode_fp4q_workspace_size(1, 8, 2, 128, 8, 0)
+
+    def call(Hq=8, Hkv=2, d=128, fmt=0, q=fake, ws_bytes=ws):
+        return L.fa4q_decode_fp4q(q, *ptrs[1:], 16, 1, Hq, Hkv, d, 8, fmt, F(1), F(1), F(0), fake, fake,
+                                  ws_bytes, 0, None)
+    assert call(fmt=1) == 2                  # MXFP4 pages: the residual query is NVFP4
+    assert call(fmt=5) == 1                  # unknown format
+    assert call(q=None) == 1                 # null input
+    assert call(Hq=34, Hkv=2) == 2           # G = 17 > 16 heads on the MMA's N side
+    assert call(Hq=9, Hkv=2) == 1            # Hq not a multiple of Hkv
+    assert call(d=64) == 2                   # head dimension other than 128
+    assert call(ws_bytes=ws - 1) == 1        # workspace one byte short
