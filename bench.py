@@ -61,6 +61,29 @@ NCU_TRAFFIC = {
 }
 
 
+def max_over_ranks(values, dev=None):
+    """Element-wise maximum of per-rank timings over all ranks (the list itself with one rank).
+    NCCL reduces device tensors, gloo host tensors; every rank must call it in the same order."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    on_dev = dist.get_backend() == "nccl"
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=dev if on_dev else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def world_size() -> int:
+    import torch.distributed as dist
+    return dist.get_world_size() if dist.is_available() and dist.is_initialized() else 1
+
+
+def job_rate(units_per_rank: float, ms: float, world: int) -> float:
+    """Whole-job rate: the units all ranks processed over the slowest rank's time, per second."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def sources_sha256(names) -> str:
     import hashlib
     h = hashlib.sha256()
@@ -240,7 +263,7 @@ def hybrid_bench(run, w, dev, fa4q, flush, barrier, steps):
         call()
         ev[i][1].record()
     barrier()
-    ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    ms, = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in ev]))], dev)
     return {"kernels": "hybrid_full_kernel (BF16 mma.sync) + attn_fwd_kernel<HYB> (tcgen05 FP4)",
             "ms": ms, "TFLOP/s": run.flops / (ms * 1e-3) / 1e12, "window": W, "vertical_lines_per_kv_head": n_vl,
             "note": "FLOPs of the whole causal attention (both parts); seeded random vertical-line positions"}
@@ -317,8 +340,9 @@ def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
             drun.step()
         d1.record()
         barrier()
-    d_ms = d0.elapsed_time(d1) / dsteps
-    gbs = drun.bytes / (d_ms * 1e-3) / 1e9
+    d_ms, = max_over_ranks([d0.elapsed_time(d1) / dsteps], dev)
+    world = world_size()
+    gbs = job_rate(drun.bytes, d_ms, world) / 1e9
     # vertical-line identification (column mass + selection + mask + row gather); the method
     # refreshes it every 64 decoded tokens, so it is reported beside the step, not in it
     ws = torch.empty(fa4q.vlines_workspace_size(dw.B, dw.Hq, dw.Hkv, drun.q_obs.shape[2], dw.L),
@@ -333,7 +357,7 @@ def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
         ident()
     i1.record()
     torch.cuda.synchronize()
-    id_ms = i0.elapsed_time(i1) / 5
+    id_ms, = max_over_ranks([i0.elapsed_time(i1) / 5], dev)
     line["decode"] = {"workload": dw.name, "us_per_step": d_ms * 1e3, "higher_is_better": False,
                       "GBps": gbs, "bytes_per_step": drun.bytes, "gpu_launches": 2 * dsteps,
                       "roofline": {"kernel": "decode_split_kernel+decode_combine_kernel", "bound": "hbm",
@@ -401,8 +425,8 @@ def decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
             step()
         e1.record()
         barrier()
-    ms = e0.elapsed_time(e1) / dsteps
-    gbs = nbytes / (ms * 1e-3) / 1e9
+    ms, = max_over_ranks([e0.elapsed_time(e1) / dsteps], dev)
+    gbs = job_rate(nbytes, ms, world_size()) / 1e9
     line["decode_fp4q"] = {
         "workload": f"{dw.name} shape, all {L} keys FP4 (NVFP4 pages)", "us_per_step": ms * 1e3,
         "higher_is_better": False, "GBps": gbs, "bytes_per_step": nbytes, "gpu_launches": 3 * dsteps,
@@ -541,11 +565,8 @@ def main():
     attn_ms = [a.elapsed_time(b) for a, b in aev]
     t_ms = float(np.mean(step_ms))
     a_ms = float(np.mean(attn_ms))
-    if world > 1:
-        t = torch.tensor([t_ms, a_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_ms, a_ms = float(t[0]), float(t[1])
-    value = world * run.flops / (t_ms * 1e-3) / 1e12
+    t_ms, a_ms = max_over_ranks([t_ms, a_ms], dev)
+    value = job_rate(run.flops, t_ms, world) / 1e12
 
     # ablation beside the headline: conditional rescaling (reference maximum kept within 8
     # binades, fa4q_attn_fwd_ex; MXFP4 only), the attention kernel alone on the same operands
@@ -564,7 +585,7 @@ def main():
             tau_run()
             tev[i][1].record()
         barrier()
-        tau_ms = float(np.mean([a.elapsed_time(b) for a, b in tev]))
+        tau_ms, = max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in tev]))], dev)
 
     # end to end through the public API: pinned host inputs -> device, quantise, attend, output -> host
     q_h = torch.from_numpy(run.host[0]).to(torch.bfloat16).pin_memory()
@@ -590,11 +611,7 @@ def main():
         e2e_step()
     e1.record()
     barrier()
-    e_ms = e0.elapsed_time(e1) / e_steps
-    if world > 1:
-        t = torch.tensor([e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e_ms = float(t[0])
+    e_ms, = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)
     h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
     d2h = o_h.numel() * 2
 
@@ -613,7 +630,7 @@ def main():
                    "step": "quantize Q,K,V + fused FP4 attention",
                    "l2": "flushed before each timed step (256 MB write, untimed)"},
         "gpu_launches": run.launches_per_step * args.steps,
-        "e2e": {"value": world * run.flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_rate(run.flops, e_ms, world) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
         "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
                      "unit": "TFLOP/s", "frac": achieved / fp4_peak,
@@ -637,7 +654,7 @@ def main():
             fn()
             e[i][1].record()
         barrier()
-        return float(np.mean([a.elapsed_time(b) for a, b in e]))
+        return max_over_ranks([float(np.mean([a.elapsed_time(b) for a, b in e]))], dev)[0]
     rot_ms = time_q(lambda: (fa4q.quantize_rotated(run.q, w.fmt, w.qmax), fa4q.quantize_rotated(run.k, w.fmt, w.qmax)))
     inn_ms = time_q(lambda: (fa4q.quantize(run.q, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax),
                              fa4q.quantize(run.k, w.fmt, fa4q.FA4Q_AXIS_INNER, w.qmax)))
