@@ -442,23 +442,40 @@ def decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
 
 
 # ------------------------------------------------------------------------------ CPU oracle timing
-def oracle_prefill_sample(w, budget_s: float, host=None):
+def oracle_prefill_sample(w, budget_s: float, host=None, gpu_out=None, accuracy=None):
     """Time the oracle on sampled (head, row) work of workload w for about budget_s seconds;
-    returns (TFLOP/s, description, seconds)."""
+    returns (TFLOP/s, description, seconds).
+
+    With gpu_out (the GPU's output [B, Hq, S, d] for the same inputs, batch 0 used) and a dict
+    `accuracy`, the sampled rows also give the accuracy report (untimed): GPU vs oracle, and
+    GPU and oracle each vs unquantised FP64 softmax attention on the bf16 inputs (sums of
+    absolute differences over sums of absolute reference values, and maxima)."""
     from oracle import attention as OA
     from oracle import smooth as OS
     q, k, v = host if host is not None else synth.prefill_inputs(w)
     lam = OS.calibrate(*synth.calibration_inputs(w)) if w.smooth else None
     rng = np.random.default_rng(0)
     done_flops, t_used, n_rows, heads_used = 0.0, 0.0, 0, 0
+    sums = np.zeros(5)    # sums of |g-o|, |o|, |g-u|, |o-u|, |u| over the reported rows
+    maxs = np.zeros(3)    # max |g-o|, |g-u|, |o-u|
+    acc_rows = 0
     R = 64
     while t_used < budget_s and heads_used < w.Hq:
         h = int(rng.integers(w.Hq))
         rows = np.sort(rng.choice(w.S, R, replace=False))
         t0 = time.perf_counter()
-        OA.prefill(q, k, v, causal=w.causal, fmt=w.fmt, qmax=w.qmax, qmax_p=w.qmax_p, lam=lam, rows=rows,
-                   heads=[(0, h)])
+        res = OA.prefill(q, k, v, causal=w.causal, fmt=w.fmt, qmax=w.qmax, qmax_p=w.qmax_p, lam=lam, rows=rows,
+                         heads=[(0, h)])
         dt = time.perf_counter() - t0
+        if gpu_out is not None and accuracy is not None and heads_used < 6:   # bounded extra host time
+            o = np.asarray(res[(0, h)], dtype=np.float64)
+            hk = h // (w.Hq // w.Hkv)
+            u = OA.attention_plain(q[0, h], k[0, hk], v[0, hk], causal=w.causal, rows=rows)
+            g = np.asarray(gpu_out[0, h][rows], dtype=np.float64)
+            sums += [np.abs(g - o).sum(), np.abs(o).sum(), np.abs(g - u).sum(), np.abs(o - u).sum(),
+                     np.abs(u).sum()]
+            acc_rows += len(rows)
+            maxs = np.maximum(maxs, [np.abs(g - o).max(), np.abs(g - u).max(), np.abs(o - u).max()])
         keys = (rows + 1) if w.causal else np.full(R, w.S)
         done_flops += float(4.0 * w.d * keys.sum())
         t_used += dt
@@ -467,6 +484,13 @@ def oracle_prefill_sample(w, budget_s: float, host=None):
         if dt < budget_s / 8:
             R = min(w.S, R * 2)
     desc = f"{n_rows} query rows over {heads_used} heads of {w.name} (all keys per row, oracle as is)"
+    if gpu_out is not None and accuracy is not None and sums[1] > 0:
+        accuracy.update({
+            "rows": acc_rows, "what": "query rows of the first sampled heads of the cpu_baseline sample; "
+                                      "mean_rel = sum|x - ref| / sum|ref|",
+            "gpu_vs_oracle": {"max_abs": float(maxs[0]), "mean_rel": float(sums[0] / sums[1])},
+            "gpu_vs_unquantized": {"max_abs": float(maxs[1]), "mean_rel": float(sums[2] / sums[4])},
+            "oracle_vs_unquantized": {"max_abs": float(maxs[2]), "mean_rel": float(sums[3] / sums[4])}})
     return done_flops / t_used / 1e12, desc, t_used
 
 
@@ -676,6 +700,9 @@ def main():
             "note": "P quantised against a reference maximum kept within 8 binades "
                     "(FlashAttention-4 conditional rescaling); not the headline reading"}
 
+    # the GPU's output of this batch, for the accuracy report beside the CPU baseline
+    gpu_out = (run.out.float().cpu().numpy() if rank == 0 and world == 1 and not args.no_cpu_baseline
+               else None)
     if not args.no_decode:
         del run, flush
         torch.cuda.empty_cache()
@@ -684,9 +711,12 @@ def main():
         decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, _ = oracle_prefill_sample(w, 12.0)
+        acc = {}
+        v, desc, _ = oracle_prefill_sample(w, 12.0, gpu_out=gpu_out, accuracy=acc)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
                                 "sample": desc}
+        if acc:
+            line["accuracy"] = acc
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
