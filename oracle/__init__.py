@@ -23,6 +23,8 @@ A plain, slow, obviously-correct numpy implementation, written from the pages:
                 the rest FP4, one online softmax.
 * `bitdecode` - decode with a dual-residual FP4 query and FP4 probabilities against
                 the FP4 paged cache.
+* `report_accuracy` - (run by hand) the method's error against unquantised attention on
+                the synthetic workloads, from the oracle alone.
 
 Every function states the passage it follows.  Floating point is FP64 except
 where the method fixes FP32 decisions (scale selection and element rounding),
