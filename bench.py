@@ -56,7 +56,7 @@ NCU_TRAFFIC = {
                "bytes_per_sequence": (358936576 + 5338368) // 8},
     # profiles/decode_fp4q_paged_nvfp4_b32_l32k.md: 1,209,192,704 + 5,807,616 B (bench workload)
     "decode_fp4q": {"sources": ("decode_tc.cu", "fa4q_common.cuh"),
-                    "sha256": "f71a491ab8410525e88baddbb8aba5a3043c66af813ea227d7bc4fd0891e9b6e",
+                    "sha256": "8ef392cbb9624318b89523367dcdf313789e897d7bbb9704f6acd340aadc562c",
                     "bytes_per_launch": 1209192704 + 5807616},
 }
 

@@ -16,8 +16,7 @@
 //   S^T[128 keys x (16 + 16)]     = K_hat[128 x d] [Q_hat1 ; Q_hat2]^T      2 MMAs
 //   O^T[128 channels x 16 heads] += V_hat^T[128 x 128 keys] P_hat^T           2 MMAs
 // (the four S^T partials, residual x half of d, are added by the softmax, the two O^T
-// accumulators in the epilogue).  Every tcgen05 operation of the tile costs a similar time
-// in the tensor pipe whatever its size, so the tile is built from as few as it allows.
+// accumulators in the epilogue).
 // A softmax thread owns one key of the tile (its TMEM lane): the 16-key P blocks are 16
 // lanes (block maxima by shuffles), the tile maximum goes through shared memory, and P_hat^T
 // is packed by shuffles into the K-major [heads][keys] operand.  The normaliser is summed
