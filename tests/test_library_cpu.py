@@ -128,3 +128,53 @@ def test_decode_fp4q_plan_workspace_and_arguments(L):
     assert call(Hq=9, Hkv=2) == 1            # Hq not a multiple of Hkv
     assert call(d=64) == 2                   # head dimension other than 128
     assert call(ws_bytes=ws - 1) == 1        # workspace one byte short
+
+
+def test_more_entry_points_reject_bad_arguments_without_gpu(L):
+    """Hybrid prefill, fused Q/K/V quantisation, page quantisation, smoothing calibration and
+    vertical-line selection: each error below is caught before any device call."""
+    P_, F, D = ctypes.c_void_p, ctypes.c_float, ctypes.c_double
+    fake = P_(0x1000)
+    # hybrid prefill: workspace rule, bad format, window, head dim, missing vertical-line
+    # arrays, short workspace; an empty batch is a no-op
+    assert L.fa4q_attn_fwd_hybrid_workspace_size(1, 4, 128, 128) == 1 * 4 * 128 * (128 + 4) * 4
+    assert L.fa4q_attn_fwd_hybrid_workspace_size(0, 4, 128, 128) == 0
+    ws = L.fa4q_attn_fwd_hybrid_workspace_size(1, 4, 128, 128)
+
+    def hyb(fmt=0, window=16, d=128, max_vl=0, vl=fake, B=1, ws_bytes=ws):
+        return L.fa4q_attn_fwd_hybrid(*([fake] * 9), vl, vl, vl, vl, max_vl, vl, F(1), F(1), F(1), B, 4, 1, 128,
+                                      d, window, fmt, F(0), F(0), fake, 1, None, fake, ws_bytes, None)
+    assert hyb(fmt=3) == 1
+    assert hyb(window=0) == 1
+    assert hyb(d=64) == 2
+    assert hyb(max_vl=8, vl=None) == 1
+    assert hyb(ws_bytes=ws - 1) == 1
+    assert hyb(B=0) == 0
+    # fused Q/K/V quantisation: head dim, null input, GQA mismatch
+    qkv = lambda q=fake, Hq=4, d=128: L.fa4q_quantize_qkv(q, fake, fake, 1, Hq, 2, 128, 128, d, 0, F(0), F(1),
+                                                          F(1), F(1), None, None, *([fake] * 6), None)
+    assert qkv(d=96) == 2
+    assert qkv(q=None) == 1
+    assert qkv(Hq=3) == 1
+    # page quantisation: head dim, format, null input, empty length
+    pages = lambda k=fake, L_=128, d=128, fmt=0: L.fa4q_quantize_kv_pages(
+        k, fake, 1, 2, L_, d, fake, None, fake, 2, fmt, F(1), F(1), fake, fake, fake, fake, None)
+    assert pages(d=64) == 2
+    assert pages(fmt=4) == 1
+    assert pages(k=None) == 1
+    assert pages(L_=0) == 1
+    # smoothing calibration: null input, GQA mismatch
+    assert L.fa4q_smooth_calibrate(None, fake, 4, 2, 64, 128, fake, fake, None) == 1
+    assert L.fa4q_smooth_calibrate(fake, fake, 5, 2, 64, 128, fake, fake, None) == 1
+    # vertical-line selection: rho, head dim, too few selection slots, short workspace
+    vws = L.fa4q_vlines_workspace_size(1, 4, 1, 64, 1024)
+    assert vws > 0
+
+    def vl(rho=0.05, d=128, max_select=64, ws_bytes=vws):
+        return L.fa4q_select_vertical_lines(fake, fake, fake, fake, 1, 4, 1, 64, 1024, d, D(rho), F(0), fake, fake,
+                                            fake, max_select, None, 0, None, None, fake, ws_bytes, None)
+    assert vl(rho=0.0) == 1
+    assert vl(rho=1.5) == 1
+    assert vl(d=96) == 2
+    assert vl(max_select=51) == 1           # ceil(0.05 * 1024) = 52 slots needed
+    assert vl(ws_bytes=vws - 1) == 1
