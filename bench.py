@@ -1,16 +1,20 @@
 """Benchmark of the fused 4-bit microscaled FlashAttention path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 2|3|5] [--no-decode] [--no-cpu-baseline]
+                    [--workload 5|2|3] [--no-sub] [--no-decode] [--no-cpu-baseline]
 
-One step = one pass of the prefill hot path over one synthetic batch of the causal GQA
-MXFP4 workload (B=1, 32/8 heads, S=4096, d=128, Smooth-QK on): block quantisation of Q and K
-(with the calibrated per-channel multipliers) and of V (transposed), then the fused FP4
-attention kernel.  Inputs are resident in HBM; L2 (126 MB) is flushed by a 256 MB write
-before every timed step.  The metric is prefill TFLOP/s (4*B*Hq*S^2*d, halved for causal).
-The decode path (batch 32, 32/8 heads, 32768 keys, NVFP4 pages + 5% BF16 vertical lines +
-128-token BF16 window) is timed in the same run and reported under "decode" (us/step, GB/s),
-and the FP4 tensor-core decode (dual-residual query) on the same shape under "decode_fp4q".
+One step = one pass of the prefill hot path over one synthetic batch: block quantisation of
+Q, K (with the calibrated per-channel multipliers where the workload smooths) and V
+(transposed), then the fused FP4 attention kernel.  The headline workload is the largest
+single-GPU prefill: non-causal MXFP4 with the scale bound Qmax = 7.25 (B=1, H=40, S=32768,
+d=128, 1% of tokens x8).  Inputs are resident in HBM; L2 (126 MB) is flushed by a 256 MB
+write before every timed step.  The metric is prefill TFLOP/s (4*B*Hq*S^2*d, halved for
+causal).  The two other prefill workloads (causal GQA MXFP4 + Smooth-QK at S=4096, causal
+GQA NVFP4 at S=16384) are timed the same way and reported under "prefill_workloads".  The
+decode path (batch 32, 32/8 heads, 32768 keys, NVFP4 pages + 5% BF16 vertical lines +
+128-token BF16 window) is timed in the same run and reported under "decode" (us/step,
+GB/s), and the FP4 tensor-core decode (dual-residual query) on the same shape under
+"decode_fp4q".
 
 N > 1 (torchrun): every rank runs its own independent batch (weak scaling, no collective on
 the data path); the step time is the max over ranks.  `--impl reference` times the CPU oracle
@@ -46,8 +50,8 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # The decode capture ran 8 of the 32 sequences: its traffic is per sequence (it grows with the
 # number of sequences) and is scaled to the timed batch.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,531,904 + 136,192 B (bench workload)
-    "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"),
+    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,531,904 + 136,192 B (that workload only)
+    "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"), "workload": "causal_gqa_mxfp4_smooth_s4096",
                  "sha256": "db57444a96ac2c0fc3d32578247edcc5c9d91eb1e8a86729799f1ec73df0e70f",
                  "bytes_per_launch": 13531904 + 136192},
     # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,936,576 + 5,338,368 B for 8 sequences
@@ -93,9 +97,11 @@ def sources_sha256(names) -> str:
     return h.hexdigest()
 
 
-def ncu_traffic(kernel: str, sequences: int = 0):
+def ncu_traffic(kernel: str, sequences: int = 0, workload: str | None = None):
     e = NCU_TRAFFIC[kernel]
     if e["sha256"] is None or sources_sha256(e["sources"]) != e["sha256"]:
+        return None
+    if workload is not None and e.get("workload") not in (None, workload):
         return None
     return e["bytes_per_launch"] if "bytes_per_launch" in e else e["bytes_per_sequence"] * sequences
 
@@ -401,10 +407,12 @@ def decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
         del k, v
     q = (torch.randn((B, Hq, d), generator=gen, device=dev) * 1.5).to(torch.bfloat16)
     out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(int(fa4q.lib().fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, d, P, 0)),
+    tps = args.fp4q_tiles_per_split
+    splits = -(-((P + 1) // 2) // tps)
+    ws = torch.empty(int(fa4q.lib().fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, d, P, tps)),
                      dtype=torch.uint8, device=dev)
-    splits, tps = fa4q.decode_fp4q_plan(B, Hq, Hkv, P)
-    step = lambda: fa4q.decode_fp4q(q, kp, ks, vp, vs, table, lens, B * P, out=out, workspace=ws)
+    step = lambda: fa4q.decode_fp4q(q, kp, ks, vp, vs, table, lens, B * P, out=out, workspace=ws,
+                                    tiles_per_split=tps)
     for _ in range(max(3, args.warmup)):
         step()
     torch.cuda.synchronize()
@@ -495,6 +503,58 @@ def oracle_prefill_sample(w, budget_s: float, host=None, gpu_out=None, accuracy=
     return done_flops / t_used / 1e12, desc, t_used
 
 
+# ------------------------------------------------------------------------------ prefill timing
+def time_prefill(run, flush, steps, barrier, gpu_index, soak_s, dev):
+    """Time `steps` prefill steps (L2 flushed by an untimed write before each) and, inside
+    each, the attention kernel alone (CUDA events on the launching stream).  Clocks are
+    sampled during a soak of back-to-back steps and the timed loop.  Returns (mean step ms,
+    mean attention ms, clock summary), the times as the max over ranks."""
+    import torch
+    for _ in range(3):
+        run.step()
+    barrier()
+    sampler = ClockSampler(gpu_index)
+    with sampler:
+        t_end = time.time() + soak_s
+        while time.time() < t_end:
+            for _ in range(20):
+                run.step()
+            torch.cuda.synchronize()
+        barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        aev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(float(i))                      # evict L2 (untimed)
+            ev[i][0].record()
+            run.step(attn_events=aev[i])
+            ev[i][1].record()
+        barrier()
+    t_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    a_ms = float(np.mean([a.elapsed_time(b) for a, b in aev]))
+    t_ms, a_ms = max_over_ranks([t_ms, a_ms], dev)
+    return t_ms, a_ms, sampler.summary()
+
+
+def attn_roofline(w, flops, a_ms, fp4_peak, peak_src, world):
+    """Roofline record of the attention kernel: algorithmic FLOPs per launch over its mean
+    launch time, against the FP4 dense peak; `traffic` from the ncu capture of this
+    workload when the kernel is unchanged since, else null."""
+    achieved = flops / (a_ms * 1e-3) / 1e12
+    sm_mhz = load_sm_max_mhz()
+    # exponential ceiling: every score needs one 2^x; six of every eight run on MUFU at
+    # 16 per clock per SM (the FMA pipe takes the other two), 4*d FLOPs per score
+    exp_peak = 16.0 / (6.0 / 8.0) * 4 * w.d * 148 * sm_mhz * 1e6 / 1e12
+    return {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+            "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+            "traffic": ncu_traffic("attn_fwd", workload=w.name),
+            "traffic_note": "dram read + write of one launch; the bf16 output (B*Hq*S*d*2 B) can stay in L2 "
+                            "during a captured launch, so its write-back may fall outside the figure",
+            "peak_source": peak_src, "ms_per_launch": a_ms, "launches_per_step": 1,
+            "exp_ceiling": {"peak": exp_peak, "unit": "TFLOP/s", "frac": achieved / exp_peak,
+                            "what": "MUFU ex2 at 16/clk/SM for 6 of 8 exponentials, 148 SMs at "
+                                    f"{sm_mhz:.0f} MHz, 4*d FLOPs per score"}}
+
+
 # ------------------------------------------------------------------------------ main
 def main():
     ap = argparse.ArgumentParser()
@@ -502,13 +562,16 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 5])
+    ap.add_argument("--workload", type=int, default=5, choices=[2, 3, 5])
+    ap.add_argument("--no-sub", action="store_true", help="skip the other prefill workloads")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true", help="time only the decode path")
     ap.add_argument("--decode-fp4q-only", action="store_true",
                     help="time only the FP4 tensor-core decode (dual-residual query)")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="decode batch (0 = the workload's 32); smaller batches are for profiling")
+    ap.add_argument("--fp4q-tiles-per-split", type=int, default=32,
+                    help="range length of the FP4 tensor-core decode (part of its result)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--soak-s", type=float, default=2.0)
     args = ap.parse_args()
@@ -569,28 +632,8 @@ def main():
     for _ in range(max(3, args.warmup)):
         run.step()
     barrier()
-    # soak: run steps back to back so the clock sampler sees the part under load
-    sampler = ClockSampler(dev.index if world == 1 else local_rank)
-    with sampler:
-        t_end = time.time() + args.soak_s
-        while time.time() < t_end:
-            for _ in range(20):
-                run.step()
-            torch.cuda.synchronize()
-        barrier()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        aev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for i in range(args.steps):
-            flush.fill_(float(i))                      # evict L2 (untimed)
-            ev[i][0].record()
-            run.step(attn_events=aev[i])
-            ev[i][1].record()
-        barrier()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    attn_ms = [a.elapsed_time(b) for a, b in aev]
-    t_ms = float(np.mean(step_ms))
-    a_ms = float(np.mean(attn_ms))
-    t_ms, a_ms = max_over_ranks([t_ms, a_ms], dev)
+    gpu_index = dev.index if world == 1 else local_rank
+    t_ms, a_ms, clocks = time_prefill(run, flush, args.steps, barrier, gpu_index, args.soak_s, dev)
     value = job_rate(run.flops, t_ms, world) / 1e12
 
     # ablation beside the headline: conditional rescaling (reference maximum kept within 8
@@ -639,33 +682,24 @@ def main():
     e_ms, = max_over_ranks([e0.elapsed_time(e1) / e_steps], dev)
     h2d = (q_h.numel() + k_h.numel() + v_h.numel()) * 2
     d2h = o_h.numel() * 2
+    del q_h, k_h, v_h, o_h, qd, kd, vd
 
     fp4_peak = bf16_tf * FP4_PER_BF16
-    achieved = run.flops / (a_ms * 1e-3) / 1e12
-    # exponential ceiling: every score needs one 2^x; six of every eight run on MUFU at
-    # 16 per clock per SM (the FMA pipe takes the other two), 4*d FLOPs per score
-    sm_mhz = load_sm_max_mhz()
-    exp_peak = 16.0 / (6.0 / 8.0) * 4 * w.d * 148 * sm_mhz * 1e6 / 1e12
+    peak_src = f"{peak_kind} bf16 burst {bf16_tf:.1f} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4/BF16)"
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": t_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.fmt, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "S": w.S, "d": w.d, "causal": w.causal,
-                   "fmt": w.fmt, "smooth": w.smooth, "qmax": w.qmax, "parallelism": f"replicas x{world}",
+                   "fmt": w.fmt, "smooth": w.smooth, "qmax": w.qmax, "qmax_p": w.qmax_p,
+                   "parallelism": f"replicas x{world}",
                    "step": "quantize Q,K,V + fused FP4 attention",
                    "l2": "flushed before each timed step (256 MB write, untimed)"},
         "gpu_launches": run.launches_per_step * args.steps,
         "e2e": {"value": job_rate(run.flops, e_ms, world) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e_ms},
-        "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
-                     "unit": "TFLOP/s", "frac": achieved / fp4_peak,
-                     "traffic": ncu_traffic("attn_fwd") if w.name == synth.WORKLOADS[2].name else None,
-                     "peak_source": f"{peak_kind} bf16 burst {bf16_tf:.1f} TFLOP/s x {FP4_PER_BF16:g} (nominal FP4/BF16)",
-                     "ms_per_launch": a_ms,
-                     "exp_ceiling": {"peak": exp_peak, "unit": "TFLOP/s", "frac": achieved / exp_peak,
-                                     "what": "MUFU ex2 at 16/clk/SM for 6 of 8 exponentials, 148 SMs at "
-                                             f"{sm_mhz:.0f} MHz, 4*d FLOPs per score"}},
-        "clocks": sampler.summary(),
+        "roofline": attn_roofline(w, run.flops, a_ms, fp4_peak, peak_src, world),
+        "clocks": clocks,
     }
     # ablation beside the headline: Hadamard-rotated Q and K (fa4q_quantize_rotated, the
     # alternative to Smooth-QK) against the plain inner quantisation of the same tensors
@@ -690,9 +724,6 @@ def main():
         "GBps": qk_bytes / (rot_ms * 1e-3) / 1e9, "plain_inner_ms": inn_ms,
         "plain_inner_GBps": qk_bytes / (inn_ms * 1e-3) / 1e9,
         "note": "Walsh-Hadamard rotation of every Q/K row fused into the quantiser; not on the headline path"}
-    # next row beside the headline: the hybrid-precision prefill (HyQuant) on the same
-    # inputs, 5% vertical lines per kv-head (seeded positions) and a 128-token window
-    line["hybrid_prefill"] = hybrid_bench(run, w, dev, fa4q, flush, barrier, args.steps)
     if tau_ms is not None:
         line["ablation_rescale_tau8"] = {
             "kernel": "attn_fwd_kernel via fa4q_attn_fwd_ex(rescale_tau=8)", "ms_per_launch": tau_ms,
@@ -704,8 +735,34 @@ def main():
     # the GPU's output of this batch, for the accuracy report beside the CPU baseline
     gpu_out = (run.out.float().cpu().numpy() if rank == 0 and world == 1 and not args.no_cpu_baseline
                else None)
+    # the other prefill workloads, each timed as the headline (its own clocks); the hybrid
+    # prefill (HyQuant) runs beside the causal MXFP4 one, on the same inputs
+    if not args.no_sub:
+        del run
+        torch.cuda.empty_cache()
+        subs = {}
+        for wid in (5, 2, 3):
+            if wid == args.workload:
+                continue
+            ws_ = synth.WORKLOADS[wid]
+            r2 = PrefillRun(ws_, dev, fa4q, seed_offset=rank)
+            ts, as_, cl = time_prefill(r2, flush, args.steps, barrier, gpu_index, min(1.0, args.soak_s), dev)
+            subs[ws_.name] = {
+                "ms_per_step": ts, "TFLOP/s": job_rate(r2.flops, ts, world) / 1e12,
+                "config": {"B": ws_.B, "Hq": ws_.Hq, "Hkv": ws_.Hkv, "S": ws_.S, "d": ws_.d, "causal": ws_.causal,
+                           "fmt": ws_.fmt, "smooth": ws_.smooth, "qmax": ws_.qmax, "qmax_p": ws_.qmax_p},
+                "gpu_launches": r2.launches_per_step * args.steps,
+                "roofline": attn_roofline(ws_, r2.flops, as_, fp4_peak, peak_src, world), "clocks": cl}
+            if ws_.causal and ws_.fmt == "mxfp4":
+                line["hybrid_prefill"] = dict(workload=ws_.name, **hybrid_bench(r2, ws_, dev, fa4q, flush, barrier,
+                                                                               args.steps))
+            del r2
+            torch.cuda.empty_cache()
+        line["prefill_workloads"] = subs
     if not args.no_decode:
-        del run, flush
+        if args.no_sub:
+            del run
+        del flush
         torch.cuda.empty_cache()
         decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier)
         torch.cuda.empty_cache()

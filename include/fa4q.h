@@ -333,9 +333,9 @@ fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const uint8_t* k_
  * q2 = NVFP4(r); scores = (deq(q1) + deq(q2)) . k_hat; the keys of a sequence are scanned in
  * tiles of 128 positions (page pairs, in position order) with pre-normalisation quantisation
  * of P against the running maximum (NVFP4, g_P = 1/(6*448)) and the normaliser from P_hat,
- * as the prefill; the scan is cut into splits of T = ceil(ceil(max_pages / 2) / S) tiles,
- * S = num_splits or, for 0, ceil(1184 / (B * Hkv)), clamped to [1, ceil(max_pages / 2)];
- * each split restarts the running state and the splits merge exactly (log-sum-exp), so T is
+ * as the prefill; the scan of each sequence is cut into ranges of T = tiles_per_split whole
+ * tiles (0 -> 32 tiles = 4096 keys), positions [0, 128 T), [128 T, 256 T), ...; each range
+ * restarts the running state and the ranges merge exactly (log-sum-exp), so T is
  * part of the result.  The GQA heads of a kv-head share one MMA operand: the kernel computes
  * S^T = K_hat [Q_hat1 ; Q_hat2]^T and O^T += V_hat^T P_hat^T with the keys and channels on
  * the MMA's M side and the heads on N, so the result is the definition's up to FP32
@@ -351,12 +351,12 @@ fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const uint8_t* k_
  * MXFP4 pages -> FA4Q_ERR_UNSUPPORTED.  Other errors as fa4q_decode.  Three launches
  * (query tiles, the tcgen05 scan, the combine), asynchronous on `stream`.
  */
-size_t fa4q_decode_fp4q_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int num_splits);
+size_t fa4q_decode_fp4q_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int tiles_per_split);
 fa4q_status fa4q_decode_fp4q(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
                              const uint8_t* vt_pages, const uint8_t* vt_sf, const int32_t* block_table,
                              const int32_t* fp4_len, int n_phys_pages, int B, int Hq, int Hkv, int d,
                              int max_pages, fa4q_format fmt, float g_k, float g_v, float sm_scale,
-                             void* out, void* workspace, size_t workspace_bytes, int num_splits,
+                             void* out, void* workspace, size_t workspace_bytes, int tiles_per_split,
                              void* stream);
 
 /*

@@ -212,18 +212,11 @@ def attn_fwd_hybrid(q, q_sf, k, k_sf, vt, vt_sf, q_bf16, k_bf16, v_bf16, vl_pos,
     return out
 
 
-def decode_fp4q_plan(B, Hq, Hkv, max_pages, num_splits=0):
-    """(splits, tiles per split) fa4q_decode_fp4q uses (the rule in fa4q.h)."""
-    tiles = (max_pages + 1) // 2
-    s = num_splits if num_splits > 0 else -(-148 * 8 // (B * Hkv))
-    s = max(1, min(s, max(1, tiles)))
-    tps = max(1, -(-tiles // s))
-    return max(1, -(-tiles // tps)), tps
-
-
 def decode_fp4q(q, k_pages, k_sf, vt_pages, vt_sf, block_table, fp4_len, n_phys_pages, *, fmt="nvfp4",
-                g_k=1.0, g_v=1.0, sm_scale=0.0, num_splits=0, out=None, workspace=None, stream=None):
-    """FP4 tensor-core decode with a dual-residual query (fa4q_decode_fp4q); out [B, Hq, d]."""
+                g_k=1.0, g_v=1.0, sm_scale=0.0, tiles_per_split=0, out=None, workspace=None, stream=None):
+    """FP4 tensor-core decode with a dual-residual query (fa4q_decode_fp4q); out [B, Hq, d].
+    tiles_per_split: the scan restarts every that many 128-key tiles (0: the library's fixed
+    default, 32); it is part of the result."""
     import torch
     B, Hq, d = q.shape
     Hkv = k_pages.shape[1]
@@ -231,12 +224,12 @@ def decode_fp4q(q, k_pages, k_sf, vt_pages, vt_sf, block_table, fp4_len, n_phys_
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=q.device)
     if workspace is None:
-        need = int(lib().fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, d, max_pages, num_splits))
+        need = int(lib().fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, d, max_pages, tiles_per_split))
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     _check("fa4q_decode_fp4q", lib().fa4q_decode_fp4q(
         _ptr(q), _ptr(k_pages), _ptr(k_sf), _ptr(vt_pages), _ptr(vt_sf), _ptr(block_table), _ptr(fp4_len),
         n_phys_pages, B, Hq, Hkv, d, max_pages, _fmt(fmt), g_k, g_v, sm_scale, _ptr(out), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), num_splits, _stream(stream)))
+        workspace.numel() * workspace.element_size(), tiles_per_split, _stream(stream)))
     return out
 
 

@@ -30,17 +30,33 @@ def _stale() -> bool:
 
 
 def build(force: bool = False, verbose: bool = True) -> str:
-    """Compile every CUDA source of the library into one shared object (sm_100a)."""
+    """Compile every CUDA source of the library for sm_100a (one nvcc process per source, in
+    parallel) and link them into one shared object."""
     if not force and not _stale():
         return LIB_PATH
-    cmd = [nvcc_path(), "-std=c++17", "-O3", "-lineinfo", "-shared", "-Xcompiler", "-fPIC",
-           "-gencode", "arch=compute_100a,code=sm_100a", "-I", INCLUDE, "-o", LIB_PATH + ".tmp"]
-    cmd += [os.path.join(CSRC, s) for s in SOURCES]
+    from concurrent.futures import ThreadPoolExecutor
+    nvcc = nvcc_path()
+    flags = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC",
+             "-gencode", "arch=compute_100a,code=sm_100a", "-I", INCLUDE]
+    obj_dir = os.path.join(PKG_DIR, "_build")
+    os.makedirs(obj_dir, exist_ok=True)
     if verbose:
         print("[fa4q] building", os.path.relpath(LIB_PATH, ROOT), file=sys.stderr)
-    res = subprocess.run(cmd, capture_output=True, text=True)
+
+    def compile_one(src):
+        obj = os.path.join(obj_dir, src.replace(".cu", ".o"))
+        res = subprocess.run([nvcc, *flags, "-c", os.path.join(CSRC, src), "-o", obj], capture_output=True, text=True)
+        return obj, res
+
+    with ThreadPoolExecutor(max_workers=len(SOURCES)) as ex:
+        results = list(ex.map(compile_one, SOURCES))
+    errors = [r.stdout + r.stderr for _, r in results if r.returncode != 0]
+    if errors:
+        raise RuntimeError("nvcc failed:\n" + "\n".join(errors))
+    res = subprocess.run([nvcc, "-shared", "-gencode", "arch=compute_100a,code=sm_100a", "-o", LIB_PATH + ".tmp",
+                          *[o for o, _ in results]], capture_output=True, text=True)
     if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
+        raise RuntimeError("nvcc link failed:\n" + res.stdout + res.stderr)
     os.replace(LIB_PATH + ".tmp", LIB_PATH)
     return LIB_PATH
 

@@ -590,9 +590,9 @@ static int decode_chunks(int max_pages, int max_hp, int W) {
 static int decode_auto_splits(int B, int Hkv, int chunks) {
   const int target_ctas = 148 * 8;                        // 1184: ~2.9 waves of 3 CTAs per SM at B*Hkv = 256
   int s = (target_ctas + B * Hkv - 1) / (B * Hkv);
-  s = s < 1 ? 1 : s;
   const int max_s = (chunks + kDecWarps - 1) / kDecWarps;  // at least a chunk per warp
-  return s > max_s ? max_s : s;
+  s = s > max_s ? max_s : s;
+  return s < 1 ? 1 : s;
 }
 
 }  // namespace fa4q
@@ -635,6 +635,7 @@ extern "C" fa4q_status fa4q_decode(const void* q, const uint8_t* k_pages, const 
     return FA4Q_ERR_INVALID_ARG;
   if (B > 65535 || Hkv > 65535) return FA4Q_ERR_UNSUPPORTED;
   const int chunks = decode_chunks(max_pages, max_hp, W);
+  if (chunks == 0) return FA4Q_ERR_INVALID_ARG;   // no key slot at all: nothing to attend to
   const int splits = num_splits > 0 ? num_splits : decode_auto_splits(B, Hkv, chunks);
   const size_t need = (size_t)B * Hq * splits * (kDecD + 2) * sizeof(float);
   if (workspace_bytes < need) return FA4Q_ERR_INVALID_ARG;
@@ -733,10 +734,12 @@ extern "C" fa4q_status fa4q_decode_noalloc(const void* q, const uint8_t* k_pages
   if (d != kDecD) return FA4Q_ERR_UNSUPPORTED;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_pages < 0 || max_hp < 0 || W < 0 || num_splits < 0)
     return FA4Q_ERR_INVALID_ARG;
+  const int chunks = decode_chunks(max_pages, max_hp, W);
+  if (chunks == 0) return FA4Q_ERR_INVALID_ARG;   // no key slot at all: nothing to attend to
   const size_t per_split = (size_t)B * Hq * (kDecD + 2) * sizeof(float);
   int splits = num_splits;
   if (splits == 0) {
-    splits = decode_auto_splits(B, Hkv, decode_chunks(max_pages, max_hp, W));
+    splits = decode_auto_splits(B, Hkv, chunks);
     const size_t cap = kNoAllocScratchBytes / per_split;
     if (cap < 1) return FA4Q_ERR_UNSUPPORTED;  // even one split's partials exceed the array
     if ((size_t)splits > cap) splits = (int)cap;

@@ -39,6 +39,7 @@ constexpr int kTcD = 128;                 // head dimension
 constexpr int kTcN = 16;                  // query heads per MMA (the N side)
 constexpr int kTcStages = 5;
 constexpr int kTcThreads = 384;
+constexpr int kTcDefaultTilesPerSplit = 32;   // 4096 keys per range when the caller passes 0
 constexpr float kTcLog2e = 1.4426950408889634f;
 constexpr float kTcGp = 1.0f / 2688.0f;   // g_P = 1/(6*448), rounded to FP32
 constexpr float kTcInvSixGp = 1.0f / (6.0f * kTcGp);
@@ -606,15 +607,15 @@ struct TcPlan {
   size_t off_qt, off_qsf, total;
 };
 
-// splits: S = num_splits, or ceil(1184 / (B * Hkv)) for 0, clamped to [1, tiles]; tiles per
-// split T = ceil(tiles / S); the split count actually used is ceil(tiles / T)
-static TcPlan tc_plan(int B, int Hq, int Hkv, int max_pages, int num_splits) {
+// The scan of each sequence restarts its running state every T tiles (T = tiles_per_split,
+// 0 -> kTcDefaultTilesPerSplit): T is part of the result, so it never depends on the batch,
+// the head count or the GPU.  The split count follows from the longest sequence the block
+// table can map: ceil(ceil(max_pages / 2) / T).
+static TcPlan tc_plan(int B, int Hq, int Hkv, int max_pages, int tiles_per_split) {
   TcPlan pl;
-  const int tiles = (max_pages + 1) / 2;
-  int s = num_splits > 0 ? num_splits : (148 * 8 + B * Hkv - 1) / (B * Hkv);
-  s = std::max(1, std::min(s, std::max(1, tiles)));
-  pl.tiles_per_split = std::max(1, (tiles + s - 1) / s);
-  pl.splits = std::max(1, (tiles + pl.tiles_per_split - 1) / pl.tiles_per_split);
+  const int tiles = std::max(1, (max_pages + 1) / 2);
+  pl.tiles_per_split = tiles_per_split > 0 ? tiles_per_split : kTcDefaultTilesPerSplit;
+  pl.splits = (tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
   const size_t part = (size_t)B * Hq * pl.splits * (kTcD + 2) * sizeof(float);
   pl.off_qt = (part + 1023) / 1024 * 1024;
   pl.off_qsf = pl.off_qt + (size_t)B * Hkv * 2 * 128 * (kTcD / 2);
@@ -648,9 +649,10 @@ static fa4q_status launch_tc(const CUtensorMap& tq, const CUtensorMap& tk, const
 
 using namespace fa4q;
 
-extern "C" size_t fa4q_decode_fp4q_workspace_size(int B, int Hq, int Hkv, int d, int max_pages, int num_splits) {
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || d != kTcD || max_pages <= 0 || num_splits < 0) return 0;
-  return tc_plan(B, Hq, Hkv, max_pages, num_splits).total;
+extern "C" size_t fa4q_decode_fp4q_workspace_size(int B, int Hq, int Hkv, int d, int max_pages,
+                                                  int tiles_per_split) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || d != kTcD || max_pages <= 0 || tiles_per_split < 0) return 0;
+  return tc_plan(B, Hq, Hkv, max_pages, tiles_per_split).total;
 }
 
 extern "C" fa4q_status fa4q_decode_fp4q(const void* q, const uint8_t* k_pages, const uint8_t* k_sf,
@@ -658,13 +660,13 @@ extern "C" fa4q_status fa4q_decode_fp4q(const void* q, const uint8_t* k_pages, c
                                         const int32_t* block_table, const int32_t* fp4_len,
                                         int n_phys_pages, int B, int Hq, int Hkv, int d, int max_pages,
                                         fa4q_format fmt, float g_k, float g_v, float sm_scale, void* out,
-                                        void* workspace, size_t workspace_bytes, int num_splits,
+                                        void* workspace, size_t workspace_bytes, int tiles_per_split,
                                         void* stream) {
   if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
   if (fmt == FA4Q_MXFP4) return FA4Q_ERR_UNSUPPORTED;          // the query residuals are NVFP4
   if (!q || !k_pages || !k_sf || !vt_pages || !vt_sf || !block_table || !fp4_len || !out || !workspace)
     return FA4Q_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_pages <= 0 || n_phys_pages <= 0 || num_splits < 0)
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || max_pages <= 0 || n_phys_pages <= 0 || tiles_per_split < 0)
     return FA4Q_ERR_INVALID_ARG;
   if (d != kTcD || Hq / Hkv > kTcN) return FA4Q_ERR_UNSUPPORTED;
   if (!(g_k > 0.0f) || !(g_v > 0.0f)) return FA4Q_ERR_INVALID_ARG;
@@ -672,7 +674,7 @@ extern "C" fa4q_status fa4q_decode_fp4q(const void* q, const uint8_t* k_pages, c
       !aligned16(out) || !aligned16(workspace))
     return FA4Q_ERR_INVALID_ARG;
   if ((int64_t)n_phys_pages * Hkv > 0x7fffffff || (int64_t)B * Hkv * 2 > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
-  const TcPlan pl = tc_plan(B, Hq, Hkv, max_pages, num_splits);
+  const TcPlan pl = tc_plan(B, Hq, Hkv, max_pages, tiles_per_split);
   if (workspace_bytes < pl.total) return FA4Q_ERR_INVALID_ARG;
   if ((int64_t)B * Hkv * pl.splits > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -30,14 +30,26 @@ def tile_sf(sf_rm, rows, cols, blk):
 
 
 def assert_close(got, ref, max_abs=2e-2, mean_rel=2e-3, what=""):
+    """max |got - ref| <= max_abs and sum |got - ref| / sum |ref| <= mean_rel; prints the
+    observed pair (visible with pytest -s or in the report of a failure)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     assert got.shape == ref.shape, (got.shape, ref.shape)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     err = np.abs(got - ref)
     mr = err.sum() / max(np.abs(ref).sum(), 1e-30)
+    print(f"[parity] {what}: max_abs={err.max():.3e} mean_rel={mr:.3e} (bounds {max_abs:g} / {mean_rel:g})")
     assert err.max() <= max_abs and mr <= mean_rel, f"{what}: max_abs={err.max():.3e} mean_rel={mr:.3e}"
     return err.max(), mr
+
+
+def bf16_ref(ref):
+    """An FP64 oracle output rounded as the kernels round a bf16 output (to FP32, then to
+    bfloat16 by round-to-nearest-even), for comparison with a bf16 result."""
+    x = np.ascontiguousarray(np.asarray(ref, dtype=np.float64).astype(np.float32))
+    u = x.view(np.uint32)
+    r = (u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) & np.uint32(0xFFFF0000)
+    return r.view(np.float32).astype(np.float64)
 
 
 def to_dev_bf16(a, dev):

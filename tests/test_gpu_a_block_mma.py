@@ -1,7 +1,6 @@
 """One block-scaled FP4 tensor-core MMA (the prefill kernel's MMA path) against an FP64
 product of the oracle-dequantised operands: pins operand swizzle, descriptors, scale-factor
 TMEM layout and the per-format scale selection."""
-import os
 
 import numpy as np
 import pytest
@@ -46,7 +45,4 @@ def test_block_mma_matches_fp64(fmt, K, N):
     torch.cuda.synchronize()
     bound = 1e-5 * (np.abs(A) @ np.abs(Bm).T) + 1e-30
     bad = np.abs(got - ref) > bound
-    if bad.any() and os.environ.get("FA4Q_DUMP"):
-        os.makedirs("gpurun_out", exist_ok=True)
-        np.savez(f"gpurun_out/mma_{fmt}_{N}_{K}.npz", ca=ca, cb=cb, sa=sa, sb=sb, got=got, ref=ref)
     assert not bad.any(), f"{bad.sum()} of {bad.size} wrong; max err {np.abs(got - ref).max():.4g}"

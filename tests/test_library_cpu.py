@@ -81,6 +81,10 @@ def test_argument_errors_without_gpu(L):
     dargs = [fake] * 14
     assert L.fa4q_decode(*dargs, 1, 32, 2, 128, 4, 0, 0, 0, F(1), F(1), F(0), fake, fake, 1 << 30, 0, None) == 2
     assert L.fa4q_decode(*dargs, 1, 8, 2, 128, 4, 0, 0, 0, F(1), F(1), F(0), fake, fake, 16, 0, None) == 1
+    # decode over a cache with no key slot at all (no pages, no BF16 set, no window), with the
+    # automatic split count: refused as an argument error, with and without a workspace
+    assert L.fa4q_decode(*dargs, 1, 8, 2, 128, 0, 0, 0, 0, F(1), F(1), F(0), fake, fake, 1 << 30, 0, None) == 1
+    assert L.fa4q_decode_noalloc(*dargs, 1, 8, 2, 128, 0, 0, 0, 0, F(1), F(1), F(0), fake, 0, None) == 1
     # selftest: bad shapes
     assert L.fa4q_selftest_block_mma(fake, fake, fake, fake, 24, 64, 0, fake, None) == 2
     assert L.fa4q_selftest_block_mma(fake, fake, fake, fake, 128, 96, 0, fake, None) == 2
@@ -96,21 +100,19 @@ def test_binding_refuses_without_device(L):
 
 
 def test_decode_fp4q_plan_workspace_and_arguments(L):
-    """The FP4 tensor-core decode's split rule and workspace size as fa4q.h states them, and
-    its argument checks (all return before any device call)."""
-    import microscaled_fp4_flashattention_b200 as fa4q
-    for B, Hq, Hkv, P, ns in [(32, 32, 8, 512, 0), (2, 8, 2, 11, 0), (2, 8, 2, 16, 3), (1, 16, 1, 9, 0),
-                              (1, 4, 1, 1, 0), (3, 8, 2, 32, 4)]:
+    """The FP4 tensor-core decode's range rule and workspace size as fa4q.h states them (the
+    split count is ceil(ceil(max_pages / 2) / T), T = tiles_per_split or 32, whatever the
+    batch), and its argument checks (all return before any device call)."""
+    for B, Hq, Hkv, P, tps in [(32, 32, 8, 512, 0), (2, 8, 2, 11, 0), (2, 8, 2, 16, 3), (1, 16, 1, 9, 0),
+                               (1, 4, 1, 1, 0), (3, 8, 2, 32, 4), (1, 32, 8, 512, 0), (64, 32, 8, 512, 0)]:
         tiles = (P + 1) // 2
-        s = ns if ns > 0 else -(-1184 // (B * Hkv))
-        s = max(1, min(s, max(1, tiles)))
-        tps = max(1, -(-tiles // s))
-        splits = max(1, -(-tiles // tps))
-        assert fa4q.decode_fp4q_plan(B, Hq, Hkv, P, ns) == (splits, tps)
+        T = tps if tps > 0 else 32
+        splits = -(-tiles // T)
         part = B * Hq * splits * (128 + 2) * 4
         off_qt = -(-part // 1024) * 1024
         total = off_qt + B * Hkv * 2 * 128 * 64 + B * Hkv * 2 * 2 * 512
-        assert L.fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, 128, P, ns) == total
+        assert L.fa4q_decode_fp4q_workspace_size(B, Hq, Hkv, 128, P, tps) == total
+    assert L.fa4q_decode_fp4q_workspace_size(1, 4, 1, 128, 8, -1) == 0   # negative range length
     assert L.fa4q_decode_fp4q_workspace_size(1, 4, 1, 64, 8, 0) == 0     # d != 128
     assert L.fa4q_decode_fp4q_workspace_size(1, 4, 1, 128, 0, 0) == 0    # no pages
     P_, F = ctypes.c_void_p, ctypes.c_float
@@ -118,9 +120,10 @@ def test_decode_fp4q_plan_workspace_and_arguments(L):
     ptrs = [fake] * 7
     ws = L.fa4q_decode_fp4q_workspace_size(1, 8, 2, 128, 8, 0)
 
-    def call(Hq=8, Hkv=2, d=128, fmt=0, q=fake, ws_bytes=ws):
+    def call(Hq=8, Hkv=2, d=128, fmt=0, q=fake, ws_bytes=ws, tps=0):
         return L.fa4q_decode_fp4q(q, *ptrs[1:], 16, 1, Hq, Hkv, d, 8, fmt, F(1), F(1), F(0), fake, fake,
-                                  ws_bytes, 0, None)
+                                  ws_bytes, tps, None)
+    assert call(tps=-1) == 1                 # negative range length
     assert call(fmt=1) == 2                  # MXFP4 pages: the residual query is NVFP4
     assert call(fmt=5) == 1                  # unknown format
     assert call(q=None) == 1                 # null input
