@@ -481,10 +481,11 @@ def oracle_prefill_sample(w, budget_s: float, host=None, gpu_out=None, accuracy=
             hk = h // (w.Hq // w.Hkv)
             u = OA.attention_plain(q[0, h], k[0, hk], v[0, hk], causal=w.causal, rows=rows[sel])
             g = np.asarray(gpu_out[0, h][rows[sel]], dtype=np.float64)
-            sums += [np.abs(g - o).sum(), np.abs(o).sum(), np.abs(g - u).sum(), np.abs(o - u).sum(),
+            ob = synth.round_to_bf16(o.astype(np.float32)).astype(np.float64)   # the GPU output is bf16
+            sums += [np.abs(g - ob).sum(), np.abs(ob).sum(), np.abs(g - u).sum(), np.abs(o - u).sum(),
                      np.abs(u).sum()]
             acc_rows += len(rows[sel])
-            maxs = np.maximum(maxs, [np.abs(g - o).max(), np.abs(g - u).max(), np.abs(o - u).max()])
+            maxs = np.maximum(maxs, [np.abs(g - ob).max(), np.abs(g - u).max(), np.abs(o - u).max()])
         keys = (rows + 1) if w.causal else np.full(R, w.S)
         done_flops += float(4.0 * w.d * keys.sum())
         t_used += dt
@@ -496,7 +497,8 @@ def oracle_prefill_sample(w, budget_s: float, host=None, gpu_out=None, accuracy=
     if gpu_out is not None and accuracy is not None and sums[1] > 0:
         accuracy.update({
             "rows": acc_rows, "what": "query rows of the first sampled heads of the cpu_baseline sample; "
-                                      "mean_rel = sum|x - ref| / sum|ref|",
+                                      "mean_rel = sum|x - ref| / sum|ref|; the bf16 GPU output is compared "
+                                      "with the oracle rounded to bf16",
             "gpu_vs_oracle": {"max_abs": float(maxs[0]), "mean_rel": float(sums[0] / sums[1])},
             "gpu_vs_unquantized": {"max_abs": float(maxs[1]), "mean_rel": float(sums[2] / sums[4])},
             "oracle_vs_unquantized": {"max_abs": float(maxs[2]), "mean_rel": float(sums[3] / sums[4])}})

@@ -123,6 +123,10 @@ struct AttnParams {
   float score_scale_log2;  // sm_scale * g_q * g_k * log2(e)
   float g_v;
   float qmax_p;
+  // MXFP4 P scale without an exponential: with x = (bmax - m) * sc the block maximum is 2^x,
+  // so the OCP exponent floor(log2 amax) - 2 is floor(x) - 2 and the bound-Q rule (smallest
+  // e with amax <= Q 2^e) is ceil(x - log2 Q).
+  float log2_qmax_p;
   // Conditional rescaling (FlashAttention-4, as named in the FLAMIA page's abstract): the
   // reference maximum moves only when a tile's maximum exceeds it by more than tau binades
   // (tau = 0: the exact running maximum).  NVFP4 P then takes the tensor scale
@@ -182,6 +186,13 @@ FA4Q_DEVINL bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 FA4Q_DEVINL bool warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag, uint32_t code) {
   if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
   return __all_sync(0xffffffffu, cta_wait(bar, parity, abort_flag, code));
+}
+
+// Wait of the MMA-issuing thread: a non-blocking test first (its inputs are usually ready),
+// then the bounded suspending wait.
+FA4Q_DEVINL bool mma_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return cta_wait(bar, parity, abort_flag, kStatusTimeoutMma);
 }
 
 FA4Q_DEVINL float ex2_approx(float x) {
@@ -457,9 +468,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one()) {
-      const uint32_t ones_addr = smem_u32(sm.ones);
-      for (int a = 0; a < C::kSfTileAtoms; ++a)
-        tmem_cp_sf_atom(tmem + kColSfOne + 4 * a, smem_u32(sm.sfone + 512 * a));
+      // Every shared-memory descriptor is formed once: a tile at byte offset o from the
+      // shared-memory base has the base's descriptor plus o/16 (the start-address field;
+      // shared memory is below 256 KB, so the field never carries), so issuing an MMA is a
+      // few integer adds (this single thread's latency sits on the softmax groups' path).
+      using SM = Smem<D, MX>;
+      const uint32_t base = smem_u32(&sm);
+      const uint64_t d_qk = make_smem_desc(base, 16, C::kQKSbo, C::kQKSwizzle);   // Q and K tiles
+      const uint64_t d_pv = make_smem_desc(base, 16, 512, kSwiz64);               // P, V^T, ones
+      const uint64_t d_sf = make_smem_desc(base, 0, 128, kSwizNone);              // scale atoms
+      constexpr uint64_t oq = offsetof(SM, q) >> 4, ok_ = offsetof(SM, k) >> 4, ov = offsetof(SM, v) >> 4;
+      constexpr uint64_t op = offsetof(SM, p) >> 4, oones = offsetof(SM, ones) >> 4;
+      constexpr uint64_t osfq = offsetof(SM, sfq) >> 4, osfk = offsetof(SM, sfk) >> 4;
+      constexpr uint64_t osfv = offsetof(SM, sfv) >> 4, osfp = offsetof(SM, sfp) >> 4;
+      constexpr uint64_t osfone = offsetof(SM, sfone) >> 4;
+      constexpr uint64_t kQStride = C::kQBytes >> 4, kKStride = C::kKBytes >> 4, kVStride = C::kVBytes >> 4;
+      constexpr uint64_t kPStride = C::kPBytes >> 4, kSfStride = 1024 >> 4;
+      // instruction descriptors (MXFP4: the 64-element step selects its scale byte pair)
+      const uint32_t id_s[2] = {make_idesc_fp4(kBN, MX, 0, 0), make_idesc_fp4(kBN, MX, MX ? 2 : 0, MX ? 2 : 0)};
+      const uint32_t id_o[2] = {make_idesc_fp4(D, MX, 0, 0), make_idesc_fp4(D, MX, MX ? 2 : 0, MX ? 2 : 0)};
+      const uint32_t id_l[2] = {make_idesc_fp4(16, MX, 0, 0), make_idesc_fp4(16, MX, MX ? 2 : 0, MX ? 2 : 0)};
+      // TMEM scale column of the 64-element step kk (MXFP4: two steps share a 4-column atom)
+      auto sf_step = [](int kk) -> uint32_t { return MX ? 4u * (kk >> 1) : 4u * kk; };
+      auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t sfa, uint32_t sfb, uint32_t acc) {
+        if constexpr (MX) mma_mxf4(d, ad, bd, idesc, sfa, sfb, acc);
+        else mma_nvf4(d, ad, bd, idesc, sfa, sfb, acc);
+      };
+      for (int a = 0; a < C::kSfTileAtoms; ++a) tmem_cp_sf_desc(tmem + kColSfOne + 4 * a, d_sf + osfone + 32 * a);
       bool ok = true;
       int T = 0;                                   // key tiles of all earlier items
       int n_pv0 = 0, n_pv1 = 0;                    // PV products issued per softmax group
@@ -468,28 +503,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u < 0) break;
         const Item it = decode_item(u);
         const int qs = k & 1, T0 = T, n_tiles = it.n_tiles;
-        if (!cta_wait(&sm.bar_q[qs], (k >> 1) & 1, abort_flag, kStatusTimeoutMma)) break;
+        if (!mma_wait(&sm.bar_q[qs], (k >> 1) & 1, abort_flag)) break;
         tc_fence_after();
         // item k-2 used this scale slot; all of its products completed before item k-1 ended
-        for (int a = 0; a < C::kSfQAtoms; ++a)
-          tmem_cp_sf_atom(tmem + kColSfQ + 8 * qs + 4 * a, smem_u32(sm.sfq[qs] + 512 * a));
-        const uint32_t q_addr = smem_u32(sm.q[qs]);
+        for (int a = 0; a < C::kSfQAtoms; ++a) tmem_cp_sf_desc(tmem + kColSfQ + 8 * qs + 4 * a, d_sf + osfq + qs * kSfStride + 32 * a);
+        const uint64_t qd = d_qk + oq + qs * kQStride;
         // S_j = Q K_j^T into the single S buffer once the softmax group of the previous key
         // tile (of this item or the last) holds its scores in registers
         auto issue_s = [&](int j) -> bool {
           const int t = T0 + j, s = t % kStages, kb = t & 1;
-          if (!cta_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag, kStatusTimeoutMma)) return false;
-          if (t >= 1 && !cta_wait(&sm.s_free, (t - 1) & 1, abort_flag, kStatusTimeoutMma)) return false;
+          if (!mma_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag)) return false;
+          if (t >= 1 && !mma_wait(&sm.s_free, (t - 1) & 1, abort_flag)) return false;
           tc_fence_after();
           for (int a = 0; a < C::kSfQAtoms; ++a)
-            tmem_cp_sf_atom(tmem + kColSfK + 8 * kb + 4 * a, smem_u32(sm.sfk[s] + 512 * a));
-          const uint32_t k_addr = smem_u32(sm.k[s]);
+            tmem_cp_sf_desc(tmem + kColSfK + 8 * kb + 4 * a, d_sf + osfk + s * kSfStride + 32 * a);
+          const uint64_t kd = d_qk + ok_ + s * kKStride;
 #pragma unroll
-          for (int ks = 0; ks < C::kKStepsQK; ++ks) {
-            const uint64_t ad = make_smem_desc(q_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-            const uint64_t bd = make_smem_desc(k_addr + 32 * ks, 16, C::kQKSbo, C::kQKSwizzle);
-            mma_step<MX>(tmem + kColS, ad, bd, kBN, ks, tmem + kColSfQ + 8 * qs, tmem + kColSfK + 8 * kb, ks > 0);
-          }
+          for (int kk = 0; kk < C::kKStepsQK; ++kk)
+            mma(tmem + kColS, qd + 2 * kk, kd + 2 * kk, id_s[kk & 1], tmem + kColSfQ + 8 * qs + sf_step(kk),
+                tmem + kColSfK + 8 * kb + sf_step(kk), kk > 0);
           tc_commit(&sm.s_full[j & 1]);
           return true;
         };
@@ -497,28 +529,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // product of an item waits until the previous item's epilogue has read O and l
         auto issue_pv = [&](int jp) -> bool {
           const int t = T0 + jp, s = t % kStages, pb = jp & 1;
-          if (jp == 0 && k >= 1 && !cta_wait(&sm.o_free, (k - 1) & 1, abort_flag, kStatusTimeoutMma))
-            return false;
+          if (jp == 0 && k >= 1 && !mma_wait(&sm.o_free, (k - 1) & 1, abort_flag)) return false;
           int& n_pv = pb ? n_pv1 : n_pv0;
-          if (!cta_wait(&sm.p_full[pb], n_pv & 1, abort_flag, kStatusTimeoutMma)) return false;
+          if (!mma_wait(&sm.p_full[pb], n_pv & 1, abort_flag)) return false;
           ++n_pv;
           tc_fence_after();
           for (int a = 0; a < C::kSfTileAtoms; ++a) {
-            tmem_cp_sf_atom(tmem + kColSfP + 8 * pb + 4 * a, smem_u32(sm.sfp[pb] + 512 * a));
-            tmem_cp_sf_atom(tmem + kColSfV + 8 * pb + 4 * a, smem_u32(sm.sfv[s] + 512 * a));
+            tmem_cp_sf_desc(tmem + kColSfP + 8 * pb + 4 * a, d_sf + osfp + pb * kSfStride + 32 * a);
+            tmem_cp_sf_desc(tmem + kColSfV + 8 * pb + 4 * a, d_sf + osfv + s * kSfStride + 32 * a);
           }
-          const uint32_t p_addr = smem_u32(sm.p[pb]);
-          const uint32_t v_addr = smem_u32(sm.v[s]);
+          const uint64_t pd = d_pv + op + pb * kPStride, vd = d_pv + ov + s * kVStride, od = d_pv + oones;
           const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const uint64_t ad = make_smem_desc(p_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint64_t vd = make_smem_desc(v_addr + 32 * ks, 16, 512, kSwiz64);
-            const uint64_t od = make_smem_desc(ones_addr + 32 * ks, 16, 512, kSwiz64);
+          for (int kk = 0; kk < 2; ++kk) {
             // (hybrid: group A's accumulator starts from the full-precision part)
-            const uint32_t acc = (jp >= 2 || ks > 0 || (HYB && jp == 0)) ? 1u : 0u;
-            mma_step<MX>(tmem + o_col, ad, vd, D, ks, tmem + kColSfP + 8 * pb, tmem + kColSfV + 8 * pb, acc);
-            mma_step<MX>(tmem + l_col, ad, od, 16, ks, tmem + kColSfP + 8 * pb, tmem + kColSfOne, acc);
+            const uint32_t acc = (jp >= 2 || kk > 0 || (HYB && jp == 0)) ? 1u : 0u;
+            mma(tmem + o_col, pd + 2 * kk, vd + 2 * kk, id_o[kk], tmem + kColSfP + 8 * pb + sf_step(kk),
+                tmem + kColSfV + 8 * pb + sf_step(kk), acc);
+            mma(tmem + l_col, pd + 2 * kk, od + 2 * kk, id_l[kk], tmem + kColSfP + 8 * pb + sf_step(kk),
+                tmem + kColSfOne + sf_step(kk), acc);
           }
           tc_commit(&sm.o_done[pb]);
           tc_commit(&sm.kv_empty[s]);
@@ -651,22 +680,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       sm.m_xchg[j & 1][r] = m_new;
       named_bar_arrive(bar_send, 64);
       const float mref = m_new * sc;
-      // per block: amax = exp2((bmax - m)*sc); scale; y_i = exp2(s_i*sc - m*sc - log2(scale))
+      // per block: scale from the block maximum 2^((bmax - m)*sc); y_i = exp2(s_i*sc - m*sc -
+      // log2(scale)).  MXFP4 takes the exponent from (bmax - m)*sc directly, so its scales
+      // need no MUFU work (the MUFU unit is the softmax's scarcest resource); NVFP4 rounds
+      // amax / (6 g_P) to UE4M3 and takes the logarithm of the decoded scale.
+      const float gp = ABL ? p.gp : kGpNvfp4;
       float lsc[kNB];                              // log2 of each block's scale (+inf: zero block)
-      const float gp = ABL ? p.gp : kGpNvfp4, inv6gp = ABL ? p.inv6gp : kInvSixGp;
+      const float inv6gp = ABL ? p.inv6gp : kInvSixGp;
       uint32_t sfw[kNB / 4];
 #pragma unroll
       for (int w = 0; w < kNB / 4; ++w) sfw[w] = 0;
 #pragma unroll
       for (int bi = 0; bi < kNB; ++bi) {
-        const float amax = ex2_approx((bmax[bi] - m_new) * sc);
+        const float x = (bmax[bi] - m_new) * sc;   // log2 of the block maximum, <= 0
         uint32_t code;
         if constexpr (MX) {
-          const int e = mx_exponent(amax, p.qmax_p);
+          int e = -127;
+          if (x > -160.0f) {
+            e = p.qmax_p == 0.0f ? static_cast<int>(floorf(x)) - 2 : static_cast<int>(ceilf(x - p.log2_qmax_p));
+            e = max(e, -127);
+          }
           code = static_cast<uint32_t>(e + 127);
-          lsc[bi] = amax > 0.0f ? static_cast<float>(e) : INFINITY;
+          lsc[bi] = x > -INFINITY ? static_cast<float>(e) : INFINITY;
         } else {
-          const float t = amax * inv6gp;                           // amax / (6 * gp)
+          const float t = ex2_approx(x) * inv6gp;                  // amax / (6 * gp)
           code = ue4m3_encode(t);
           const float sf = ue4m3_decode(code);
           lsc[bi] = sf > 0.0f ? lg2_approx(sf * gp) : INFINITY;
@@ -1005,6 +1042,11 @@ cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word) {
   return cudaStreamSynchronize(st);
 }
 
+// Host side of the MXFP4 P scale rule: log2 of the bound (rounded once to FP32).
+static void fill_p_scale_rule(AttnParams& prm) {
+  prm.log2_qmax_p = prm.qmax_p > 0.0f ? static_cast<float>(std::log2(static_cast<double>(prm.qmax_p))) : 0.0f;
+}
+
 template <int D, bool MX, bool CAUSAL, bool ABL = false, bool HYB = false>
 static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t* vt,
                                const AttnParams& prm, cudaStream_t st) {
@@ -1085,6 +1127,7 @@ extern "C" fa4q_status fa4q_attn_fwd_ex(const uint8_t* q, const uint8_t* q_sf, c
   prm.tau = static_cast<float>(rescale_tau);
   prm.gp = kGpNvfp4 * static_cast<float>(1u << rescale_tau);     // exact power-of-two multiple
   prm.inv6gp = 1.0f / (6.0f * prm.gp);
+  fill_p_scale_rule(prm);
   prm.l_from_ptilde = l_from_ptilde;
   prm.causal = causal;
   prm.out_fp32 = out_is_fp32;
@@ -1219,6 +1262,9 @@ extern "C" fa4q_status fa4q_attn_fwd_hybrid(
   prm.qmax_p = qmax_p;
   prm.causal = 1;
   prm.out_fp32 = out_is_fp32;
+  prm.gp = kGpNvfp4;
+  prm.inv6gp = kInvSixGp;
+  fill_p_scale_rule(prm);
   prm.hy_part = static_cast<const float*>(workspace);
   prm.hy_window = window;
   prm.hy_excl_words = max_vl > 0 ? (S + 63) / 64 : 0;

@@ -234,6 +234,12 @@ FA4Q_DEVINL void tmem_cp_sf_atom(uint32_t taddr, uint32_t atom_saddr) {
                : "memory");
 }
 
+// The same with the atom's shared-memory descriptor already formed.
+FA4Q_DEVINL void tmem_cp_sf_desc(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc)
+               : "memory");
+}
+
 // 32 consecutive 32-bit TMEM columns of this warp's lane quadrant -> 32 registers / thread.
 FA4Q_DEVINL void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(

@@ -584,58 +584,74 @@ namespace fa4q {
 // Dual-residual NVFP4 query tiles for the FP4 tensor-core decode (BitDecoding-FP4, "Error
 // Sources": the query as the sum of two FP4 tensors, the second quantising the residual of
 // the first).  Per (sequence, kv-head) group: two 128-row tiles (residual 0 and 1) whose
-// rows 0..G-1 are the group's q-heads and the rest zero, packed [128][d/2] with tiled scale
-// atoms, exactly the layout the prefill kernel reads for a query tile.
+// rows 0..G-1 are the group's q-heads, packed [128][d/2] with tiled scale atoms, the layout
+// the decode kernel reads for its query operand.
 //   q1 = NVFP4(q);  r = q - deq(q1) (FP32, deq exact);  q2 = NVFP4(r)
-// grid: groups; 128 threads, thread = tile row.
 // ---------------------------------------------------------------------------------------
+// Signed E2M1 value of a 4-bit code, from its bit fields (exponent e, mantissa m):
+// e = 0 -> m * 0.5, e > 0 -> 2^(e-1) * (1 + m/2).
 FA4Q_DEVINL float e2m1_value(uint32_t code) {
-  const float mag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
-  const float v = mag[code & 7u];
-  return (code & 8u) ? -v : v;
+  const uint32_t c = code & 7u, e = c >> 1, m = c & 1u;
+  const uint32_t mag = e ? (((e + 126u) << 23) | (m << 22)) : (m ? 0x3F000000u : 0u);
+  return __uint_as_float(mag | ((code & 8u) << 28));
 }
 
-__global__ void __launch_bounds__(128) dec_query_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv,
-                                                        uint8_t* __restrict__ qt, uint8_t* __restrict__ qt_sf) {
+// Query tiles of the FP4 tensor-core decode: one warp per (sequence, kv-head) group; lane l
+// quantises elements [64 (l & 1), 64 (l & 1) + 64) of query head l / 2 of the group, first
+// q (NVFP4, 16-element blocks, UE4M3, tensor scale 1), then the FP32 residual
+// r = q - deq(q1) (exact: deq(q1) is an FP32 product).  Heads G..15 are zero rows.  The
+// decode reads rows 0..15 of each 128-row tile (and of its two scale atoms), so only those
+// are written: per lane and pass 32 bytes of codes (two 16-byte stores) and one 4-byte
+// scale word.
+__global__ void __launch_bounds__(128) dec_query_kernel(const uint16_t* __restrict__ q, int n_groups, int Hq,
+                                                        int Hkv, uint8_t* __restrict__ qt,
+                                                        uint8_t* __restrict__ qt_sf) {
   constexpr int D = 128;
-  // row r holds q-head r % 32 of the group (zero when r % 32 >= G); the FP4 tensor-core
-  // decode reads rows 0..15 as the N side of its score products
-  const int grp = blockIdx.x, r = threadIdx.x;
+  const int grp = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (grp >= n_groups) return;
+  const int lane = threadIdx.x & 31, h = lane >> 1, half = lane & 1;
   const int G = Hq / Hkv;
-  const int b = grp / Hkv, hk = grp % Hkv;
-  float x[D];
-  if ((r & 31) < G) {
-    const uint16_t* src = q + ((int64_t)b * Hq + hk * G + (r & 31)) * D;
+  const int b = grp / Hkv, hk = grp - b * Hkv;
+  float x[64];
+  if (h < G) {
+    const uint16_t* src = q + ((int64_t)b * Hq + hk * G + h) * D + 64 * half;
 #pragma unroll
-    for (int c = 0; c < D; c += 8) load_bf16x8(src + c, x + c);
+    for (int c = 0; c < 64; c += 8) load_bf16x8(src + c, x + c);
   } else {
 #pragma unroll
-    for (int c = 0; c < D; ++c) x[c] = 0.0f;
+    for (int c = 0; c < 64; ++c) x[c] = 0.0f;
   }
-  for (int res = 0; res < 2; ++res) {
-    uint8_t* dst = qt + ((int64_t)grp * 2 + res) * 128 * (D / 2) + r * (D / 2);
-    uint8_t* sdst = qt_sf + ((int64_t)grp * 2 + res) * 2 * 512;
 #pragma unroll
-    for (int kb = 0; kb < D / 16; ++kb) {
-      uint2 pk;
-      const uint32_t sc = quant_block16_nvfp4(x + 16 * kb, 6.0f, 1.0f, pk);
-      *reinterpret_cast<uint2*>(dst + 8 * kb) = pk;
-      sdst[sf_tiled_offset(r, kb, 2)] = static_cast<uint8_t>(sc);
+  for (int res = 0; res < 2; ++res) {
+    uint32_t pk[8], sfw = 0;
+#pragma unroll
+    for (int kb = 0; kb < 4; ++kb) {
+      uint2 p2;
+      const uint32_t sc = quant_block16_nvfp4(x + 16 * kb, 6.0f, 1.0f, p2);
+      pk[2 * kb] = p2.x;
+      pk[2 * kb + 1] = p2.y;
+      sfw |= sc << (8 * kb);
       if (res == 0) {
         // residual of this block: x - code * scale (the product is exact in FP32)
-        const float s = ue4m3_decode(sc);
-        const uint32_t w[2] = {pk.x, pk.y};
+        const float sv = ue4m3_decode(sc);
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          x[16 * kb + i] = __fsub_rn(x[16 * kb + i], e2m1_value(w[i >> 3] >> (4 * (i & 7))) * s);
+          x[16 * kb + i] = __fsub_rn(x[16 * kb + i], e2m1_value(pk[2 * kb + (i >> 3)] >> (4 * (i & 7))) * sv);
       }
     }
+    uint4* dst = reinterpret_cast<uint4*>(qt + ((int64_t)grp * 2 + res) * 128 * (D / 2) + h * (D / 2) + 32 * half);
+    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    // tiled scale layout: row h (< 32), scale columns 4 half .. 4 half + 3 -> atom `half`,
+    // bytes h * 16 + 0..3
+    *reinterpret_cast<uint32_t*>(qt_sf + ((int64_t)grp * 2 + res) * 2 * 512 + half * 512 + h * 16) = sfw;
   }
 }
 
 fa4q_status launch_dec_query(const uint16_t* q, int B, int Hq, int Hkv, uint8_t* qt, uint8_t* qt_sf,
                              cudaStream_t st) {
-  dec_query_kernel<<<B * Hkv, 128, 0, st>>>(q, Hq, Hkv, qt, qt_sf);
+  const int n_groups = B * Hkv;
+  dec_query_kernel<<<(n_groups + 3) / 4, 128, 0, st>>>(q, n_groups, Hq, Hkv, qt, qt_sf);
   return launch_status();
 }
 
