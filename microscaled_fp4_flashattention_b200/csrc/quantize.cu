@@ -596,62 +596,52 @@ FA4Q_DEVINL float e2m1_value(uint32_t code) {
   return __uint_as_float(mag | ((code & 8u) << 28));
 }
 
-// Query tiles of the FP4 tensor-core decode: one warp per (sequence, kv-head) group; lane l
-// quantises elements [64 (l & 1), 64 (l & 1) + 64) of query head l / 2 of the group, first
-// q (NVFP4, 16-element blocks, UE4M3, tensor scale 1), then the FP32 residual
-// r = q - deq(q1) (exact: deq(q1) is an FP32 product).  Heads G..15 are zero rows.  The
-// decode reads rows 0..15 of each 128-row tile (and of its two scale atoms), so only those
-// are written: per lane and pass 32 bytes of codes (two 16-byte stores) and one 4-byte
-// scale word.
-__global__ void __launch_bounds__(128) dec_query_kernel(const uint16_t* __restrict__ q, int n_groups, int Hq,
-                                                        int Hkv, uint8_t* __restrict__ qt,
-                                                        uint8_t* __restrict__ qt_sf) {
+// Query tiles of the FP4 tensor-core decode: one CTA of 128 threads per (sequence, kv-head)
+// group, thread t quantising NVFP4 block t % 8 (elements 16 (t % 8) .. +15) of query head
+// t / 8 of the group, first q (16-element blocks, UE4M3, tensor scale 1), then the FP32
+// residual r = q - deq(q1) (exact: deq(q1) is an FP32 product).  Heads G..15 are zero rows.
+// The decode reads rows 0..15 of each 128-row tile (and of its two scale atoms), so only
+// those are written: 8 bytes of codes per thread and pass (a warp covers four whole rows),
+// and per four blocks one 4-byte scale word gathered by shuffles.
+__global__ void __launch_bounds__(128) dec_query_kernel(const uint16_t* __restrict__ q, int Hq, int Hkv,
+                                                        uint8_t* __restrict__ qt, uint8_t* __restrict__ qt_sf) {
   constexpr int D = 128;
-  const int grp = blockIdx.x * 4 + (threadIdx.x >> 5);
-  if (grp >= n_groups) return;
-  const int lane = threadIdx.x & 31, h = lane >> 1, half = lane & 1;
+  const int grp = blockIdx.x, t = threadIdx.x, h = t >> 3, kb = t & 7, lane = t & 31;
   const int G = Hq / Hkv;
   const int b = grp / Hkv, hk = grp - b * Hkv;
-  float x[64];
+  float x[16];
   if (h < G) {
-    const uint16_t* src = q + ((int64_t)b * Hq + hk * G + h) * D + 64 * half;
-#pragma unroll
-    for (int c = 0; c < 64; c += 8) load_bf16x8(src + c, x + c);
+    const uint16_t* src = q + ((int64_t)b * Hq + hk * G + h) * D + 16 * kb;
+    load_bf16x8(src, x);
+    load_bf16x8(src + 8, x + 8);
   } else {
 #pragma unroll
-    for (int c = 0; c < 64; ++c) x[c] = 0.0f;
+    for (int c = 0; c < 16; ++c) x[c] = 0.0f;
   }
 #pragma unroll
   for (int res = 0; res < 2; ++res) {
-    uint32_t pk[8], sfw = 0;
+    uint2 pk;
+    const uint32_t sc = quant_block16_nvfp4(x, 6.0f, 1.0f, pk);
+    *reinterpret_cast<uint2*>(qt + ((int64_t)grp * 2 + res) * 128 * (D / 2) + h * (D / 2) + 8 * kb) = pk;
+    // tiled scale layout: row h (< 32), scale column kb -> atom kb / 4, byte h * 16 + kb % 4;
+    // lanes 4i..4i+3 hold one row's four bytes of an atom
+    const uint32_t w = sc | (__shfl_down_sync(0xffffffffu, sc, 1) << 8) | (__shfl_down_sync(0xffffffffu, sc, 2) << 16) |
+                       (__shfl_down_sync(0xffffffffu, sc, 3) << 24);
+    if ((lane & 3) == 0)
+      *reinterpret_cast<uint32_t*>(qt_sf + ((int64_t)grp * 2 + res) * 2 * 512 + (kb >> 2) * 512 + h * 16) = w;
+    if (res == 0) {
+      // residual of this block: x - code * scale (the product is exact in FP32)
+      const float sv = ue4m3_decode(sc);
 #pragma unroll
-    for (int kb = 0; kb < 4; ++kb) {
-      uint2 p2;
-      const uint32_t sc = quant_block16_nvfp4(x + 16 * kb, 6.0f, 1.0f, p2);
-      pk[2 * kb] = p2.x;
-      pk[2 * kb + 1] = p2.y;
-      sfw |= sc << (8 * kb);
-      if (res == 0) {
-        // residual of this block: x - code * scale (the product is exact in FP32)
-        const float sv = ue4m3_decode(sc);
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          x[16 * kb + i] = __fsub_rn(x[16 * kb + i], e2m1_value(pk[2 * kb + (i >> 3)] >> (4 * (i & 7))) * sv);
-      }
+      for (int i = 0; i < 16; ++i)
+        x[i] = __fsub_rn(x[i], e2m1_value((i < 8 ? pk.x : pk.y) >> (4 * (i & 7))) * sv);
     }
-    uint4* dst = reinterpret_cast<uint4*>(qt + ((int64_t)grp * 2 + res) * 128 * (D / 2) + h * (D / 2) + 32 * half);
-    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    // tiled scale layout: row h (< 32), scale columns 4 half .. 4 half + 3 -> atom `half`,
-    // bytes h * 16 + 0..3
-    *reinterpret_cast<uint32_t*>(qt_sf + ((int64_t)grp * 2 + res) * 2 * 512 + half * 512 + h * 16) = sfw;
   }
 }
 
 fa4q_status launch_dec_query(const uint16_t* q, int B, int Hq, int Hkv, uint8_t* qt, uint8_t* qt_sf,
                              cudaStream_t st) {
-  const int n_groups = B * Hkv;
-  dec_query_kernel<<<(n_groups + 3) / 4, 128, 0, st>>>(q, n_groups, Hq, Hkv, qt, qt_sf);
+  dec_query_kernel<<<B * Hkv, 128, 0, st>>>(q, Hq, Hkv, qt, qt_sf);
   return launch_status();
 }
 
