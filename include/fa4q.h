@@ -445,6 +445,17 @@ fa4q_status fa4q_selftest_block_mma(const uint8_t* a, const uint8_t* a_sf, const
                                     float* d_out, void* stream);
 
 /*
+ * fa4q_selftest_bf16_mma - diagnostic: one 128 x N x K BF16 tensor-core product D = A * B
+ * (FP32), through the operand layouts of the full-precision tiles of the hybrid prefill
+ * (HyQuant: vertical-line and window keys in BF16): A bf16 [128][K] K-major; B bf16 [N][K]
+ * (b_mn_major = 0, D = A B^T) or [K][N] (b_mn_major = 1, D = A B); both staged as 128-byte
+ * swizzled 64-element column chunks.  d_out FP32 [128][N].  K in {64, 128}; N in {16, 64,
+ * 128} (K-major B) or {64, 128} (MN-major B).  Synchronous errors as fa4q_attn_fwd.
+ */
+fa4q_status fa4q_selftest_bf16_mma(const void* a, const void* b, int N, int K, int b_mn_major,
+                                   float* d_out, void* stream);
+
+/*
  * fa4q_selftest_exp2 - diagnostic: y[i] = 2^x[i] through the FMA-pipe polynomial that the
  * prefill kernel uses for part of the unnormalised exponentials P~ = exp(S - m).  Source:
  * FLAMIA (FLAsh MIcroscaling Attention ... on Blackwell), Abstract - its FlashAttention-4

@@ -30,6 +30,7 @@ EXPORTED = [
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
     "fa4q_vlines_workspace_size", "fa4q_select_vertical_lines", "fa4q_quantize_qkv",
+    "fa4q_selftest_bf16_mma",
 ]
 
 _LIB = None
@@ -86,6 +87,8 @@ def lib() -> ctypes.CDLL:
                                           F, F, F, P, I, P]
         L.fa4q_selftest_block_mma.restype = I
         L.fa4q_selftest_block_mma.argtypes = [P, P, P, P, I, I, I, P, P]
+        L.fa4q_selftest_bf16_mma.restype = I
+        L.fa4q_selftest_bf16_mma.argtypes = [P, P, I, I, I, P, P]
         L.fa4q_device_status.restype = I
         L.fa4q_device_status.argtypes = [P, ctypes.POINTER(U32)]
         L.fa4q_selftest_wait_timeout.restype = I
@@ -402,6 +405,16 @@ def selftest_block_mma(a, a_sf, b, b_sf, N, K, fmt, stream=None):
     _check("fa4q_selftest_block_mma", lib().fa4q_selftest_block_mma(
         _ptr(a), _ptr(a_sf), _ptr(b), _ptr(b_sf), N, K, _fmt(fmt), _ptr(d), _stream(stream)))
     return d
+
+
+def selftest_bf16_mma(a, b, N, K, b_mn_major, stream=None):
+    """One BF16 tensor-core product (fa4q_selftest_bf16_mma); returns FP32 [128, N]."""
+    import torch
+    out = torch.empty((128, N), dtype=torch.float32, device=a.device)
+    _check("fa4q_selftest_bf16_mma", lib().fa4q_selftest_bf16_mma(_ptr(a), _ptr(b), N, K, int(b_mn_major),
+                                                                  _ptr(out), _stream(stream)))
+    torch.cuda.synchronize()
+    return out
 
 
 def device_status(stream=None):

@@ -202,6 +202,38 @@ FA4Q_DEVINL uint32_t make_idesc_fp4(int N, bool ue8m0, uint32_t a_sf_id, uint32_
   return d;
 }
 
+// Instruction descriptor of the BF16 MMA (kind::f16, FP32 accumulate), M = 128.  Fields:
+// D format (F32 = 1) [4,6), A / B format (BF16 = 1) [7,10) / [10,13), A major [15] (0: K-major),
+// B major [16] (0: K-major, 1: MN-major), N>>3 [17,23), M>>4 [24,29).
+FA4Q_DEVINL uint32_t make_idesc_bf16(int N, bool b_mn_major) {
+  uint32_t d = 0;
+  d |= 1u << 4;
+  d |= 1u << 7;
+  d |= 1u << 10;
+  d |= (b_mn_major ? 1u : 0u) << 16;
+  d |= (static_cast<uint32_t>(N) >> 3) << 17;
+  d |= (128u >> 4) << 24;
+  return d;
+}
+
+// D[tmem] (+)= A[smem] * B[smem] (BF16 operands, FP32 accumulate), K = 16 per instruction.
+FA4Q_DEVINL void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// byte offset of (row r, 16-byte chunk c) in a tile of 128-byte rows with the 128-byte swizzle
+// (1024-byte atoms of 8 rows; chunk c of row r stored at chunk c ^ (r % 8)) - the layout TMA
+// writes with CU_TENSOR_MAP_SWIZZLE_128B and the MMA reads with the 128B swizzle mode
+FA4Q_DEVINL uint32_t swz128_offset(uint32_t r, uint32_t c) {
+  return (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T with per-16-element UE4M3 scales (NVFP4).
 FA4Q_DEVINL void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                           uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {

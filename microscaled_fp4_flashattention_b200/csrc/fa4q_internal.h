@@ -95,5 +95,6 @@ fa4q_status launch_decode_combine(const float* ws, int rows, int splits, uint16_
 cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word);
 cudaError_t decode_status_fetch(cudaStream_t st, uint32_t* host_word);
 cudaError_t dectc_status_fetch(cudaStream_t st, uint32_t* host_word);
+cudaError_t hy_status_fetch(cudaStream_t st, uint32_t* host_word);
 
 }  // namespace fa4q
