@@ -224,32 +224,34 @@ fa4q_status fa4q_attn_fwd_ex(const uint8_t* q, const uint8_t* q_sf, const uint8_
 
 /*
  * fa4q_attn_fwd_hybrid - hybrid-precision causal prefill: window and vertical-line keys in
- * BF16, the rest in FP4, under one online softmax.
+ * BF16, the rest in FP4, under one online softmax, in one kernel.
  *
  * Source: HyQuant (Hybrid-Precision Quantization for LLM Attention): the keys of each query
  * are split into vertical-line positions, a recent sliding window and the 4-bit remainder;
  * vertical lines and the window stay in FP16/BF16; low-bit and full-precision GEMMs share
- * one FlashAttention-style online softmax.  Reading (the pages give no order or masks):
- * query row i takes the window {j : i - window < j <= i} and the vertical lines
+ * one FlashAttention-style kernel and one online softmax.  Reading (the pages give no order
+ * or masks): query row i takes the window {j : i - window < j <= i} and the vertical lines
  * {v : v <= i - window} from the BF16 inputs first (unquantised P), then the FP4 key tiles
  * (width 128, in order) with the keys of those two classes masked out, pre-normalisation
  * quantisation of P against the running maximum that started from the BF16 part, and the
- * normaliser from P_hat; every visible key counts once.
+ * normaliser from P_hat; every visible key counts once.  The kernel runs the BF16 part as
+ * tensor-core tiles of 64 keys (window band, then vertical lines) ahead of the FP4 tiles of
+ * each 128-row query tile; the BF16 probabilities enter their PV products rounded to bf16.
  *
  * q, q_sf, k, k_sf, vt, vt_sf  FP4 operands as for fa4q_attn_fwd (S_q = S_k = S), quantised
  *             from Q, K, V with the vertical-line rows of K and V zeroed first (as the decode
  *             cache; the window keys keep their FP4 copies, later rows read them).
  * q_bf16, k_bf16, v_bf16  bf16 [B][H][S][d] (H = Hq for q, Hkv for k, v).
  * vl_pos      int32 [B][Hkv][max_vl] vertical-line positions, ascending; vl_count int32
- *             [B][Hkv] (<= max_vl); vl_k, vl_v bf16 [B][Hkv][max_vl][d] their K / V rows;
- *             vl_excl uint64 [B][Hkv][ceil(S/64)] their bit mask (bit p%64 of word p/64).
+ *             [B][Hkv] (<= max_vl); vl_k, vl_v bf16 [B][Hkv][max_vl][d] their K / V rows
+ *             (rows past vl_count must hold finite values, e.g. zeros); vl_excl uint64
+ *             [B][Hkv][ceil(S/64)] their bit mask (bit p%64 of word p/64).
  *             max_vl = 0: no vertical lines (the pointers may be null).
  * window      >= 1 (128 in the pages' study).  d = 128 (else FA4Q_ERR_UNSUPPORTED).
- * workspace   device, >= fa4q_attn_fwd_hybrid_workspace_size(B, Hq, S, d) bytes, 16-byte
- *             aligned: the per-row BF16-part state, written by the first of the two launches.
- * Other arguments, layouts and errors as fa4q_attn_fwd (causal implied).
+ * g_v         (NVFP4) must be a bf16 value (the BF16 part's normaliser is formed with it in
+ *             bf16), else FA4Q_ERR_UNSUPPORTED.
+ * Other arguments, layouts and errors as fa4q_attn_fwd (causal implied).  No workspace.
  */
-size_t fa4q_attn_fwd_hybrid_workspace_size(int B, int Hq, int S, int d);
 fa4q_status fa4q_attn_fwd_hybrid(const uint8_t* q, const uint8_t* q_sf, const uint8_t* k,
                                  const uint8_t* k_sf, const uint8_t* vt, const uint8_t* vt_sf,
                                  const void* q_bf16, const void* k_bf16, const void* v_bf16,
@@ -257,8 +259,7 @@ fa4q_status fa4q_attn_fwd_hybrid(const uint8_t* q, const uint8_t* q_sf, const ui
                                  const void* vl_v, int max_vl, const uint64_t* vl_excl, float g_q,
                                  float g_k, float g_v, int B, int Hq, int Hkv, int S, int d,
                                  int window, fa4q_format fmt, float qmax_p, float sm_scale,
-                                 void* out, int out_is_fp32, float* lse, void* workspace,
-                                 size_t workspace_bytes, void* stream);
+                                 void* out, int out_is_fp32, float* lse, void* stream);
 
 /*
  * Paged FP4 KV cache (BitDecoding-FP4, "System-Level Optimization": fixed-size token

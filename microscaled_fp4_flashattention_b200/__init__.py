@@ -25,7 +25,7 @@ STATUS = {0: "FA4Q_OK", 1: "FA4Q_ERR_INVALID_ARG", 2: "FA4Q_ERR_UNSUPPORTED", 3:
 EXPORTED = [
     "fa4q_status_string", "fa4q_version", "fa4q_sf_tiled_bytes", "fa4q_quantize",
     "fa4q_smooth_calibrate", "fa4q_attn_fwd", "fa4q_attn_fwd_ex", "fa4q_quantize_kv_pages",
-    "fa4q_quantize_rotated", "fa4q_attn_fwd_hybrid", "fa4q_attn_fwd_hybrid_workspace_size",
+    "fa4q_quantize_rotated", "fa4q_attn_fwd_hybrid",
     "fa4q_decode_fp4q", "fa4q_decode_fp4q_workspace_size",
     "fa4q_decode_workspace_size", "fa4q_decode", "fa4q_decode_noalloc", "fa4q_selftest_block_mma",
     "fa4q_device_status", "fa4q_selftest_wait_timeout", "fa4q_selftest_exp2",
@@ -58,11 +58,9 @@ def lib() -> ctypes.CDLL:
         L.fa4q_sf_tiled_bytes.argtypes = [I64, I64, I]
         L.fa4q_quantize.restype = I
         L.fa4q_quantize.argtypes = [P, I64, I64, I64, I64, I, I, F, F, P, I64, I64, I, P, P, P]
-        L.fa4q_attn_fwd_hybrid_workspace_size.restype = Z
-        L.fa4q_attn_fwd_hybrid_workspace_size.argtypes = [I, I, I, I]
         L.fa4q_attn_fwd_hybrid.restype = I
         L.fa4q_attn_fwd_hybrid.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, I, P, F, F, F, I, I, I, I, I,
-                                           I, I, F, F, P, I, P, P, Z, P]
+                                           I, I, F, F, P, I, P, P]
         L.fa4q_decode_fp4q_workspace_size.restype = Z
         L.fa4q_decode_fp4q_workspace_size.argtypes = [I, I, I, I, I, I]
         L.fa4q_decode_fp4q.restype = I
@@ -196,22 +194,19 @@ def quantize_rotated(x, fmt, qmax: float = 0.0, tensor_scale: float = 1.0, smoot
 
 def attn_fwd_hybrid(q, q_sf, k, k_sf, vt, vt_sf, q_bf16, k_bf16, v_bf16, vl_pos, vl_count, vl_k, vl_v,
                     vl_excl, *, B, Hq, Hkv, S, d, window, fmt, g_q=1.0, g_k=1.0, g_v=1.0, qmax_p=0.0,
-                    sm_scale=0.0, out=None, out_fp32=False, lse=None, workspace=None, stream=None):
+                    sm_scale=0.0, out=None, out_fp32=False, lse=None, stream=None):
     """Hybrid-precision causal prefill (fa4q_attn_fwd_hybrid); vl_* may be None (no vertical
     lines).  Returns out [B, Hq, S, d]."""
     import torch
     if out is None:
         out = torch.empty((B, Hq, S, d), dtype=torch.float32 if out_fp32 else torch.bfloat16,
                           device=q.device)
-    need = int(lib().fa4q_attn_fwd_hybrid_workspace_size(B, Hq, S, d))
-    if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     max_vl = 0 if vl_pos is None else int(vl_pos.shape[-1])
     _check("fa4q_attn_fwd_hybrid", lib().fa4q_attn_fwd_hybrid(
         _ptr(q), _ptr(q_sf), _ptr(k), _ptr(k_sf), _ptr(vt), _ptr(vt_sf), _ptr(q_bf16), _ptr(k_bf16),
         _ptr(v_bf16), _ptr(vl_pos), _ptr(vl_count), _ptr(vl_k), _ptr(vl_v), max_vl, _ptr(vl_excl), g_q, g_k,
         g_v, B, Hq, Hkv, S, d, window, _fmt(fmt), qmax_p, sm_scale, _ptr(out), int(out_fp32), _ptr(lse),
-        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+        _stream(stream)))
     return out
 
 

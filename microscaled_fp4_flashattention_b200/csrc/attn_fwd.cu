@@ -35,6 +35,8 @@
 // skips the remaining waits, drains its own copies and MMAs and exits.
 #include <math.h>
 
+#include <cstring>
+
 #include "fa4q_common.cuh"
 #include "fa4q_internal.h"
 
@@ -81,24 +83,45 @@ struct Cfg {
   static constexpr int kQKSbo = D == 128 ? 512 : 256;
 };
 
-template <int D, bool MX>
+// Full-precision tiles of the hybrid prefill (HYB): bf16 Q, K, V as 64-column (128-byte)
+// chunks with the 128-byte swizzle, 64 keys per tile.
+constexpr int kHyKeys = 64;       // keys per full-precision tile
+constexpr int kHyStages = 2;      // K/V stages of the full-precision tiles
+template <bool HYB>
+struct HybSmem {
+  uint8_t unused;
+};
+template <>
+struct __align__(1024) HybSmem<true> {
+  uint8_t q[2][128 * 128];          // bf16 Q of the work item: two chunks of 128 rows x 128 B
+  uint8_t kv[kHyStages][4][kHyKeys * 128];   // K chunk 0, K chunk 1, V chunk 0, V chunk 1
+  uint8_t ones[16 * kHyKeys * 2];   // B operand of the normaliser: 16 rows of g_v (bf16)
+  uint64_t bar_q, q_free;
+  // K and V of a stage have their own barriers: the K slot frees as soon as its S product
+  // completes, so S can run two tiles ahead of PV with two stages
+  uint64_t kfull[kHyStages], kempty[kHyStages], vfull[kHyStages], vempty[kHyStages];
+};
+
+template <int D, bool MX, bool HYB = false>
 struct __align__(1024) Smem {
   using C = Cfg<D, MX>;
+  static constexpr int kNst = HYB ? 3 : kStages;   // FP4 K/V stages (the hybrid's BF16 tiles take room)
   uint8_t q[2][C::kQBytes];                 // double-buffered by work item
-  uint8_t k[kStages][C::kKBytes];
-  uint8_t v[kStages][C::kVBytes];
-  uint8_t p[2][C::kPBytes];
+  uint8_t k[kNst][C::kKBytes];
+  uint8_t v[kNst][C::kVBytes];
+  uint8_t p[2][HYB ? 128 * kHyKeys * 2 : C::kPBytes];   // P^ per group (hybrid: bf16 P as well)
   uint8_t ones[1024];
   uint8_t sfq[2][2 * 512];
-  uint8_t sfk[kStages][2 * 512];
-  uint8_t sfv[kStages][2 * 512];
+  uint8_t sfk[kNst][2 * 512];
+  uint8_t sfv[kNst][2 * 512];
   uint8_t sfp[2][2 * 512];
   uint8_t sfone[2 * 512];
+  HybSmem<HYB> hy;
   uint64_t bar_q[2];         // Q tile (and its scales) of work item k landed, slot k % 2
   uint64_t q_free[2];        // all S products of work item k issued and complete
   uint64_t o_free;           // all eight softmax warps have read O and l in the epilogue
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t kv_full[kNst];
+  uint64_t kv_empty[kNst];
   uint64_t s_full[2];        // S of an even / odd key tile ready (one per softmax group)
   uint64_t s_free;
   uint64_t p_full[2];
@@ -141,14 +164,21 @@ struct AttnParams {
   // feeds the PV product; the numerator is unchanged, so each output row is scaled by
   // sum P_hat / sum P~.
   int l_from_ptilde;
-  // Hybrid-precision prefill (HyQuant): per row the full-precision part of the softmax,
-  // [m0 (log2 units), l0, o0[D]] in FP32, has already been computed over the window and
-  // vertical-line keys; this kernel starts from it and masks those keys out of its FP4
-  // tiles (window: key > row - hy_window; vertical lines: bit set in hy_excl).
-  const float* hy_part;      // [B][Hq][S_q][D + 4]: m0, l0, -, -, o0[D]
+  // Hybrid-precision prefill (HyQuant): each work item first takes its full-precision keys
+  // in BF16 tiles of 64 - the window band {j : i - W < j <= i}, then the vertical lines
+  // {v : v <= i - W} from their gathered rows - and then its FP4 tiles with those keys
+  // masked out (window: key > row - W; vertical lines: bit set in hy_excl), all under one
+  // online softmax.
   const uint64_t* hy_excl;   // [B][Hkv][hy_excl_words]
+  const int32_t* hy_vl_pos;  // [B][Hkv][hy_max_vl] ascending positions of the vertical lines
+  const int32_t* hy_vl_count;  // [B][Hkv]
   int hy_window;
   int hy_excl_words;
+  int hy_max_vl;
+  float hy_inv_gqgk;         // BF16 scores -> the FP4 products' units (1 / (g_q g_k))
+  float hy_lp16;             // log2 of the units of P in the FP4 PV products, times g_v (NVFP4:
+                             // g_P g_v; MXFP4: 1) - a BF16 tile's P is 2^(s sc - m sc - hy_lp16)
+  uint32_t hy_ones_bits;     // bf16 bits of g_v (exact): the full-precision normaliser's operand
   int causal;
   int out_fp32;
 };
@@ -205,6 +235,13 @@ FA4Q_DEVINL float lg2_approx(float x) {
   float y;
   asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// (lo, hi) -> bf16x2 (round to nearest even), lo in the low half
+FA4Q_DEVINL uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
 }
 
 FA4Q_DEVINL float fmax3(float a, float b, float c) {
@@ -326,14 +363,20 @@ FA4Q_DEVINL void mma_step(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, int N
 
 // ABL: the ablations of fa4q_attn_fwd_ex (conditional rescaling, normaliser from P~) are
 // compiled into separate instantiations so the default kernel carries none of their work.
-// HYB: the FP4 part of the hybrid-precision prefill (causal only).
+// HYB: the hybrid-precision prefill (causal only, D = 128): full-precision tiles first, then
+// the FP4 tiles; tm_q16 .. tm_vlv are its bf16 operands (unused by the other instantiations).
 template <int D, bool MX, bool CAUSAL, bool PERSIST, bool ABL, bool HYB = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q16,
+                    const __grid_constant__ CUtensorMap tm_k16, const __grid_constant__ CUtensorMap tm_v16,
+                    const __grid_constant__ CUtensorMap tm_vlk, const __grid_constant__ CUtensorMap tm_vlv,
+                    const AttnParams p) {
   using C = Cfg<D, MX>;
+  using SM = Smem<D, MX, HYB>;
+  constexpr int NST = SM::kNst;
   extern __shared__ uint8_t smem_raw[];
-  Smem<D, MX>& sm = *reinterpret_cast<Smem<D, MX>*>(
+  SM& sm = *reinterpret_cast<SM*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   volatile uint32_t* abort_flag = &sm.abort_flag;
 
@@ -344,8 +387,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   // K/V tiles stay in L2.  CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... (G CTAs): a snake
   // over the longest-first list that evens out the work.  Every role walks the same items,
   // so the barrier phases below follow from counters each role keeps itself.
+  // n_tiles counts every key tile of the item; the hybrid's are nw window tiles (64 keys,
+  // starting at key 64 w0), then nv vertical-line tiles (64 gathered rows each), then FP4.
   struct Item {
     int b, h, qt, n_tiles;
+    int nw, w0, nv;
   };
   const int n_ktiles_all = (p.S_k + kBN - 1) / kBN;
   auto item_index = [&](int k) -> int {
@@ -362,11 +408,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       it.b = rem / p.Hq;
       it.h = rem % p.Hq;
       it.n_tiles = min(it.qt + 1, n_ktiles_all);
+      it.nw = it.w0 = it.nv = 0;
       if constexpr (HYB) {
-        // the last FP4 key of the tile's last row is row - window; at least one (possibly
-        // fully masked) tile, so every item runs its epilogue
-        const int last = min(it.qt * kBM + kBM - 1, p.S_q - 1) - p.hy_window;
-        it.n_tiles = max(1, min(it.n_tiles, last >= 0 ? last / kBN + 1 : 0));
+        // rows [r0, r1] of the item: window keys (r0 - W, r1], vertical lines up to r1 - W,
+        // FP4 keys up to r1 - W (the window tiles always hold each row's own key)
+        const int r0 = it.qt * kBM, r1 = min(r0 + kBM - 1, p.S_q - 1), last = r1 - p.hy_window;
+        it.w0 = max(0, r0 - p.hy_window + 1) / kHyKeys;
+        it.nw = r1 / kHyKeys - it.w0 + 1;
+        int nvis = 0;
+        if (p.hy_max_vl > 0 && last >= 0) {
+          const int bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
+          const int32_t* pos = p.hy_vl_pos + (int64_t)bh_k * p.hy_max_vl;
+          int lo = 0, hi = min(p.hy_vl_count[bh_k], p.hy_max_vl);     // first position > last
+          while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (pos[mid] <= last) lo = mid + 1;
+            else hi = mid;
+          }
+          nvis = lo;
+        }
+        it.nv = (nvis + kHyKeys - 1) / kHyKeys;
+        it.n_tiles = it.nw + it.nv + min(it.n_tiles, last >= 0 ? last / kBN + 1 : 0);
       }
     } else {
       const int per = p.Hq * p.n_qtiles, rem = u % per;
@@ -374,6 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       it.h = rem / p.n_qtiles;
       it.qt = rem % p.n_qtiles;
       it.n_tiles = n_ktiles_all;
+      it.nw = it.w0 = it.nv = 0;
     }
     return it;
   };
@@ -384,9 +447,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.bar_q[s], 1);
       mbar_init(&sm.q_free[s], 1);
     }
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&sm.kv_full[s], 1);
       mbar_init(&sm.kv_empty[s], 1);
+    }
+    if constexpr (HYB) {
+      mbar_init(&sm.hy.bar_q, 1);
+      mbar_init(&sm.hy.q_free, 1);
+      for (int s = 0; s < kHyStages; ++s) {
+        mbar_init(&sm.hy.kfull[s], 1);
+        mbar_init(&sm.hy.kempty[s], 1);
+        mbar_init(&sm.hy.vfull[s], 1);
+        mbar_init(&sm.hy.vempty[s], 1);
+      }
     }
     mbar_init(&sm.s_free, 4);
     for (int s = 0; s < 2; ++s) {
@@ -406,6 +479,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* s32 = reinterpret_cast<uint32_t*>(sm.sfone);
     const uint32_t one = MX ? 0x7F7F7F7Fu : 0x38383838u;
     for (int i = lane; i < 256; i += 32) s32[i] = one;
+    if constexpr (HYB) {
+      // B operand of the full-precision tiles' normaliser: 16 rows of g_v in bf16 (every
+      // element equal, so the swizzle is immaterial)
+      uint32_t* h32 = reinterpret_cast<uint32_t*>(sm.hy.ones);
+      for (int i = lane; i < 16 * kHyKeys / 2; i += 32) h32[i] = p.hy_ones_bits * 0x10001u;
+    }
     fence_proxy_async_smem();
   }
   if (warp == 1) {
@@ -425,9 +504,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      if constexpr (HYB) {
+        prefetch_tmap(&tm_q16);
+        prefetch_tmap(&tm_k16);
+        prefetch_tmap(&tm_v16);
+        prefetch_tmap(&tm_vlk);
+        prefetch_tmap(&tm_vlv);
+      }
       const int nrt_q = (p.S_q + 127) / 128, nrt_k = (p.S_k + 127) / 128;
       const int ng_v = ((p.S_kpad + 127) / 128) * C::kSfGroups;
-      int T = 0, q_issued = 0;                     // key tiles / Q tiles issued so far
+      int T = 0, q_issued = 0;                     // FP4 key tiles / Q tiles issued so far
+      int Tb = 0, Tbv = 0;                         // full-precision K / V tiles issued so far
+      int q16_issued = 0;                          // bf16 Q tiles issued so far
       bool go = true;
       for (int k = 0; go && (PERSIST || k < 1); ++k) {
         const int u = item_index(k);
@@ -435,6 +523,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Item it = decode_item(u);
         const int bh_q = it.b * p.Hq + it.h, bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
         const int qs = k & 1;
+        if constexpr (HYB) {
+          // bf16 Q: the slot was last read by the full-precision S products of item k-1
+          if (k >= 1 && !cta_wait(&sm.hy.q_free, (k - 1) & 1, abort_flag, kStatusTimeoutTmaFull)) break;
+          mbar_arrive_expect_tx(&sm.hy.bar_q, 2 * 128 * 128);
+          tma_load_3d(sm.hy.q[0], &tm_q16, 0, it.qt * kBM, bh_q, &sm.hy.bar_q);
+          tma_load_3d(sm.hy.q[1], &tm_q16, 128, it.qt * kBM, bh_q, &sm.hy.bar_q);
+          q16_issued = k + 1;
+        }
         // Q slot qs was last read by the S products of item k-2
         if (k >= 2 && !cta_wait(&sm.q_free[qs], ((k - 2) >> 1) & 1, abort_flag, kStatusTimeoutTmaFull)) break;
         mbar_arrive_expect_tx(&sm.bar_q[qs], C::kQBytes + C::kSfQAtoms * 512);
@@ -442,10 +538,40 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_load(sm.sfq[qs], p.q_sf + ((int64_t)bh_q * nrt_q + it.qt) * C::kSfGroups * 512,
                   C::kSfQAtoms * 512, &sm.bar_q[qs]);
         q_issued = k + 1;
-        for (int j = 0; j < it.n_tiles; ++j, ++T) {
-          const int s = T % kStages;
-          if (T >= kStages && !cta_wait(&sm.kv_empty[s], ((T / kStages) - 1) & 1, abort_flag,
-                                        kStatusTimeoutTmaFull)) {
+        if constexpr (HYB) {
+          // full-precision tiles: K and V rows of the window band, then the gathered
+          // vertical-line rows (past the sequence / the row count TMA fills zeros)
+          for (int i = 0; i < it.nw + it.nv; ++i, ++Tb) {
+            const int hs = Tb % kHyStages;
+            const uint32_t ph = ((Tb / kHyStages) - 1) & 1;
+            const bool win = i < it.nw;
+            const CUtensorMap* mk = win ? &tm_k16 : &tm_vlk;
+            const CUtensorMap* mv = win ? &tm_v16 : &tm_vlv;
+            const int y = win ? (it.w0 + i) * kHyKeys : (i - it.nw) * kHyKeys;
+            if (Tb >= kHyStages && !cta_wait(&sm.hy.kempty[hs], ph, abort_flag, kStatusTimeoutTmaFull)) {
+              go = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&sm.hy.kfull[hs], 2 * kHyKeys * 128);
+            tma_load_3d(sm.hy.kv[hs][0], mk, 0, y, bh_k, &sm.hy.kfull[hs]);
+            tma_load_3d(sm.hy.kv[hs][1], mk, 128, y, bh_k, &sm.hy.kfull[hs]);
+            if (Tb >= kHyStages && !cta_wait(&sm.hy.vempty[hs], ph, abort_flag, kStatusTimeoutTmaFull)) {
+              go = false;
+              ++Tb;                                // its K copy is in flight (drained below)
+              break;
+            }
+            mbar_arrive_expect_tx(&sm.hy.vfull[hs], 2 * kHyKeys * 128);
+            tma_load_3d(sm.hy.kv[hs][2], mv, 0, y, bh_k, &sm.hy.vfull[hs]);
+            tma_load_3d(sm.hy.kv[hs][3], mv, 128, y, bh_k, &sm.hy.vfull[hs]);
+            ++Tbv;
+          }
+          if (!go) break;
+        }
+        const int nf = it.n_tiles - it.nw - it.nv;
+        for (int j = 0; j < nf; ++j, ++T) {
+          const int s = T % NST;
+          if (T >= NST && !cta_wait(&sm.kv_empty[s], ((T / NST) - 1) & 1, abort_flag,
+                                    kStatusTimeoutTmaFull)) {
             go = false;
             break;
           }
@@ -460,10 +586,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // drain: every issued copy must have landed before the CTA may exit
-      for (int t = max(0, T - kStages); t < T; ++t)
-        mbar_wait(&sm.kv_full[t % kStages], (t / kStages) & 1, &g_attn_status, kStatusTimeoutDrain);
+      for (int t = max(0, T - NST); t < T; ++t)
+        mbar_wait(&sm.kv_full[t % NST], (t / NST) & 1, &g_attn_status, kStatusTimeoutDrain);
       for (int k = max(0, q_issued - 2); k < q_issued; ++k)
         mbar_wait(&sm.bar_q[k & 1], (k >> 1) & 1, &g_attn_status, kStatusTimeoutDrain);
+      if constexpr (HYB) {
+        for (int t = max(0, Tb - kHyStages); t < Tb; ++t)
+          mbar_wait(&sm.hy.kfull[t % kHyStages], (t / kHyStages) & 1, &g_attn_status, kStatusTimeoutDrain);
+        for (int t = max(0, Tbv - kHyStages); t < Tbv; ++t)
+          mbar_wait(&sm.hy.vfull[t % kHyStages], (t / kHyStages) & 1, &g_attn_status, kStatusTimeoutDrain);
+        if (q16_issued > 0) mbar_wait(&sm.hy.bar_q, (q16_issued - 1) & 1, &g_attn_status, kStatusTimeoutDrain);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -472,7 +605,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // shared-memory base has the base's descriptor plus o/16 (the start-address field;
       // shared memory is below 256 KB, so the field never carries), so issuing an MMA is a
       // few integer adds (this single thread's latency sits on the softmax groups' path).
-      using SM = Smem<D, MX>;
       const uint32_t base = smem_u32(&sm);
       const uint64_t d_qk = make_smem_desc(base, 16, C::kQKSbo, C::kQKSwizzle);   // Q and K tiles
       const uint64_t d_pv = make_smem_desc(base, 16, 512, kSwiz64);               // P, V^T, ones
@@ -483,7 +615,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint64_t osfv = offsetof(SM, sfv) >> 4, osfp = offsetof(SM, sfp) >> 4;
       constexpr uint64_t osfone = offsetof(SM, sfone) >> 4;
       constexpr uint64_t kQStride = C::kQBytes >> 4, kKStride = C::kKBytes >> 4, kVStride = C::kVBytes >> 4;
-      constexpr uint64_t kPStride = C::kPBytes >> 4, kSfStride = 1024 >> 4;
+      constexpr uint64_t kPStride = sizeof(sm.p[0]) >> 4, kSfStride = 1024 >> 4;
+      // full-precision tiles (hybrid): bf16 chunks of 128-byte rows, 128-byte swizzle
+      const uint64_t d_h = make_smem_desc(base, 16, 1024, kSwiz128);               // K-major (Q, K, P, ones)
+      const uint64_t d_hv = make_smem_desc(base, kHyKeys * 128, 1024, kSwiz128);   // V, MN-major
+      constexpr uint64_t ohq = HYB ? offsetof(SM, hy) >> 4 : 0;
+      constexpr uint64_t kHq = 128 * 128 >> 4, kHc = kHyKeys * 128 >> 4, kHst = 4 * kHc;
+      constexpr uint64_t ohkv = ohq + 2 * kHq, ohones = ohkv + kHyStages * kHst;
+      const uint32_t id_hs = make_idesc_bf16(kHyKeys, false), id_ho = make_idesc_bf16(D, true);
+      const uint32_t id_hl = make_idesc_bf16(16, false);
       // instruction descriptors (MXFP4: the 64-element step selects its scale byte pair)
       const uint32_t id_s[2] = {make_idesc_fp4(kBN, MX, 0, 0), make_idesc_fp4(kBN, MX, MX ? 2 : 0, MX ? 2 : 0)};
       const uint32_t id_o[2] = {make_idesc_fp4(D, MX, 0, 0), make_idesc_fp4(D, MX, MX ? 2 : 0, MX ? 2 : 0)};
@@ -497,23 +637,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int a = 0; a < C::kSfTileAtoms; ++a) tmem_cp_sf_desc(tmem + kColSfOne + 4 * a, d_sf + osfone + 32 * a);
       bool ok = true;
       int T = 0;                                   // key tiles of all earlier items
+      int T4 = 0, T4p = 0;                         // FP4 tiles whose S / PV products were issued
+      int Tb = 0, Tbp = 0;                         // full-precision tiles (hybrid), S / PV
       int n_pv0 = 0, n_pv1 = 0;                    // PV products issued per softmax group
       for (int k = 0; ok && (PERSIST || k < 1); ++k) {
         const int u = item_index(k);
         if (u < 0) break;
         const Item it = decode_item(u);
-        const int qs = k & 1, T0 = T, n_tiles = it.n_tiles;
+        const int qs = k & 1, T0 = T, n_tiles = it.n_tiles, nb = it.nw + it.nv;
         if (!mma_wait(&sm.bar_q[qs], (k >> 1) & 1, abort_flag)) break;
         tc_fence_after();
         // item k-2 used this scale slot; all of its products completed before item k-1 ended
         for (int a = 0; a < C::kSfQAtoms; ++a) tmem_cp_sf_desc(tmem + kColSfQ + 8 * qs + 4 * a, d_sf + osfq + qs * kSfStride + 32 * a);
         const uint64_t qd = d_qk + oq + qs * kQStride;
+        if constexpr (HYB) {
+          if (!mma_wait(&sm.hy.bar_q, k & 1, abort_flag)) break;
+        }
         // S_j = Q K_j^T into the single S buffer once the softmax group of the previous key
         // tile (of this item or the last) holds its scores in registers
         auto issue_s = [&](int j) -> bool {
-          const int t = T0 + j, s = t % kStages, kb = t & 1;
-          if (!mma_wait(&sm.kv_full[s], (t / kStages) & 1, abort_flag)) return false;
+          const int t = T0 + j;
           if (t >= 1 && !mma_wait(&sm.s_free, (t - 1) & 1, abort_flag)) return false;
+          if constexpr (HYB) {
+            if (j < nb) {
+              // full-precision tile: S = Q K^T on bf16 (M = 128, N = 64, K = 16 per MMA)
+              const int hs = Tb % kHyStages;
+              if (!mma_wait(&sm.hy.kfull[hs], (Tb / kHyStages) & 1, abort_flag)) return false;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16(tmem + kColS, d_h + ohq + (kk >> 2) * kHq + 2 * (kk & 3),
+                         d_h + ohkv + hs * kHst + (kk >> 2) * kHc + 2 * (kk & 3), id_hs, kk > 0);
+              tc_commit(&sm.s_full[j & 1]);
+              tc_commit(&sm.hy.kempty[hs]);
+              ++Tb;
+              if (j == nb - 1) tc_commit(&sm.hy.q_free);   // every product that read the bf16 Q
+              return true;
+            }
+          }
+          const int s = T4 % NST, kb = T4 & 1;
+          if (!mma_wait(&sm.kv_full[s], (T4 / NST) & 1, abort_flag)) return false;
           tc_fence_after();
           for (int a = 0; a < C::kSfQAtoms; ++a)
             tmem_cp_sf_desc(tmem + kColSfK + 8 * kb + 4 * a, d_sf + osfk + s * kSfStride + 32 * a);
@@ -523,27 +686,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma(tmem + kColS, qd + 2 * kk, kd + 2 * kk, id_s[kk & 1], tmem + kColSfQ + 8 * qs + sf_step(kk),
                 tmem + kColSfK + 8 * kb + sf_step(kk), kk > 0);
           tc_commit(&sm.s_full[j & 1]);
+          ++T4;
           return true;
         };
         // [O | l]_{j%2} (+)= P^_j [V_j | 1] once the softmax group has written P^_j; the first
         // product of an item waits until the previous item's epilogue has read O and l
         auto issue_pv = [&](int jp) -> bool {
-          const int t = T0 + jp, s = t % kStages, pb = jp & 1;
+          const int pb = jp & 1;
           if (jp == 0 && k >= 1 && !mma_wait(&sm.o_free, (k - 1) & 1, abort_flag)) return false;
           int& n_pv = pb ? n_pv1 : n_pv0;
           if (!mma_wait(&sm.p_full[pb], n_pv & 1, abort_flag)) return false;
           ++n_pv;
           tc_fence_after();
+          const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
+          if constexpr (HYB) {
+            if (jp < nb) {
+              // full-precision tile: [O | l] (+)= P [V | g_v] on bf16 (K = 16 keys per MMA; V is
+              // [keys][d], the MN-major B operand, in two 64-channel chunks)
+              const int hs = Tbp % kHyStages;
+              if (!mma_wait(&sm.hy.vfull[hs], (Tbp / kHyStages) & 1, abort_flag)) return false;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < kHyKeys / 16; ++kk) {
+                const uint32_t acc = (jp >= 2 || kk > 0) ? 1u : 0u;
+                const uint64_t pd = d_h + op + pb * kPStride + 2 * kk;
+                mma_bf16(tmem + o_col, pd, d_hv + ohkv + hs * kHst + 2 * kHc + kk * 128, id_ho, acc);
+                mma_bf16(tmem + l_col, pd, d_h + ohones + 2 * kk, id_hl, acc);
+              }
+              tc_commit(&sm.o_done[pb]);
+              tc_commit(&sm.hy.vempty[hs]);
+              ++Tbp;
+              return true;
+            }
+          }
+          const int s = T4p % NST;
           for (int a = 0; a < C::kSfTileAtoms; ++a) {
             tmem_cp_sf_desc(tmem + kColSfP + 8 * pb + 4 * a, d_sf + osfp + pb * kSfStride + 32 * a);
             tmem_cp_sf_desc(tmem + kColSfV + 8 * pb + 4 * a, d_sf + osfv + s * kSfStride + 32 * a);
           }
           const uint64_t pd = d_pv + op + pb * kPStride, vd = d_pv + ov + s * kVStride, od = d_pv + oones;
-          const uint32_t o_col = pb ? kColO1 : kColO0, l_col = pb ? kColL1 : kColL0;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
-            // (hybrid: group A's accumulator starts from the full-precision part)
-            const uint32_t acc = (jp >= 2 || kk > 0 || (HYB && jp == 0)) ? 1u : 0u;
+            const uint32_t acc = (jp >= 2 || kk > 0) ? 1u : 0u;
             mma(tmem + o_col, pd + 2 * kk, vd + 2 * kk, id_o[kk], tmem + kColSfP + 8 * pb + sf_step(kk),
                 tmem + kColSfV + 8 * pb + sf_step(kk), acc);
             mma(tmem + l_col, pd + 2 * kk, od + 2 * kk, id_l[kk], tmem + kColSfP + 8 * pb + sf_step(kk),
@@ -551,6 +735,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_commit(&sm.o_done[pb]);
           tc_commit(&sm.kv_empty[s]);
+          ++T4p;
           return true;
         };
         // Issue order S_0, S_1, PV_0, S_2, PV_1, ...: S runs two products ahead of PV, so the
@@ -605,9 +790,106 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_acc = -INFINITY;                       // maximum of this group's last tile
     float lpt = 0.0f;                              // sum of P~ of this group (ABL), MMA units
     const float gp_item = ABL ? p.gp : kGpNvfp4;
+    const int nb = it.nw + it.nv;                  // full-precision tiles (hybrid) come first
+    // bring accumulator g from the maximum it holds (tile j-2) to m_new (rows whose maximum
+    // did not move keep alpha = 1; -inf to -inf, a row without a visible key yet, too)
+    auto rescale_to = [&](int j, float m_new) {
+      if (j >= 2) {
+        tc_fence_after();
+        const float alpha = m_acc == m_new ? 1.0f : ex2_approx((m_acc - m_new) * sc);
+        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+          const uint32_t o_col = g ? kColO1 : kColO0, l_col = g ? kColL1 : kColL0;
+          uint32_t raw[D / 32][32];
+          uint32_t lr;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + o_col + 32 * c, raw[c]);
+          tmem_ld1(lane_base + l_col, lr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) fmul2_inplace(raw[c][i], raw[c][i + 1], alpha);
+            tmem_st32(lane_base + o_col + 32 * c, raw[c]);
+          }
+          tmem_st1(lane_base + l_col, __float_as_uint(__uint_as_float(lr) * alpha));
+          tmem_wait_st();
+        }
+      }
+      m_acc = m_new;
+    };
     for (int j = g; j < n_tiles; j += 2) {
       ok = warp_wait(&sm.s_full[g], (done_g + (j >> 1)) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
       tc_fence_after();
+      if constexpr (HYB) {
+        if (j < nb) {
+          // ---- full-precision tile (64 keys): scores, masks, maximum, unquantised P in bf16
+          float sh[kHyKeys];
+          {
+            uint32_t raw[2][32];
+            tmem_ld32(lane_base + kColS, raw[0]);
+            tmem_ld32(lane_base + kColS + 32, raw[1]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int i = 0; i < 32; ++i) sh[32 * c + i] = __uint_as_float(raw[c][i]) * p.hy_inv_gqgk;
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_free);
+          if (j < it.nw) {
+            // window band: row - W < key <= row, key < S_k
+            const int k0 = (it.w0 + j) * kHyKeys;
+#pragma unroll
+            for (int i = 0; i < kHyKeys; ++i) {
+              const int key = k0 + i;
+              if (!(key <= row && key > row - p.hy_window && key < p.S_k)) sh[i] = -INFINITY;
+            }
+          } else {
+            // gathered vertical lines: entry e (< the kv-head's count) at position <= row - W
+            const int e0 = (j - it.nw) * kHyKeys, bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
+            const int cnt = min(p.hy_vl_count[bh_k], p.hy_max_vl), lim = row - p.hy_window;
+            const int32_t* pos = p.hy_vl_pos + (int64_t)bh_k * p.hy_max_vl;
+#pragma unroll
+            for (int i = 0; i < kHyKeys; ++i) {
+              const int e = e0 + i;
+              if (!(e < cnt && pos[min(e, cnt - 1)] <= lim)) sh[i] = -INFINITY;
+            }
+          }
+          const float tmax = block_max<kHyKeys>(sh);
+          float m_prev = -INFINITY;
+          if (j > 0) {
+            named_bar_sync(bar_recv, 64);
+            m_prev = sm.m_xchg[(j - 1) & 1][r];
+          }
+          const float m_new = fmaxf(m_prev, tmax);
+          sm.m_xchg[j & 1][r] = m_new;
+          named_bar_arrive(bar_send, 64);
+          // P = 2^(s sc - m sc - lp16): the FP4 PV products' units, divided by g_v (the
+          // normaliser's B operand holds g_v); a row with no visible key yet gets P = 0
+          const float off = m_new > -INFINITY ? m_new * sc + p.hy_lp16 : 0.0f;
+          uint32_t pk[kHyKeys / 2];
+#pragma unroll
+          for (int i = 0; i < kHyKeys / 2; ++i) {
+            float y0, y1;
+            ffma2(y0, y1, sh[2 * i], sh[2 * i + 1], sc, sc, -off, -off);
+            pk[i] = pack_bf16x2(ex2_approx(y0), ex2_approx(y1));
+          }
+          // P buffer g was last read by this group's previous PV product
+          if (j >= 2)
+            ok = warp_wait(&sm.o_done[g], (done_g + (j >> 1) - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
+#pragma unroll
+          for (int c = 0; c < kHyKeys / 8; ++c)
+            *reinterpret_cast<uint4*>(sm.p[g] + swz128_offset(r, c)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          fence_proxy_async_smem();
+          rescale_to(j, m_new);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full[g]);
+          continue;
+        }
+      }
       float s[kBN];
       {
         uint32_t raw[kBN / 32][32];
@@ -623,7 +905,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.s_free);
       // masking: keys beyond S_k, and (causal) keys after this query
-      const int key0 = j * kBN;
+      const int key0 = (HYB ? j - nb : j) * kBN;
       if constexpr (HYB) {
         // FP4 keys of row i: key <= i - window and not a vertical line
         const int lim = min(p.S_k - key0, row - p.hy_window - key0 + 1);
@@ -663,11 +945,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int bi = 1; bi < kNB; ++bi) tmax = fmaxf(tmax, bmax[bi]);
       // running maximum: take m_{j-1} from the other group, publish m_j
       float m_prev = -INFINITY;
-      float hy_m0 = -INFINITY;                     // full-precision part, raw score units
-      if constexpr (HYB) {
-        if (j == 0 && row < p.S_q) hy_m0 = p.hy_part[((int64_t)bh_q * p.S_q + row) * (D + 4)] / sc;
-        if (j == 0) m_prev = hy_m0;
-      }
       if (j > 0) {
         named_bar_sync(bar_recv, 64);
         m_prev = sm.m_xchg[(j - 1) & 1][r];
@@ -782,54 +1059,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         lpt = (j >= 2 ? lpt * ex2_approx((m_acc - m_new) * sc) : 0.0f) + add;
       }
-      if (HYB && j == 0) {
-        // group A's accumulator := the full-precision part, brought from m0 to m_new
-        // (O in MMA units: the PV products carry neither g_P nor g_v)
-        if (PERSIST && k >= 1)
-          ok = warp_wait(&sm.o_free, (k - 1) & 1, abort_flag, kStatusTimeoutSoftmax) && ok;
-        tc_fence_after();
-        const float* src = p.hy_part + ((int64_t)bh_q * p.S_q + min(row, p.S_q - 1)) * (D + 4);
-        const float a0 = row < p.S_q ? ex2_approx((hy_m0 - m_new) * sc) : 0.0f;
-        const float gpl = MX ? 1.0f : kGpNvfp4;
-        const float so = a0 / (gpl * p.g_v), sl = a0 / gpl;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t raw[32];
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const float4 v4 = *reinterpret_cast<const float4*>(src + 4 + 32 * c + i);
-            raw[i] = __float_as_uint(v4.x * so);
-            raw[i + 1] = __float_as_uint(v4.y * so);
-            raw[i + 2] = __float_as_uint(v4.z * so);
-            raw[i + 3] = __float_as_uint(v4.w * so);
-          }
-          tmem_st32(lane_base + kColO0 + 32 * c, raw);
-        }
-        tmem_st1(lane_base + kColL0, __float_as_uint(src[1] * sl));
-        tmem_wait_st();
-      }
-      if (j >= 2) {
-        tc_fence_after();
-        const float alpha = ex2_approx((m_acc - m_new) * sc);
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-          const uint32_t o_col = g ? kColO1 : kColO0, l_col = g ? kColL1 : kColL0;
-          uint32_t raw[D / 32][32];
-          uint32_t lr;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) tmem_ld32(lane_base + o_col + 32 * c, raw[c]);
-          tmem_ld1(lane_base + l_col, lr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) fmul2_inplace(raw[c][i], raw[c][i + 1], alpha);
-            tmem_st32(lane_base + o_col + 32 * c, raw[c]);
-          }
-          tmem_st1(lane_base + l_col, __float_as_uint(__uint_as_float(lr) * alpha));
-          tmem_wait_st();
-        }
-      }
-      m_acc = m_new;
+      rescale_to(j, m_new);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.p_full[g]);
@@ -1047,9 +1277,16 @@ static void fill_p_scale_rule(AttnParams& prm) {
   prm.log2_qmax_p = prm.qmax_p > 0.0f ? static_cast<float>(std::log2(static_cast<double>(prm.qmax_p))) : 0.0f;
 }
 
+// bf16 operands of the hybrid prefill's full-precision tiles (rows of d = 128 bf16 = 256 bytes,
+// loaded as two 128-byte chunks with the 128-byte swizzle)
+struct HyOperands {
+  const void *q, *k, *v, *vl_k, *vl_v;
+  int max_vl;
+};
+
 template <int D, bool MX, bool CAUSAL, bool ABL = false, bool HYB = false>
 static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t* vt,
-                               const AttnParams& prm, cudaStream_t st) {
+                               const AttnParams& prm, cudaStream_t st, const HyOperands* hy = nullptr) {
   CUtensorMap tq, tk, tv;
   const CUtensorMapSwizzle qk_swz = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   if (!make_map_3d(&tq, q, D / 2, prm.S_q, (uint64_t)prm.B * prm.Hq, D / 2, kBM, qk_swz) ||
@@ -1057,7 +1294,19 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
       !make_map_3d(&tv, vt, prm.S_kpad / 2, D, (uint64_t)prm.B * prm.Hkv, kBN / 2, D,
                    CU_TENSOR_MAP_SWIZZLE_64B))
     return FA4Q_ERR_CUDA;
-  const size_t smem = sizeof(Smem<D, MX>) + 1024;
+  CUtensorMap tq16 = tq, tk16 = tq, tv16 = tq, tvlk = tq, tvlv = tq;   // unused unless hybrid
+  if (HYB) {
+    const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    const uint64_t nq = (uint64_t)prm.B * prm.Hq, nk = (uint64_t)prm.B * prm.Hkv;
+    if (!hy || !make_map_3d(&tq16, hy->q, 2 * D, prm.S_q, nq, 128, kBM, sw) ||
+        !make_map_3d(&tk16, hy->k, 2 * D, prm.S_k, nk, 128, kHyKeys, sw) ||
+        !make_map_3d(&tv16, hy->v, 2 * D, prm.S_k, nk, 128, kHyKeys, sw))
+      return FA4Q_ERR_CUDA;
+    if (hy->max_vl > 0 && (!make_map_3d(&tvlk, hy->vl_k, 2 * D, hy->max_vl, nk, 128, kHyKeys, sw) ||
+                           !make_map_3d(&tvlv, hy->vl_v, 2 * D, hy->max_vl, nk, 128, kHyKeys, sw)))
+      return FA4Q_ERR_CUDA;
+  }
+  const size_t smem = sizeof(Smem<D, MX, HYB>) + 1024;
   // Short items (few key tiles on average, as in causal attention over a few thousand keys)
   // run persistently, one CTA per SM walking the item list, so the per-CTA setup and the
   // pipeline fill and drain of an item overlap the neighbouring items.  Long items run one
@@ -1070,7 +1319,7 @@ static fa4q_status launch_attn(const uint8_t* q, const uint8_t* k, const uint8_t
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return FA4Q_ERR_CUDA;
   const dim3 grid(static_cast<unsigned>(persist ? num_sms() : prm.n_items));
-  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, prm);
+  kern<<<grid, kThreads, smem, st>>>(tq, tk, tv, tq16, tk16, tv16, tvlk, tvlv, prm);
   return launch_status();
 }
 
@@ -1189,22 +1438,17 @@ extern "C" fa4q_status fa4q_selftest_wait_timeout(uint32_t wait_us, void* stream
 }
 
 // =======================================================================================
-// hybrid-precision prefill: the full-precision part (hybrid.cu), then the FP4 part here
+// hybrid-precision prefill: one kernel, the full-precision tiles first, then the FP4 tiles
 // =======================================================================================
-extern "C" size_t fa4q_attn_fwd_hybrid_workspace_size(int B, int Hq, int S, int d) {
-  if (B <= 0 || Hq <= 0 || S <= 0 || d <= 0) return 0;
-  return (size_t)B * Hq * S * (d + 4) * sizeof(float);
-}
-
 extern "C" fa4q_status fa4q_attn_fwd_hybrid(
     const uint8_t* q, const uint8_t* q_sf, const uint8_t* k, const uint8_t* k_sf, const uint8_t* vt,
     const uint8_t* vt_sf, const void* q_bf16, const void* k_bf16, const void* v_bf16,
     const int32_t* vl_pos, const int32_t* vl_count, const void* vl_k, const void* vl_v, int max_vl,
     const uint64_t* vl_excl, float g_q, float g_k, float g_v, int B, int Hq, int Hkv, int S, int d,
     int window, fa4q_format fmt, float qmax_p, float sm_scale, void* out, int out_is_fp32, float* lse,
-    void* workspace, size_t workspace_bytes, void* stream) {
+    void* stream) {
   if (fmt != FA4Q_NVFP4 && fmt != FA4Q_MXFP4) return FA4Q_ERR_INVALID_ARG;
-  if (!q || !q_sf || !k || !k_sf || !vt || !vt_sf || !q_bf16 || !k_bf16 || !v_bf16 || !out || !workspace)
+  if (!q || !q_sf || !k || !k_sf || !vt || !vt_sf || !q_bf16 || !k_bf16 || !v_bf16 || !out)
     return FA4Q_ERR_INVALID_ARG;
   if (B < 0 || Hq <= 0 || Hkv <= 0 || S < 0 || Hq % Hkv != 0 || window < 1 || max_vl < 0)
     return FA4Q_ERR_INVALID_ARG;
@@ -1213,36 +1457,19 @@ extern "C" fa4q_status fa4q_attn_fwd_hybrid(
   if (!(qmax_p >= 0.0f) || !isfinite(qmax_p)) return FA4Q_ERR_INVALID_ARG;
   if (fmt == FA4Q_MXFP4) { g_q = g_k = g_v = 1.0f; }
   if (!(g_q > 0.0f) || !(g_k > 0.0f) || !(g_v > 0.0f)) return FA4Q_ERR_INVALID_ARG;
+  // the full-precision normaliser multiplies by g_v in bf16: g_v must be a bf16 value
+  uint32_t gv_bits;
+  std::memcpy(&gv_bits, &g_v, sizeof(gv_bits));
+  if ((gv_bits & 0xFFFFu) != 0u) return FA4Q_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(vt) || !aligned16(q_sf) || !aligned16(k_sf) ||
       !aligned16(vt_sf) || !aligned16(out) || !aligned16(q_bf16) || !aligned16(k_bf16) ||
-      !aligned16(v_bf16) || !aligned16(workspace) || (vl_k && !aligned16(vl_k)) || (vl_v && !aligned16(vl_v)))
+      !aligned16(v_bf16) || (vl_k && !aligned16(vl_k)) || (vl_v && !aligned16(vl_v)))
     return FA4Q_ERR_INVALID_ARG;
   if (B == 0 || S == 0) return FA4Q_OK;
-  if (workspace_bytes < fa4q_attn_fwd_hybrid_workspace_size(B, Hq, S, d)) return FA4Q_ERR_INVALID_ARG;
   const int n_qtiles = (S + kBM - 1) / kBM;
   if (static_cast<int64_t>(B) * Hq * n_qtiles > 0x7fffffff || B > 65535 || Hq > 65535) return FA4Q_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const float sms = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf((float)d);
-  // 1. full-precision part: window and vertical-line keys, bf16, unquantised P
-  HyParams hp;
-  hp.q = static_cast<const uint16_t*>(q_bf16);
-  hp.k = static_cast<const uint16_t*>(k_bf16);
-  hp.v = static_cast<const uint16_t*>(v_bf16);
-  hp.vl_pos = max_vl > 0 ? vl_pos : nullptr;
-  hp.vl_count = max_vl > 0 ? vl_count : nullptr;
-  hp.vl_k = static_cast<const uint16_t*>(vl_k);
-  hp.vl_v = static_cast<const uint16_t*>(vl_v);
-  hp.part = static_cast<float*>(workspace);
-  hp.B = B;
-  hp.Hq = Hq;
-  hp.Hkv = Hkv;
-  hp.S = S;
-  hp.W = window;
-  hp.max_vl = max_vl;
-  hp.c2 = sms * kLog2e;
-  fa4q_status stt = launch_hybrid_full(hp, st);
-  if (stt != FA4Q_OK) return stt;
-  // 2. FP4 part, continuing each row's softmax from the full-precision state
   AttnParams prm{};
   prm.q_sf = q_sf;
   prm.k_sf = k_sf;
@@ -1265,10 +1492,17 @@ extern "C" fa4q_status fa4q_attn_fwd_hybrid(
   prm.gp = kGpNvfp4;
   prm.inv6gp = kInvSixGp;
   fill_p_scale_rule(prm);
-  prm.hy_part = static_cast<const float*>(workspace);
   prm.hy_window = window;
   prm.hy_excl_words = max_vl > 0 ? (S + 63) / 64 : 0;
   prm.hy_excl = max_vl > 0 ? vl_excl : nullptr;     // read only while a word index is < hy_excl_words
-  if (fmt == FA4Q_MXFP4) return launch_attn<128, true, true, false, true>(q, k, vt, prm, st);
-  return launch_attn<128, false, true, false, true>(q, k, vt, prm, st);
+  prm.hy_vl_pos = max_vl > 0 ? vl_pos : nullptr;
+  prm.hy_vl_count = max_vl > 0 ? vl_count : nullptr;
+  prm.hy_max_vl = max_vl;
+  prm.hy_inv_gqgk = 1.0f / (g_q * g_k);
+  const double units = fmt == FA4Q_MXFP4 ? 1.0 : static_cast<double>(kGpNvfp4) * g_v;
+  prm.hy_lp16 = static_cast<float>(std::log2(units));
+  prm.hy_ones_bits = gv_bits >> 16;
+  const HyOperands hy{q_bf16, k_bf16, v_bf16, vl_k, vl_v, max_vl};
+  if (fmt == FA4Q_MXFP4) return launch_attn<128, true, true, false, true>(q, k, vt, prm, st, &hy);
+  return launch_attn<128, false, true, false, true>(q, k, vt, prm, st, &hy);
 }

@@ -64,26 +64,10 @@ inline int num_sms() {
   return cached[dev];
 }
 
-// Full-precision part of the hybrid-precision prefill (hybrid.cu): per query row, the online
-// softmax state [m0 (log2 units), l0, -, -, o0[d]] (row stride d + 4) over the window and
-// vertical-line keys.
-struct HyParams {
-  const uint16_t* q;        // [B][Hq][S][d] bf16
-  const uint16_t* k;        // [B][Hkv][S][d] bf16
-  const uint16_t* v;        // [B][Hkv][S][d] bf16
-  const int32_t* vl_pos;    // [B][Hkv][max_vl] ascending positions (nullable: none)
-  const int32_t* vl_count;  // [B][Hkv]
-  const uint16_t* vl_k;     // [B][Hkv][max_vl][d] bf16 rows of the vertical lines
-  const uint16_t* vl_v;
-  float* part;              // [B][Hq][S][d + 4]
-  int B, Hq, Hkv, S, W, max_vl;
-  float c2;                 // sm_scale * log2(e)
-};
-fa4q_status launch_hybrid_full(const HyParams& p, cudaStream_t st);
-
 // Dual-residual NVFP4 query tiles of the FP4 tensor-core decode (quantize.cu): q bf16
-// [B][Hq][128] -> qt [B*Hkv][2][128][64] packed, qt_sf [B*Hkv][2][2][512] tiled atoms
-// (row r holds q-head r % 32 of the group, zero when r % 32 >= G).
+// [B][Hq][128] -> qt [B*Hkv][2][128][64] packed, qt_sf [B*Hkv][2][2][512] tiled atoms; rows
+// 0..G-1 hold the group's q-heads and rows G..15 are zero (rows 16..127, which the decode does
+// not read, are not written).
 fa4q_status launch_dec_query(const uint16_t* q, int B, int Hq, int Hkv, uint8_t* qt, uint8_t* qt_sf,
                              cudaStream_t st);
 // log-sum-exp merge of decode split partials [rows][splits][d + 2] (m in log2 units, l, o)

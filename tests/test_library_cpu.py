@@ -138,21 +138,18 @@ def test_more_entry_points_reject_bad_arguments_without_gpu(L):
     vertical-line selection: each error below is caught before any device call."""
     P_, F, D = ctypes.c_void_p, ctypes.c_float, ctypes.c_double
     fake = P_(0x1000)
-    # hybrid prefill: workspace rule, bad format, window, head dim, missing vertical-line
-    # arrays, short workspace; an empty batch is a no-op
-    assert L.fa4q_attn_fwd_hybrid_workspace_size(1, 4, 128, 128) == 1 * 4 * 128 * (128 + 4) * 4
-    assert L.fa4q_attn_fwd_hybrid_workspace_size(0, 4, 128, 128) == 0
-    ws = L.fa4q_attn_fwd_hybrid_workspace_size(1, 4, 128, 128)
-
-    def hyb(fmt=0, window=16, d=128, max_vl=0, vl=fake, B=1, ws_bytes=ws):
-        return L.fa4q_attn_fwd_hybrid(*([fake] * 9), vl, vl, vl, vl, max_vl, vl, F(1), F(1), F(1), B, 4, 1, 128,
-                                      d, window, fmt, F(0), F(0), fake, 1, None, fake, ws_bytes, None)
+    # hybrid prefill: bad format, window, head dim, missing vertical-line arrays, an NVFP4
+    # V tensor scale that is not a bf16 value; an empty batch is a no-op
+    def hyb(fmt=0, window=16, d=128, max_vl=0, vl=fake, B=1, g_v=1.0):
+        return L.fa4q_attn_fwd_hybrid(*([fake] * 9), vl, vl, vl, vl, max_vl, vl, F(1), F(1), F(g_v), B, 4, 1, 128,
+                                      d, window, fmt, F(0), F(0), fake, 1, None, None)
     assert hyb(fmt=3) == 1
     assert hyb(window=0) == 1
     assert hyb(d=64) == 2
     assert hyb(max_vl=8, vl=None) == 1
-    assert hyb(ws_bytes=ws - 1) == 1
-    assert hyb(B=0) == 0
+    assert hyb(g_v=1.1) == 2                 # 1.1 is not a bf16 value
+    assert hyb(B=0, g_v=0.5) == 0
+    assert hyb(B=0, fmt=1, g_v=1.1) == 0     # MXFP4 carries no tensor scale
     # fused Q/K/V quantisation: head dim, null input, GQA mismatch
     qkv = lambda q=fake, Hq=4, d=128: L.fa4q_quantize_qkv(q, fake, fake, 1, Hq, 2, 128, 128, d, 0, F(0), F(1),
                                                           F(1), F(1), None, None, *([fake] * 6), None)
