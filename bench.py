@@ -47,21 +47,23 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture
 # of each roofline kernel (summaries and commands in profiles/).  A figure is reported only
 # while the kernel's sources hash to the ones it was taken on; any change makes it null.
-# The decode capture ran 8 of the 32 sequences: its traffic is per sequence (it grows with the
-# number of sequences) and is scaled to the timed batch.
+# Each capture ran a smaller batch of the same kernel (fewer heads, fewer sequences), so
+# that it stays small; the traffic is stored per unit (query head, sequence) and scaled to
+# the timed batch, the operand reads growing in proportion to the units.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_causal_gqa_mxfp4_s4096.md: 13,531,904 + 136,192 B (that workload only)
-    "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"), "workload": "causal_gqa_mxfp4_smooth_s4096",
-                 "sha256": "db57444a96ac2c0fc3d32578247edcc5c9d91eb1e8a86729799f1ec73df0e70f",
-                 "bytes_per_launch": 13531904 + 136192},
-    # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,936,576 + 5,338,368 B for 8 sequences
-    "decode": {"sources": ("decode.cu", "fa4q_common.cuh"),
-               "sha256": "30d1b993fd9dfb1d0f3e4d581d55f6a1d1ef7f27afa37ebdeb49f3c9b5fbb0c2",
-               "bytes_per_sequence": (358936576 + 5338368) // 8},
-    # profiles/decode_fp4q_paged_nvfp4_b32_l32k.md: 1,209,192,704 + 5,807,616 B (bench workload)
-    "decode_fp4q": {"sources": ("decode_tc.cu", "fa4q_common.cuh"),
-                    "sha256": "8ef392cbb9624318b89523367dcdf313789e897d7bbb9704f6acd340aadc562c",
-                    "bytes_per_launch": 1209192704 + 5807616},
+    # profiles/attn_fwd_noncausal_mxfp4_uos_s32768.md: 107,913,216 + 89,085,952 B for 16 of the
+    # 40 heads (the output write-back that stays in L2 at the end of the launch is not in it)
+    "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"), "workload": "noncausal_mxfp4_uos_h40_s32768",
+                 "sha256": "e61074644556cdc84fc4497f71b3015106c756dfd1f6d1c04e52995747f62f52",
+                 "bytes_per_unit": (107913216 + 89085952) / 16},
+    # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,902,272 + 8,193,536 B for 8 sequences
+    "decode": {"sources": ("decode.cu", "fa4q_common.cuh"), "workload": None,
+               "sha256": "ba940cd89265356d949f7a42e68a6b04591dda9da095edeabffefb29fc940c4f",
+               "bytes_per_unit": (358902272 + 8193536) / 8},
+    # profiles/decode_fp4q_paged_nvfp4_b8_l32k.md: 302,323,968 + 4,372,992 B for 8 sequences
+    "decode_fp4q": {"sources": ("decode_tc.cu", "fa4q_common.cuh"), "workload": None,
+                    "sha256": "67d20327f671a0249d5eeebd7395234a3a23deb9e11d7f9fc995909bfe115a1d",
+                    "bytes_per_unit": (302323968 + 4372992) / 8},
 }
 
 
@@ -97,13 +99,15 @@ def sources_sha256(names) -> str:
     return h.hexdigest()
 
 
-def ncu_traffic(kernel: str, sequences: int = 0, workload: str | None = None):
+def ncu_traffic(kernel: str, units: int, workload: str | None = None):
+    """DRAM bytes of one launch over `units` heads or sequences, or None when the kernel
+    changed since the capture or the capture was of another workload."""
     e = NCU_TRAFFIC[kernel]
     if e["sha256"] is None or sources_sha256(e["sources"]) != e["sha256"]:
         return None
-    if workload is not None and e.get("workload") not in (None, workload):
+    if e["workload"] is not None and workload != e["workload"]:
         return None
-    return e["bytes_per_launch"] if "bytes_per_launch" in e else e["bytes_per_sequence"] * sequences
+    return int(round(e["bytes_per_unit"] * units))
 
 
 # ------------------------------------------------------------------------------ helpers
@@ -440,7 +444,7 @@ def decode_fp4q_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
         "splits": splits, "tiles_per_split": tps,
         "roofline": {"kernel": "decode_tc_kernel+dec_query_kernel+decode_combine_kernel", "bound": "hbm",
                      "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
-                     "traffic": ncu_traffic("decode_fp4q") if not args.decode_batch else None,
+                     "traffic": ncu_traffic("decode_fp4q", dw.B),
                      "peak_source": f"{peak_kind} hbm copy"},
         "note": "dual-residual NVFP4 query and PNQ probabilities on the block-scaled tensor cores "
                 "(BitDecoding-FP4); seeded gaussian cache, not the hybrid cache of line['decode']",
@@ -547,9 +551,10 @@ def attn_roofline(w, flops, a_ms, fp4_peak, peak_src, world):
     exp_peak = 16.0 / (6.0 / 8.0) * 4 * w.d * 148 * sm_mhz * 1e6 / 1e12
     return {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
             "unit": "TFLOP/s", "frac": achieved / fp4_peak,
-            "traffic": ncu_traffic("attn_fwd", workload=w.name),
-            "traffic_note": "dram read + write of one launch; the bf16 output (B*Hq*S*d*2 B) can stay in L2 "
-                            "during a captured launch, so its write-back may fall outside the figure",
+            "traffic": ncu_traffic("attn_fwd", w.B * w.Hq, workload=w.name),
+            "traffic_note": "dram read + write per launch, scaled by heads from a 16-head ncu capture of the "
+                            "same kernel; the part of the bf16 output (B*Hq*S*d*2 B) still in L2 when the "
+                            "launch ends is written back later and falls outside the figure",
             "peak_source": peak_src, "ms_per_launch": a_ms, "launches_per_step": 1,
             "exp_ceiling": {"peak": exp_peak, "unit": "TFLOP/s", "frac": achieved / exp_peak,
                             "what": "MUFU ex2 at 16/clk/SM for 6 of 8 exponentials, 148 SMs at "
@@ -573,6 +578,9 @@ def main():
                     help="decode batch (0 = the workload's 32); smaller batches are for profiling")
     ap.add_argument("--fp4q-tiles-per-split", type=int, default=32,
                     help="range length of the FP4 tensor-core decode (part of its result)")
+    ap.add_argument("--prefill-heads", type=int, default=0,
+                    help="query heads of the prefill batch (0 = the workload's; the group ratio is kept); "
+                         "fewer heads are for profiling and never the headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--soak-s", type=float, default=2.0)
     args = ap.parse_args()
@@ -581,6 +589,13 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = synth.WORKLOADS[args.workload]
+    if args.prefill_heads > 0 and args.prefill_heads != w.Hq:
+        import dataclasses
+        g = w.Hq // w.Hkv
+        if args.prefill_heads % g:
+            ap.error(f"--prefill-heads must be a multiple of the group size {g}")
+        w = dataclasses.replace(w, name=f"{w.name}_heads{args.prefill_heads}", Hq=args.prefill_heads,
+                                Hkv=args.prefill_heads // g)
 
     if args.impl == "reference":
         if rank != 0:
