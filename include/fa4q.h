@@ -421,11 +421,13 @@ fa4q_status fa4q_decode_noalloc(const void* q, const uint8_t* k_pages, const uin
  *            fa4q_quantize_kv_pages and fa4q_decode.
  * hp_k, hp_v nullable out, bf16 [B][Hkv][max_select][d]: the kept rows of k and v in
  *            position order (the decode's full-precision set; rows past counts not written).
- * workspace  device, >= fa4q_vlines_workspace_size(B, Hq, Hkv, n_obs, L) bytes, 8-aligned.
+ * workspace  device, >= fa4q_vlines_workspace_size(B, Hq, Hkv, n_obs, L) bytes, 16-byte
+ *            aligned.
  * The candidates of one (sequence, kv-head) are selected in shared memory: L up to ~55,000
  * keys (4 L + 4 max_select + 8 max_pages bytes <= 227 KB), else FA4Q_ERR_UNSUPPORTED.
  * Errors: null required pointers, bad sizes, short workspace or misaligned (16-byte) bf16
- * pointers -> FA4Q_ERR_INVALID_ARG.  Asynchronous on `stream`.
+ * pointers or workspace -> FA4Q_ERR_INVALID_ARG.  A device wait that expires sets the
+ * status fa4q_device_status reports.  Asynchronous on `stream`.
  */
 size_t fa4q_vlines_workspace_size(int B, int Hq, int Hkv, int n_obs, int L);
 fa4q_status fa4q_select_vertical_lines(const void* q_obs, const void* k, const void* v,

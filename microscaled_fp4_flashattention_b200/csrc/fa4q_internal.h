@@ -80,5 +80,6 @@ cudaError_t attn_status_fetch(cudaStream_t st, uint32_t* host_word);
 cudaError_t decode_status_fetch(cudaStream_t st, uint32_t* host_word);
 cudaError_t dectc_status_fetch(cudaStream_t st, uint32_t* host_word);
 cudaError_t hy_status_fetch(cudaStream_t st, uint32_t* host_word);
+cudaError_t vl_status_fetch(cudaStream_t st, uint32_t* host_word);
 
 }  // namespace fa4q

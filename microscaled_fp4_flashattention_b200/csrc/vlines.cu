@@ -14,66 +14,58 @@
 // gathered from a set of observation queries.
 //
 // Kernels:
-//   colmass_kernel<0>  grid (key chunk, kv-head, sequence), 8 warps, 32 query rows each:
-//                      BF16 mma.sync m16n8k16 scores of the R rows against the chunk's keys
-//                      (K streamed through a two-stage cp.async ring), per row a running
-//                      maximum and sum of exp2 -> partials (m, l) per (row, chunk)
-//   lse_kernel         partials -> lse2[row] = m + log2(l)   (log2 domain)
-//   colmass_kernel<1>  the same scores again; mass_j = sum_i exp2(s2_ij - lse2_i), reduced
-//                      over the rows of a warp by shuffles and over the warps in shared memory
-//   select_kernel      grid (kv-head, sequence): the masses in shared memory, an 8-bit radix
-//                      select of the threshold (4 passes), an ordered compaction (positions
-//                      ascending), the exclusion-mask words and the gather of the kept rows
+//   colmass_kernel<D, 0>  persistent CTAs over (sequence, kv-head, 1024-key chunk) items:
+//                         S = Q K^T on the tensor cores (tcgen05 kind::f16, M = 128 rows,
+//                         N = 128 keys, FP32 in TMEM), one observation row per TMEM lane, so
+//                         each thread keeps its row's running maximum and sum of exp2 alone
+//                         -> partials (m, l) per (row, chunk)
+//   vl_lse_kernel         partials -> lse2[row] = m + log2(l)   (log2 domain)
+//   colmass_kernel<D, 1>  the same products transposed, S^T = K Q^T (M = 128 keys, N = 256
+//                         rows), one key per TMEM lane: each thread sums exp2(s2_ij - lse2_i)
+//                         over the rows of its key alone; the two warpgroups (rows 0..127,
+//                         128..255) add their halves into the zeroed mass array (a sum of two
+//                         terms, so the result does not depend on their order)
+//   vl_select_kernel      grid (kv-head, sequence): the masses in shared memory, an 8-bit
+//                         radix select of the threshold (4 passes), an ordered compaction
+//                         (positions ascending), the exclusion-mask words and the gather of
+//                         the kept rows
 // The scores are computed twice rather than stored (R x n_prefix FP32 per group would be
 // 33 MB per (sequence, kv-head) at 32K keys).
 #include <math.h>
+#include <stddef.h>
 
 #include "fa4q_common.cuh"
 #include "fa4q_internal.h"
 
 namespace fa4q {
 
-constexpr int kVlThreads = 256;          // 8 warps x 32 query rows = up to 256 rows
-constexpr int kVlTile = 64;              // keys per sub-tile
-constexpr int kVlChunk = 1024;           // keys per CTA
-constexpr int kVlPad = 8;                // bf16 elements of row padding (16 bytes)
+static __device__ uint32_t g_vl_status;
+
+cudaError_t vl_status_fetch(cudaStream_t st, uint32_t* host_word) {
+  cudaError_t e = cudaMemcpyFromSymbolAsync(host_word, g_vl_status, sizeof(uint32_t), 0, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return e;
+  const uint32_t zero = 0;
+  e = cudaMemcpyToSymbolAsync(g_vl_status, &zero, sizeof(uint32_t), 0, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return e;
+  return cudaStreamSynchronize(st);
+}
+
+constexpr int kVlChunk = 1024;           // keys per work item (one partial per row)
+constexpr int kCmKeys = 128;             // keys per tile
+constexpr int kCmRows = 256;             // observation rows held per group (R <= 256)
+constexpr int kCmStages = 3;             // K tiles in flight
+constexpr int kCmThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2..9 two warpgroups
 constexpr int kSelThreads = 1024;
 constexpr float kVlLog2e = 1.4426950408889634f;
 
 struct VlParams {
-  const uint16_t* q_obs;     // [B][Hq][n_obs][d]
-  const uint16_t* k;         // [B][Hkv][L][d]
   const int32_t* n_prefix;   // [B]
   float* part;               // [B][Hkv][R][chunks][2]
   float* lse2;               // [B][Hkv][R]
   float* mass;               // [B][Hkv][L]
-  int B, Hq, Hkv, n_obs, L, d, R, chunks;
+  int B, Hq, Hkv, n_obs, L, d, R, chunks, n_items;
   float c2;                  // sm_scale * log2(e)
 };
-
-FA4Q_DEVINL void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-// D (16x8, FP32) += A (16x16, row) * B (16x8, col), BF16 inputs
-FA4Q_DEVINL void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// 16-byte async copy global -> shared; src_bytes = 0 fills zeros without reading
-FA4Q_DEVINL void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-FA4Q_DEVINL void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-FA4Q_DEVINL void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 FA4Q_DEVINL float vl_ex2(float x) {
   float y;
@@ -89,189 +81,316 @@ FA4Q_DEVINL void merge_ml(float& m, float& l, float m2, float l2) {
   m = mn;
 }
 
-template <int D, int PASS>
-__global__ void __launch_bounds__(kVlThreads, 2) colmass_kernel(const VlParams p) {
-  constexpr int kRow = D + kVlPad;                 // padded row, bf16 elements
-  constexpr int kKs = D / 16;                      // k-steps
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  uint16_t* sq = reinterpret_cast<uint16_t*>(smem_raw);                 // [R][kRow]
-  uint16_t* sk = sq + kVlThreads * kRow;                                // [2][kVlTile][kRow]
-  float* red = reinterpret_cast<float*>(sk + 2 * kVlTile * kRow);       // [8][kVlTile]
+// Shared memory of the column-mass kernel: the group's observation rows and a ring of key
+// tiles, both as 64-element column chunks of 128-byte rows with the 128-byte swizzle (the
+// layout TMA writes and the K-major MMA operand reads), 1024-byte aligned.
+template <int D>
+struct CmSmem {
+  static constexpr int kChunks = D / 64;
+  uint8_t q[kChunks][kCmRows * 128];
+  uint8_t k[kCmStages][kChunks][kCmKeys * 128];
+  float lse[kCmRows];                    // pass 1: lse2 of the group's rows, +inf past R
+  uint64_t q_full, q_free;
+  uint64_t k_full[kCmStages], k_empty[kCmStages];
+  uint64_t s_full[2], s_free[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  uint32_t abort_flag;
+};
 
-  const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+// Bounded wait shared by the roles of one CTA: a wait that expires records `code` and sets
+// the CTA's abort flag, after which every later wait returns false at once.
+FA4Q_DEVINL bool cm_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag, uint32_t code) {
+  if (*abort_flag) return false;
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitNs) break;
+  }
+  atomicOr(&g_vl_status, code);
+  *abort_flag = 1;
+  return false;
+}
+
+FA4Q_DEVINL bool cm_warp_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag, uint32_t code) {
+  return __all_sync(0xffffffffu, cm_wait(bar, parity, abort_flag, code));
+}
+
+struct CmItem {
+  int bh, b, h, chunk, key_begin, key_end, n_tiles;
+};
+
+FA4Q_DEVINL CmItem cm_item(const VlParams& p, int u) {
+  CmItem it;
+  it.bh = u / p.chunks;
+  it.chunk = u - it.bh * p.chunks;
+  it.b = it.bh / p.Hkv;
+  it.h = it.bh - it.b * p.Hkv;
+  const int n_pre = min(max(p.n_prefix[it.b], 0), p.L);
+  it.key_begin = it.chunk * kVlChunk;
+  it.key_end = min(it.key_begin + kVlChunk, n_pre);
+  it.n_tiles = it.key_end > it.key_begin ? (it.key_end - it.key_begin + kCmKeys - 1) / kCmKeys : 0;
+  return it;
+}
+
+// Persistent column-mass pass (PASS 0: per-row partials of the log-sum-exp; PASS 1: column
+// masses).  CTA c takes the contiguous item range [c n / G, (c+1) n / G) of the
+// (sequence, kv-head, chunk) list, so it changes group (and reloads the observation rows)
+// once or twice; every role walks the same items and derives its barrier phases from its own
+// counters.
+template <int D, int PASS>
+__global__ void __launch_bounds__(kCmThreads, 1)
+    colmass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const VlParams p) {
+  using SM = CmSmem<D>;
+  constexpr int kCh = SM::kChunks;
+  extern __shared__ uint8_t smem_raw[];
+  SM& sm = *reinterpret_cast<SM*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  volatile uint32_t* abort_flag = &sm.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.Hq / p.Hkv;
-  const int n_pre = min(max(p.n_prefix[b], 0), p.L);
-  const int key_begin = chunk * kVlChunk;
-  const int key_end = min(key_begin + kVlChunk, n_pre);
-  const int n_tiles = key_end > key_begin ? (key_end - key_begin + kVlTile - 1) / kVlTile : 0;
-  const bool active = warp * 32 < p.R;             // rows [32 warp, 32 warp + 32)
-  const int64_t bh = static_cast<int64_t>(b) * p.Hkv + h;
+  const int u0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.n_items / gridDim.x);
+  const int u1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.n_items / gridDim.x);
 
-  // observation rows -> shared memory (row i = g * n_obs + t of q-head h*G + g)
-  for (int idx = threadIdx.x; idx < p.R * (D / 8); idx += kVlThreads) {
-    const int i = idx / (D / 8), c = idx % (D / 8);
-    const int g = i / p.n_obs, t = i % p.n_obs;
-    const uint16_t* src = p.q_obs + ((static_cast<int64_t>(b) * p.Hq + h * G + g) * p.n_obs + t) * D + 8 * c;
-    *reinterpret_cast<uint4*>(sq + i * kRow + 8 * c) = *reinterpret_cast<const uint4*>(src);
-  }
-  const uint16_t* kbase = p.k + bh * p.L * D;
-  auto load_tile = [&](int tile, int buf) {
-    const int key0 = key_begin + tile * kVlTile;
-    for (int idx = threadIdx.x; idx < kVlTile * (D / 8); idx += kVlThreads) {
-      const int r = idx / (D / 8), c = idx % (D / 8);
-      const int key = key0 + r;
-      const bool in = key < p.L;
-      const uint16_t* src = kbase + static_cast<int64_t>(in ? key : 0) * D + 8 * c;
-      cp_async16(smem_u32(sk + (buf * kVlTile + r) * kRow + 8 * c), src, in ? 16u : 0u);
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_free, PASS == 1 ? 9 : 1);      // the MMA commit (+ the 8 softmax warps)
+    for (int s = 0; s < kCmStages; ++s) {
+      mbar_init(&sm.k_full[s], 1);
+      mbar_init(&sm.k_empty[s], 1);
     }
-    cp_async_commit();
-  };
-  if (n_tiles > 0) load_tile(0, 0);
-  __syncthreads();
-
-  // ldmatrix addresses of this warp's A fragments (rows 32 warp + 16 mt + ...), k-step 0
-  const uint32_t a_addr0 = smem_u32(sq + (warp * 32 + ((lane >> 3) & 1) * 8 + (lane & 7)) * kRow + (lane >> 4) * 8);
-  // per thread: rows r(mt, hf) = 32 warp + 16 mt + g + 8 hf, g = lane / 4
-  const int g4 = lane >> 2, t4 = lane & 3;
-  float m_run[2][2], l_run[2][2], lse[2][2];
-#pragma unroll
-  for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      m_run[mt][hf] = -INFINITY;
-      l_run[mt][hf] = 0.0f;
-      const int row = warp * 32 + mt * 16 + g4 + 8 * hf;
-      lse[mt][hf] = (PASS == 1 && active) ? p.lse2[bh * p.R + row] : 0.0f;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sm.s_full[s], 1);
+      mbar_init(&sm.s_free[s], 8);
     }
-
-  for (int tile = 0; tile < n_tiles; ++tile) {
-    const int buf = tile & 1;
-    if (tile + 1 < n_tiles) {
-      load_tile(tile + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const int key0 = key_begin + tile * kVlTile;
-    float acc[2][8][4];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[mt][nt][e] = 0.0f;
-    if (active) {
-#pragma unroll
-      for (int ks = 0; ks < kKs; ++ks) {
-        uint32_t a[2][4];
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-          ldsm_x4(a_addr0 + (mt * 16 * kRow + ks * 16) * 2, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-#pragma unroll
-        for (int np2 = 0; np2 < 4; ++np2) {
-          const int key = np2 * 16 + (lane >> 4) * 8 + (lane & 7);
-          const int col = ks * 16 + ((lane >> 3) & 1) * 8;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(smem_u32(sk + (buf * kVlTile + key) * kRow + col), b0, b1, b2, b3);
-#pragma unroll
-          for (int mt = 0; mt < 2; ++mt) {
-            mma_bf16(acc[mt][2 * np2], a[mt], b0, b1);
-            mma_bf16(acc[mt][2 * np2 + 1], a[mt], b2, b3);
-          }
-        }
-      }
-    }
-    // scores in the log2 domain; keys outside the candidate prefix do not take part
-    float colsum[8][2];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) colsum[nt][0] = colsum[nt][1] = 0.0f;
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v[16];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int key = key0 + nt * 8 + 2 * t4 + c;
-            v[2 * nt + c] = key < key_end ? acc[mt][nt][2 * hf + c] * p.c2 : -INFINITY;
-          }
-        if constexpr (PASS == 0) {
-          float tmax = v[0];
-#pragma unroll
-          for (int i = 1; i < 16; ++i) tmax = fmaxf(tmax, v[i]);
-          const float mn = fmaxf(m_run[mt][hf], tmax);
-          if (mn != -INFINITY) {
-            float s = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) s += vl_ex2(v[i] - mn);
-            l_run[mt][hf] = (m_run[mt][hf] == -INFINITY ? 0.0f : l_run[mt][hf] * vl_ex2(m_run[mt][hf] - mn)) + s;
-            m_run[mt][hf] = mn;
-          }
-        } else {
-#pragma unroll
-          for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) colsum[nt][c] += vl_ex2(v[2 * nt + c] - lse[mt][hf]);
-        }
-      }
-    if constexpr (PASS == 1) {
-      // sum over the 8 row groups of the warp (lanes with the same t4), then over the warps
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          float x = colsum[nt][c];
-          x += __shfl_xor_sync(0xffffffffu, x, 4);
-          x += __shfl_xor_sync(0xffffffffu, x, 8);
-          x += __shfl_xor_sync(0xffffffffu, x, 16);
-          colsum[nt][c] = x;
-        }
-      if (g4 == 0) {
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) red[warp * kVlTile + nt * 8 + 2 * t4 + c] = active ? colsum[nt][c] : 0.0f;
-      }
-      __syncthreads();
-      if (threadIdx.x < kVlTile) {
-        const int key = key0 + threadIdx.x;
-        float sum = 0.0f;
-#pragma unroll
-        for (int w = 0; w < kVlThreads / 32; ++w) sum += red[w * kVlTile + threadIdx.x];
-        if (key < key_end) p.mass[bh * p.L + key] = sum;
-      }
-    }
-    __syncthreads();   // the buffer is refilled two tiles later; red is reused next tile
+    mbar_init(&sm.drain, 1);
+    sm.abort_flag = 0;
+    fence_barrier_init();
   }
   if constexpr (PASS == 1) {
-    // positions of this chunk outside the candidate prefix carry no mass
-    const int z0 = max(key_begin, n_pre), z1 = min(key_begin + kVlChunk, p.L);
-    for (int key = z0 + threadIdx.x; key < z1; key += kVlThreads) p.mass[bh * p.L + key] = 0.0f;
+    // rows past R take no part: exp2(s - inf) = 0 (the copies below write only [0, R))
+    for (int i = p.R + static_cast<int>(threadIdx.x); i < kCmRows; i += kCmThreads) sm.lse[i] = INFINITY;
   }
-  if constexpr (PASS == 0) {
-    // merge the four threads of each row (t4), then one lane writes the row's partial
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float m = m_run[mt][hf], l = l_run[mt][hf];
-#pragma unroll
-        for (int o = 1; o <= 2; o <<= 1) {
-          const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-          const float l2 = __shfl_xor_sync(0xffffffffu, l, o);
-          merge_ml(m, l, m2, l2);
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      int T = 0, nq = 0, cur = -1;
+      bool go = true;
+      for (int u = u0; go && u < u1; ++u) {
+        const CmItem it = cm_item(p, u);
+        if (it.n_tiles == 0) continue;
+        if (it.bh != cur) {
+          // the observation rows of the new group (+ its lse2 in pass 1) once every product
+          // (and, in pass 1, every softmax warp) is done with the previous group's
+          if (nq > 0 && !cm_wait(&sm.q_free, (nq - 1) & 1, abort_flag, kStatusTimeoutTmaFull)) break;
+          const int row0 = (it.b * p.Hq + it.h * G) * p.n_obs;
+          mbar_arrive_expect_tx(&sm.q_full, kCh * kCmRows * 128 + (PASS == 1 ? p.R * 4 : 0));
+          for (int c = 0; c < kCh; ++c) {
+            tma_load_3d(sm.q[c], &tm_q, 128 * c, row0, 0, &sm.q_full);
+            tma_load_3d(sm.q[c] + 128 * 128, &tm_q, 128 * c, row0 + 128, 0, &sm.q_full);
+          }
+          if constexpr (PASS == 1) bulk_load(sm.lse, p.lse2 + static_cast<int64_t>(it.bh) * p.R, p.R * 4, &sm.q_full);
+          ++nq;
+          cur = it.bh;
         }
-        const int row = warp * 32 + mt * 16 + g4 + 8 * hf;
-        if (active && t4 == 0) {
-          float* dst = p.part + ((bh * p.R + row) * p.chunks + chunk) * 2;
-          dst[0] = m;
-          dst[1] = l;
+        for (int j = 0; j < it.n_tiles; ++j, ++T) {
+          const int s = T % kCmStages;
+          if (T >= kCmStages &&
+              !cm_wait(&sm.k_empty[s], ((T / kCmStages) - 1) & 1, abort_flag, kStatusTimeoutTmaFull)) {
+            go = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&sm.k_full[s], kCh * kCmKeys * 128);
+          for (int c = 0; c < kCh; ++c)
+            tma_load_3d(sm.k[s][c], &tm_k, 128 * c, it.key_begin + j * kCmKeys, it.bh, &sm.k_full[s]);
         }
       }
+      // drain: every issued copy lands before the CTA may exit
+      for (int t = max(0, T - kCmStages); t < T; ++t)
+        mbar_wait(&sm.k_full[t % kCmStages], (t / kCmStages) & 1, &g_vl_status, kStatusTimeoutDrain);
+      if (nq > 0) mbar_wait(&sm.q_full, (nq - 1) & 1, &g_vl_status, kStatusTimeoutDrain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      // descriptors: base descriptor + byte offset / 16 (shared memory < 256 KB: no carry)
+      const uint64_t dsc = make_smem_desc(smem_u32(&sm), 16, 1024, kSwiz128);
+      constexpr uint64_t oq = offsetof(SM, q) >> 4, ok = offsetof(SM, k) >> 4;
+      constexpr uint64_t kQc = kCmRows * 128 >> 4, kKc = kCmKeys * 128 >> 4, kKs = kCh * kKc;
+      constexpr uint64_t kQh = 128 * 128 >> 4;
+      const uint32_t idesc = make_idesc_bf16(PASS == 0 ? kCmKeys : kCmRows, false);
+      int T = 0, nq = 0, cur = -1;
+      bool ok_run = true;
+      for (int u = u0; ok_run && u < u1; ++u) {
+        const CmItem it = cm_item(p, u);
+        if (it.n_tiles == 0) continue;
+        if (it.bh != cur) {
+          if (nq > 0) tc_commit(&sm.q_free);
+          if (!cm_wait(&sm.q_full, nq & 1, abort_flag, kStatusTimeoutMma)) break;
+          tc_fence_after();
+          ++nq;
+          cur = it.bh;
+        }
+        for (int j = 0; j < it.n_tiles; ++j, ++T) {
+          const int s = T % kCmStages, buf = T & 1;
+          if (!cm_wait(&sm.k_full[s], (T / kCmStages) & 1, abort_flag, kStatusTimeoutMma) ||
+              (T >= 2 && !cm_wait(&sm.s_free[buf], ((T >> 1) - 1) & 1, abort_flag, kStatusTimeoutMma))) {
+            ok_run = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t dcol = tmem + 256u * buf;
+          if constexpr (PASS == 0) {
+            // S[row][key] for rows 0..127 and 128..255 (two M = 128 products)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+              for (int kk = 0; kk < D / 16; ++kk)
+                mma_bf16(dcol + 128u * hh, dsc + oq + (kk >> 2) * kQc + hh * kQh + 2 * (kk & 3),
+                         dsc + ok + s * kKs + (kk >> 2) * kKc + 2 * (kk & 3), idesc, kk > 0);
+          } else {
+            // S^T[key][row] for all 256 rows (M = 128 keys, N = 256)
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              mma_bf16(dcol, dsc + ok + s * kKs + (kk >> 2) * kKc + 2 * (kk & 3),
+                       dsc + oq + (kk >> 2) * kQc + 2 * (kk & 3), idesc, kk > 0);
+          }
+          tc_commit(&sm.s_full[buf]);
+          tc_commit(&sm.k_empty[s]);
+        }
+      }
+      // drain: every product this thread issued completes before TMEM is released
+      tc_commit(&sm.drain);
+      mbar_wait(&sm.drain, 0, &g_vl_status, kStatusTimeoutDrain);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warpgroups
+    // warp w reads TMEM lanes 32 (w % 4) ..; warpgroup wg = 0, 1 takes S columns
+    // [128 wg, 128 wg + 128) of each buffer (pass 0: the rows 128 wg + lane of its own;
+    // pass 1: rows 128 wg .. 128 wg + 127 of the key in its lane)
+    const int wg = (warp - 2) >> 2, lq = 32 * (warp & 3) + lane;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 128u * wg;
+    int T = 0, nq = 0, cur = -1;
+    bool ok_run = true;
+    for (int u = u0; ok_run && u < u1; ++u) {
+      const CmItem it = cm_item(p, u);
+      const int64_t bh = it.bh;
+      if constexpr (PASS == 0) {
+        float m_run = -INFINITY, l_run = 0.0f;
+        for (int j = 0; j < it.n_tiles; ++j, ++T) {
+          const int buf = T & 1;
+          if (!cm_warp_wait(&sm.s_full[buf], (T >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) {
+            ok_run = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t r[4][32];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(trow + 256u * buf + 32u * q4, r[q4]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_free[buf]);
+          const int valid = min(kCmKeys, it.key_end - (it.key_begin + j * kCmKeys));
+          if (valid < kCmKeys) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (32 * q4 + i >= valid) r[q4][i] = __float_as_uint(-INFINITY);
+          }
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+            for (int i = 0; i < 32; i += 2) {
+              mx0 = fmaxf(mx0, __uint_as_float(r[q4][i]));
+              mx1 = fmaxf(mx1, __uint_as_float(r[q4][i + 1]));
+            }
+          const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * p.c2);
+          const float nm = -m_new;
+          float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              a0 += vl_ex2(fmaf(__uint_as_float(r[q4][i]), p.c2, nm));
+              a1 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 1]), p.c2, nm));
+              a2 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 2]), p.c2, nm));
+              a3 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 3]), p.c2, nm));
+            }
+          l_run = (m_run == -INFINITY ? 0.0f : l_run * vl_ex2(m_run - m_new)) + ((a0 + a1) + (a2 + a3));
+          m_run = m_new;
+        }
+        if (!ok_run) break;
+        const int row = 128 * wg + lq;
+        if (row < p.R) {
+          float* dst = p.part + ((bh * p.R + row) * p.chunks + it.chunk) * 2;
+          dst[0] = m_run;
+          dst[1] = l_run;
+        }
+      } else {
+        if (it.n_tiles == 0) continue;                 // the mass array was zeroed
+        if (it.bh != cur) {
+          if (nq > 0) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.q_free);     // done with the previous group's lse2
+          }
+          if (!cm_warp_wait(&sm.q_full, nq & 1, abort_flag, kStatusTimeoutSoftmax)) break;
+          ++nq;
+          cur = it.bh;
+        }
+        const float4* lse4 = reinterpret_cast<const float4*>(sm.lse + 128 * wg);
+        for (int j = 0; j < it.n_tiles; ++j, ++T) {
+          const int buf = T & 1;
+          if (!cm_warp_wait(&sm.s_full[buf], (T >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) {
+            ok_run = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t r[4][32];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(trow + 256u * buf + 32u * q4, r[q4]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.s_free[buf]);
+          float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 l4 = lse4[8 * q4 + i / 4];
+              a0 += vl_ex2(fmaf(__uint_as_float(r[q4][i]), p.c2, -l4.x));
+              a1 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 1]), p.c2, -l4.y));
+              a2 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 2]), p.c2, -l4.z));
+              a3 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 3]), p.c2, -l4.w));
+            }
+          const int key = it.key_begin + j * kCmKeys + lq;
+          if (key < it.key_end) atomicAdd(p.mass + bh * p.L + key, (a0 + a1) + (a2 + a3));
+        }
+      }
+    }
+  }
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -300,31 +419,37 @@ struct SelParams {
   double rho;
 };
 
-// exclusive prefix count of `flag` over the block in thread order; *total = the block's count
-FA4Q_DEVINL uint32_t block_excl_count(bool flag, uint32_t* wsum, uint32_t* total) {
+// exclusive prefix sum of `v` over the block in thread order; *total = the block's sum
+// (every thread of the block calls it; wsum holds 33 words)
+FA4Q_DEVINL uint32_t block_excl_sum(uint32_t v, uint32_t* wsum, uint32_t* total) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t ballot = __ballot_sync(0xffffffffu, flag);
-  const uint32_t lane_rank = __popc(ballot & ((1u << lane) - 1u));
-  if (lane == 0) wsum[warp] = __popc(ballot);
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    const uint32_t v = lane < (kSelThreads / 32) ? wsum[lane] : 0u;
-    uint32_t incl = v;
+    const uint32_t w = lane < (kSelThreads / 32) ? wsum[lane] : 0u;
+    uint32_t wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
+      const uint32_t y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
     }
-    if (lane < (kSelThreads / 32)) wsum[lane] = incl - v;
-    if (lane == 31) wsum[32] = incl;
+    if (lane < (kSelThreads / 32)) wsum[lane] = wi - w;
+    if (lane == 31) wsum[32] = wi;
   }
   __syncthreads();
-  const uint32_t rank = wsum[warp] + lane_rank;
+  const uint32_t r = wsum[warp] + incl - v;
   *total = wsum[32];
   __syncthreads();
-  return rank;
+  return r;
 }
 
+// one CTA per (kv-head, sequence); the candidates' masses live in shared memory
 __global__ void __launch_bounds__(kSelThreads, 1) vl_select_kernel(const SelParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   unsigned long long* mask = reinterpret_cast<unsigned long long*>(smem_raw);   // [max_pages]
@@ -335,7 +460,7 @@ __global__ void __launch_bounds__(kSelThreads, 1) vl_select_kernel(const SelPara
   __shared__ uint32_t s_prefix, s_remaining;
   const int h = blockIdx.x, b = blockIdx.y;
   const int64_t bh = static_cast<int64_t>(b) * p.Hkv + h;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int n = min(max(p.n_prefix[b], 0), p.L);
   int cnt = static_cast<int>(ceil(p.rho * static_cast<double>(n) - 1e-9));
   cnt = min(max(cnt, 0), n);
@@ -346,15 +471,21 @@ __global__ void __launch_bounds__(kSelThreads, 1) vl_select_kernel(const SelPara
   __syncthreads();
 
   // radix select of the cnt-th largest pattern T, 8 bits at a time from the top; at the end
-  // `remaining` is how many of the elements equal to T belong to the top cnt
+  // `remaining` is how many of the elements equal to T belong to the top cnt.  Masses of one
+  // group share few exponents, so the lanes of a warp that fall in the same bin add their
+  // count with one atomic (lanes grouped by __match_any_sync).
   uint32_t prefix = 0, pmask = 0, remaining = static_cast<uint32_t>(cnt);
   if (cnt > 0) {
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += kSelThreads) hist[i] = 0;
       __syncthreads();
-      for (int j = tid; j < n; j += kSelThreads) {
-        const uint32_t x = bits[j];
-        if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+      for (int j0 = 0; j0 < n; j0 += kSelThreads) {       // uniform per warp
+        const int j = j0 + tid;
+        const uint32_t x = j < n ? bits[j] : 0u;
+        const bool in = j < n && (x & pmask) == prefix;
+        const uint32_t bin = in ? (x >> shift) & 255u : 256u;
+        const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(peers)));
       }
       __syncthreads();
       if (tid == 0) {
@@ -373,23 +504,40 @@ __global__ void __launch_bounds__(kSelThreads, 1) vl_select_kernel(const SelPara
       pmask |= 255u << shift;
     }
     // ordered compaction: every element above T, and the first `remaining` equal to T in
-    // position order (the lowest positions win ties); positions come out ascending
-    uint32_t base_eq = 0, base_sel = 0;
-    for (int t0 = 0; t0 < n; t0 += kSelThreads) {
-      const int j = t0 + tid;
-      const uint32_t x = j < n ? bits[j] : 0u;
-      const bool eq = j < n && x == prefix;
-      const bool gt = j < n && x > prefix;
-      uint32_t tot_eq, tot_sel;
-      const uint32_t eq_rank = block_excl_count(eq, wsum, &tot_eq);
-      const bool sel = gt || (eq && base_eq + eq_rank < remaining);
-      const uint32_t sel_rank = block_excl_count(sel, wsum, &tot_sel);
-      if (sel && base_sel + sel_rank < static_cast<uint32_t>(cnt)) {
-        pos[base_sel + sel_rank] = j;
-        atomicOr(&mask[j >> 6], 1ull << (j & 63));
+    // position order (the lowest positions win ties); positions come out ascending.  Thread
+    // t takes the 32 consecutive positions base + 32 t .. (read in a lane-rotated order, so
+    // the shared-memory loads of a warp hit 32 banks), as bit masks.
+    uint32_t eq_before = 0, sel_before = 0;
+    for (int base = 0; base < n; base += 32 * kSelThreads) {
+      const int j0 = base + 32 * tid;
+      uint32_t gtm = 0, eqm = 0;
+#pragma unroll 8
+      for (int i = 0; i < 32; ++i) {
+        const int bi = (i + lane) & 31;
+        const int j = j0 + bi;
+        if (j < n) {
+          const uint32_t x = bits[j];
+          gtm |= static_cast<uint32_t>(x > prefix) << bi;
+          eqm |= static_cast<uint32_t>(x == prefix) << bi;
+        }
       }
-      base_eq += tot_eq;
-      base_sel += tot_sel;
+      uint32_t eq_tot, sel_tot;
+      const uint32_t eq_rank = eq_before + block_excl_sum(__popc(eqm), wsum, &eq_tot);
+      // the lowest `take` equal elements of this thread are kept
+      const uint32_t take = remaining > eq_rank ? min(remaining - eq_rank, static_cast<uint32_t>(__popc(eqm))) : 0u;
+      uint32_t selm = gtm, e = eqm;
+      for (uint32_t t = 0; t < take; ++t) {
+        selm |= e & (0u - e);                             // lowest set bit
+        e &= e - 1u;
+      }
+      const uint32_t sel_rank = sel_before + block_excl_sum(__popc(selm), wsum, &sel_tot);
+      uint32_t k = sel_rank;
+      for (uint32_t s = selm; s != 0u && k < static_cast<uint32_t>(cnt); s &= s - 1u, ++k)
+        pos[k] = j0 + __ffs(s) - 1;
+      if (selm != 0u && p.max_pages > 0)
+        atomicOr(&mask[j0 >> 6], static_cast<unsigned long long>(selm) << (j0 & 63));
+      eq_before += eq_tot;
+      sel_before += sel_tot;
     }
   }
   __syncthreads();
@@ -397,16 +545,32 @@ __global__ void __launch_bounds__(kSelThreads, 1) vl_select_kernel(const SelPara
   for (int i = tid; i < cnt; i += kSelThreads) p.positions[bh * p.max_select + i] = pos[i];
   if (p.excl != nullptr)
     for (int i = tid; i < p.max_pages; i += kSelThreads) p.excl[bh * p.max_pages + i] = mask[i];
-  // the kept rows, 16 bytes per lane
-  const int warp = tid >> 5, lane = tid & 31, chunks = p.d / 8;
-  for (int i = warp; i < cnt; i += kSelThreads / 32) {
-    if (lane >= chunks) continue;
-    const int64_t src = (bh * p.L + pos[i]) * p.d + 8 * lane;
-    const int64_t dst = (bh * p.max_select + i) * p.d + 8 * lane;
-    if (p.hp_k != nullptr)
-      *reinterpret_cast<uint4*>(p.hp_k + dst) = *reinterpret_cast<const uint4*>(p.k + src);
-    if (p.hp_v != nullptr)
-      *reinterpret_cast<uint4*>(p.hp_v + dst) = *reinterpret_cast<const uint4*>(p.v + src);
+  // the kept rows in 16-byte pieces, four pieces of K and V per thread in flight at a time
+  const int shift_c = p.d == 128 ? 4 : 3;                // 16-byte pieces per row: d / 8
+  const int total = cnt << shift_c;
+  constexpr int kU = 4;
+  for (int i0 = 0; i0 < total; i0 += kU * kSelThreads) {
+    uint4 kk[kU], vv[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int idx = i0 + u * kSelThreads + tid;
+      if (idx < total) {
+        const int r = idx >> shift_c, c = idx & ((1 << shift_c) - 1);
+        const int64_t src = (bh * p.L + pos[r]) * p.d + 8 * c;
+        if (p.hp_k != nullptr) kk[u] = *reinterpret_cast<const uint4*>(p.k + src);
+        if (p.hp_v != nullptr) vv[u] = *reinterpret_cast<const uint4*>(p.v + src);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int idx = i0 + u * kSelThreads + tid;
+      if (idx < total) {
+        const int r = idx >> shift_c, c = idx & ((1 << shift_c) - 1);
+        const int64_t dst = (bh * p.max_select + r) * p.d + 8 * c;
+        if (p.hp_k != nullptr) *reinterpret_cast<uint4*>(p.hp_k + dst) = kk[u];
+        if (p.hp_v != nullptr) *reinterpret_cast<uint4*>(p.hp_v + dst) = vv[u];
+      }
+    }
   }
 }
 
@@ -418,21 +582,31 @@ size_t vl_select_smem(int L, int max_select, int max_pages) {
   return static_cast<size_t>(max_pages) * 8 + static_cast<size_t>(L) * 4 + static_cast<size_t>(max_select) * 4 +
          (256 + 33) * 4;
 }
-size_t vl_colmass_smem(int d) {
-  return static_cast<size_t>(kVlThreads + 2 * kVlTile) * (d + kVlPad) * 2 + (kVlThreads / 32) * kVlTile * 4;
-}
+template <int D>
+size_t vl_colmass_smem() { return sizeof(CmSmem<D>) + 1024; }
 
 template <int D>
-fa4q_status vl_launch(const VlParams& vp, const SelParams& sp, cudaStream_t st, size_t sel_smem) {
-  const size_t cm = vl_colmass_smem(D);
+fa4q_status vl_launch(const VlParams& vp, const SelParams& sp, const void* q_obs, const void* k, cudaStream_t st,
+                      size_t sel_smem) {
+  const size_t cm = vl_colmass_smem<D>();
   if (cudaFuncSetAttribute(colmass_kernel<D, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cm) != cudaSuccess ||
       cudaFuncSetAttribute(colmass_kernel<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cm) != cudaSuccess ||
       cudaFuncSetAttribute(vl_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem) != cudaSuccess)
     return FA4Q_ERR_CUDA;
-  const dim3 grid(vp.chunks, vp.Hkv, vp.B);
-  colmass_kernel<D, 0><<<grid, kVlThreads, cm, st>>>(vp);
+  // observation rows as one [B*Hq*n_obs][2D bytes] matrix, keys as [B*Hkv][L][2D bytes]; 128-byte
+  // boxes (one 64-element column chunk) of 128 rows, 128-byte swizzle; rows past either
+  // tensor's end read as zeros
+  CUtensorMap tq, tk;
+  const uint64_t q_rows = static_cast<uint64_t>(vp.B) * vp.Hq * vp.n_obs;
+  if (!make_map_3d(&tq, q_obs, 2 * D, q_rows, 1, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_3d(&tk, k, 2 * D, vp.L, static_cast<uint64_t>(vp.B) * vp.Hkv, 128, kCmKeys, CU_TENSOR_MAP_SWIZZLE_128B))
+    return FA4Q_ERR_CUDA;
+  if (cudaMemsetAsync(vp.mass, 0, static_cast<size_t>(vp.B) * vp.Hkv * vp.L * sizeof(float), st) != cudaSuccess)
+    return FA4Q_ERR_CUDA;
+  const int grid = std::min(vp.n_items, num_sms());
+  colmass_kernel<D, 0><<<grid, kCmThreads, cm, st>>>(tq, tk, vp);
   vl_lse_kernel<<<vp.B * vp.Hkv, vp.R, 0, st>>>(vp.part, vp.lse2, vp.R, vp.chunks);
-  colmass_kernel<D, 1><<<grid, kVlThreads, cm, st>>>(vp);
+  colmass_kernel<D, 1><<<grid, kCmThreads, cm, st>>>(tq, tk, vp);
   vl_select_kernel<<<dim3(vp.Hkv, vp.B), kSelThreads, sel_smem, st>>>(sp);
   return launch_status();
 }
@@ -459,13 +633,13 @@ extern "C" fa4q_status fa4q_select_vertical_lines(
   if (!(rho > 0.0) || rho > 1.0 || !(sm_scale >= 0.0f) || !isfinite(sm_scale)) return FA4Q_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA4Q_ERR_UNSUPPORTED;
   const int R = vl_rows(Hq, Hkv, n_obs);
-  if (R % 32 != 0 || R > kVlThreads) return FA4Q_ERR_UNSUPPORTED;
+  if (R % 32 != 0 || R > kCmRows) return FA4Q_ERR_UNSUPPORTED;
   const double need = ceil(rho * static_cast<double>(L) - 1e-9);
   if (static_cast<double>(max_select) < need || max_select <= 0) return FA4Q_ERR_INVALID_ARG;
   if (excl_mask != nullptr && static_cast<int64_t>(max_pages) * 64 < L) return FA4Q_ERR_INVALID_ARG;
   if (excl_mask == nullptr) max_pages = 0;
   if (!aligned16(q_obs) || !aligned16(k) || (v && !aligned16(v)) || (hp_k && !aligned16(hp_k)) ||
-      (hp_v && !aligned16(hp_v)) || (reinterpret_cast<uintptr_t>(workspace) & 7) ||
+      (hp_v && !aligned16(hp_v)) || !aligned16(workspace) ||
       (reinterpret_cast<uintptr_t>(mass) & 3))
     return FA4Q_ERR_INVALID_ARG;
   if (workspace_bytes < fa4q_vlines_workspace_size(B, Hq, Hkv, n_obs, L)) return FA4Q_ERR_INVALID_ARG;
@@ -473,10 +647,10 @@ extern "C" fa4q_status fa4q_select_vertical_lines(
   const size_t sel_smem = vl_select_smem(L, max_select, max_pages);
   if (sel_smem > 227 * 1024) return FA4Q_ERR_UNSUPPORTED;   // candidates held in shared memory
   VlParams vp;
-  vp.q_obs = static_cast<const uint16_t*>(q_obs);
-  vp.k = static_cast<const uint16_t*>(k);
   vp.n_prefix = n_prefix;
   vp.chunks = vl_chunks(L);
+  if (static_cast<int64_t>(B) * Hkv * vp.chunks > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
+  vp.n_items = B * Hkv * vp.chunks;
   vp.part = static_cast<float*>(workspace);
   vp.lse2 = vp.part + static_cast<size_t>(B) * Hkv * R * vp.chunks * 2;
   vp.mass = mass;
@@ -496,5 +670,5 @@ extern "C" fa4q_status fa4q_select_vertical_lines(
   sp.L = L; sp.d = d; sp.Hkv = Hkv; sp.max_select = max_select; sp.max_pages = max_pages;
   sp.rho = rho;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return d == 128 ? vl_launch<128>(vp, sp, st, sel_smem) : vl_launch<64>(vp, sp, st, sel_smem);
+  return d == 128 ? vl_launch<128>(vp, sp, q_obs, k, st, sel_smem) : vl_launch<64>(vp, sp, q_obs, k, st, sel_smem);
 }
