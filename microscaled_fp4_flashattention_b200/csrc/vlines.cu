@@ -17,18 +17,19 @@
 //   colmass_kernel<D, 0>  persistent CTAs over (sequence, kv-head, 1024-key chunk) items:
 //                         S = Q K^T on the tensor cores (tcgen05 kind::f16, M = 128 rows,
 //                         N = 128 keys, FP32 in TMEM), one observation row per TMEM lane, so
-//                         each thread keeps its row's running maximum and sum of exp2 alone
-//                         -> partials (m, l) per (row, chunk)
-//   vl_lse_kernel         partials -> lse2[row] = m + log2(l)   (log2 domain)
-//   colmass_kernel<D, 1>  the same products transposed, S^T = K Q^T (M = 128 keys, N = 256
-//                         rows), one key per TMEM lane: each thread sums exp2(s2_ij - lse2_i)
-//                         over the rows of its key alone; the two warpgroups (rows 0..127,
-//                         128..255) add their halves into the zeroed mass array (a sum of two
-//                         terms, so the result does not depend on their order)
+//                         each thread keeps its rows' running maximum and sum of exp2 alone;
+//                         two softmax groups take alternate key tiles -> partials (m, l) per
+//                         (row, chunk, group)
+//   vl_lse_kernel         partials -> -lse2[row] = -(m + log2(l))   (log2 domain)
+//   colmass_kernel<D, 1>  the same products transposed, S^T = K Q^T (M = 128 keys, N = 128
+//                         rows, twice), one key per TMEM lane: each thread sums exp2(s2_ij - lse2_i)
+//                         over the 256 rows of its key alone and writes the key's mass
 //   vl_select_kernel      grid (kv-head, sequence): the masses in shared memory, an 8-bit
 //                         radix select of the threshold (4 passes), an ordered compaction
-//                         (positions ascending), the exclusion-mask words and the gather of
-//                         the kept rows
+//                         (positions ascending) and the exclusion-mask words
+//   vl_gather_kernel      the kept rows of K and V, position order
+// In both column-mass passes ten of every sixteen exponentials run on MUFU, six on the FMA
+// pipe.
 // The scores are computed twice rather than stored (R x n_prefix FP32 per group would be
 // 33 MB per (sequence, kv-head) at 32K keys).
 #include <math.h>
@@ -53,15 +54,15 @@ cudaError_t vl_status_fetch(cudaStream_t st, uint32_t* host_word) {
 constexpr int kVlChunk = 1024;           // keys per work item (one partial per row)
 constexpr int kCmKeys = 128;             // keys per tile
 constexpr int kCmRows = 256;             // observation rows held per group (R <= 256)
-constexpr int kCmStages = 3;             // K tiles in flight
+constexpr int kCmStages = 4;             // K tiles in flight
 constexpr int kCmThreads = 320;          // warp 0 TMA, warp 1 MMA, warps 2..9 two warpgroups
 constexpr int kSelThreads = 1024;
 constexpr float kVlLog2e = 1.4426950408889634f;
 
 struct VlParams {
   const int32_t* n_prefix;   // [B]
-  float* part;               // [B][Hkv][R][chunks][2]
-  float* lse2;               // [B][Hkv][R]
+  float* part;               // [B][Hkv][R][chunks][2 softmax groups][2]: (m, l)
+  float* nlse2;              // [B][Hkv][R]: -log2 sum_j 2^(s2_ij) per row
   float* mass;               // [B][Hkv][L]
   int B, Hq, Hkv, n_obs, L, d, R, chunks, n_items;
   float c2;                  // sm_scale * log2(e)
@@ -71,6 +72,76 @@ FA4Q_DEVINL float vl_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed FP32 pairs (f32x2 instructions: one issue slot for two lanes of work)
+FA4Q_DEVINL float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+FA4Q_DEVINL float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+FA4Q_DEVINL float vl_max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of values on the FMA pipe (the MUFU pipe is the column-mass passes' limit,
+// so six of every sixteen exponentials take this path):
+//   x clamped at -126 (2^-126 stands for anything smaller: far below any mass that counts)
+//   t = x + 1.5*2^23 rounded toward -inf -> floor(x) in the low mantissa bits of t
+//   f = x - (t - 1.5*2^23) in [0, 1), exact
+//   p = c0 + f (c1 + f (c2 + f (c3 + f c4)))   2^f, minimax (relative) on [0, 1),
+//                                              max relative error 2.7e-6
+//   2^x = p * 2^floor(x): floor(x) added to the exponent field of p (bits of t << 23)
+// Coefficients: degree-4 Lawson fit of 2^f on [0, 1) (fit_exp2_poly.py beside this file).
+constexpr float kVlE0 = 1.0000026226043701f, kVlE1 = 0.6930038332939148f, kVlE2 = 0.2414427399635315f;
+constexpr float kVlE3 = 0.05201146751642227f, kVlE4 = 0.01353417057543993f;
+FA4Q_DEVINL float2 vl_ex2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  uint32_t t0, t1, p0, p1;
+  asm("{\n\t.reg .b64 rx, rt, rj, rf, rp, rm, c0, c1, c2, c3, c4;\n\t"
+      "mov.b64 rx, {%4, %5};\n\tmov.b64 rm, {%6, %6};\n\t"
+      "add.rm.f32x2 rt, rx, rm;\n\tsub.rn.f32x2 rj, rt, rm;\n\tsub.rn.f32x2 rf, rx, rj;\n\t"
+      "mov.b64 c4, {%11, %11};\n\tmov.b64 c3, {%10, %10};\n\tmov.b64 c2, {%9, %9};\n\t"
+      "mov.b64 c1, {%8, %8};\n\tmov.b64 c0, {%7, %7};\n\t"
+      "fma.rn.f32x2 rp, c4, rf, c3;\n\tfma.rn.f32x2 rp, rp, rf, c2;\n\t"
+      "fma.rn.f32x2 rp, rp, rf, c1;\n\tfma.rn.f32x2 rp, rp, rf, c0;\n\t"
+      "mov.b64 {%0, %1}, rt;\n\tmov.b64 {%2, %3}, rp;\n\t}"
+      : "=r"(t0), "=r"(t1), "=r"(p0), "=r"(p1)
+      : "f"(x.x), "f"(x.y), "f"(12582912.0f), "f"(kVlE0), "f"(kVlE1), "f"(kVlE2), "f"(kVlE3), "f"(kVlE4));
+  return make_float2(__uint_as_float(p0 + (t0 << 23)), __uint_as_float(p1 + (t1 << 23)));
+}
+
+// sum of 2^x over sixteen values (x = s * c2 + o, pairs): ten on MUFU, six on the FMA pipe,
+// as two packed partial sums
+FA4Q_DEVINL void vl_sum16(const uint32_t* s, float2 c2, const float2* o, float2& acc0, float2& acc1) {
+  float2 x[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) x[k] = fma2(make_float2(__uint_as_float(s[2 * k]), __uint_as_float(s[2 * k + 1])), c2, o[k]);
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    const float2 y = make_float2(vl_ex2(x[k].x), vl_ex2(x[k].y));
+    if (k & 1) acc1 = add2(acc1, y);
+    else acc0 = add2(acc0, y);
+  }
+  acc1 = add2(acc1, vl_ex2_fma2(x[5]));
+  acc0 = add2(acc0, vl_ex2_fma2(x[6]));
+  acc1 = add2(acc1, vl_ex2_fma2(x[7]));
 }
 
 // (m, l) of two partial softmax sums merged (m = -inf means empty)
@@ -89,10 +160,10 @@ struct CmSmem {
   static constexpr int kChunks = D / 64;
   uint8_t q[kChunks][kCmRows * 128];
   uint8_t k[kCmStages][kChunks][kCmKeys * 128];
-  float lse[kCmRows];                    // pass 1: lse2 of the group's rows, +inf past R
+  float nlse[kCmRows];                   // pass 1: -lse2 of the group's rows, -inf past R
   uint64_t q_full, q_free;
   uint64_t k_full[kCmStages], k_empty[kCmStages];
-  uint64_t s_full[2], s_free[2];
+  uint64_t s_full[2][2], s_free[2][2];   // [buffer][128-column half]
   uint64_t drain;
   uint32_t tmem_base;
   uint32_t abort_flag;
@@ -161,17 +232,19 @@ __global__ void __launch_bounds__(kCmThreads, 1)
       mbar_init(&sm.k_full[s], 1);
       mbar_init(&sm.k_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.s_free[s], 8);
-    }
+    for (int s = 0; s < 2; ++s)
+      for (int hh = 0; hh < 2; ++hh) {
+        mbar_init(&sm.s_full[s][hh], 1);
+        mbar_init(&sm.s_free[s][hh], 4);          // the four warps of softmax group s
+      }
     mbar_init(&sm.drain, 1);
     sm.abort_flag = 0;
     fence_barrier_init();
   }
   if constexpr (PASS == 1) {
-    // rows past R take no part: exp2(s - inf) = 0 (the copies below write only [0, R))
-    for (int i = p.R + static_cast<int>(threadIdx.x); i < kCmRows; i += kCmThreads) sm.lse[i] = INFINITY;
+    // rows past R take no part: 2^(s - inf) = 0 on MUFU, 2^-126 on the FMA path (the copies
+    // below write only [0, R))
+    for (int i = p.R + static_cast<int>(threadIdx.x); i < kCmRows; i += kCmThreads) sm.nlse[i] = -INFINITY;
   }
   if (warp == 1) {
     tmem_alloc(&sm.tmem_base, 512);
@@ -193,7 +266,7 @@ __global__ void __launch_bounds__(kCmThreads, 1)
         const CmItem it = cm_item(p, u);
         if (it.n_tiles == 0) continue;
         if (it.bh != cur) {
-          // the observation rows of the new group (+ its lse2 in pass 1) once every product
+          // the observation rows of the new group (+ its -lse2 in pass 1) once every product
           // (and, in pass 1, every softmax warp) is done with the previous group's
           if (nq > 0 && !cm_wait(&sm.q_free, (nq - 1) & 1, abort_flag, kStatusTimeoutTmaFull)) break;
           const int row0 = (it.b * p.Hq + it.h * G) * p.n_obs;
@@ -202,7 +275,7 @@ __global__ void __launch_bounds__(kCmThreads, 1)
             tma_load_3d(sm.q[c], &tm_q, 128 * c, row0, 0, &sm.q_full);
             tma_load_3d(sm.q[c] + 128 * 128, &tm_q, 128 * c, row0 + 128, 0, &sm.q_full);
           }
-          if constexpr (PASS == 1) bulk_load(sm.lse, p.lse2 + static_cast<int64_t>(it.bh) * p.R, p.R * 4, &sm.q_full);
+          if constexpr (PASS == 1) bulk_load(sm.nlse, p.nlse2 + static_cast<int64_t>(it.bh) * p.R, p.R * 4, &sm.q_full);
           ++nq;
           cur = it.bh;
         }
@@ -231,7 +304,7 @@ __global__ void __launch_bounds__(kCmThreads, 1)
       constexpr uint64_t oq = offsetof(SM, q) >> 4, ok = offsetof(SM, k) >> 4;
       constexpr uint64_t kQc = kCmRows * 128 >> 4, kKc = kCmKeys * 128 >> 4, kKs = kCh * kKc;
       constexpr uint64_t kQh = 128 * 128 >> 4;
-      const uint32_t idesc = make_idesc_bf16(PASS == 0 ? kCmKeys : kCmRows, false);
+      const uint32_t idesc = make_idesc_bf16(128, false);
       int T = 0, nq = 0, cur = -1;
       bool ok_run = true;
       for (int u = u0; ok_run && u < u1; ++u) {
@@ -244,31 +317,32 @@ __global__ void __launch_bounds__(kCmThreads, 1)
           ++nq;
           cur = it.bh;
         }
-        for (int j = 0; j < it.n_tiles; ++j, ++T) {
+        for (int j = 0; j < it.n_tiles && ok_run; ++j, ++T) {
           const int s = T % kCmStages, buf = T & 1;
-          if (!cm_wait(&sm.k_full[s], (T / kCmStages) & 1, abort_flag, kStatusTimeoutMma) ||
-              (T >= 2 && !cm_wait(&sm.s_free[buf], ((T >> 1) - 1) & 1, abort_flag, kStatusTimeoutMma))) {
+          if (!cm_wait(&sm.k_full[s], (T / kCmStages) & 1, abort_flag, kStatusTimeoutMma)) {
             ok_run = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t dcol = tmem + 256u * buf;
-          if constexpr (PASS == 0) {
-            // S[row][key] for rows 0..127 and 128..255 (two M = 128 products)
+          // the two 128-column halves of the buffer (rows 0..127 and 128..255), each issued
+          // as soon as the softmax group has read that half of the tile two steps back
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
+          for (int hh = 0; hh < 2; ++hh) {
+            if (T >= 2 && !cm_wait(&sm.s_free[buf][hh], ((T >> 1) - 1) & 1, abort_flag, kStatusTimeoutMma)) {
+              ok_run = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t dcol = tmem + 256u * buf + 128u * hh;
 #pragma unroll
-              for (int kk = 0; kk < D / 16; ++kk)
-                mma_bf16(dcol + 128u * hh, dsc + oq + (kk >> 2) * kQc + hh * kQh + 2 * (kk & 3),
-                         dsc + ok + s * kKs + (kk >> 2) * kKc + 2 * (kk & 3), idesc, kk > 0);
-          } else {
-            // S^T[key][row] for all 256 rows (M = 128 keys, N = 256)
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              mma_bf16(dcol, dsc + ok + s * kKs + (kk >> 2) * kKc + 2 * (kk & 3),
-                       dsc + oq + (kk >> 2) * kQc + 2 * (kk & 3), idesc, kk > 0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t qd = dsc + oq + (kk >> 2) * kQc + hh * kQh + 2 * (kk & 3);
+              const uint64_t kd = dsc + ok + s * kKs + (kk >> 2) * kKc + 2 * (kk & 3);
+              if constexpr (PASS == 0) mma_bf16(dcol, qd, kd, idesc, kk > 0);   // S[row][key]
+              else mma_bf16(dcol, kd, qd, idesc, kk > 0);                       // S^T[key][row]
+            }
+            tc_commit(&sm.s_full[buf][hh]);
           }
-          tc_commit(&sm.s_full[buf]);
+          if (!ok_run) break;
           tc_commit(&sm.k_empty[s]);
         }
       }
@@ -277,111 +351,131 @@ __global__ void __launch_bounds__(kCmThreads, 1)
       mbar_wait(&sm.drain, 0, &g_vl_status, kStatusTimeoutDrain);
     }
   } else {
-    // ------------------------------------------------------------ softmax warpgroups
-    // warp w reads TMEM lanes 32 (w % 4) ..; warpgroup wg = 0, 1 takes S columns
-    // [128 wg, 128 wg + 128) of each buffer (pass 0: the rows 128 wg + lane of its own;
-    // pass 1: rows 128 wg .. 128 wg + 127 of the key in its lane)
-    const int wg = (warp - 2) >> 2, lq = 32 * (warp & 3) + lane;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 128u * wg;
+    // ------------------------------------------------------------ softmax groups
+    // Two groups of four warps take alternate key tiles (group g the tiles T with T % 2 = g,
+    // whose products sit in S buffer g), so one group's wait for its products and its TMEM
+    // loads overlap the other group's exponentials.  Warp w reads TMEM lanes 32 (w % 4) ..;
+    // a thread takes the buffer's two 128-column halves one after the other (pass 0: rows
+    // lq and 128 + lq, a running maximum and sum each; pass 1: rows 0..255 of key lq).
+    const int g = (warp - 2) >> 2, lq = 32 * (warp & 3) + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + 256u * g;
+    const float2 c2 = make_float2(p.c2, p.c2);
     int T = 0, nq = 0, cur = -1;
     bool ok_run = true;
     for (int u = u0; ok_run && u < u1; ++u) {
       const CmItem it = cm_item(p, u);
       const int64_t bh = it.bh;
+      const int T0 = T;
+      T += it.n_tiles;
       if constexpr (PASS == 0) {
-        float m_run = -INFINITY, l_run = 0.0f;
-        for (int j = 0; j < it.n_tiles; ++j, ++T) {
-          const int buf = T & 1;
-          if (!cm_warp_wait(&sm.s_full[buf], (T >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) {
-            ok_run = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t r[4][32];
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(trow + 256u * buf + 32u * q4, r[q4]);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_free[buf]);
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+        for (int j = ((T0 & 1) == g) ? 0 : 1; j < it.n_tiles; j += 2) {
+          const int t = T0 + j;
           const int valid = min(kCmKeys, it.key_end - (it.key_begin + j * kCmKeys));
-          if (valid < kCmKeys) {
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            if (!cm_warp_wait(&sm.s_full[g][hh], (t >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) {
+              ok_run = false;
+              break;
+            }
+            tc_fence_after();
+            uint32_t r[4][32];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tl + 128u * hh + 32u * q4, r[q4]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.s_free[g][hh]);
+            if (valid < kCmKeys) {
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (32 * q4 + i >= valid) r[q4][i] = __float_as_uint(-INFINITY);
+            }
+            float mx[4];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              float tt[11];
+#pragma unroll
+              for (int i = 0; i < 10; ++i)
+                tt[i] = vl_max3(__uint_as_float(r[q4][3 * i]), __uint_as_float(r[q4][3 * i + 1]),
+                                __uint_as_float(r[q4][3 * i + 2]));
+              tt[10] = fmaxf(__uint_as_float(r[q4][30]), __uint_as_float(r[q4][31]));
+              const float u0 = vl_max3(tt[0], tt[1], tt[2]), u1 = vl_max3(tt[3], tt[4], tt[5]);
+              const float u2 = vl_max3(tt[6], tt[7], tt[8]), u3 = fmaxf(tt[9], tt[10]);
+              mx[q4] = fmaxf(vl_max3(u0, u1, u2), u3);
+            }
+            const float m_old = m_run[hh];
+            const float m_new = fmaxf(m_old, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.c2);
+            const float2 nm2 = make_float2(-m_new, -m_new);
+            const float2 o[8] = {nm2, nm2, nm2, nm2, nm2, nm2, nm2, nm2};
+            float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (32 * q4 + i >= valid) r[q4][i] = __float_as_uint(-INFINITY);
+              for (int i = 0; i < 32; i += 16) vl_sum16(&r[q4][i], c2, o, acc0, acc1);
+            l_run[hh] = (m_old == -INFINITY ? 0.0f : l_run[hh] * vl_ex2(m_old - m_new)) +
+                        ((acc0.x + acc0.y) + (acc1.x + acc1.y));
+            m_run[hh] = m_new;
           }
-          float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              mx0 = fmaxf(mx0, __uint_as_float(r[q4][i]));
-              mx1 = fmaxf(mx1, __uint_as_float(r[q4][i + 1]));
-            }
-          const float m_new = fmaxf(m_run, fmaxf(mx0, mx1) * p.c2);
-          const float nm = -m_new;
-          float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              a0 += vl_ex2(fmaf(__uint_as_float(r[q4][i]), p.c2, nm));
-              a1 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 1]), p.c2, nm));
-              a2 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 2]), p.c2, nm));
-              a3 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 3]), p.c2, nm));
-            }
-          l_run = (m_run == -INFINITY ? 0.0f : l_run * vl_ex2(m_run - m_new)) + ((a0 + a1) + (a2 + a3));
-          m_run = m_new;
+          if (!ok_run) break;
         }
         if (!ok_run) break;
-        const int row = 128 * wg + lq;
-        if (row < p.R) {
-          float* dst = p.part + ((bh * p.R + row) * p.chunks + it.chunk) * 2;
-          dst[0] = m_run;
-          dst[1] = l_run;
+        // this group's partial of rows lq and 128 + lq over its tiles of the chunk
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int row = 128 * hh + lq;
+          if (row < p.R) {
+            float* dst = p.part + (((bh * p.R + row) * p.chunks + it.chunk) * 2 + g) * 2;
+            dst[0] = m_run[hh];
+            dst[1] = l_run[hh];
+          }
         }
       } else {
-        if (it.n_tiles == 0) continue;                 // the mass array was zeroed
-        if (it.bh != cur) {
-          if (nq > 0) {
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.q_free);     // done with the previous group's lse2
-          }
-          if (!cm_warp_wait(&sm.q_full, nq & 1, abort_flag, kStatusTimeoutSoftmax)) break;
-          ++nq;
-          cur = it.bh;
-        }
-        const float4* lse4 = reinterpret_cast<const float4*>(sm.lse + 128 * wg);
-        for (int j = 0; j < it.n_tiles; ++j, ++T) {
-          const int buf = T & 1;
-          if (!cm_warp_wait(&sm.s_full[buf], (T >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) {
-            ok_run = false;
-            break;
-          }
-          tc_fence_after();
-          uint32_t r[4][32];
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(trow + 256u * buf + 32u * q4, r[q4]);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sm.s_free[buf]);
-          float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 l4 = lse4[8 * q4 + i / 4];
-              a0 += vl_ex2(fmaf(__uint_as_float(r[q4][i]), p.c2, -l4.x));
-              a1 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 1]), p.c2, -l4.y));
-              a2 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 2]), p.c2, -l4.z));
-              a3 += vl_ex2(fmaf(__uint_as_float(r[q4][i + 3]), p.c2, -l4.w));
+        const int zero_end = min(it.key_begin + kVlChunk, p.L);
+        if (it.n_tiles > 0) {
+          if (it.bh != cur) {
+            if (nq > 0) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.q_free);   // done with the previous group's -lse2
             }
-          const int key = it.key_begin + j * kCmKeys + lq;
-          if (key < it.key_end) atomicAdd(p.mass + bh * p.L + key, (a0 + a1) + (a2 + a3));
+            if (!cm_warp_wait(&sm.q_full, nq & 1, abort_flag, kStatusTimeoutSoftmax)) break;
+            ++nq;
+            cur = it.bh;
+          }
+          const float2* nlse2 = reinterpret_cast<const float2*>(sm.nlse);
+          for (int j = ((T0 & 1) == g) ? 0 : 1; j < it.n_tiles; j += 2) {
+            const int t = T0 + j;
+            float2 acc0 = make_float2(0.0f, 0.0f), acc1 = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              if (!cm_warp_wait(&sm.s_full[g][hh], (t >> 1) & 1, abort_flag, kStatusTimeoutSoftmax)) {
+                ok_run = false;
+                break;
+              }
+              tc_fence_after();
+              uint32_t r[4][32];
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tl + 128u * hh + 32u * q4, r[q4]);
+              tmem_wait_ld();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sm.s_free[g][hh]);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+                for (int i = 0; i < 32; i += 16)
+                  vl_sum16(&r[q4][i], c2, &nlse2[(128 * hh + 32 * q4 + i) / 2], acc0, acc1);
+            }
+            if (!ok_run) break;
+            const int key = it.key_begin + j * kCmKeys + lq;
+            if (key < it.key_end) p.mass[bh * p.L + key] = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+          }
         }
+        // positions of the chunk past the candidate prefix carry no mass
+        if (g == 0)
+          for (int key = max(it.key_end, it.key_begin) + lq; key < zero_end; key += 128) p.mass[bh * p.L + key] = 0.0f;
       }
     }
   }
@@ -394,15 +488,15 @@ __global__ void __launch_bounds__(kCmThreads, 1)
   }
 }
 
-// partials (m, l) of every chunk -> lse2 = m + log2(l) per observation row
-__global__ void vl_lse_kernel(const float* __restrict__ part, float* __restrict__ lse2, int R, int chunks) {
+// partials (m, l) of every chunk and softmax group -> -lse2 = -(m + log2(l)) per row
+__global__ void vl_lse_kernel(const float* __restrict__ part, float* __restrict__ nlse2, int R, int chunks) {
   const int64_t bh = blockIdx.x;
   const int row = threadIdx.x;
   if (row >= R) return;
-  const float* src = part + (bh * R + row) * chunks * 2;
+  const float* src = part + (bh * R + row) * chunks * 4;
   float m = -INFINITY, l = 0.0f;
-  for (int c = 0; c < chunks; ++c) merge_ml(m, l, src[2 * c], src[2 * c + 1]);
-  lse2[bh * R + row] = l > 0.0f ? m + log2f(l) : INFINITY;
+  for (int c = 0; c < 2 * chunks; ++c) merge_ml(m, l, src[2 * c], src[2 * c + 1]);
+  nlse2[bh * R + row] = l > 0.0f ? -(m + log2f(l)) : -INFINITY;
 }
 
 struct SelParams {
@@ -545,15 +639,23 @@ __global__ void __launch_bounds__(kSelThreads, 1) vl_select_kernel(const SelPara
   for (int i = tid; i < cnt; i += kSelThreads) p.positions[bh * p.max_select + i] = pos[i];
   if (p.excl != nullptr)
     for (int i = tid; i < p.max_pages; i += kSelThreads) p.excl[bh * p.max_pages + i] = mask[i];
-  // the kept rows in 16-byte pieces, four pieces of K and V per thread in flight at a time
-  const int shift_c = p.d == 128 ? 4 : 3;                // 16-byte pieces per row: d / 8
-  const int total = cnt << shift_c;
-  constexpr int kU = 4;
-  for (int i0 = 0; i0 < total; i0 += kU * kSelThreads) {
-    uint4 kk[kU], vv[kU];
+}
+
+// The kept rows of K and V in 16-byte pieces (d / 8 per row), four pieces of each per thread
+// in flight at a time; grid (piece blocks, kv-head, sequence), after vl_select_kernel.
+constexpr int kGatherThreads = 256, kGatherUnroll = 4;
+__global__ void __launch_bounds__(kGatherThreads) vl_gather_kernel(const SelParams p) {
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int64_t bh = static_cast<int64_t>(b) * p.Hkv + h;
+  const int shift_c = p.d == 128 ? 4 : 3;
+  const int total = p.counts[bh] << shift_c;
+  const int32_t* pos = p.positions + bh * p.max_select;
+  for (int i0 = blockIdx.x * kGatherThreads * kGatherUnroll; i0 < total;
+       i0 += gridDim.x * kGatherThreads * kGatherUnroll) {
+    uint4 kk[kGatherUnroll], vv[kGatherUnroll];
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int idx = i0 + u * kSelThreads + tid;
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const int idx = i0 + u * kGatherThreads + static_cast<int>(threadIdx.x);
       if (idx < total) {
         const int r = idx >> shift_c, c = idx & ((1 << shift_c) - 1);
         const int64_t src = (bh * p.L + pos[r]) * p.d + 8 * c;
@@ -562,8 +664,8 @@ __global__ void __launch_bounds__(kSelThreads, 1) vl_select_kernel(const SelPara
       }
     }
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int idx = i0 + u * kSelThreads + tid;
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const int idx = i0 + u * kGatherThreads + static_cast<int>(threadIdx.x);
       if (idx < total) {
         const int r = idx >> shift_c, c = idx & ((1 << shift_c) - 1);
         const int64_t dst = (bh * p.max_select + r) * p.d + 8 * c;
@@ -601,13 +703,16 @@ fa4q_status vl_launch(const VlParams& vp, const SelParams& sp, const void* q_obs
   if (!make_map_3d(&tq, q_obs, 2 * D, q_rows, 1, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_3d(&tk, k, 2 * D, vp.L, static_cast<uint64_t>(vp.B) * vp.Hkv, 128, kCmKeys, CU_TENSOR_MAP_SWIZZLE_128B))
     return FA4Q_ERR_CUDA;
-  if (cudaMemsetAsync(vp.mass, 0, static_cast<size_t>(vp.B) * vp.Hkv * vp.L * sizeof(float), st) != cudaSuccess)
-    return FA4Q_ERR_CUDA;
   const int grid = std::min(vp.n_items, num_sms());
   colmass_kernel<D, 0><<<grid, kCmThreads, cm, st>>>(tq, tk, vp);
-  vl_lse_kernel<<<vp.B * vp.Hkv, vp.R, 0, st>>>(vp.part, vp.lse2, vp.R, vp.chunks);
+  vl_lse_kernel<<<vp.B * vp.Hkv, vp.R, 0, st>>>(vp.part, vp.nlse2, vp.R, vp.chunks);
   colmass_kernel<D, 1><<<grid, kCmThreads, cm, st>>>(tq, tk, vp);
   vl_select_kernel<<<dim3(vp.Hkv, vp.B), kSelThreads, sel_smem, st>>>(sp);
+  if (sp.hp_k != nullptr || sp.hp_v != nullptr) {
+    const int pieces = sp.max_select * (D / 8);
+    const int gx = (pieces + kGatherThreads * kGatherUnroll - 1) / (kGatherThreads * kGatherUnroll);
+    vl_gather_kernel<<<dim3(gx, vp.Hkv, vp.B), kGatherThreads, 0, st>>>(sp);
+  }
   return launch_status();
 }
 
@@ -619,7 +724,7 @@ using namespace fa4q;
 extern "C" size_t fa4q_vlines_workspace_size(int B, int Hq, int Hkv, int n_obs, int L) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || n_obs <= 0 || L <= 0) return 0;
   const size_t rows = static_cast<size_t>(B) * Hkv * vl_rows(Hq, Hkv, n_obs);
-  return rows * (2 * static_cast<size_t>(vl_chunks(L)) + 1) * sizeof(float);
+  return rows * (4 * static_cast<size_t>(vl_chunks(L)) + 1) * sizeof(float);
 }
 
 extern "C" fa4q_status fa4q_select_vertical_lines(
@@ -652,7 +757,7 @@ extern "C" fa4q_status fa4q_select_vertical_lines(
   if (static_cast<int64_t>(B) * Hkv * vp.chunks > 0x7fffffff) return FA4Q_ERR_UNSUPPORTED;
   vp.n_items = B * Hkv * vp.chunks;
   vp.part = static_cast<float*>(workspace);
-  vp.lse2 = vp.part + static_cast<size_t>(B) * Hkv * R * vp.chunks * 2;
+  vp.nlse2 = vp.part + static_cast<size_t>(B) * Hkv * R * vp.chunks * 4;
   vp.mass = mass;
   vp.B = B; vp.Hq = Hq; vp.Hkv = Hkv; vp.n_obs = n_obs; vp.L = L; vp.d = d; vp.R = R;
   const float sm = sm_scale > 0.0f ? sm_scale : 1.0f / sqrtf(static_cast<float>(d));
