@@ -168,22 +168,25 @@ FA4Q_DEVINL void inner_store(const InnerArgs& a, const InnerGeom& q, int64_t gi,
     a.sf[gi * q.sf_group_bytes + (int64_t)r * q.nblk + kb] = (uint8_t)s;
 }
 
-// slots 2*pair and 2*pair + 1 (the same row: ncol_sp is even), both loads issued before
-// either block is quantised (NVFP4: twice the bytes in flight per thread at little register
-// cost; MXFP4 blocks are already 64 bytes and run one per thread)
+// flat slots 2*pair and 2*pair + 1 of a group, each decoded to its own row and block (a row
+// with an odd number of slots ends inside a pair), both loads issued before either block is
+// quantised (NVFP4: twice the bytes in flight per thread at little register cost; MXFP4
+// blocks are already 64 bytes and run one per thread)
 template <int BLK>
 FA4Q_DEVINL void quant_inner_pair(const InnerArgs& a, int64_t gi, int pair) {
   const InnerGeom q = inner_geom<BLK>(a);
+  const int total = q.rows_sp * q.ncol_sp;
   const int idx = 2 * pair;
-  if (idx >= q.rows_sp * q.ncol_sp) return;
-  const int r = idx / q.ncol_sp;
-  const int kb = idx - r * q.ncol_sp;
-  const bool real0 = r < q.rows_i && kb < q.nblk, real1 = r < q.rows_i && kb + 1 < q.nblk;
+  if (idx >= total) return;
+  const int r0 = idx / q.ncol_sp, kb0 = idx - r0 * q.ncol_sp;
+  const bool has1 = idx + 1 < total;
+  const int r1 = kb0 + 1 < q.ncol_sp ? r0 : r0 + 1, kb1 = kb0 + 1 < q.ncol_sp ? kb0 + 1 : 0;
+  const bool real0 = r0 < q.rows_i && kb0 < q.nblk, real1 = has1 && r1 < q.rows_i && kb1 < q.nblk;
   float v0[BLK], v1[BLK];
-  if (real0) inner_load<BLK>(a, gi, r, kb, v0);
-  if (real1) inner_load<BLK>(a, gi, r, kb + 1, v1);
-  inner_store<BLK>(a, q, gi, r, kb, v0, real0);
-  inner_store<BLK>(a, q, gi, r, kb + 1, v1, real1);
+  if (real0) inner_load<BLK>(a, gi, r0, kb0, v0);
+  if (real1) inner_load<BLK>(a, gi, r1, kb1, v1);
+  inner_store<BLK>(a, q, gi, r0, kb0, v0, real0);
+  if (has1) inner_store<BLK>(a, q, gi, r1, kb1, v1, real1);
 }
 
 // slots handled by one thread of the inner quantiser
@@ -378,7 +381,8 @@ __global__ void __launch_bounds__(256) quant_qkv_kernel(const InnerArgs aq, cons
   if (cta < gr.n_q + gr.n_k) {
     const bool is_q = cta < gr.n_q;
     const int64_t flat = (is_q ? cta : cta - gr.n_q) * 256 + threadIdx.x;
-    const int64_t per = (is_q ? gr.per_group_q : gr.per_group_k) / inner_slots_per_thread<BLK>();
+    constexpr int64_t spt = inner_slots_per_thread<BLK>();
+    const int64_t per = ((is_q ? gr.per_group_q : gr.per_group_k) + spt - 1) / spt;
     const int64_t gi = flat / per;
     if (gi < (is_q ? gr.groups_q : gr.groups_k)) quant_inner_work<BLK>(is_q ? aq : ak, gi, (int)(flat - gi * per));
     return;
@@ -554,7 +558,7 @@ extern "C" fa4q_status fa4q_quantize(const void* x, int64_t groups, int64_t rows
     const int64_t per_group = rows_sp * ncol_sp;
     if (groups > 65535 || per_group > (int64_t)1 << 30 || rows > ((int64_t)1 << 30)) return FA4Q_ERR_UNSUPPORTED;
     const int64_t spt = blk == 16 ? inner_slots_per_thread<16>() : inner_slots_per_thread<32>();
-    dim3 grid((unsigned)((per_group / spt + 255) / 256), (unsigned)groups);
+    dim3 grid((unsigned)(((per_group + spt - 1) / spt + 255) / 256), (unsigned)groups);
     const int64_t mh = smooth_heads > 0 ? smooth_heads : 1, mr = smooth_ratio > 0 ? smooth_ratio : 1;
     const InnerArgs ia{(const uint16_t*)x, rows, cols, row_stride, qm, g, smooth_mul, mh, mr, tiled,
                        packed_out, scales_out};
@@ -718,8 +722,8 @@ extern "C" fa4q_status fa4q_quantize_qkv(const void* q, const void* k, const voi
   gr.groups_q = static_cast<int64_t>(B) * Hq;
   gr.groups_k = gr.groups_v = static_cast<int64_t>(B) * Hkv;
   const int64_t spt = blk == 16 ? inner_slots_per_thread<16>() : inner_slots_per_thread<32>();
-  gr.n_q = S_q > 0 ? (gr.groups_q * gr.per_group_q / spt + 255) / 256 : 0;
-  gr.n_k = S_k > 0 ? (gr.groups_k * gr.per_group_k / spt + 255) / 256 : 0;
+  gr.n_q = S_q > 0 ? (gr.groups_q * ((gr.per_group_q + spt - 1) / spt) + 255) / 256 : 0;
+  gr.n_k = S_k > 0 ? (gr.groups_k * ((gr.per_group_k + spt - 1) / spt) + 255) / 256 : 0;
   const int64_t rows_pad_v = (static_cast<int64_t>(S_k) + 31) / 32 * 32;
   gr.tok_tiles = S_k > 0 ? (rows_pad_v + 127) / 128 : 0;
   gr.ch_tiles = (d + 127) / 128 * 2;                  // tiled layout: channels padded to 128

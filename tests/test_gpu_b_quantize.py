@@ -51,6 +51,19 @@ def test_inner_bit_exact(fmt, qmax, g, tiled):
             assert np.array_equal(s[gi], rs), f"scales group {gi}"
 
 
+@pytest.mark.parametrize("fmt,cols", [("nvfp4", 48), ("nvfp4", 80), ("mxfp4", 96)])
+def test_inner_odd_blocks_per_row(fmt, cols):
+    """Row-major scales with an odd number of blocks per row: a work unit of two slots then
+    spans the end of one row and the start of the next, and an odd slot count ends in a
+    single slot."""
+    x = _wide((3, 51, cols), 5 + cols, F.block_size(fmt))
+    p, s = _run_inner(x, fmt, tiled=False)
+    for gi in range(3):
+        rp, rs = F.quantize_rows(x[gi], fmt)
+        assert np.array_equal(p[gi], rp), f"packed mismatch in group {gi}"
+        assert np.array_equal(s[gi], rs), f"scales group {gi}"
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
 def test_inner_head_dim_64(fmt):
     blk = F.block_size(fmt)
