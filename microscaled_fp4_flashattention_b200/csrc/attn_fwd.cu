@@ -51,6 +51,10 @@ constexpr int kThreads = 384;
 // 16128 of the scheduler's 16384); warpgroup 0 (TMA, MMA, 2 idle warps) drops to 56 and the
 // two softmax warpgroups rise to 224: 56*32 + 2*224*32 = 16128, the launch total exactly.
 constexpr int kRegsIssue = 56, kRegsSoftmax = 224;
+// The hybrid instantiation's TMA and MMA warps carry the full-precision rings' counters,
+// barriers and descriptors on top: 56 registers made them spill 156 bytes; 104 / 200 keeps
+// the block's total (4 x 32 x 104 + 8 x 32 x 200 = 384 x 168) and spills 4 bytes.
+constexpr int kRegsIssueHyb = 104, kRegsSoftmaxHyb = 200;
 constexpr int kStages = 4;      // K/V tile stages (tiles mostly served from L2)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kGpNvfp4 = 1.0f / 2688.0f;  // g_P = 1/(6*448), rounded to FP32
@@ -497,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
 
   if (warp < 4) {
-  setmaxnreg_dec<kRegsIssue>();
+  setmaxnreg_dec<HYB ? kRegsIssueHyb : kRegsIssue>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
@@ -756,7 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   } else {
-    setmaxnreg_inc<kRegsSoftmax>();
+    setmaxnreg_inc<HYB ? kRegsSoftmaxHyb : kRegsSoftmax>();
     // ------------------------------------------------------------ softmax / PNQ / epilogue
     // Two softmax groups of four warps: group A (warps 4-7) takes the even key tiles, group B
     // (warps 8-11) the odd ones; each thread owns one full query row of its tiles, and the TMEM
