@@ -795,6 +795,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     float lpt = 0.0f;                              // sum of P~ of this group (ABL), MMA units
     const float gp_item = ABL ? p.gp : kGpNvfp4;
     const int nb = it.nw + it.nv;                  // full-precision tiles (hybrid) come first
+    // vertical-line entries visible to this row (positions ascending: those <= row - W), so a
+    // vertical-line tile masks by entry index alone
+    int nvis_row = 0;
+    if constexpr (HYB) {
+      if (it.nv > 0) {
+        const int bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv), lim = row - p.hy_window;
+        const int32_t* pos = p.hy_vl_pos + (int64_t)bh_k * p.hy_max_vl;
+        int lo = 0, hi = min(p.hy_vl_count[bh_k], p.hy_max_vl);
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (pos[mid] <= lim) lo = mid + 1;
+          else hi = mid;
+        }
+        nvis_row = lo;
+      }
+    }
     // bring accumulator g from the maximum it holds (tile j-2) to m_new (rows whose maximum
     // did not move keep alpha = 1; -inf to -inf, a row without a visible key yet, too)
     auto rescale_to = [&](int j, float m_new) {
@@ -850,15 +866,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!(key <= row && key > row - p.hy_window && key < p.S_k)) sh[i] = -INFINITY;
             }
           } else {
-            // gathered vertical lines: entry e (< the kv-head's count) at position <= row - W
-            const int e0 = (j - it.nw) * kHyKeys, bh_k = it.b * p.Hkv + it.h / (p.Hq / p.Hkv);
-            const int cnt = min(p.hy_vl_count[bh_k], p.hy_max_vl), lim = row - p.hy_window;
-            const int32_t* pos = p.hy_vl_pos + (int64_t)bh_k * p.hy_max_vl;
+            // gathered vertical lines: entry e visible to this row when e < nvis_row
+            const int e0 = (j - it.nw) * kHyKeys;
 #pragma unroll
-            for (int i = 0; i < kHyKeys; ++i) {
-              const int e = e0 + i;
-              if (!(e < cnt && pos[min(e, cnt - 1)] <= lim)) sh[i] = -INFINITY;
-            }
+            for (int i = 0; i < kHyKeys; ++i)
+              if (e0 + i >= nvis_row) sh[i] = -INFINITY;
           }
           const float tmax = block_max<kHyKeys>(sh);
           float m_prev = -INFINITY;
