@@ -51,11 +51,11 @@ FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS = 6650.0, 1590.0
 # that it stays small; the traffic is stored per unit (query head, sequence) and scaled to
 # the timed batch, the operand reads growing in proportion to the units.
 NCU_TRAFFIC = {
-    # profiles/attn_fwd_noncausal_mxfp4_uos_s32768.md: 107,093,760 + 88,925,952 B for 16 of the
+    # profiles/attn_fwd_noncausal_mxfp4_uos_s32768.md: 107,980,544 + 89,369,088 B for 16 of the
     # 40 heads (the output write-back that stays in L2 at the end of the launch is not in it)
     "attn_fwd": {"sources": ("attn_fwd.cu", "fa4q_common.cuh"), "workload": "noncausal_mxfp4_uos_h40_s32768",
-                 "sha256": "5bfd3825d05e16abfe8379c50ffa1ef171f2fd1182a69fb777ee28ff4433e925",
-                 "bytes_per_unit": (107093760 + 88925952) / 16},
+                 "sha256": "de54c21559c148c16d65baacc7df36b6f7fab41261fa03952cb237cee838653d",
+                 "bytes_per_unit": (107980544 + 89369088) / 16},
     # profiles/decode_split_paged_nvfp4_b8_l32k.md: 358,902,272 + 8,193,536 B for 8 sequences
     "decode": {"sources": ("decode.cu", "fa4q_common.cuh"), "workload": None,
                "sha256": "ba940cd89265356d949f7a42e68a6b04591dda9da095edeabffefb29fc940c4f",

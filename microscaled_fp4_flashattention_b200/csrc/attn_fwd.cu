@@ -852,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
-              for (int i = 0; i < 32; ++i) sh[32 * c + i] = __uint_as_float(raw[c][i]) * p.hy_inv_gqgk;
+              for (int i = 0; i < 32; ++i) sh[32 * c + i] = __uint_as_float(raw[c][i]);
           }
           tc_fence_before();
           __syncwarp();
@@ -872,7 +872,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < kHyKeys; ++i)
               if (e0 + i >= nvis_row) sh[i] = -INFINITY;
           }
-          const float tmax = block_max<kHyKeys>(sh);
+          // the bf16 products times hy_inv_gqgk are in the FP4 tiles' score units (a positive
+          // factor: the maximum converts after the fact, the exponent takes it in its scale)
+          const float tmax = block_max<kHyKeys>(sh) * p.hy_inv_gqgk;
           float m_prev = -INFINITY;
           if (j > 0) {
             named_bar_sync(bar_recv, 64);
@@ -884,11 +886,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           // P = 2^(s sc - m sc - lp16): the FP4 PV products' units, divided by g_v (the
           // normaliser's B operand holds g_v); a row with no visible key yet gets P = 0
           const float off = m_new > -INFINITY ? m_new * sc + p.hy_lp16 : 0.0f;
+          const float sch = sc * p.hy_inv_gqgk;
           uint32_t pk[kHyKeys / 2];
 #pragma unroll
           for (int i = 0; i < kHyKeys / 2; ++i) {
             float y0, y1;
-            ffma2(y0, y1, sh[2 * i], sh[2 * i + 1], sc, sc, -off, -off);
+            ffma2(y0, y1, sh[2 * i], sh[2 * i + 1], sch, sch, -off, -off);
             pk[i] = pack_bf16x2(ex2_approx(y0), ex2_approx(y1));
           }
           // P buffer g was last read by this group's previous PV product
