@@ -30,6 +30,29 @@ def test_tiled_loop_identity_quantizer_is_softmax(causal, S):
     assert np.max(np.abs(out - ref)) <= 1e-12
 
 
+def test_attention_plain_closed_forms():
+    """The unquantised reference against closed forms: zero queries weight every visible key
+    equally (the output is the mean of all values, or under the causal mask the mean of the
+    prefix); two keys whose scores differ by delta get the logistic weights 1 / (1 + e^-delta)
+    and 1 / (1 + e^delta); sm_scale multiplies delta."""
+    rng = np.random.default_rng(17)
+    S, d = 7, 4
+    q = np.zeros((S, d))
+    k, v = rng.normal(size=(S, d)), rng.normal(size=(S, d))
+    assert np.max(np.abs(A.attention_plain(q, k, v, causal=False) - v.mean(axis=0))) <= 1e-15
+    out = A.attention_plain(q, k, v, causal=True)
+    for i in range(S):
+        assert np.max(np.abs(out[i] - v[: i + 1].mean(axis=0))) <= 1e-15
+    q2 = np.array([[1.0, 0.0, 0.0, 0.0]])
+    k2 = np.array([[3.0, 0.0, 0.0, 0.0], [0.4, 0.0, 0.0, 0.0]])
+    v2 = np.array([[1.0, 0.0, 0.0, 0.0], [0.0, 1.0, 0.0, 0.0]])
+    for sm in (None, 0.3):
+        delta = (3.0 - 0.4) * (0.5 if sm is None else sm)          # 1 / sqrt(4) by default
+        w0 = 1.0 / (1.0 + math.exp(-delta))
+        got = A.attention_plain(q2, k2, v2, causal=False, sm_scale=sm)[0]
+        assert abs(got[0] - w0) <= 1e-15 and abs(got[1] - (1.0 - w0)) <= 1e-15 and got[2] == got[3] == 0.0
+
+
 def _scalar_pnq(q, k, v, causal, fmt, qmax_p=0.0, tau=0, stats=None):
     """Brute-force restatement with scalar Python loops (tiny inputs only).  tau > 0: the
     reference maximum moves only when a tile's maximum exceeds it by more than tau binades

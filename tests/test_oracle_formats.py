@@ -243,3 +243,29 @@ def test_smoothing_multiplier_enters_before_amax():
     p1, s1 = F.quantize_rows(x * 4.0, "nvfp4")
     p2, s2 = F.quantize_rows(x, "nvfp4", mul=mul)
     assert np.array_equal(p1, p2) and np.array_equal(s1, s2)
+
+
+def test_transposed_quantisation_hand_worked():
+    """quantize_cols_transposed against bytes worked out by hand (NVFP4, blocks of 16 tokens,
+    one block per channel and half of the 32 tokens):
+      channel 0, tokens 0..3 = 6, 3, -1.5, 0.5: amax 6 -> t = 6 / 6 = 1 -> UE4M3 0x38 (exponent
+        field 7), codes 7 (6), 5 (3), 8|3 (-1.5), 1 (0.5) -> bytes 0x57, 0x1B (low nibble first);
+      channel 1, tokens 0..3 = 2, 1, 0.5, -2: t = 2 / 6 rounds to 1.375 * 2^-2 = 0.34375 ->
+        UE4M3 0x2B; y = 5.818, 2.909, 1.455, -5.818 round to 6, 3, 1.5, -6 -> codes 7, 5, 3,
+        8|7 -> bytes 0x57, 0xF3;
+      every other token is 0, so the second block of each channel has scale byte 0."""
+    v = np.zeros((32, 2), dtype=np.float32)
+    v[:4, 0] = [6.0, 3.0, -1.5, 0.5]
+    v[:4, 1] = [2.0, 1.0, 0.5, -2.0]
+    p, s = F.quantize_cols_transposed(v, "nvfp4")
+    assert p.shape == (2, 16) and s.shape == (2, 2)
+    expect_p = np.zeros((2, 16), dtype=np.uint8)
+    expect_p[0, :2] = [0x57, 0x1B]
+    expect_p[1, :2] = [0x57, 0xF3]
+    assert p.tolist() == expect_p.tolist()
+    assert s.tolist() == [[0x38, 0x00], [0x2B, 0x00]]
+    # MXFP4 (blocks of 32 tokens, OCP rule): amax 6 -> e = floor(log2 6) - 2 = 0 -> E8M0 127,
+    # the values are their own codes; a channel of zeros gets the smallest exponent (E8M0 0)
+    pm, sm = F.quantize_cols_transposed(v[:, :1] * np.float32(1.0), "mxfp4")
+    assert pm.shape == (1, 16) and sm.tolist() == [[127]]
+    assert pm[0, :2].tolist() == [0x57, 0x1B] and not pm[0, 2:].any()
