@@ -1,4 +1,6 @@
-"""Fit the polynomial 2^f ~ c0 + c1 f + c2 f^2 + c3 f^3 on [0, 1) used by ex2_poly2 in attn_fwd.cu.
+"""Fit the polynomials 2^f ~ c0 + c1 f + ... on [0, 1) of the FMA-pipe exponentials:
+degree 3 for ex2_poly2 in attn_fwd.cu (its result feeds E2M1 rounding) and degree 4 for
+vl_ex2_fma2 in vlines.cu (column masses, relative error 2.7e-6).
 
 Minimax in relative error by Lawson's algorithm (iteratively reweighted least squares on a
 dense grid), then rounded to float32.  Prints the coefficients and the maximum relative error
@@ -26,6 +28,7 @@ def fit(deg: int = 3, n: int = 20001, iters: int = 2000):
 
 
 if __name__ == "__main__":
-    c, err = fit()
-    print("coefficients (c0..c3):", ", ".join(repr(float(x)) for x in c))
-    print("max relative error on [0, 1): %.3e" % err)
+    for deg in (3, 4):
+        c, err = fit(deg)
+        print(f"degree {deg} coefficients (c0..c{deg}):", ", ".join(repr(float(x)) for x in c))
+        print("  max relative error on [0, 1): %.3e" % err)
