@@ -373,6 +373,7 @@ def decode_bench(args, dev, fa4q, line, hbm_gbs, peak_kind, barrier):
                                    "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
                                    "traffic": ncu_traffic("decode", dw.B), "peak_source": f"{peak_kind} hbm copy"},
                       "identify": {"ms": id_ms, "every_tokens": 64, "us_per_step_amortized": id_ms * 1e3 / 64,
+                                   "share_of_decode_step": (id_ms / 64) / (d_ms + id_ms / 64),
                                    "what": "column mass of 64 observation queries x 4 q-heads over the 32640-token "
                                            "prefix, top-5% selection, exclusion mask, BF16 row gather (all 32 x 8 groups)"},
                       "l2": "working set 1.4 GB > L2", "clocks": dsampler.summary()}
