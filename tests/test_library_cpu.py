@@ -170,11 +170,12 @@ def test_more_entry_points_reject_bad_arguments_without_gpu(L):
     vws = L.fa4q_vlines_workspace_size(1, 4, 1, 64, 1024)
     assert vws > 0
 
-    def vl(rho=0.05, d=128, max_select=64, ws_bytes=vws):
+    def vl(rho=0.05, d=128, max_select=64, ws_bytes=vws, ws=fake):
         return L.fa4q_select_vertical_lines(fake, fake, fake, fake, 1, 4, 1, 64, 1024, d, D(rho), F(0), fake, fake,
-                                            fake, max_select, None, 0, None, None, fake, ws_bytes, None)
+                                            fake, max_select, None, 0, None, None, ws, ws_bytes, None)
     assert vl(rho=0.0) == 1
     assert vl(rho=1.5) == 1
     assert vl(d=96) == 2
     assert vl(max_select=51) == 1           # ceil(0.05 * 1024) = 52 slots needed
     assert vl(ws_bytes=vws - 1) == 1
+    assert vl(ws=P_(0x1008)) == 1           # the workspace must be 16-byte aligned (bulk copies)
